@@ -1,0 +1,190 @@
+"""fp64 CPU oracle for the fused SDPA forward -- test infrastructure.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never imports it and shares no code with it.
+
+The arithmetic lives in ``sdpa_oracle.c`` (plain C, fp64, OpenMP over rows);
+this module only compiles it with gcc and marshals numpy / torch CPU arrays.
+See that file's header for the formula and the passages it follows.
+
+Parity status of each function (what pins it, in ``tests/test_oracle.py``):
+  sdpa_fwd         pinned: closed forms (Sk=1, Sk=2 logistic, d=1, first causal
+                   row), invariants (rows of weights sum to 1, constant V,
+                   affine V, key permutation, LSE shift, GQA == repeated-KV
+                   MHA, causal prefix independence), a dominant key, and a
+                   40-digit mpmath evaluation on tiny inputs.
+  sdpa_rows        pinned: equals sdpa_fwd on the same rows (same per-row code
+                   reached through a different index path) and the pins above.
+  sdpa_bruteforce  pinned: mpmath evaluation, weights-sum, V = identity.
+  decode_*         pinned: all 256 e4m3 codes and all 65536 fp16 / bf16 codes
+                   against torch's own casts.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sdpa_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+F64, BF16, F16, E4M3 = 0, 1, 2, 3
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile sdpa_oracle.c into liboracle.so next to it (gcc, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+               "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        vp, i32, f64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
+        lib.oracle_sdpa_fwd.argtypes = [vp, vp, vp, i32, f64, f64, f64, vp, vp,
+                                        i32, i32, i32, i32, i32, i32, f64, i32, i32]
+        lib.oracle_sdpa_rows.argtypes = [vp, vp, vp, i32, f64, f64, f64, vp, ctypes.c_int64,
+                                         vp, vp, i32, i32, i32, i32, i32, i32, f64, i32, i32]
+        lib.oracle_sdpa_bruteforce.argtypes = [vp, vp, vp, i32, f64, f64, f64, vp, vp, vp,
+                                               i32, i32, i32, i32, i32, i32, f64, i32]
+        lib.oracle_decode_bf16.argtypes = [ctypes.c_uint16]
+        lib.oracle_decode_bf16.restype = f64
+        lib.oracle_decode_f16.argtypes = [ctypes.c_uint16]
+        lib.oracle_decode_f16.restype = f64
+        lib.oracle_decode_e4m3.argtypes = [ctypes.c_uint8]
+        lib.oracle_decode_e4m3.restype = f64
+        for fn in (lib.oracle_sdpa_fwd, lib.oracle_sdpa_rows, lib.oracle_sdpa_bruteforce):
+            fn.restype = i32
+        lib.oracle_max_threads.restype = i32
+        _lib = lib
+    return _lib
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def _raw(x):
+    """(contiguous numpy array of the storage bits, dtype code)."""
+    try:
+        import torch
+    except ImportError:  # pragma: no cover
+        torch = None
+    if torch is not None and isinstance(x, torch.Tensor):
+        x = x.detach().contiguous().cpu()
+        if x.dtype == torch.bfloat16:
+            return x.view(torch.int16).numpy().view(np.uint16), BF16
+        if x.dtype == torch.float16:
+            return x.view(torch.int16).numpy().view(np.uint16), F16
+        if x.dtype == torch.float8_e4m3fn:
+            return x.view(torch.uint8).numpy(), E4M3
+        return x.to(torch.float64).numpy(), F64
+    a = np.ascontiguousarray(x)
+    if a.dtype != np.float64:
+        a = a.astype(np.float64)
+    return a, F64
+
+
+def _shape(q, k):
+    B, Hq, Sq, d = (int(s) for s in q.shape)
+    Bk, Hkv, Sk, dk = (int(s) for s in k.shape)
+    if Bk != B or dk != d:
+        raise ValueError("q and k shapes disagree")
+    return B, Hq, Hkv, Sq, Sk, d
+
+
+def _check(rc):
+    if rc == 1:
+        raise ValueError("oracle: invalid arguments")
+    if rc == 2:
+        raise ValueError("oracle: causal attention needs Sq == Sk")
+    if rc != 0:
+        raise MemoryError("oracle: allocation failed")
+
+
+def _prep(q, k, v):
+    qa, tq = _raw(q)
+    ka, tk = _raw(k)
+    va, tv = _raw(v)
+    if not (tq == tk == tv):
+        raise ValueError("q, k, v must share one storage type")
+    return qa, ka, va, tq
+
+
+def sdpa_fwd(q, k, v, scale: float, causal: bool = False, descales=(1.0, 1.0, 1.0),
+             nthreads: int | None = None):
+    """Full forward.  q [B,Hq,Sq,d], k/v [B,Hkv,Sk,d] (torch CPU tensors in bf16,
+    fp16, float8_e4m3fn or any float, or numpy).  Returns (O, LSE) as float64
+    numpy arrays [B,Hq,Sq,d] and [B,Hq,Sq]."""
+    lib = _load()
+    qa, ka, va, t = _prep(q, k, v)
+    B, Hq, Hkv, Sq, Sk, d = _shape(q, k)
+    o = np.empty((B, Hq, Sq, d), np.float64)
+    lse = np.empty((B, Hq, Sq), np.float64)
+    nt = nthreads or max_threads()
+    _check(lib.oracle_sdpa_fwd(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, t,
+                               float(descales[0]), float(descales[1]), float(descales[2]),
+                               o.ctypes.data, lse.ctypes.data,
+                               B, Hq, Hkv, Sq, Sk, d, float(scale), int(bool(causal)), nt))
+    return o, lse
+
+
+def sdpa_rows(q, k, v, rows, scale: float, causal: bool = False, descales=(1.0, 1.0, 1.0),
+              nthreads: int | None = None):
+    """Selected rows: rows are flat indices (b*Hq + hq)*Sq + i.  Returns
+    (O_rows [n,d], LSE_rows [n]) float64."""
+    lib = _load()
+    qa, ka, va, t = _prep(q, k, v)
+    B, Hq, Hkv, Sq, Sk, d = _shape(q, k)
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    o = np.empty((r.size, d), np.float64)
+    lse = np.empty((r.size,), np.float64)
+    nt = nthreads or max_threads()
+    _check(lib.oracle_sdpa_rows(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, t,
+                                float(descales[0]), float(descales[1]), float(descales[2]),
+                                r.ctypes.data, r.size, o.ctypes.data, lse.ctypes.data,
+                                B, Hq, Hkv, Sq, Sk, d, float(scale), int(bool(causal)), nt))
+    return o, lse
+
+
+def sdpa_bruteforce(q, k, v, scale: float, causal: bool = False, descales=(1.0, 1.0, 1.0),
+                    return_weights: bool = False):
+    """Explicit-matrix forward for tiny inputs.  Returns (O, LSE) or
+    (O, LSE, W) with W the [B,Hq,Sq,Sk] attention weights."""
+    lib = _load()
+    qa, ka, va, t = _prep(q, k, v)
+    B, Hq, Hkv, Sq, Sk, d = _shape(q, k)
+    o = np.empty((B, Hq, Sq, d), np.float64)
+    lse = np.empty((B, Hq, Sq), np.float64)
+    w = np.empty((B, Hq, Sq, Sk), np.float64) if return_weights else None
+    _check(lib.oracle_sdpa_bruteforce(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, t,
+                                      float(descales[0]), float(descales[1]), float(descales[2]),
+                                      o.ctypes.data, lse.ctypes.data,
+                                      None if w is None else w.ctypes.data,
+                                      B, Hq, Hkv, Sq, Sk, d, float(scale), int(bool(causal))))
+    return (o, lse, w) if return_weights else (o, lse)
+
+
+def decode_bf16(bits: int) -> float:
+    return float(_load().oracle_decode_bf16(int(bits)))
+
+
+def decode_f16(bits: int) -> float:
+    return float(_load().oracle_decode_f16(int(bits)))
+
+
+def decode_e4m3(code: int) -> float:
+    return float(_load().oracle_decode_e4m3(int(code)))

@@ -1,0 +1,291 @@
+/*
+ * sdpa_oracle.c -- fp64 CPU oracle for the fused scaled-dot-product attention
+ * forward.  TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the
+ * benchmark's CPU-baseline leg may call it; the product path never does, and
+ * this file shares no code, header, table or helper with the CUDA library.
+ *
+ * What it computes (codelab "JAX on GPU, Lab 5: attention on GPU", section 1
+ * "How attention works", the formula Attention(Q,K,V) = softmax(Q K^T / sqrt(d_k)) V
+ * and its four steps score -> scale+softmax -> attend -> output of Q's shape;
+ * article "Self-attention, CUDA kernels and FlashAttention", section 1, the
+ * same formula for one head and "run per head in parallel"):
+ *
+ *   for every batch b, query head hq, query row i:
+ *     hk  = hq / (Hq / Hkv)                         (codelab section 9: KV heads
+ *                                                    are shared by groups of
+ *                                                    query heads; contiguous groups)
+ *     J_i = {0 .. Sk-1}, or {0 .. i} when causal     (codelab section 7: each
+ *                                                    position sees earlier ones)
+ *     s_j = scale * sum_c Q[b,hq,i,c] * K[b,hk,j,c]  for j in J_i
+ *     m   = max_j s_j ;  l = sum_j exp(s_j - m)
+ *     O[b,hq,i,:] = sum_j exp(s_j - m) / l * V[b,hk,j,:]
+ *     LSE[b,hq,i] = m + ln(l)                        (article section 3: only the
+ *                                                    small per-row normalisation
+ *                                                    statistic is kept; natural log
+ *                                                    of the scaled scores)
+ *
+ * Two passes over the row (max, then exp/sum/accumulate) in fp64; no tiling, no
+ * online rescaling.  A second routine materialises the whole score matrix of a
+ * head, applies a row softmax and multiplies by V, the structure of the
+ * codelab's from-scratch attention (section 4); it serves tiny inputs only.
+ *
+ * Layouts: Q [B,Hq,Sq,d], K and V [B,Hkv,Sk,d], O [B,Hq,Sq,d], LSE [B,Hq,Sq],
+ * all contiguous row-major.  Inputs are read in their storage type and widened
+ * exactly to double: bf16, fp16, e4m3 (OCP "fn" variant, times a per-tensor
+ * descale) or fp64.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { ORC_F64 = 0, ORC_BF16 = 1, ORC_F16 = 2, ORC_E4M3 = 3 };
+
+/* ---- exact widening of the storage formats to double ------------------- */
+
+/* bf16 is the upper half of an IEEE binary32 pattern. */
+double oracle_decode_bf16(uint16_t h) {
+    uint32_t bits = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+/* IEEE binary16: 1 sign, 5 exponent (bias 15), 10 fraction bits. */
+double oracle_decode_f16(uint16_t h) {
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1f;
+    int f = h & 0x3ff;
+    double mag;
+    if (e == 0) {
+        mag = ldexp((double)f, -24);            /* subnormal: f * 2^-10 * 2^-14 */
+    } else if (e == 31) {
+        mag = f ? NAN : INFINITY;
+    } else {
+        mag = ldexp((double)(1024 + f), e - 25); /* (1 + f/1024) * 2^(e-15) */
+    }
+    return sign ? -mag : mag;
+}
+
+/* OCP FP8 E4M3 ("fn": finite, no infinities): 1 sign, 4 exponent (bias 7),
+ * 3 fraction bits; S.1111.111 is NaN, the largest finite is 448. */
+double oracle_decode_e4m3(uint8_t c) {
+    int sign = (c >> 7) & 1;
+    int e = (c >> 3) & 0xf;
+    int f = c & 0x7;
+    double mag;
+    if (e == 15 && f == 7) {
+        mag = NAN;
+    } else if (e == 0) {
+        mag = ldexp((double)f, -9);             /* subnormal: f/8 * 2^-6 */
+    } else {
+        mag = ldexp((double)(8 + f), e - 10);   /* (1 + f/8) * 2^(e-7) */
+    }
+    return sign ? -mag : mag;
+}
+
+static double load_elem(const void* base, int dtype, size_t idx, double descale) {
+    switch (dtype) {
+    case ORC_BF16: return oracle_decode_bf16(((const uint16_t*)base)[idx]);
+    case ORC_F16:  return oracle_decode_f16(((const uint16_t*)base)[idx]);
+    case ORC_E4M3: return oracle_decode_e4m3(((const uint8_t*)base)[idx]) * descale;
+    default:       return ((const double*)base)[idx];
+    }
+}
+
+typedef struct {
+    const void *q, *k, *v;
+    int dtype;
+    double dq, dk, dv;
+    int B, Hq, Hkv, Sq, Sk, d;
+    double scale;
+    int causal;
+} problem_t;
+
+static int check_problem(const problem_t* p) {
+    if (!p->q || !p->k || !p->v) return 1;
+    if (p->B <= 0 || p->Hq <= 0 || p->Hkv <= 0 || p->Sq <= 0 || p->Sk <= 0 || p->d <= 0) return 1;
+    if (p->Hq % p->Hkv != 0) return 1;
+    if (p->causal && p->Sq != p->Sk) return 2;
+    if (p->dtype < ORC_F64 || p->dtype > ORC_E4M3) return 1;
+    return 0;
+}
+
+/* One output row (b, hq, i).  `work` holds Sk doubles. */
+static void one_row(const problem_t* p, int b, int hq, int i, double* work,
+                    double* o_row, double* lse_out) {
+    const int group = p->Hq / p->Hkv;
+    const int hk = hq / group;
+    const size_t qoff = (((size_t)b * p->Hq + hq) * p->Sq + i) * p->d;
+    const size_t kvhead = ((size_t)b * p->Hkv + hk) * p->Sk;
+    const int nkeys = p->causal ? i + 1 : p->Sk;
+
+    /* score step: s_j = scale * q_i . k_j */
+    double m = -INFINITY;
+    for (int j = 0; j < nkeys; ++j) {
+        const size_t koff = (kvhead + j) * p->d;
+        double acc = 0.0;
+        for (int c = 0; c < p->d; ++c)
+            acc += load_elem(p->q, p->dtype, qoff + c, p->dq) *
+                   load_elem(p->k, p->dtype, koff + c, p->dk);
+        work[j] = p->scale * acc;
+        if (work[j] > m) m = work[j];
+    }
+    /* softmax step (second pass) and attend step */
+    double l = 0.0;
+    for (int c = 0; c < p->d; ++c) o_row[c] = 0.0;
+    for (int j = 0; j < nkeys; ++j) {
+        const double w = exp(work[j] - m);
+        l += w;
+        const size_t voff = (kvhead + j) * p->d;
+        for (int c = 0; c < p->d; ++c)
+            o_row[c] += w * load_elem(p->v, p->dtype, voff + c, p->dv);
+    }
+    for (int c = 0; c < p->d; ++c) o_row[c] /= l;
+    *lse_out = m + log(l);
+}
+
+/*
+ * Full forward.  o: [B,Hq,Sq,d] doubles, lse: [B,Hq,Sq] doubles.
+ * Returns 0 on success, 1 for invalid arguments, 2 for causal with Sq != Sk.
+ */
+int oracle_sdpa_fwd(const void* q, const void* k, const void* v, int dtype,
+                    double dq, double dk, double dv, double* o, double* lse,
+                    int B, int Hq, int Hkv, int Sq, int Sk, int d,
+                    double scale, int causal, int nthreads) {
+    problem_t p = {q, k, v, dtype, dq, dk, dv, B, Hq, Hkv, Sq, Sk, d, scale, causal};
+    int rc = check_problem(&p);
+    if (rc) return rc;
+    if (!o || !lse) return 1;
+    const long long nrows = (long long)B * Hq * Sq;
+    if (nthreads <= 0) nthreads = 1;
+    int failed = 0;
+#pragma omp parallel num_threads(nthreads)
+    {
+        double* work = (double*)malloc(sizeof(double) * (size_t)Sk);
+        if (!work) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (long long r = 0; r < nrows; ++r) {
+                const int i = (int)(r % Sq);
+                const int hq = (int)((r / Sq) % Hq);
+                const int b = (int)(r / ((long long)Sq * Hq));
+                one_row(&p, b, hq, i, work, o + (size_t)r * d, lse + r);
+            }
+            free(work);
+        }
+    }
+    return failed ? 3 : 0;
+}
+
+/*
+ * Selected rows only: rows[t] is the flat row index (b*Hq + hq)*Sq + i.
+ * o_rows: [nrows, d], lse_rows: [nrows].  Used where the full problem is too
+ * large for the CPU (the output of every row depends on its own row only).
+ */
+int oracle_sdpa_rows(const void* q, const void* k, const void* v, int dtype,
+                     double dq, double dk, double dv,
+                     const int64_t* rows, int64_t nrows, double* o_rows, double* lse_rows,
+                     int B, int Hq, int Hkv, int Sq, int Sk, int d,
+                     double scale, int causal, int nthreads) {
+    problem_t p = {q, k, v, dtype, dq, dk, dv, B, Hq, Hkv, Sq, Sk, d, scale, causal};
+    int rc = check_problem(&p);
+    if (rc) return rc;
+    if (!rows || !o_rows || !lse_rows || nrows < 0) return 1;
+    const long long total = (long long)B * Hq * Sq;
+    for (int64_t t = 0; t < nrows; ++t)
+        if (rows[t] < 0 || rows[t] >= total) return 1;
+    if (nthreads <= 0) nthreads = 1;
+    int failed = 0;
+#pragma omp parallel num_threads(nthreads)
+    {
+        double* work = (double*)malloc(sizeof(double) * (size_t)Sk);
+        if (!work) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+#pragma omp for schedule(dynamic, 4)
+            for (int64_t t = 0; t < nrows; ++t) {
+                const long long r = rows[t];
+                const int i = (int)(r % Sq);
+                const int hq = (int)((r / Sq) % Hq);
+                const int b = (int)(r / ((long long)Sq * Hq));
+                one_row(&p, b, hq, i, work, o_rows + (size_t)t * d, lse_rows + t);
+            }
+            free(work);
+        }
+    }
+    return failed ? 3 : 0;
+}
+
+/*
+ * Brute force, the explicit-matrix structure of the codelab's from-scratch
+ * attention (section 4): per head, build the whole Sq x Sk score matrix
+ * (masked entries = -inf), scale it, apply a row softmax in place (weights),
+ * then multiply the weight matrix by V.  The weights are also returned when
+ * `weights` is non-null ([B,Hq,Sq,Sk]).  Meant for tiny inputs.
+ */
+int oracle_sdpa_bruteforce(const void* q, const void* k, const void* v, int dtype,
+                           double dq, double dk, double dv, double* o, double* lse,
+                           double* weights,
+                           int B, int Hq, int Hkv, int Sq, int Sk, int d,
+                           double scale, int causal) {
+    problem_t p = {q, k, v, dtype, dq, dk, dv, B, Hq, Hkv, Sq, Sk, d, scale, causal};
+    int rc = check_problem(&p);
+    if (rc) return rc;
+    if (!o || !lse) return 1;
+    double* S = (double*)malloc(sizeof(double) * (size_t)Sq * Sk);
+    if (!S) return 3;
+    const int group = Hq / Hkv;
+    for (int b = 0; b < B; ++b) {
+        for (int hq = 0; hq < Hq; ++hq) {
+            const int hk = hq / group;
+            const size_t qh = ((size_t)b * Hq + hq) * Sq;
+            const size_t kh = ((size_t)b * Hkv + hk) * Sk;
+            /* scores = (Q K^T) * scale, causal entries above the diagonal -inf */
+            for (int i = 0; i < Sq; ++i)
+                for (int j = 0; j < Sk; ++j) {
+                    double acc = 0.0;
+                    for (int c = 0; c < d; ++c)
+                        acc += load_elem(q, dtype, (qh + i) * d + c, dq) *
+                               load_elem(k, dtype, (kh + j) * d + c, dk);
+                    S[(size_t)i * Sk + j] = (causal && j > i) ? -INFINITY : acc * scale;
+                }
+            /* row softmax in place; keep each row's log normaliser */
+            for (int i = 0; i < Sq; ++i) {
+                double* row = S + (size_t)i * Sk;
+                double m = -INFINITY;
+                for (int j = 0; j < Sk; ++j) m = row[j] > m ? row[j] : m;
+                double l = 0.0;
+                for (int j = 0; j < Sk; ++j) { row[j] = exp(row[j] - m); l += row[j]; }
+                for (int j = 0; j < Sk; ++j) row[j] /= l;
+                lse[qh + i] = m + log(l);
+            }
+            if (weights)
+                memcpy(weights + qh * (size_t)Sk, S, sizeof(double) * (size_t)Sq * Sk);
+            /* weights @ V */
+            for (int i = 0; i < Sq; ++i)
+                for (int c = 0; c < d; ++c) {
+                    double acc = 0.0;
+                    for (int j = 0; j < Sk; ++j)
+                        acc += S[(size_t)i * Sk + j] * load_elem(v, dtype, (kh + j) * d + c, dv);
+                    o[(qh + i) * d + c] = acc;
+                }
+        }
+    }
+    free(S);
+    return 0;
+}
+
+int oracle_max_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
