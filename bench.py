@@ -1,0 +1,350 @@
+"""Benchmark of the fused SDPA forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one fused forward (one kernel launch) over the whole workload with
+Q, K, V resident in HBM.  Default workload: causal LM attention, B=8, Hq=Hkv=16,
+Sq=Sk=4096, d=128, bf16 -- the Sk >= 4096, d = 128 case the tensor-core target
+is stated on.  Q+K+V are 402 MB, above the 126 MB L2, so no step starts with
+its inputs in L2.  Under torchrun every rank runs its own copy of the workload
+(independent batches, weak scaling, no data-path collective); the process
+group only carries the barrier and the max-over-ranks of the timings.
+
+`--impl reference` times the fp64 CPU oracle on the host cores instead (rank
+0 only), each step a bounded random sample of the workload's rows.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd TFLOP/s on 1 B200 and % of dense BF16/FP8 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="lm_causal")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic(workload_name):
+    """DRAM bytes per launch from the committed ncu summary of this kernel
+    and workload, if one exists for the current kernel build."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload_name)
+    return None if e is None else e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only; nothing is changed)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
+
+    def __init__(self, index):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.error = str(e)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                self.samples.append(mhz)
+                for b, name in self.REASONS.items():
+                    if bits & b and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.02)
+
+    def start(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (reported baseline, and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_rows_tflops(w, q, k, v, nrows, seed, nthreads, descales=(1.0, 1.0, 1.0)):
+    """Time the oracle on `nrows` random rows; returns (seconds, flops)."""
+    import numpy as np
+    import oracle
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.integers(0, w.B * w.Hq * w.Sq, size=nrows))
+    i = rows % w.Sq
+    keys = (i + 1) if w.causal else np.full_like(i, w.Sk)
+    flops = float(4.0 * w.d * keys.sum())
+    t0 = time.perf_counter()
+    oracle.sdpa_rows(q, k, v, rows, w.scale, w.causal, descales=descales, nthreads=nthreads)
+    return time.perf_counter() - t0, flops
+
+
+def cpu_inputs(w):
+    from sdpa_workloads import make_qkv, make_qkv_fp8
+    if w.dtype == "e4m3":
+        q8, k8, v8, ds, _ = make_qkv_fp8(w)
+        return q8, k8, v8, ds
+    q, k, v = make_qkv(w)
+    return q, k, v, (1.0, 1.0, 1.0)
+
+
+def cpu_baseline(w, seconds):
+    import oracle
+    nt = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    q, k, v, ds = cpu_inputs(w)
+    t, f = oracle_rows_tflops(w, q, k, v, 64, 1, nt, ds)          # calibrate
+    nrows = int(max(64, min(200000, 64 * seconds / max(t, 1e-6))))
+    t, f = oracle_rows_tflops(w, q, k, v, nrows, 2, nt, ds)
+    return {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": nt, "kind": "oracle",
+            "sample": "%d random rows of %s (all batches/heads), fp64 C oracle, OpenMP, %.1f s"
+                      % (nrows, w.name, t)}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    nt = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    q, k, v, ds = cpu_inputs(w)
+    t, _ = oracle_rows_tflops(w, q, k, v, 32, 7, nt, ds)
+    per_row = t / 32
+    budget = 90.0
+    rows_per_step = int(max(1, min(4096, budget / max(1, args.steps + args.warmup) / per_row)))
+    for s in range(args.warmup):
+        oracle_rows_tflops(w, q, k, v, rows_per_step, 100 + s, nt, ds)
+    tot_t, tot_f = 0.0, 0.0
+    for s in range(args.steps):
+        t, f = oracle_rows_tflops(w, q, k, v, rows_per_step, 1000 + s, nt, ds)
+        tot_t += t
+        tot_f += f
+    value = tot_f / tot_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": dict(w.describe(), parallelism="none (host cores)"),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": nt, "kind": "oracle",
+                         "sample": "%d random rows per step of %s, fp64 C oracle, OpenMP"
+                                   % (rows_per_step, w.name)},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def main():
+    args = parse()
+    from sdpa_workloads import WORKLOADS, make_qkv, make_qkv_fp8, sample_rows
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE %d" % (args.gpus, world))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    import scaled_dot_product_11_b200 as sdpa
+    fp8 = w.dtype == "e4m3"
+    if fp8:
+        q, k, v, ds, _ = make_qkv_fp8(w, dev)
+        run = lambda: sdpa.attention_fp8(q, k, v, ds, causal=w.causal, scale=w.scale, out=o, lse=lse)
+    else:
+        q, k, v = make_qkv(w, dev)
+        run = lambda: sdpa.attention(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse)
+    o = torch.empty((w.B, w.Hq, w.Sq, w.d), dtype=torch.bfloat16 if fp8 or w.dtype == "bf16"
+                    else torch.float16, device=dev)
+    lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # warm-up (also the parity spot check of this exact launch configuration)
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+    st, detail = sdpa.sdpa_device_status(clear=True)
+    if st != 0:
+        raise SystemExit("device status %d (%#x) after warm-up" % (st, detail))
+    parity = None
+    if rank == 0:
+        import oracle
+        rows = sample_rows(w, n_random=32)[:: max(1, len(sample_rows(w, n_random=32)) // 96)]
+        qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
+        ro, rl = oracle.sdpa_rows(qc, kc, vc, rows, w.scale, w.causal,
+                                  descales=ds if fp8 else (1.0, 1.0, 1.0))
+        idx = torch.tensor(rows, device=dev)
+        go = o.reshape(-1, w.d).index_select(0, idx).double().cpu().numpy()
+        gl = lse.reshape(-1).index_select(0, idx).double().cpu().numpy()
+        parity = {"rows": len(rows), "max_abs_o": float(np.abs(go - ro).max()),
+                  "max_abs_lse": float(np.abs(gl - rl).max())}
+
+    # timed region: device time with CUDA events on the launching stream
+    stream = torch.cuda.current_stream(dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        run()
+    e1.record(stream)
+    e1.synchronize()
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    st, detail = sdpa.sdpa_device_status(clear=True)
+    if st != 0:
+        raise SystemExit("device status %d (%#x) after timing" % (st, detail))
+    ms_per_step = ms_total / args.steps
+    value = world * w.flops * args.steps / (ms_total * 1e-3) / 1e12
+
+    # end to end through the public API: pinned host inputs -> device -> fused
+    # forward -> O and LSE back to pinned host memory, all inside the region
+    e2e_steps = max(3, min(20, args.steps // 20))
+    hq_, hk_, hv_ = (t.cpu().pin_memory() for t in (q, k, v))
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def run_e2e():
+        dq.copy_(hq_, non_blocking=True)
+        dk.copy_(hk_, non_blocking=True)
+        dv.copy_(hv_, non_blocking=True)
+        if fp8:
+            sdpa.attention_fp8(dq, dk, dv, ds, causal=w.causal, scale=w.scale, out=o, lse=lse)
+        else:
+            sdpa.attention(dq, dk, dv, causal=w.causal, scale=w.scale, out=o, lse=lse)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    run_e2e()
+    torch.cuda.synchronize()
+    barrier()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        run_e2e()
+    e1.record(stream)
+    e1.synchronize()
+    barrier()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1))
+    h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
+    d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
+    e2e_value = world * w.flops * e2e_steps / (ms_e2e * 1e-3) / 1e12
+
+    if rank == 0:
+        peaks, src = load_peaks()
+        peak = float(peaks["bf16_tflops"])
+        achieved = w.flops / (ms_per_step * 1e-3) / 1e12
+        traffic = load_traffic(w.name)
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3" if fp8 else w.dtype, "data": "synthetic",
+            "config": dict(w.describe(), global_batch=w.B * world,
+                           parallelism="dp%d (independent batches per GPU)" % world,
+                           l2="inputs %.0f MB per GPU > 126 MB L2; no flush" % (
+                               sum(t.numel() * t.element_size() for t in (q, k, v)) / 1e6)),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": "%s bf16_tflops (burst); frac of sustained %.3f" % (
+                             src, achieved / float(peaks["bf16_tflops_sustained"]))},
+            "clocks": clk,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": args.steps * sdpa.sdpa_launches_per_call(),
+            "parity": parity,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

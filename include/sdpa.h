@@ -1,0 +1,139 @@
+/*
+ * sdpa.h -- C ABI of the B200 (sm_100a) fused scaled-dot-product attention
+ * forward library (libsdpa_b200.so).
+ *
+ * The operation (codelab "JAX on GPU, Lab 5: attention on GPU", section 1 "How
+ * attention works": Attention(Q,K,V) = softmax(Q K^T / sqrt(d_k)) V in four
+ * steps -- score, scale + softmax, attend, output of Q's shape; section 7: the
+ * causal (lower-triangular) mask applied inside the fused kernel; section 9:
+ * K/V heads shared by groups of query heads, MHA / GQA / MQA; article
+ * "Self-attention, CUDA kernels and FlashAttention", section 3: tiles kept on
+ * chip, online softmax with running max and sum, only the per-row
+ * normalisation statistic written to memory):
+ *
+ *   for b < B, hq < Hq, i < Sq:
+ *     hk = hq / (Hq / Hkv)                         contiguous head groups
+ *     s_j = scale * <Q[b,hq,i,:], K[b,hk,j,:]>     j < Sk  (j <= i if causal)
+ *     O[b,hq,i,:] = sum_j softmax_j(s) * V[b,hk,j,:]
+ *     LSE[b,hq,i] = ln sum_j exp(s_j)              natural log, fp32
+ *
+ * The Sq x Sk score matrix never reaches global memory.
+ *
+ * Layout (all entry points): Q [B,Hq,Sq,d], K and V [B,Hkv,Sk,d],
+ * O [B,Hq,Sq,d], LSE [B,Hq,Sq]; every tensor dense row-major ("BHSD"), device
+ * pointers, 16-byte aligned.  (The codelab's JAX arrays are (B,T,N,H); this
+ * library takes the head-major order.)
+ *
+ * Ownership: the caller owns every buffer.  The entry points allocate no
+ * memory, keep no state between calls other than cached per-device set-up
+ * (driver entry points, kernel attributes) and a device status word, and
+ * never synchronise: work is queued on `stream` (a cudaStream_t; NULL = the
+ * legacy default stream) and errors raised while it runs surface at the
+ * caller's next synchronisation.
+ *
+ * Errors: every entry point returns an sdpa_status.  There is no fallback
+ * path: a request the kernels cannot serve is refused with a status (the
+ * codelab's cuDNN back-end likewise raises instead of silently falling back,
+ * section 6).  Q/K/V/O/LSE must not overlap; O and LSE may be any device
+ * memory of the right size.
+ */
+#ifndef SDPA_B200_H
+#define SDPA_B200_H
+
+#if defined(__GNUC__)
+#define SDPA_API __attribute__((visibility("default")))
+#else
+#define SDPA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SDPA_BF16 = 0,   /* bfloat16 Q/K/V/O */
+    SDPA_FP16 = 1    /* float16  Q/K/V/O */
+} sdpa_dtype;
+
+typedef enum {
+    SDPA_OK = 0,
+    SDPA_ERR_INVALID_ARG = 1,    /* null pointer, a size <= 0, Hq % Hkv != 0,
+                                    non-finite or non-positive scale, a pointer
+                                    not 16-byte aligned, sizes whose element
+                                    counts overflow the addressing limits */
+    SDPA_ERR_UNSUPPORTED = 2,    /* d not 64 or 128, causal with Sq != Sk,
+                                    unknown dtype, device not sm_100 */
+    SDPA_ERR_CUDA = 3,           /* the CUDA runtime or driver reported an
+                                    error while preparing or launching */
+    SDPA_ERR_DEVICE_TIMEOUT = 4  /* a kernel's bounded wait expired (reported
+                                    by sdpa_device_status only) */
+} sdpa_status;
+
+/*
+ * sdpa_fwd -- fused attention forward, bf16 or fp16.
+ *
+ *   q    [B,Hq,Sq,d]  in,  dtype
+ *   k, v [B,Hkv,Sk,d] in,  dtype
+ *   o    [B,Hq,Sq,d]  out, dtype (rounded to nearest even from fp32)
+ *   lse  [B,Hq,Sq]    out, float32, natural-log logsumexp of the scaled
+ *                     scores of each row (may be NULL to skip it)
+ *   scale            applied to Q K^T as given; pass 1/sqrt(d) for the
+ *                    codelab's default (section 4, scale = 1/sqrt(H))
+ *   causal           0: every key; 1: key j only for query i >= j (needs
+ *                    Sq == Sk)
+ *   dtype            an sdpa_dtype
+ *   stream           cudaStream_t to enqueue on
+ *
+ * Accumulation is fp32 in tensor memory; the softmax weights are rounded to
+ * the input dtype before the P*V product while the row sums use fp32.
+ */
+SDPA_API int sdpa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+             int B, int Hq, int Hkv, int Sq, int Sk, int d,
+             float scale, int causal, int dtype, void* stream);
+
+/*
+ * sdpa_fwd_fp8 -- the same forward with FP8 E4M3 ("fn", max 448) Q/K/V.
+ *
+ * The codelab runs attention in E4M3 for the forward pass with per-tensor
+ * scaling factors (section 10, "Check the FP8 path").  Here the scaling is
+ * per tensor and current: the caller quantises x8 = e4m3(x / descale_x) with
+ * descale_x = amax(|x|) / 448 and passes descale_x, so the value a code
+ * stands for is code * descale_x.
+ *
+ *   q8, k8, v8       e4m3 codes, layouts as above
+ *   descale_q/k/v    host floats, > 0 and finite
+ *   o                bf16 [B,Hq,Sq,d]
+ *   lse              float32 [B,Hq,Sq] or NULL
+ *
+ * The softmax weights p in [0, 1] are themselves quantised to e4m3 as
+ * e4m3(448 * p) (the amax rule with amax(p) = 1) for the P*V product, whose
+ * result is multiplied back by descale_v / 448; row sums use fp32 p.
+ * Errors as sdpa_fwd; d must be 128 (SDPA_ERR_UNSUPPORTED otherwise).
+ */
+SDPA_API int sdpa_fwd_fp8(const void* q8, const void* k8, const void* v8,
+                 float descale_q, float descale_k, float descale_v,
+                 void* o, float* lse,
+                 int B, int Hq, int Hkv, int Sq, int Sk, int d,
+                 float scale, int causal, void* stream);
+
+/* Static, NUL-terminated description of a status code. */
+SDPA_API const char* sdpa_strerror(int status);
+
+/*
+ * sdpa_device_status -- read (and with clear != 0, reset) the device status
+ * word of the current device.  The kernels never trap: a wait that does not
+ * complete within about one second stops the kernel and records
+ * SDPA_ERR_DEVICE_TIMEOUT here.  *status receives SDPA_OK or that code and
+ * *detail a kernel-specific location code (0 when none).  This call
+ * synchronises the current device.  Returns SDPA_OK or SDPA_ERR_CUDA.
+ */
+SDPA_API int sdpa_device_status(int* status, int* detail, int clear);
+
+/* Number of kernel launches sdpa_fwd / sdpa_fwd_fp8 issue per call (1). */
+SDPA_API int sdpa_launches_per_call(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SDPA_B200_H */

@@ -1,0 +1,156 @@
+"""B200-native fused scaled-dot-product attention forward.
+
+Python binding of ``libsdpa_b200.so`` (C ABI in ``include/sdpa.h``).  The
+functions with the C names take raw device pointers and sizes and only
+marshal arguments; :func:`attention` and :func:`attention_fp8` add the torch
+conveniences a user wants (output allocation with torch, the current stream,
+error translation).  Every step of the computation runs in the library's
+CUDA kernels; there is no fallback, and importing this package fails loudly
+when the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+__all__ = [
+    "SDPA_BF16", "SDPA_FP16", "SDPA_OK", "SDPA_ERR_INVALID_ARG", "SDPA_ERR_UNSUPPORTED",
+    "SDPA_ERR_CUDA", "SDPA_ERR_DEVICE_TIMEOUT", "SdpaError", "LIB_PATH",
+    "sdpa_fwd", "sdpa_fwd_fp8", "sdpa_strerror", "sdpa_device_status",
+    "sdpa_launches_per_call", "attention", "attention_fp8",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsdpa_b200.so")
+
+SDPA_BF16, SDPA_FP16 = 0, 1
+SDPA_OK, SDPA_ERR_INVALID_ARG, SDPA_ERR_UNSUPPORTED, SDPA_ERR_CUDA, SDPA_ERR_DEVICE_TIMEOUT = range(5)
+
+
+class SdpaError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = int(status)
+        super().__init__("%s%s (status %d)" % (what + ": " if what else "",
+                                                sdpa_strerror(self.status), self.status))
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError("libsdpa_b200.so is not built at %s; run "
+                      "`python -m scaled_dot_product_11_b200.build` (nvcc, sm_100a)" % LIB_PATH)
+
+_lib = ctypes.CDLL(LIB_PATH)
+_vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+_lib.sdpa_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _vp]
+_lib.sdpa_fwd.restype = _i
+_lib.sdpa_fwd_fp8.argtypes = [_vp, _vp, _vp, _f, _f, _f, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]
+_lib.sdpa_fwd_fp8.restype = _i
+_lib.sdpa_strerror.argtypes = [_i]
+_lib.sdpa_strerror.restype = ctypes.c_char_p
+_lib.sdpa_device_status.argtypes = [ctypes.POINTER(_i), ctypes.POINTER(_i), _i]
+_lib.sdpa_device_status.restype = _i
+_lib.sdpa_launches_per_call.argtypes = []
+_lib.sdpa_launches_per_call.restype = _i
+
+
+# ---- the C entry points, same names, raw arguments ------------------------
+
+def sdpa_fwd(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal, dtype, stream) -> int:
+    """Raw call: pointers are ints (device addresses, lse may be 0/None),
+    stream an int cudaStream_t (0 = default stream).  Returns the status."""
+    return int(_lib.sdpa_fwd(q, k, v, o, lse or None, B, Hq, Hkv, Sq, Sk, d, float(scale),
+                             int(causal), int(dtype), stream or None))
+
+
+def sdpa_fwd_fp8(q8, k8, v8, descale_q, descale_k, descale_v, o, lse, B, Hq, Hkv, Sq, Sk, d,
+                 scale, causal, stream) -> int:
+    return int(_lib.sdpa_fwd_fp8(q8, k8, v8, float(descale_q), float(descale_k), float(descale_v),
+                                 o, lse or None, B, Hq, Hkv, Sq, Sk, d, float(scale), int(causal),
+                                 stream or None))
+
+
+def sdpa_strerror(status: int) -> str:
+    return _lib.sdpa_strerror(int(status)).decode()
+
+
+def sdpa_device_status(clear: bool = True):
+    """(status, detail) of the current device; synchronises the device."""
+    st, dt = _i(0), _i(0)
+    rc = _lib.sdpa_device_status(ctypes.byref(st), ctypes.byref(dt), int(bool(clear)))
+    if rc != SDPA_OK:
+        raise SdpaError(rc, "sdpa_device_status")
+    return st.value, dt.value
+
+
+def sdpa_launches_per_call() -> int:
+    return int(_lib.sdpa_launches_per_call())
+
+
+# ---- torch conveniences -------------------------------------------------------
+
+def _dims(q, k, v):
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be 4-D [B, H, S, d]")
+    B, Hq, Sq, d = q.shape
+    Bk, Hkv, Sk, dk = k.shape
+    if tuple(v.shape) != (Bk, Hkv, Sk, dk) or Bk != B or dk != d:
+        raise ValueError("shape mismatch: q %s k %s v %s" % (tuple(q.shape), tuple(k.shape),
+                                                              tuple(v.shape)))
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous CUDA tensors")
+    return int(B), int(Hq), int(Hkv), int(Sq), int(Sk), int(d)
+
+
+def _stream_handle(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream(torch.cuda.current_device())
+    return int(s.cuda_stream)
+
+
+def attention(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
+              return_lse: bool = True, stream=None):
+    """O (and LSE) = softmax(q k^T * scale [causal]) v for bf16 / fp16 CUDA
+    tensors q [B,Hq,Sq,d], k/v [B,Hkv,Sk,d].  Enqueued on `stream` (default:
+    torch's current stream); raises SdpaError on a refused call."""
+    import torch
+    B, Hq, Hkv, Sq, Sk, d = _dims(q, k, v)
+    if q.dtype not in (torch.bfloat16, torch.float16) or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share dtype bfloat16 or float16")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    with torch.cuda.device(q.device):
+        if out is None:
+            out = torch.empty_like(q)
+        if lse is None and return_lse:
+            lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+        rc = sdpa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                      lse.data_ptr() if lse is not None else 0, B, Hq, Hkv, Sq, Sk, d, scale,
+                      causal, SDPA_BF16 if q.dtype == torch.bfloat16 else SDPA_FP16,
+                      _stream_handle(stream))
+    if rc != SDPA_OK:
+        raise SdpaError(rc, "sdpa_fwd")
+    return (out, lse) if return_lse else out
+
+
+def attention_fp8(q8, k8, v8, descales, causal: bool = False, scale: float | None = None,
+                  out=None, lse=None, stream=None):
+    """FP8 E4M3 forward: q8/k8/v8 torch.float8_e4m3fn CUDA tensors holding
+    codes, descales = (dq, dk, dv) so that value = code * descale.  Returns
+    (O bf16, LSE fp32)."""
+    import torch
+    B, Hq, Hkv, Sq, Sk, d = _dims(q8, k8, v8)
+    for t in (q8, k8, v8):
+        if t.dtype != torch.float8_e4m3fn:
+            raise ValueError("q8, k8, v8 must be float8_e4m3fn")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    with torch.cuda.device(q8.device):
+        if out is None:
+            out = torch.empty((B, Hq, Sq, d), dtype=torch.bfloat16, device=q8.device)
+        if lse is None:
+            lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q8.device)
+        rc = sdpa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), descales[0], descales[1],
+                          descales[2], out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, Sq, Sk, d,
+                          scale, causal, _stream_handle(stream))
+    if rc != SDPA_OK:
+        raise SdpaError(rc, "sdpa_fwd_fp8")
+    return out, lse

@@ -1,0 +1,192 @@
+// sdpa_api.cu -- the C ABI declared in include/sdpa.h: argument checks,
+// TMA tensor-map encoding, kernel selection and launch.  No allocation, no
+// synchronisation, no fallback path.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "sdpa.h"
+#include "sdpa_fwd_sm100.cuh"
+
+namespace {
+
+using sdpa::FwdCfg;
+using sdpa::FwdParams;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (fn == nullptr) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 0 ok, else an sdpa_status.  Caches the answer per device.
+int check_device() {
+    static int verdict[64];   // 0 unknown, 1 ok, 2 unsupported
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SDPA_ERR_CUDA;
+    if (dev >= 0 && dev < 64 && verdict[dev] != 0) return verdict[dev] == 1 ? SDPA_OK : SDPA_ERR_UNSUPPORTED;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        return SDPA_ERR_CUDA;
+    const bool ok = (major == 10 && minor == 0);
+    if (dev >= 0 && dev < 64) verdict[dev] = ok ? 1 : 2;
+    return ok ? SDPA_OK : SDPA_ERR_UNSUPPORTED;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Common argument checks of both entry points.
+int check_args(const void* q, const void* k, const void* v, const void* o, const float* lse,
+               int B, int Hq, int Hkv, int Sq, int Sk, int d, float scale, int causal) {
+    if (!q || !k || !v || !o) return SDPA_ERR_INVALID_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Sq <= 0 || Sk <= 0 || d <= 0) return SDPA_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return SDPA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.0f)) return SDPA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SDPA_ERR_INVALID_ARG;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return SDPA_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return SDPA_ERR_INVALID_ARG;
+    // addressing limits: head counts and row indices fit the 32-bit TMA
+    // coordinates and the grid, element offsets fit 64-bit size_t trivially
+    const long long bhq = (long long)B * Hq, bhk = (long long)B * Hkv;
+    const long long qblocks = (Sq + 255) / 256;
+    if (bhq > INT32_MAX || bhk > INT32_MAX || bhq * qblocks > INT32_MAX) return SDPA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return SDPA_ERR_UNSUPPORTED;
+    if (causal && Sq != Sk) return SDPA_ERR_UNSUPPORTED;
+    return SDPA_OK;
+}
+
+bool encode_3d(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* base, int d,
+               int rows, long long heads, int box_inner) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)heads};
+    const cuuint64_t strides[2] = {(cuuint64_t)d * elem_bytes, (cuuint64_t)d * elem_bytes * rows};
+    const cuuint32_t box[3] = {(cuuint32_t)box_inner, 128u, 1u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int KIND, int NS>
+int launch(const void* q, const void* k, const void* v, const FwdParams& prm, cudaStream_t stream) {
+    using C = FwdCfg<D, KIND, NS>;
+    const CUtensorMapDataType dt = KIND == sdpa::KIND_BF16   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                   : KIND == sdpa::KIND_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                             : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    CUtensorMap tq, tk, tv;
+    if (!encode_3d(&tq, dt, C::kElem, q, D, prm.Sq, (long long)prm.B * prm.Hq, C::kElemsPerSw) ||
+        !encode_3d(&tk, dt, C::kElem, k, D, prm.Sk, (long long)prm.B * prm.Hkv, C::kElemsPerSw) ||
+        !encode_3d(&tv, dt, C::kElem, v, D, prm.Sk, (long long)prm.B * prm.Hkv, C::kElemsPerSw))
+        return SDPA_ERR_CUDA;
+    auto kern = sdpa::sdpa_fwd_sm100_kernel<D, KIND, NS>;
+    static bool attr_set[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+            cudaSuccess)
+            return SDPA_ERR_CUDA;
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+    const unsigned grid = (unsigned)((long long)prm.n_qblocks * prm.B * prm.Hq);
+    kern<<<grid, sdpa::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, prm);
+    return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
+FwdParams make_params(void* o, float* lse, int B, int Hq, int Hkv, int Sq, int Sk, int causal) {
+    FwdParams prm;
+    prm.o = o;
+    prm.lse = lse;
+    prm.B = B;
+    prm.Hq = Hq;
+    prm.Hkv = Hkv;
+    prm.Sq = Sq;
+    prm.Sk = Sk;
+    prm.group = Hq / Hkv;
+    prm.n_qblocks = (Sq + 255) / 256;
+    prm.causal = causal;
+    prm.score_log2 = 0.f;
+    prm.out_mul = 1.f;
+    prm.p_mul = 1.f;
+    return prm;
+}
+
+}  // namespace
+
+extern "C" int sdpa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int Hq, int Hkv, int Sq, int Sk, int d, float scale, int causal, int dtype,
+                        void* stream) {
+    int rc = check_args(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal);
+    if (rc != SDPA_OK) return rc;
+    if (dtype != SDPA_BF16 && dtype != SDPA_FP16) return SDPA_ERR_UNSUPPORTED;
+    rc = check_device();
+    if (rc != SDPA_OK) return rc;
+    FwdParams prm = make_params(o, lse, B, Hq, Hkv, Sq, Sk, causal);
+    prm.score_log2 = scale * sdpa::kLog2e;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (dtype == SDPA_BF16)
+        return d == 128 ? launch<128, sdpa::KIND_BF16, 4>(q, k, v, prm, s)
+                        : launch<64, sdpa::KIND_BF16, 8>(q, k, v, prm, s);
+    return d == 128 ? launch<128, sdpa::KIND_FP16, 4>(q, k, v, prm, s)
+                    : launch<64, sdpa::KIND_FP16, 8>(q, k, v, prm, s);
+}
+
+extern "C" int sdpa_fwd_fp8(const void* q8, const void* k8, const void* v8, float descale_q,
+                            float descale_k, float descale_v, void* o, float* lse, int B, int Hq,
+                            int Hkv, int Sq, int Sk, int d, float scale, int causal, void* stream) {
+    int rc = check_args(q8, k8, v8, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal);
+    if (rc != SDPA_OK) return rc;
+    for (float ds : {descale_q, descale_k, descale_v})
+        if (!std::isfinite(ds) || !(ds > 0.0f)) return SDPA_ERR_INVALID_ARG;
+    if (d != 128) return SDPA_ERR_UNSUPPORTED;
+    rc = check_device();
+    if (rc != SDPA_OK) return rc;
+    FwdParams prm = make_params(o, lse, B, Hq, Hkv, Sq, Sk, causal);
+    prm.score_log2 = scale * descale_q * descale_k * sdpa::kLog2e;
+    prm.p_mul = 448.0f;
+    prm.out_mul = descale_v / 448.0f;
+    return launch<128, sdpa::KIND_E4M3, 8>(q8, k8, v8, prm, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" const char* sdpa_strerror(int status) {
+    switch (status) {
+    case SDPA_OK: return "success";
+    case SDPA_ERR_INVALID_ARG: return "invalid argument";
+    case SDPA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SDPA_ERR_CUDA: return "CUDA runtime or driver error";
+    case SDPA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+    }
+}
+
+extern "C" int sdpa_device_status(int* status, int* detail, int clear) {
+    unsigned int h[2] = {0u, 0u};
+    if (cudaDeviceSynchronize() != cudaSuccess) return SDPA_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(h, sdpa::g_sdpa_status, sizeof h) != cudaSuccess) return SDPA_ERR_CUDA;
+    if (status) *status = (int)h[0];
+    if (detail) *detail = (int)h[1];
+    if (clear) {
+        const unsigned int z[2] = {0u, 0u};
+        if (cudaMemcpyToSymbol(sdpa::g_sdpa_status, z, sizeof z) != cudaSuccess) return SDPA_ERR_CUDA;
+    }
+    return SDPA_OK;
+}
+
+extern "C" int sdpa_launches_per_call(void) { return 1; }

@@ -1,0 +1,501 @@
+// sdpa_fwd_sm100.cuh -- fused scaled-dot-product attention forward for
+// sm_100a (B200): TMA-fed K/V ring, tcgen05 MMAs with accumulators in tensor
+// memory, warp-specialised roles, exp2 online softmax, causal tile skipping,
+// GQA/MQA K/V heads shared by index.
+//
+// Method (article "Self-attention, CUDA kernels and FlashAttention", section
+// 3): Q, K, V are cut into on-chip tiles, scores of a tile are turned into
+// weights with a softmax that keeps a running row maximum and row sum, the
+// partial output is rescaled when the maximum moves, and only the output and
+// the per-row normaliser (LSE) are written to global memory; the Sq x Sk
+// score matrix never leaves the SM.  Formula and steps: codelab "JAX on GPU,
+// Lab 5: attention on GPU", section 1; causal mask section 7; MHA/GQA/MQA
+// section 9; FP8 E4M3 forward section 10.
+//
+// One CTA owns 2 x 128 query rows of one (batch, query head) and walks the
+// K/V tiles of that head's KV head.  Warp roles (320 threads):
+//   warps 0-3  softmax group 0: query tile 0, thread = row = TMEM lane
+//   warps 4-7  softmax group 1: query tile 1
+//   warp  8    TMA producer: Q tiles once, then K_0, V_0, K_1, V_1, ...
+//   warp  9    MMA issuer (one thread) and TMEM owner
+// Tensor memory (512 columns x 128 lanes, fp32):
+//   [0,128) S0   [128,256) S1   [256,256+d) O0   [384,384+d) O1
+//   P_w (the weights, packed 2 x 16-bit or 4 x e4m3 per column) overwrites
+//   the upper half of S_w once the softmax group has read S_w.
+// MMA issue order per K/V tile i: S0=Q0 K_i^T, O1+=P1(i-1) V_(i-1),
+// S1=Q1 K_i^T, O0+=P0(i) V_i -- while one softmax group works, the tensor
+// pipe always has the other group's products queued.  tcgen05 MMAs from one
+// thread execute in issue order, so an S_w write queued after the P_w read
+// of the previous tile cannot overtake it, and the commit that signals S_w(i)
+// also covers O_w += P_w(i-1) V_(i-1): when a softmax group sees S_w(i) its
+// O_w is quiescent and may be rescaled in place.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include "sm100_ptx.cuh"
+
+namespace sdpa {
+
+enum Kind { KIND_BF16 = 0, KIND_FP16 = 1, KIND_E4M3 = 2 };
+
+constexpr int kBlockM = 128;        // query rows per tile (= TMEM lanes)
+constexpr int kBlockN = 128;        // keys per K/V tile
+constexpr int kQTiles = 2;          // query tiles per CTA
+constexpr int kThreads = 320;
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLn2 = 0.69314718055994530942f;
+constexpr float kLog2e = 1.44269504088896340736f;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // bounded waits: 1 s
+
+// Device status word: [0] status (0 ok, 4 = device timeout), [1] location.
+__device__ unsigned int g_sdpa_status[2];
+
+struct FwdParams {
+    void* o;            // [B,Hq,Sq,D] 16-bit
+    float* lse;         // [B,Hq,Sq] or null
+    int B, Hq, Hkv, Sq, Sk;
+    int group;          // Hq / Hkv
+    int n_qblocks;      // ceil(Sq / 256)
+    int causal;
+    float score_log2;   // multiplier from raw MMA score to log2 units
+    float out_mul;      // multiplier on sum_j p_j v_j before / l
+    float p_mul;        // multiplier on p before it is rounded for the PV MMA
+};
+
+template <int D, int KIND, int NS>
+struct FwdCfg {
+    static constexpr int kElem = (KIND == KIND_E4M3) ? 1 : 2;
+    static constexpr int kRowBytes = D * kElem;
+    static constexpr int kElemsPerSw = 128 / kElem;      // elements in one 128-byte swizzle row
+    static constexpr int kSwBlocks = kRowBytes / 128;    // 128-byte column blocks per row
+    static constexpr int kSwBlockBytes = 128 * 128;      // one column block of a 128-row tile
+    static constexpr int kTileBytes = 128 * kRowBytes;
+    static constexpr int kQkSteps = kRowBytes / 32;      // every MMA consumes 32 bytes of K
+    static constexpr int kPvKeysPerStep = 32 / kElem;
+    static constexpr int kPvSteps = kBlockN / kPvKeysPerStep;
+    static constexpr int kPCols = kBlockN * kElem / 4;   // TMEM columns of one P row
+    static constexpr float kRescaleThreshold = (KIND == KIND_E4M3) ? 0.0f : 8.0f;
+    // shared memory map (offsets from a 1024-byte aligned base)
+    static constexpr int kSmemQ = 0;
+    static constexpr int kSmemKV = kQTiles * kTileBytes;
+    static constexpr int kSmemBar = kSmemKV + NS * kTileBytes;
+    // barriers: q_full[2] kv_full[NS] kv_empty[NS] s_full[2] p_full[2] o_full[2] drain[1]
+    static constexpr int kBarQFull = 0;
+    static constexpr int kBarKVFull = 2;
+    static constexpr int kBarKVEmpty = 2 + NS;
+    static constexpr int kBarSFull = 2 + 2 * NS;
+    static constexpr int kBarPFull = 4 + 2 * NS;
+    static constexpr int kBarOFull = 6 + 2 * NS;
+    static constexpr int kBarDrain = 8 + 2 * NS;
+    static constexpr int kNumBars = 9 + 2 * NS;
+    static constexpr int kSmemTmemSlot = kSmemBar + 8 * kNumBars;
+    static constexpr int kSmemAbort = kSmemTmemSlot + 4;
+    static constexpr int kSmemUsed = kSmemAbort + 4;
+    static constexpr int kSmemBytes = kSmemUsed + 1024;  // slack for the 1024-byte alignment
+    // TMEM columns
+    static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
+    static constexpr uint32_t kPOffset = 64;
+    static_assert(kRowBytes % 128 == 0, "rows must fill whole 128-byte swizzle rows");
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+    static_assert(D <= 128, "O tile must fit its 128 TMEM columns");
+};
+
+// ---------------------------------------------------------------------------
+// bounded waiting
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t v) {
+    asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// Wait for the phase of `bar` with parity `parity`.  Gives up (returning
+// false) when another role of the CTA has aborted, or after kWaitLimitNs, in
+// which case it records the timeout and `where` in the device status word and
+// raises the CTA's abort flag.
+__device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, uint32_t abort_addr,
+                                           uint32_t where) {
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t k = 1;; ++k) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((k & 63u) == 0) {
+            if (ld_shared_u32(abort_addr) != 0u) return false;
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                st_shared_u32(abort_addr, 1u);
+                if (atomicCAS(&g_sdpa_status[0], 0u, 4u) == 0u)
+                    atomicExch(&g_sdpa_status[1], where);
+                return false;
+            }
+        }
+    }
+}
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, uint32_t abort_addr,
+                                         uint32_t where) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait_bar_slow(bar, parity, abort_addr, where);
+}
+
+// Row-tile key counts of one CTA: number of K/V tiles query tile w needs.
+__device__ __forceinline__ int tiles_for(int row0, int Sq, int Sk, int causal) {
+    if (row0 >= Sq) return 0;
+    const int kend = causal ? min(Sk, row0 + kBlockM) : Sk;
+    return (kend + kBlockN - 1) / kBlockN;
+}
+
+template <int D, int KIND, int NS>
+__global__ void __launch_bounds__(kThreads, 1)
+sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
+                      const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV,
+                      const FwdParams p) {
+    using C = FwdCfg<D, KIND, NS>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // ---- work unit: longest (last) query blocks first --------------------
+    const int n_bh = p.B * p.Hq;
+    const int qblk = p.n_qblocks - 1 - (int)(blockIdx.x / (unsigned)n_bh);
+    const int bh = (int)(blockIdx.x % (unsigned)n_bh);
+    const int b = bh / p.Hq;
+    const int hq = bh - b * p.Hq;
+    const int kvh = b * p.Hkv + hq / p.group;
+    const int m0 = qblk * (kQTiles * kBlockM);
+    const int nt0 = tiles_for(m0, p.Sq, p.Sk, p.causal);
+    const int nt1 = tiles_for(m0 + kBlockM, p.Sq, p.Sk, p.causal);
+    const int n = max(nt0, nt1);
+
+    auto bar = [&](int i) -> uint32_t { return sbase + C::kSmemBar + 8u * (uint32_t)i; };
+    const uint32_t abort_addr = sbase + C::kSmemAbort;
+    const uint32_t slot_addr = sbase + C::kSmemTmemSlot;
+
+    if (threadIdx.x == 0) {
+        for (int w = 0; w < kQTiles; ++w) {
+            mbar_init(bar(C::kBarQFull + w), 1);
+            mbar_init(bar(C::kBarSFull + w), 1);
+            mbar_init(bar(C::kBarPFull + w), kBlockM);
+            mbar_init(bar(C::kBarOFull + w), 1);
+        }
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(bar(C::kBarKVFull + s), 1);
+            mbar_init(bar(C::kBarKVEmpty + s), 1);
+        }
+        mbar_init(bar(C::kBarDrain), 1);
+        st_shared_u32(abort_addr, 0u);
+        fence_barrier_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(slot_addr, kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == kLoadWarp && lane == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ld_shared_u32(slot_addr);
+
+    const uint32_t sQ = sbase + C::kSmemQ;
+    const uint32_t sKV = sbase + C::kSmemKV;
+
+    if (warp == kLoadWarp) {
+        // ================= TMA producer =================================
+        if (lane == 0) {
+            bool ok = true;
+            for (int w = 0; w < kQTiles; ++w) {
+                if ((w ? nt1 : nt0) == 0) continue;
+                const uint32_t qb = bar(C::kBarQFull + w);
+                mbar_arrive_expect_tx(qb, C::kTileBytes);
+                for (int kb = 0; kb < C::kSwBlocks; ++kb)
+                    tma_load_3d(sQ + w * C::kTileBytes + kb * C::kSwBlockBytes, &tmQ, qb,
+                                kb * C::kElemsPerSw, m0 + w * kBlockM, bh);
+            }
+            int t = 0;
+            for (; t < 2 * n && ok; ++t) {
+                const int slot = t % NS;
+                const uint32_t par = ((uint32_t)(t / NS) & 1u) ^ 1u;
+                ok = wait_bar(bar(C::kBarKVEmpty + slot), par, abort_addr, 0x10000u | (uint32_t)t);
+                if (!ok) break;
+                const uint32_t fb = bar(C::kBarKVFull + slot);
+                mbar_arrive_expect_tx(fb, C::kTileBytes);
+                const CUtensorMap* m = (t & 1) ? &tmV : &tmK;
+                for (int kb = 0; kb < C::kSwBlocks; ++kb)
+                    tma_load_3d(sKV + slot * C::kTileBytes + kb * C::kSwBlockBytes, m, fb,
+                                kb * C::kElemsPerSw, (t >> 1) * kBlockN, kvh);
+            }
+            if (!ok) {
+                // let the copies already issued land before the CTA exits
+                for (int u = max(0, t - NS); u < t; ++u) {
+                    const uint64_t t0 = global_timer_ns();
+                    while (!mbar_try_wait(bar(C::kBarKVFull + u % NS), (uint32_t)(u / NS) & 1u) &&
+                           global_timer_ns() - t0 < 100000000ull) {
+                    }
+                }
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        // ================= MMA issuer ===================================
+        if (lane == 0) {
+            constexpr uint32_t fmt = (KIND == KIND_BF16) ? 1u : 0u;
+            constexpr uint32_t idesc_qk = make_idesc(fmt, false, kBlockM, kBlockN);
+            constexpr uint32_t idesc_pv = make_idesc(fmt, true, kBlockM, D);
+            bool ok = true;
+
+            auto issue_qk = [&](int w, int slot) {
+                const uint32_t d_tmem = tmem + (w ? C::kColS1 : C::kColS0);
+                const uint32_t qa = sQ + w * C::kTileBytes;
+                const uint32_t kb_ = sKV + slot * C::kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < C::kQkSteps; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::kSwBlockBytes + (kk & 3) * 32;
+                    const uint64_t da = make_smem_desc(qa + off, 16, 1024);
+                    const uint64_t db = make_smem_desc(kb_ + off, 16, 1024);
+                    if constexpr (KIND == KIND_E4M3)
+                        mma_f8_ss(d_tmem, da, db, idesc_qk, kk > 0);
+                    else
+                        mma_f16_ss(d_tmem, da, db, idesc_qk, kk > 0);
+                }
+            };
+            auto issue_pv = [&](int w, int slot, bool acc) {
+                const uint32_t d_tmem = tmem + (w ? C::kColO1 : C::kColO0);
+                const uint32_t a_tmem = tmem + (w ? C::kColS1 : C::kColS0) + C::kPOffset;
+                const uint32_t vb = sKV + slot * C::kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < C::kPvSteps; ++kk) {
+                    const uint64_t db = make_smem_desc(vb + kk * C::kPvKeysPerStep * 128,
+                                                       C::kSwBlockBytes, 1024);
+                    if constexpr (KIND == KIND_E4M3)
+                        mma_f8_ts(d_tmem, a_tmem + kk * 8, db, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+                    else
+                        mma_f16_ts(d_tmem, a_tmem + kk * 8, db, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+                }
+            };
+
+            for (int w = 0; w < kQTiles && ok; ++w)
+                if ((w ? nt1 : nt0) > 0) ok = wait_bar(bar(C::kBarQFull + w), 0, abort_addr, 0x20000u | w);
+
+            for (int i = 0; i <= n && ok; ++i) {
+                const int tK = 2 * i, tV = 2 * i + 1;
+                const int slotK = tK % NS, slotV = tV % NS;
+                if (i < n) {
+                    ok = wait_bar(bar(C::kBarKVFull + slotK), (uint32_t)(tK / NS) & 1u, abort_addr,
+                                  0x21000u | (uint32_t)i);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (i < nt0) {
+                        issue_qk(0, slotK);
+                        mma_commit(bar(C::kBarSFull + 0));
+                    }
+                }
+                if (i >= 1) {
+                    const int j = i - 1;
+                    if (j < nt1) {
+                        ok = wait_bar(bar(C::kBarPFull + 1), (uint32_t)j & 1u, abort_addr,
+                                      0x22000u | (uint32_t)j);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_pv(1, (2 * j + 1) % NS, j > 0);
+                        if (j == nt1 - 1) mma_commit(bar(C::kBarOFull + 1));
+                    }
+                    mma_commit(bar(C::kBarKVEmpty + (2 * j + 1) % NS));   // V_(i-1) free
+                }
+                if (i < n) {
+                    if (i < nt1) {
+                        issue_qk(1, slotK);
+                        mma_commit(bar(C::kBarSFull + 1));
+                    }
+                    mma_commit(bar(C::kBarKVEmpty + slotK));               // K_i free
+                    ok = wait_bar(bar(C::kBarKVFull + slotV), (uint32_t)(tV / NS) & 1u, abort_addr,
+                                  0x23000u | (uint32_t)i);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (i < nt0) {
+                        ok = wait_bar(bar(C::kBarPFull + 0), (uint32_t)i & 1u, abort_addr,
+                                      0x24000u | (uint32_t)i);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_pv(0, slotV, i > 0);
+                        if (i == nt0 - 1) mma_commit(bar(C::kBarOFull + 0));
+                    }
+                }
+            }
+            if (!ok) {
+                // make sure no MMA is still writing tensor memory at exit
+                mma_commit(bar(C::kBarDrain));
+                const uint64_t t0 = global_timer_ns();
+                while (!mbar_try_wait(bar(C::kBarDrain), 0) && global_timer_ns() - t0 < 100000000ull) {
+                }
+            }
+        }
+    } else {
+        // ================= softmax groups (warps 0-7) ====================
+        const int w = warp >> 2;                 // query tile
+        const int quarter = warp & 3;            // TMEM lane quarter of this warp
+        const int r = (int)(threadIdx.x & 127);  // row within the tile
+        const int row = m0 + w * kBlockM + r;
+        const int nw = w ? nt1 : nt0;
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        const uint32_t tS = tmem + lane_base + (w ? C::kColS1 : C::kColS0);
+        const uint32_t tP = tS + C::kPOffset;
+        const uint32_t tO = tmem + lane_base + (w ? C::kColO1 : C::kColO0);
+        const float sl = p.score_log2;
+        float m_run = -INFINITY;   // running max of the scaled scores (log2 units)
+        float l_run = 0.0f;        // running sum of 2^(s*sl - m_run)
+        bool ok = true;
+
+        for (int i = 0; i < nw; ++i) {
+            ok = wait_bar(bar(C::kBarSFull + w), (uint32_t)i & 1u, abort_addr, 0x30000u | (w << 12) | i);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+
+            float s[kBlockN];
+#pragma unroll
+            for (int c = 0; c < kBlockN / 32; ++c)
+                tmem_ld32(tS + 32 * c, *reinterpret_cast<float(*)[32]>(&s[32 * c]));
+            tmem_wait_ld();
+
+            // mask: keys past Sk, and (causal) keys after the row
+            const int key0 = i * kBlockN;
+            const bool edge = (key0 + kBlockN > p.Sk) ||
+                              (p.causal && key0 + kBlockN - 1 > m0 + w * kBlockM);
+            if (edge) {
+                int lim = p.Sk - key0;
+                if (p.causal) lim = min(lim, row - key0 + 1);
+#pragma unroll
+                for (int c = 0; c < kBlockN; ++c)
+                    if (c >= lim) s[c] = -INFINITY;
+            }
+
+            // row max (tree) in raw score units, then to log2 units
+            float mx[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) mx[u] = s[u];
+#pragma unroll
+            for (int c = 8; c < kBlockN; c += 8)
+#pragma unroll
+                for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], s[c + u]);
+            float tile_max = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            tile_max *= sl;
+
+            // The running max only moves when the new one exceeds it by more
+            // than the threshold; weights computed against a stale max are
+            // bounded by 2^threshold and the final O / l and LSE are exact
+            // for any reference value as long as O and l share it.
+            float alpha = 1.0f;
+            if (tile_max > m_run + C::kRescaleThreshold) {
+                alpha = ex2_approx(m_run - tile_max);   // 0 on the first tile
+                m_run = tile_max;
+            }
+            l_run *= alpha;
+
+            // weights p = 2^(s*sl - m), rounded for the PV product
+            const float neg_m = -m_run;
+            float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+            if constexpr (KIND == KIND_E4M3) {
+#pragma unroll
+                for (int c = 0; c < kBlockN / 64; ++c) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        float q0 = ex2_approx(fmaf(s[64 * c + 4 * e + 0], sl, neg_m));
+                        float q1 = ex2_approx(fmaf(s[64 * c + 4 * e + 1], sl, neg_m));
+                        float q2 = ex2_approx(fmaf(s[64 * c + 4 * e + 2], sl, neg_m));
+                        float q3 = ex2_approx(fmaf(s[64 * c + 4 * e + 3], sl, neg_m));
+                        sum4[0] += q0; sum4[1] += q1; sum4[2] += q2; sum4[3] += q3;
+                        pk[e] = pack_e4m3x4(q0 * p.p_mul, q1 * p.p_mul, q2 * p.p_mul, q3 * p.p_mul);
+                    }
+                    tmem_st16(tP + 16 * c, pk);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < kBlockN / 32; ++c) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float q0 = ex2_approx(fmaf(s[32 * c + 2 * e], sl, neg_m));
+                        const float q1 = ex2_approx(fmaf(s[32 * c + 2 * e + 1], sl, neg_m));
+                        sum4[(2 * e) & 3] += q0;
+                        sum4[(2 * e + 1) & 3] += q1;
+                        pk[e] = (KIND == KIND_BF16) ? pack_bf16x2(q0, q1) : pack_f16x2(q0, q1);
+                    }
+                    tmem_st16(tP + 16 * c, pk);
+                }
+            }
+            l_run += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+            // O_w (quiescent: its last update is covered by the S_w(i) commit)
+            // takes the same factor as l before P_w(i) V_i is added to it.
+            if (i > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    float o[32];
+                    tmem_ld32(tO + 32 * c, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] *= alpha;
+                    tmem_st32(tO + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(o));
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(C::kBarPFull + w));
+        }
+
+        // ---- epilogue: O / l -> 16-bit, LSE ---------------------------------
+        if (ok && nw > 0) {
+            ok = wait_bar(bar(C::kBarOFull + w), 0, abort_addr, 0x40000u | w);
+            ok = __all_sync(0xffffffffu, ok);
+        }
+        if (ok && nw > 0) {
+            tc_fence_after();
+            const float inv_l = p.out_mul / l_run;
+            const bool live = row < p.Sq;
+            const size_t orow = ((size_t)bh * p.Sq + (size_t)(live ? row : 0)) * D;
+            uint16_t* obase = reinterpret_cast<uint16_t*>(p.o) + orow;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                float o[32];
+                tmem_ld32(tO + 32 * c, o);
+                tmem_wait_ld();
+                uint32_t u[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    u[e] = (KIND == KIND_FP16) ? pack_f16x2(o[2 * e] * inv_l, o[2 * e + 1] * inv_l)
+                                               : pack_bf16x2(o[2 * e] * inv_l, o[2 * e + 1] * inv_l);
+                if (live) {
+                    uint4* dst = reinterpret_cast<uint4*>(obase + 32 * c);
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4)
+                        dst[v4] = make_uint4(u[4 * v4], u[4 * v4 + 1], u[4 * v4 + 2], u[4 * v4 + 3]);
+                }
+            }
+            if (p.lse != nullptr && live)
+                p.lse[(size_t)bh * p.Sq + row] = (m_run + __log2f(l_run)) * kLn2;
+        }
+    }
+
+    // ---- teardown ------------------------------------------------------------
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace sdpa

@@ -1,5 +1,8 @@
 import os
+import shutil
 import sys
+
+import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
@@ -8,3 +11,16 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU and the built CUDA library")
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _built_libraries():
+    """Compile the oracle (gcc) and the CUDA library (nvcc, sm_100a) in-tree
+    when they are missing or older than their sources."""
+    import oracle
+    oracle.build()
+    from scaled_dot_product_11_b200 import build as lib_build
+    if lib_build.needs_build() and shutil.which(lib_build.nvcc()) or \
+            lib_build.needs_build() and os.path.exists(lib_build.nvcc()):
+        lib_build.build()
+    yield

@@ -1,0 +1,100 @@
+"""Host-side checks of the C-ABI library (no GPU, no kernel launch): the .so
+loads, exports every entry point include/sdpa.h declares, and refuses bad
+arguments with the documented status before touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sdpa.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return re.findall(r"SDPA_API\s+[\w\s\*]+?\b(sdpa_\w+)\s*\(", text)
+
+
+def test_header_declares_the_entry_points():
+    assert set(declared_symbols()) == {"sdpa_fwd", "sdpa_fwd_fp8", "sdpa_strerror",
+                                       "sdpa_device_status", "sdpa_launches_per_call"}
+
+
+def test_library_exports_every_declared_symbol():
+    import scaled_dot_product_11_b200 as sdpa
+    lib = ctypes.CDLL(sdpa.LIB_PATH)
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", sdpa.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    assert set(declared_symbols()) <= exported
+    # nothing else of ours leaks out of the library
+    assert not [s for s in exported if s.startswith("_ZN4sdpa")]
+
+
+def test_strerror_and_launch_count():
+    import scaled_dot_product_11_b200 as sdpa
+    assert sdpa.sdpa_strerror(0) == "success"
+    assert "invalid" in sdpa.sdpa_strerror(1)
+    assert "unsupported" in sdpa.sdpa_strerror(2)
+    assert "timed out" in sdpa.sdpa_strerror(4)
+    assert sdpa.sdpa_strerror(99) == "unknown status"
+    assert sdpa.sdpa_launches_per_call() == 1
+
+
+# Fake, never dereferenced device addresses: every call below is refused by
+# the argument checks, which run before any CUDA call.
+P = 0x10000
+GOOD = dict(B=1, Hq=4, Hkv=2, Sq=128, Sk=128, d=128, scale=0.088, causal=0, dtype=0)
+
+
+def call(**kw):
+    import scaled_dot_product_11_b200 as sdpa
+    a = dict(GOOD)
+    a.update(kw)
+    ptrs = a.pop("ptrs", (P, P + 0x1000, P + 0x2000, P + 0x3000, P + 0x4000))
+    return sdpa.sdpa_fwd(*ptrs, a["B"], a["Hq"], a["Hkv"], a["Sq"], a["Sk"], a["d"], a["scale"],
+                         a["causal"], a["dtype"], 0)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ptrs=(0, P, P, P, P)), 1),
+    (dict(ptrs=(P, P, P, 0, P)), 1),
+    (dict(B=0), 1), (dict(Hq=-1), 1), (dict(Sq=0), 1), (dict(Sk=0), 1), (dict(d=0), 1),
+    (dict(Hq=3, Hkv=2), 1),
+    (dict(scale=float("nan")), 1), (dict(scale=float("inf")), 1), (dict(scale=0.0), 1),
+    (dict(scale=-1.0), 1),
+    (dict(ptrs=(P + 8, P, P, P, P)), 1),
+    (dict(ptrs=(P, P, P, P + 4, P)), 1),
+    (dict(ptrs=(P, P, P, P, P + 2)), 1),
+    (dict(causal=2), 1),
+    (dict(B=1 << 16, Hq=1 << 16, Hkv=1 << 16), 1),
+    (dict(d=96), 2), (dict(d=256), 2), (dict(d=32), 2),
+    (dict(causal=1, Sq=128, Sk=256), 2),
+    (dict(dtype=2), 2), (dict(dtype=-1), 2),
+])
+def test_argument_checks(kw, code):
+    assert call(**kw) == code
+
+
+def test_fp8_argument_checks():
+    import scaled_dot_product_11_b200 as sdpa
+
+    def fp8(dq=1.0, dk=1.0, dv=1.0, d=128, causal=0, Sq=128, Sk=128):
+        return sdpa.sdpa_fwd_fp8(P, P, P, dq, dk, dv, P, P, 1, 2, 2, Sq, Sk, d, 0.088, causal, 0)
+    assert fp8(dq=0.0) == 1
+    assert fp8(dk=float("nan")) == 1
+    assert fp8(dv=-2.0) == 1
+    assert fp8(d=64) == 2
+    assert fp8(causal=1, Sk=64) == 2
+
+
+def test_torch_wrapper_rejects_cpu_tensors():
+    import torch
+    import scaled_dot_product_11_b200 as sdpa
+    q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        sdpa.attention(q, q, q)

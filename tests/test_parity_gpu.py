@@ -1,0 +1,226 @@
+"""GPU parity of the sm_100a kernels against the fp64 CPU oracle.
+
+Every case draws seeded inputs from sdpa_workloads, runs the library through
+its C ABI (ctypes binding) on cuda:0, and compares element by element with
+the oracle on the same inputs.  Tolerances (max absolute error): O <= 1e-2 and
+LSE <= 1e-3 for bf16 / fp16; O <= 6e-2 for FP8 E4M3 (LSE <= 2e-3 there, see
+the FP8 test).  Full-size workloads are checked on sampled rows (first, last,
+tile-boundary and seeded random rows of every (batch, head)), which the oracle
+computes one by one.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sdpa_workloads import (WORKLOADS, Workload, make_qkv, make_qkv_fp8, sample_rows, sweep,
+                            with_shape)
+
+pytestmark = pytest.mark.gpu
+
+O_TOL, LSE_TOL = 1e-2, 1e-3
+FP8_O_TOL, FP8_LSE_TOL = 6e-2, 2e-3
+
+
+@pytest.fixture(scope="module")
+def sdpa():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import scaled_dot_product_11_b200 as lib
+    lib.sdpa_device_status(clear=True)
+    return lib
+
+
+def run(lib, w: Workload):
+    q, k, v = make_qkv(w, "cuda")
+    o, lse = lib.attention(q, k, v, causal=w.causal, scale=w.scale)
+    torch.cuda.synchronize()
+    st, detail = lib.sdpa_device_status(clear=True)
+    assert st == 0, "device status %d detail %#x" % (st, detail)
+    return (q, k, v), o, lse
+
+
+def compare_full(lib, w: Workload, o_tol=O_TOL, lse_tol=LSE_TOL):
+    (q, k, v), o, lse = run(lib, w)
+    ro, rl = oracle.sdpa_fwd(q.cpu(), k.cpu(), v.cpu(), w.scale, w.causal)
+    go = o.double().cpu().numpy()
+    gl = lse.double().cpu().numpy()
+    assert np.isfinite(go).all() and np.isfinite(gl).all()
+    eo, el = np.abs(go - ro).max(), np.abs(gl - rl).max()
+    assert eo <= o_tol, "%s: max|dO| = %.3g" % (w.name, eo)
+    assert el <= lse_tol, "%s: max|dLSE| = %.3g" % (w.name, el)
+    return eo, el
+
+
+def compare_rows(lib, w: Workload, n_random=256):
+    (q, k, v), o, lse = run(lib, w)
+    rows = sample_rows(w, n_random=n_random)
+    ro, rl = oracle.sdpa_rows(q.cpu(), k.cpu(), v.cpu(), rows, w.scale, w.causal)
+    idx = torch.tensor(rows, device=o.device)
+    go = o.reshape(-1, w.d).index_select(0, idx).double().cpu().numpy()
+    gl = lse.reshape(-1).index_select(0, idx).double().cpu().numpy()
+    eo, el = np.abs(go - ro).max(), np.abs(gl - rl).max()
+    assert eo <= O_TOL, "%s: max|dO| = %.3g" % (w.name, eo)
+    assert el <= LSE_TOL, "%s: max|dLSE| = %.3g" % (w.name, el)
+    # properties that hold at any size: finite everywhere, LSE >= max row score
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+    return eo, el
+
+
+def test_tiny_config(sdpa):
+    compare_full(sdpa, WORKLOADS["tiny"])
+
+
+SMALL = [
+    # (B, Hq, Hkv, Sq, Sk, d, causal)
+    (1, 2, 2, 256, 256, 128, False),
+    (1, 2, 2, 256, 256, 128, True),
+    (2, 4, 4, 384, 384, 64, True),
+    (1, 2, 2, 1, 1, 128, False),
+    (1, 2, 2, 17, 17, 64, True),
+    (1, 3, 3, 127, 127, 128, True),
+    (1, 2, 2, 129, 129, 128, True),
+    (1, 2, 2, 255, 255, 64, False),
+    (1, 2, 2, 257, 257, 128, True),
+    (1, 2, 1, 640, 640, 128, True),
+    (2, 8, 2, 300, 300, 128, True),
+    (1, 8, 1, 200, 200, 64, False),
+    (1, 2, 2, 100, 300, 128, False),
+    (1, 2, 2, 300, 77, 64, False),
+    (1, 1, 1, 513, 1000, 128, False),
+]
+
+
+@pytest.mark.parametrize("shape", SMALL, ids=lambda s: "b%d_hq%d_hkv%d_sq%d_sk%d_d%d_%s" % (
+    *s[:6], "causal" if s[6] else "full"))
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_small_shapes(sdpa, shape, dtype):
+    B, Hq, Hkv, Sq, Sk, d, causal = shape
+    w = Workload("small", B, Hq, Hkv, Sq, Sk, d, causal, dtype=dtype, seed=Sq * 7 + Sk + d)
+    compare_full(sdpa, w)
+
+
+def test_vit_config_full(sdpa):
+    compare_full(sdpa, WORKLOADS["vit"])
+
+
+def test_lm_causal_config_sampled(sdpa):
+    compare_rows(sdpa, WORKLOADS["lm_causal"])
+
+
+@pytest.mark.parametrize("name", ["gqa", "mqa"])
+def test_gqa_mqa_configs_sampled(sdpa, name):
+    compare_rows(sdpa, WORKLOADS[name], n_random=128)
+
+
+@pytest.mark.parametrize("w", [sweep(True)[0], sweep(False)[1], sweep(True)[5]],
+                         ids=lambda w: w.name)
+def test_sweep_points_sampled(sdpa, w):
+    compare_rows(sdpa, w, n_random=128)
+
+
+def test_gqa_is_repeated_kv_mha(sdpa):
+    """K/V heads are shared by index: GQA equals MHA on repeated K/V."""
+    w = Workload("g", 2, 8, 2, 384, 384, 128, True, seed=5)
+    q, k, v = make_qkv(w, "cuda")
+    o1, l1 = sdpa.attention(q, k, v, causal=True)
+    o2, l2 = sdpa.attention(q, k.repeat_interleave(4, 1).contiguous(),
+                            v.repeat_interleave(4, 1).contiguous(), causal=True)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_guard_bands_untouched_and_no_lse(sdpa):
+    w = Workload("g", 1, 2, 2, 200, 200, 128, False, seed=11)
+    q, k, v = make_qkv(w, "cuda")
+    n = w.B * w.Hq * w.Sq * w.d
+    big = torch.full((n + 4096,), -7.0, dtype=torch.bfloat16, device="cuda")
+    o = big[2048:2048 + n].view(w.B, w.Hq, w.Sq, w.d)
+    lbig = torch.full((w.B * w.Hq * w.Sq + 256,), -9.0, device="cuda")
+    lse = lbig[128:128 + w.B * w.Hq * w.Sq].view(w.B, w.Hq, w.Sq)
+    sdpa.attention(q, k, v, out=o, lse=lse)
+    torch.cuda.synchronize()
+    assert (big[:2048] == -7.0).all() and (big[2048 + n:] == -7.0).all()
+    assert (lbig[:128] == -9.0).all() and (lbig[128 + w.B * w.Hq * w.Sq:] == -9.0).all()
+    o2 = sdpa.attention(q, k, v, return_lse=False)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2)
+
+
+def test_deterministic_and_stream(sdpa):
+    w = Workload("d", 2, 4, 2, 1000, 1000, 128, True, seed=3)
+    q, k, v = make_qkv(w, "cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        o1, l1 = sdpa.attention(q, k, v, causal=True)
+    s.synchronize()
+    o2, l2 = sdpa.attention(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_refusals_raise(sdpa):
+    q = torch.zeros(1, 2, 64, 96, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(sdpa.SdpaError) as e:
+        sdpa.attention(q, q, q)
+    assert e.value.status == sdpa.SDPA_ERR_UNSUPPORTED
+    q = torch.zeros(1, 2, 64, 64, dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros(1, 2, 32, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(sdpa.SdpaError) as e:
+        sdpa.attention(q, k, k, causal=True)
+    assert e.value.status == sdpa.SDPA_ERR_UNSUPPORTED
+
+
+def test_large_magnitude_scores(sdpa):
+    """Stress case outside the seeded workloads: scale 1 and inputs x4 give
+    scores of several hundred, so each row's weights are nearly one-hot and
+    |O| reaches the largest |V| (about 4).  The online max keeps every
+    exponent in range.  Tolerance from the arithmetic of this case rather than
+    the workload bound: bf16 rounding of O (2^-9 relative) plus bf16 rounding
+    of the weights before P*V (2^-9 relative to sum_j p_j |v_j| <= max|V|),
+    on top of the 1e-2 absolute bound; LSE (hundreds) to fp32 relative 1e-6."""
+    w = Workload("big", 1, 2, 2, 384, 384, 64, True, seed=9)
+    q, k, v = make_qkv(w, "cuda")
+    q = (q.float() * 4).to(torch.bfloat16)
+    k = (k.float() * 4).to(torch.bfloat16)
+    o, lse = sdpa.attention(q, k, v, causal=True, scale=1.0)
+    ro, rl = oracle.sdpa_fwd(q.cpu(), k.cpu(), v.cpu(), 1.0, True)
+    vmax = float(v.abs().max())
+    o_tol = O_TOL + 2.0 ** -9 * (np.abs(ro) + vmax)
+    assert (np.abs(o.double().cpu().numpy() - ro) <= o_tol).all()
+    assert (np.abs(lse.double().cpu().numpy() - rl) <= LSE_TOL + 1e-6 * np.abs(rl)).all()
+
+
+# ---- FP8 ----------------------------------------------------------------------
+
+def run_fp8(lib, w):
+    q8, k8, v8, ds, _ = make_qkv_fp8(w, "cuda")
+    o, lse = lib.attention_fp8(q8, k8, v8, ds, causal=w.causal, scale=w.scale)
+    torch.cuda.synchronize()
+    st, detail = lib.sdpa_device_status(clear=True)
+    assert st == 0, "device status %d detail %#x" % (st, detail)
+    return (q8, k8, v8, ds), o, lse
+
+
+@pytest.mark.parametrize("shape", [(1, 2, 2, 256, 256, True), (1, 2, 1, 333, 333, True),
+                                   (2, 4, 2, 200, 500, False)])
+def test_fp8_small(sdpa, shape):
+    B, Hq, Hkv, Sq, Sk, causal = shape
+    w = Workload("f8", B, Hq, Hkv, Sq, Sk, 128, causal, dtype="e4m3", seed=Sq + Sk)
+    (q8, k8, v8, ds), o, lse = run_fp8(sdpa, w)
+    ro, rl = oracle.sdpa_fwd(q8.cpu(), k8.cpu(), v8.cpu(), w.scale, causal, descales=ds)
+    assert np.abs(o.double().cpu().numpy() - ro).max() <= FP8_O_TOL
+    assert np.abs(lse.double().cpu().numpy() - rl).max() <= FP8_LSE_TOL
+
+
+def test_fp8_config_sampled(sdpa):
+    w = WORKLOADS["fp8"]
+    (q8, k8, v8, ds), o, lse = run_fp8(sdpa, w)
+    rows = sample_rows(w, n_random=128)
+    ro, rl = oracle.sdpa_rows(q8.cpu(), k8.cpu(), v8.cpu(), rows, w.scale, True, descales=ds)
+    idx = torch.tensor(rows, device=o.device)
+    go = o.reshape(-1, w.d).index_select(0, idx).double().cpu().numpy()
+    gl = lse.reshape(-1).index_select(0, idx).double().cpu().numpy()
+    assert np.abs(go - ro).max() <= FP8_O_TOL
+    assert np.abs(gl - rl).max() <= FP8_LSE_TOL
