@@ -41,6 +41,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
 
 
@@ -282,7 +283,7 @@ def main():
 
     # end to end through the public API: pinned host inputs -> device -> fused
     # forward -> O and LSE back to pinned host memory, all inside the region
-    e2e_steps = max(3, min(20, args.steps // 20))
+    e2e_steps = 0 if args.no_e2e else max(3, min(20, args.steps // 20))
     hq_, hk_, hv_ = (t.cpu().pin_memory() for t in (q, k, v))
     ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
@@ -299,19 +300,21 @@ def main():
         ho.copy_(o, non_blocking=True)
         hl.copy_(lse, non_blocking=True)
 
-    run_e2e()
-    torch.cuda.synchronize()
-    barrier()
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        run_e2e()
-    e1.record(stream)
-    e1.synchronize()
-    barrier()
-    ms_e2e = max_over_ranks(e0.elapsed_time(e1))
     h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
     d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
-    e2e_value = world * w.flops * e2e_steps / (ms_e2e * 1e-3) / 1e12
+    e2e_value = None
+    if e2e_steps:
+        run_e2e()
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            run_e2e()
+        e1.record(stream)
+        e1.synchronize()
+        barrier()
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1))
+        e2e_value = world * w.flops * e2e_steps / (ms_e2e * 1e-3) / 1e12
 
     if rank == 0:
         peaks, src = load_peaks()

@@ -124,7 +124,6 @@ FwdParams make_params(void* o, float* lse, int B, int Hq, int Hkv, int Sq, int S
     prm.causal = causal;
     prm.score_log2 = 0.f;
     prm.out_mul = 1.f;
-    prm.p_mul = 1.f;
     return prm;
 }
 
@@ -160,8 +159,7 @@ extern "C" int sdpa_fwd_fp8(const void* q8, const void* k8, const void* v8, floa
     if (rc != SDPA_OK) return rc;
     FwdParams prm = make_params(o, lse, B, Hq, Hkv, Sq, Sk, causal);
     prm.score_log2 = scale * descale_q * descale_k * sdpa::kLog2e;
-    prm.p_mul = 448.0f;
-    prm.out_mul = descale_v / 448.0f;
+    prm.out_mul = descale_v;
     return launch<128, sdpa::KIND_E4M3, 8>(q8, k8, v8, prm, reinterpret_cast<cudaStream_t>(stream));
 }
 

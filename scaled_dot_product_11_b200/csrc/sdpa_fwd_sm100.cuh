@@ -13,11 +13,13 @@
 // section 9; FP8 E4M3 forward section 10.
 //
 // One CTA owns 2 x 128 query rows of one (batch, query head) and walks the
-// K/V tiles of that head's KV head.  Warp roles (320 threads):
+// K/V tiles of that head's KV head.  Warp roles (384 threads):
 //   warps 0-3  softmax group 0: query tile 0, thread = row = TMEM lane
 //   warps 4-7  softmax group 1: query tile 1
 //   warp  8    TMA producer: Q tiles once, then K_0, V_0, K_1, V_1, ...
-//   warp  9    MMA issuer (one thread) and TMEM owner
+//   warp  9    MMA issuer (one elected lane) and TMEM owner
+//   warps 10-11 idle (they complete warpgroup 2 for the register split)
+// Registers are moved with setmaxnreg from warpgroup 2 to the softmax groups.
 // Tensor memory (512 columns x 128 lanes, fp32):
 //   [0,128) S0   [128,256) S1   [256,256+d) O0   [384,384+d) O1
 //   P_w (the weights, packed 2 x 16-bit or 4 x e4m3 per column) overwrites
@@ -43,7 +45,9 @@ enum Kind { KIND_BF16 = 0, KIND_FP16 = 1, KIND_E4M3 = 2 };
 constexpr int kBlockM = 128;        // query rows per tile (= TMEM lanes)
 constexpr int kBlockN = 128;        // keys per K/V tile
 constexpr int kQTiles = 2;          // query tiles per CTA
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;       // 3 warpgroups
+constexpr int kSoftmaxRegs = 200;   // per thread after setmaxnreg, warpgroups 0-1
+constexpr int kOtherRegs = 96;      // warpgroup 2 (TMA, MMA, two idle warps)
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
@@ -62,8 +66,7 @@ struct FwdParams {
     int n_qblocks;      // ceil(Sq / 256)
     int causal;
     float score_log2;   // multiplier from raw MMA score to log2 units
-    float out_mul;      // multiplier on sum_j p_j v_j before / l
-    float p_mul;        // multiplier on p before it is rounded for the PV MMA
+    float out_mul;      // multiplier on (sum_j p_j v_j) / l: the V descale for FP8, else 1
 };
 
 template <int D, int KIND, int NS>
@@ -79,6 +82,9 @@ struct FwdCfg {
     static constexpr int kPvSteps = kBlockN / kPvKeysPerStep;
     static constexpr int kPCols = kBlockN * kElem / 4;   // TMEM columns of one P row
     static constexpr float kRescaleThreshold = (KIND == KIND_E4M3) ? 0.0f : 8.0f;
+    // log2 of the factor applied to p before it is rounded for the PV MMA:
+    // 448 (the e4m3 maximum) for FP8, so that p in (0, 1] fills the format
+    static constexpr float kPLog2 = (KIND == KIND_E4M3) ? 8.807354922057604f : 0.0f;
     // shared memory map (offsets from a 1024-byte aligned base)
     static constexpr int kSmemQ = 0;
     static constexpr int kSmemKV = kQTiles * kTileBytes;
@@ -120,7 +126,7 @@ __device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t v) {
 // false) when another role of the CTA has aborted, or after kWaitLimitNs, in
 // which case it records the timeout and `where` in the device status word and
 // raises the CTA's abort flag.
-__device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, uint32_t abort_addr,
+__device__ __forceinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, uint32_t abort_addr,
                                            uint32_t where) {
     const uint64_t t0 = global_timer_ns();
     for (uint32_t k = 1;; ++k) {
@@ -207,10 +213,13 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ld_shared_u32(slot_addr);
+    // launch: 384 x 168 registers; split: 256 x 200 + 128 x 96 = 63488 <= 64512
+    static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * 168, "register split");
 
     const uint32_t sQ = sbase + C::kSmemQ;
     const uint32_t sKV = sbase + C::kSmemKV;
 
+    if (warp >= 8) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
     if (warp == kLoadWarp) {
         // ================= TMA producer =================================
         if (lane == 0) {
@@ -248,100 +257,119 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
     } else if (warp == kMmaWarp) {
         // ================= MMA issuer ===================================
-        if (lane == 0) {
-            constexpr uint32_t fmt = (KIND == KIND_BF16) ? 1u : 0u;
-            constexpr uint32_t idesc_qk = make_idesc(fmt, false, kBlockM, kBlockN);
-            constexpr uint32_t idesc_pv = make_idesc(fmt, true, kBlockM, D);
-            bool ok = true;
+        // The whole warp runs the loop (so descriptors and addresses stay
+        // warp-uniform); one elected lane issues the MMAs and commits.
+        const bool leader = elect_one();
+        constexpr uint32_t fmt = (KIND == KIND_BF16) ? 1u : 0u;
+        constexpr uint32_t idesc_qk = make_idesc(fmt, false, kBlockM, kBlockN);
+        constexpr uint32_t idesc_pv = make_idesc(fmt, true, kBlockM, D);
+        const uint64_t desc_q0 = make_smem_desc(sQ, 16, 1024);
+        const uint64_t desc_q1 = make_smem_desc(sQ + C::kTileBytes, 16, 1024);
+        const uint64_t desc_k = make_smem_desc(sKV, 16, 1024);
+        const uint64_t desc_v = make_smem_desc(sKV, C::kSwBlockBytes, 1024);
+        bool ok = true;
 
-            auto issue_qk = [&](int w, int slot) {
-                const uint32_t d_tmem = tmem + (w ? C::kColS1 : C::kColS0);
-                const uint32_t qa = sQ + w * C::kTileBytes;
-                const uint32_t kb_ = sKV + slot * C::kTileBytes;
+        auto wait_all = [&](uint32_t b_, uint32_t par, uint32_t where) {
+            const bool r_ = wait_bar(b_, par, abort_addr, where);
+            return __all_sync(0xffffffffu, r_);
+        };
+        auto commit = [&](uint32_t b_) {
+            if (leader) mma_commit(b_);
+            __syncwarp();
+        };
+        auto issue_qk = [&](int w, int slot) {
+            const uint32_t d_tmem = tmem + (w ? C::kColS1 : C::kColS0);
+            const uint64_t dq = w ? desc_q1 : desc_q0;
+            const uint64_t dk = desc_k + (uint64_t)((slot * C::kTileBytes) >> 4);
+            if (leader) {
 #pragma unroll
                 for (int kk = 0; kk < C::kQkSteps; ++kk) {
-                    const uint32_t off = (kk >> 2) * C::kSwBlockBytes + (kk & 3) * 32;
-                    const uint64_t da = make_smem_desc(qa + off, 16, 1024);
-                    const uint64_t db = make_smem_desc(kb_ + off, 16, 1024);
+                    const uint64_t off = (uint64_t)(((kk >> 2) * C::kSwBlockBytes + (kk & 3) * 32) >> 4);
                     if constexpr (KIND == KIND_E4M3)
-                        mma_f8_ss(d_tmem, da, db, idesc_qk, kk > 0);
+                        mma_f8_ss(d_tmem, dq + off, dk + off, idesc_qk, kk > 0);
                     else
-                        mma_f16_ss(d_tmem, da, db, idesc_qk, kk > 0);
-                }
-            };
-            auto issue_pv = [&](int w, int slot, bool acc) {
-                const uint32_t d_tmem = tmem + (w ? C::kColO1 : C::kColO0);
-                const uint32_t a_tmem = tmem + (w ? C::kColS1 : C::kColS0) + C::kPOffset;
-                const uint32_t vb = sKV + slot * C::kTileBytes;
-#pragma unroll
-                for (int kk = 0; kk < C::kPvSteps; ++kk) {
-                    const uint64_t db = make_smem_desc(vb + kk * C::kPvKeysPerStep * 128,
-                                                       C::kSwBlockBytes, 1024);
-                    if constexpr (KIND == KIND_E4M3)
-                        mma_f8_ts(d_tmem, a_tmem + kk * 8, db, idesc_pv, (acc || kk > 0) ? 1u : 0u);
-                    else
-                        mma_f16_ts(d_tmem, a_tmem + kk * 8, db, idesc_pv, (acc || kk > 0) ? 1u : 0u);
-                }
-            };
-
-            for (int w = 0; w < kQTiles && ok; ++w)
-                if ((w ? nt1 : nt0) > 0) ok = wait_bar(bar(C::kBarQFull + w), 0, abort_addr, 0x20000u | w);
-
-            for (int i = 0; i <= n && ok; ++i) {
-                const int tK = 2 * i, tV = 2 * i + 1;
-                const int slotK = tK % NS, slotV = tV % NS;
-                if (i < n) {
-                    ok = wait_bar(bar(C::kBarKVFull + slotK), (uint32_t)(tK / NS) & 1u, abort_addr,
-                                  0x21000u | (uint32_t)i);
-                    if (!ok) break;
-                    tc_fence_after();
-                    if (i < nt0) {
-                        issue_qk(0, slotK);
-                        mma_commit(bar(C::kBarSFull + 0));
-                    }
-                }
-                if (i >= 1) {
-                    const int j = i - 1;
-                    if (j < nt1) {
-                        ok = wait_bar(bar(C::kBarPFull + 1), (uint32_t)j & 1u, abort_addr,
-                                      0x22000u | (uint32_t)j);
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_pv(1, (2 * j + 1) % NS, j > 0);
-                        if (j == nt1 - 1) mma_commit(bar(C::kBarOFull + 1));
-                    }
-                    mma_commit(bar(C::kBarKVEmpty + (2 * j + 1) % NS));   // V_(i-1) free
-                }
-                if (i < n) {
-                    if (i < nt1) {
-                        issue_qk(1, slotK);
-                        mma_commit(bar(C::kBarSFull + 1));
-                    }
-                    mma_commit(bar(C::kBarKVEmpty + slotK));               // K_i free
-                    ok = wait_bar(bar(C::kBarKVFull + slotV), (uint32_t)(tV / NS) & 1u, abort_addr,
-                                  0x23000u | (uint32_t)i);
-                    if (!ok) break;
-                    tc_fence_after();
-                    if (i < nt0) {
-                        ok = wait_bar(bar(C::kBarPFull + 0), (uint32_t)i & 1u, abort_addr,
-                                      0x24000u | (uint32_t)i);
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_pv(0, slotV, i > 0);
-                        if (i == nt0 - 1) mma_commit(bar(C::kBarOFull + 0));
-                    }
+                        mma_f16_ss(d_tmem, dq + off, dk + off, idesc_qk, kk > 0);
                 }
             }
-            if (!ok) {
-                // make sure no MMA is still writing tensor memory at exit
-                mma_commit(bar(C::kBarDrain));
-                const uint64_t t0 = global_timer_ns();
-                while (!mbar_try_wait(bar(C::kBarDrain), 0) && global_timer_ns() - t0 < 100000000ull) {
+            __syncwarp();
+        };
+        auto issue_pv = [&](int w, int slot, bool acc) {
+            const uint32_t d_tmem = tmem + (w ? C::kColO1 : C::kColO0);
+            const uint32_t a_tmem = tmem + (w ? C::kColS1 : C::kColS0) + C::kPOffset;
+            const uint64_t dv = desc_v + (uint64_t)((slot * C::kTileBytes) >> 4);
+            if (leader) {
+#pragma unroll
+                for (int kk = 0; kk < C::kPvSteps; ++kk) {
+                    const uint64_t off = (uint64_t)((kk * C::kPvKeysPerStep * 128) >> 4);
+                    const uint32_t accum = (acc || kk > 0) ? 1u : 0u;
+                    if constexpr (KIND == KIND_E4M3)
+                        mma_f8_ts(d_tmem, a_tmem + kk * 8, dv + off, idesc_pv, accum);
+                    else
+                        mma_f16_ts(d_tmem, a_tmem + kk * 8, dv + off, idesc_pv, accum);
+                }
+            }
+            __syncwarp();
+        };
+
+        if (nt0 > 0) ok = wait_all(bar(C::kBarQFull + 0), 0, 0x20000u);
+        if (ok && nt1 > 0) ok = wait_all(bar(C::kBarQFull + 1), 0, 0x20001u);
+
+        for (int i = 0; i <= n && ok; ++i) {
+            const int tK = 2 * i, tV = 2 * i + 1;
+            const int slotK = tK % NS, slotV = tV % NS;
+            if (i < n) {
+                ok = wait_all(bar(C::kBarKVFull + slotK), (uint32_t)(tK / NS) & 1u, 0x21000u | (uint32_t)i);
+                if (!ok) break;
+                tc_fence_after();
+                if (i < nt0) {
+                    issue_qk(0, slotK);
+                    commit(bar(C::kBarSFull + 0));
+                }
+            }
+            if (i >= 1) {
+                const int j = i - 1;
+                if (j < nt1) {
+                    ok = wait_all(bar(C::kBarPFull + 1), (uint32_t)j & 1u, 0x22000u | (uint32_t)j);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(1, (2 * j + 1) % NS, j > 0);
+                    if (j == nt1 - 1) commit(bar(C::kBarOFull + 1));
+                }
+                commit(bar(C::kBarKVEmpty + (2 * j + 1) % NS));   // V_(i-1) free
+            }
+            if (i < n) {
+                if (i < nt1) {
+                    issue_qk(1, slotK);
+                    commit(bar(C::kBarSFull + 1));
+                }
+                commit(bar(C::kBarKVEmpty + slotK));               // K_i free
+                ok = wait_all(bar(C::kBarKVFull + slotV), (uint32_t)(tV / NS) & 1u, 0x23000u | (uint32_t)i);
+                if (!ok) break;
+                tc_fence_after();
+                if (i < nt0) {
+                    ok = wait_all(bar(C::kBarPFull + 0), (uint32_t)i & 1u, 0x24000u | (uint32_t)i);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(0, slotV, i > 0);
+                    if (i == nt0 - 1) commit(bar(C::kBarOFull + 0));
                 }
             }
         }
-    } else {
+        if (!ok) {
+            // make sure no MMA is still writing tensor memory at exit
+            commit(bar(C::kBarDrain));
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(bar(C::kBarDrain), 0) && global_timer_ns() - t0 < 100000000ull) {
+            }
+        }
+        // teardown: the softmax groups have read O for the last time
+        named_bar_sync(1, 256 + 32);
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    } else if (warp < 8) {
         // ================= softmax groups (warps 0-7) ====================
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
         const int w = warp >> 2;                 // query tile
         const int quarter = warp & 3;            // TMEM lane quarter of this warp
         const int r = (int)(threadIdx.x & 127);  // row within the tile
@@ -352,8 +380,9 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         const uint32_t tP = tS + C::kPOffset;
         const uint32_t tO = tmem + lane_base + (w ? C::kColO1 : C::kColO0);
         const float sl = p.score_log2;
+        const uint64_t sl2 = f2_pack(sl, sl);
         float m_run = -INFINITY;   // running max of the scaled scores (log2 units)
-        float l_run = 0.0f;        // running sum of 2^(s*sl - m_run)
+        float l_run = 0.0f;        // running sum of 2^(s*sl - m_run + kPLog2)
         bool ok = true;
 
         for (int i = 0; i < nw; ++i) {
@@ -362,35 +391,50 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             if (!ok) break;
             tc_fence_after();
 
+            // S row in two halves: the second half's load overlaps the first
+            // half's masking and max
             float s[kBlockN];
-#pragma unroll
-            for (int c = 0; c < kBlockN / 32; ++c)
-                tmem_ld32(tS + 32 * c, *reinterpret_cast<float(*)[32]>(&s[32 * c]));
+            tmem_ld32(tS + 0, *reinterpret_cast<float(*)[32]>(&s[0]));
+            tmem_ld32(tS + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
             tmem_wait_ld();
+            reg_fence32(&s[0]);
+            reg_fence32(&s[32]);
+            tmem_ld32(tS + 64, *reinterpret_cast<float(*)[32]>(&s[64]));
+            tmem_ld32(tS + 96, *reinterpret_cast<float(*)[32]>(&s[96]));
 
             // mask: keys past Sk, and (causal) keys after the row
             const int key0 = i * kBlockN;
             const bool edge = (key0 + kBlockN > p.Sk) ||
                               (p.causal && key0 + kBlockN - 1 > m0 + w * kBlockM);
+            int lim = p.Sk - key0;
+            if (p.causal) lim = min(lim, row - key0 + 1);
             if (edge) {
-                int lim = p.Sk - key0;
-                if (p.causal) lim = min(lim, row - key0 + 1);
 #pragma unroll
-                for (int c = 0; c < kBlockN; ++c)
+                for (int c = 0; c < kBlockN / 2; ++c)
                     if (c >= lim) s[c] = -INFINITY;
             }
-
-            // row max (tree) in raw score units, then to log2 units
-            float mx[8];
+            // first half only: columns 0..63 (64..127 are still in flight)
+            float mx0 = s[0], mx1 = s[1];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) mx[u] = s[u];
+            for (int c = 2; c + 4 <= kBlockN / 2 - 2; c += 4) {
+                mx0 = fmax3(mx0, s[c], s[c + 1]);
+                mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
+            }
+            mx0 = fmax3(mx0, s[kBlockN / 2 - 2], s[kBlockN / 2 - 1]);
+            tmem_wait_ld();
+            reg_fence32(&s[64]);
+            reg_fence32(&s[96]);
+            if (edge) {
 #pragma unroll
-            for (int c = 8; c < kBlockN; c += 8)
+                for (int c = kBlockN / 2; c < kBlockN; ++c)
+                    if (c >= lim) s[c] = -INFINITY;
+            }
 #pragma unroll
-                for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], s[c + u]);
-            float tile_max = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-            tile_max *= sl;
+            for (int c = kBlockN / 2; c < kBlockN; c += 4) {
+                mx0 = fmax3(mx0, s[c], s[c + 1]);
+                mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
+            }
+            const float tile_max = fmaxf(mx0, mx1) * sl;
 
             // The running max only moves when the new one exceeds it by more
             // than the threshold; weights computed against a stale max are
@@ -403,40 +447,47 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             }
             l_run *= alpha;
 
-            // weights p = 2^(s*sl - m), rounded for the PV product
-            const float neg_m = -m_run;
-            float sum4[4] = {0.f, 0.f, 0.f, 0.f};
-            if constexpr (KIND == KIND_E4M3) {
+            // weights p = 2^(s*sl - m [+ log2 of the P scale]): three pairs in
+            // four on the MUFU, the fourth on the FMA pipe (exp2_poly_x2);
+            // row sums from the fp32 values, P rounded for the PV product
+            const float neg_m = C::kPLog2 - m_run;
+            const uint64_t nm2 = f2_pack(neg_m, neg_m);
+            uint64_t sum2[2] = {0ull, 0ull};
 #pragma unroll
-                for (int c = 0; c < kBlockN / 64; ++c) {
-                    uint32_t pk[16];
+            for (int c = 0; c < kBlockN / 32; ++c) {
+                uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        float q0 = ex2_approx(fmaf(s[64 * c + 4 * e + 0], sl, neg_m));
-                        float q1 = ex2_approx(fmaf(s[64 * c + 4 * e + 1], sl, neg_m));
-                        float q2 = ex2_approx(fmaf(s[64 * c + 4 * e + 2], sl, neg_m));
-                        float q3 = ex2_approx(fmaf(s[64 * c + 4 * e + 3], sl, neg_m));
-                        sum4[0] += q0; sum4[1] += q1; sum4[2] += q2; sum4[3] += q3;
-                        pk[e] = pack_e4m3x4(q0 * p.p_mul, q1 * p.p_mul, q2 * p.p_mul, q3 * p.p_mul);
+                for (int e = 0; e < 16; ++e) {
+                    const uint64_t x2 = f2_fma(f2_pack(s[32 * c + 2 * e], s[32 * c + 2 * e + 1]), sl2, nm2);
+                    float x0, x1;
+                    f2_unpack(x2, x0, x1);
+                    uint64_t p2;
+                    if ((e & 3) == 3) {
+                        p2 = exp2_poly_x2(f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f)));
+                    } else {
+                        p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
                     }
-                    tmem_st16(tP + 16 * c, pk);
-                }
-            } else {
-#pragma unroll
-                for (int c = 0; c < kBlockN / 32; ++c) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float q0 = ex2_approx(fmaf(s[32 * c + 2 * e], sl, neg_m));
-                        const float q1 = ex2_approx(fmaf(s[32 * c + 2 * e + 1], sl, neg_m));
-                        sum4[(2 * e) & 3] += q0;
-                        sum4[(2 * e + 1) & 3] += q1;
+                    sum2[e & 1] = f2_add(sum2[e & 1], p2);
+                    float q0, q1;
+                    f2_unpack(p2, q0, q1);
+                    if constexpr (KIND == KIND_E4M3) {
+                        if (e & 1) pk[e >> 1] |= pack_e4m3x4(0.f, 0.f, q0, q1) & 0xFFFF0000u;
+                        else pk[e >> 1] = pack_e4m3x4(q0, q1, 0.f, 0.f) & 0x0000FFFFu;
+                    } else {
                         pk[e] = (KIND == KIND_BF16) ? pack_bf16x2(q0, q1) : pack_f16x2(q0, q1);
                     }
-                    tmem_st16(tP + 16 * c, pk);
                 }
+                if constexpr (KIND == KIND_E4M3)
+                    tmem_st8(tP + 8 * c, pk);
+                else
+                    tmem_st16(tP + 16 * c, pk);
             }
-            l_run += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+            {
+                float a0, a1, b0, b1;
+                f2_unpack(sum2[0], a0, a1);
+                f2_unpack(sum2[1], b0, b1);
+                l_run += (a0 + a1) + (b0 + b1);
+            }
             // O_w (quiescent: its last update is covered by the S_w(i) commit)
             // takes the same factor as l before P_w(i) V_i is added to it.
             if (i > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
@@ -445,6 +496,7 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                     float o[32];
                     tmem_ld32(tO + 32 * c, o);
                     tmem_wait_ld();
+                    reg_fence32(o);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) o[e] *= alpha;
                     tmem_st32(tO + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(o));
@@ -471,6 +523,7 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 float o[32];
                 tmem_ld32(tO + 32 * c, o);
                 tmem_wait_ld();
+                reg_fence32(o);
                 uint32_t u[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
@@ -484,18 +537,12 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 }
             }
             if (p.lse != nullptr && live)
-                p.lse[(size_t)bh * p.Sq + row] = (m_run + __log2f(l_run)) * kLn2;
+                p.lse[(size_t)bh * p.Sq + row] = (m_run + __log2f(l_run) - C::kPLog2) * kLn2;
         }
+        tc_fence_before();
+        named_bar_sync(1, 256 + 32);
     }
 
-    // ---- teardown ------------------------------------------------------------
-    tc_fence_before();
-    __syncthreads();
-    if (warp == kMmaWarp) {
-        __syncwarp();
-        tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
-    }
 }
 
 }  // namespace sdpa

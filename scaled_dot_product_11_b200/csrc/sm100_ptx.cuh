@@ -49,6 +49,11 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
+// Named CTA barrier `id` over `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // fences
 // ---------------------------------------------------------------------------
@@ -179,6 +184,26 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&u)[32
         : "memory");
 }
 
+// Make later uses of r depend on a preceding tcgen05.wait::ld (volatile asm
+// statements keep their order; this one "redefines" the registers).
+__device__ __forceinline__ void reg_fence32(float* r) {
+    asm volatile(""
+                 : "+f"(r[0]), "+f"(r[1]), "+f"(r[2]), "+f"(r[3]), "+f"(r[4]), "+f"(r[5]),
+                   "+f"(r[6]), "+f"(r[7]), "+f"(r[8]), "+f"(r[9]), "+f"(r[10]), "+f"(r[11]),
+                   "+f"(r[12]), "+f"(r[13]), "+f"(r[14]), "+f"(r[15]), "+f"(r[16]), "+f"(r[17]),
+                   "+f"(r[18]), "+f"(r[19]), "+f"(r[20]), "+f"(r[21]), "+f"(r[22]), "+f"(r[23]),
+                   "+f"(r[24]), "+f"(r[25]), "+f"(r[26]), "+f"(r[27]), "+f"(r[28]), "+f"(r[29]),
+                   "+f"(r[30]), "+f"(r[31]));
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* u) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+        ::"r"(taddr), "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]),
+          "r"(u[6]), "r"(u[7])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* u) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -222,13 +247,76 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t ab_format, bool b_mn_
            ((b_mn_major ? 1u : 0u) << 16) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
+// One lane of a converged warp gets true (the same lane every time the whole
+// warp executes it).
+__device__ __forceinline__ bool elect_one() {
+    uint32_t e;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(e));
+    return e != 0;
+}
+
 // ---------------------------------------------------------------------------
 // numeric helpers
 // ---------------------------------------------------------------------------
+// packed fp32 pairs (sm_100 f32x2 arithmetic on the FMA pipe)
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x for a pair of floats on the FMA pipe, for x in [-126, 64]:
+//   n = rint(x) by adding and removing 1.5 * 2^23 (the sum's low mantissa
+//   bits hold n), f = x - n in [-1/2, 1/2], 2^f by a cubic fitted to the
+//   relative error on that interval (max 1.0e-4), and 2^n by adding n to the
+//   exponent field: bits(t) << 23 is n << 23 because the constant's own bits
+//   vanish in the shift.
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
+    const uint64_t kMagic = 0x4B4000004B400000ull;       // 12582912.0f, twice
+    const uint64_t kNegMagic = 0xCB400000CB400000ull;
+    const uint64_t kMinusOne = 0xBF800000BF800000ull;
+    const uint64_t kC3 = 0x3D6150EA3D6150EAull;          // 0.05500881
+    const uint64_t kC2 = 0x3E78061B3E78061Bull;          // 0.24221079
+    const uint64_t kC1 = 0x3F317AFD3F317AFDull;          // 0.69328290
+    const uint64_t kOne = 0x3F8000003F800000ull;
+    const uint64_t t = f2_add(x, kMagic);
+    const uint64_t n = f2_add(t, kNegMagic);
+    const uint64_t f = f2_fma(n, kMinusOne, x);
+    uint64_t p = f2_fma(kC3, f, kC2);
+    p = f2_fma(p, f, kC1);
+    p = f2_fma(p, f, kOne);
+    const uint32_t tlo = (uint32_t)t, thi = (uint32_t)(t >> 32);
+    const uint32_t plo = (uint32_t)p + (tlo << 23);
+    const uint32_t phi = (uint32_t)(p >> 32) + (thi << 23);
+    return ((uint64_t)phi << 32) | plo;
 }
 
 // Pack two floats to bf16x2 / f16x2 (round to nearest even); `lo` goes to

@@ -75,6 +75,11 @@ WORKLOADS = {
                     seed=42),
     "fp8": Workload("fp8_b2_h32_s16384_d128_causal", 2, 32, 32, 16384, 16384, 128, True,
                     dtype="e4m3", seed=9000),
+    # profiling-sized cases: inputs above the 126 MB L2, a few hundred MB in all
+    "lm_causal_b4": Workload("lm_causal_b4_h16_s4096_d128", 4, 16, 16, 4096, 4096, 128, True,
+                             seed=4096),
+    "lm_full_b4": Workload("lm_full_b4_h16_s4096_d128", 4, 16, 16, 4096, 4096, 128, False,
+                           seed=4096),
 }
 
 
