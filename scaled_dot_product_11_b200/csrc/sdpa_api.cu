@@ -100,6 +100,12 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& prm, cu
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        // The kernel moves registers between warpgroups with setmaxnreg; that
+        // split is sized for exactly kLaunchRegs per thread at launch, so a
+        // build that allocated a different count must not run.
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return SDPA_ERR_CUDA;
+        if (fa.numRegs != sdpa::kLaunchRegs) return SDPA_ERR_UNSUPPORTED;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
             cudaSuccess)
             return SDPA_ERR_CUDA;
@@ -141,10 +147,10 @@ extern "C" int sdpa_fwd(const void* q, const void* k, const void* v, void* o, fl
     prm.score_log2 = scale * sdpa::kLog2e;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (dtype == SDPA_BF16)
-        return d == 128 ? launch<128, sdpa::KIND_BF16, 4>(q, k, v, prm, s)
-                        : launch<64, sdpa::KIND_BF16, 8>(q, k, v, prm, s);
-    return d == 128 ? launch<128, sdpa::KIND_FP16, 4>(q, k, v, prm, s)
-                    : launch<64, sdpa::KIND_FP16, 8>(q, k, v, prm, s);
+        return d == 128 ? launch<128, sdpa::KIND_BF16, SDPA_STAGES_D128>(q, k, v, prm, s)
+                        : launch<64, sdpa::KIND_BF16, SDPA_STAGES_D64>(q, k, v, prm, s);
+    return d == 128 ? launch<128, sdpa::KIND_FP16, SDPA_STAGES_D128>(q, k, v, prm, s)
+                    : launch<64, sdpa::KIND_FP16, SDPA_STAGES_D64>(q, k, v, prm, s);
 }
 
 extern "C" int sdpa_fwd_fp8(const void* q8, const void* k8, const void* v8, float descale_q,

@@ -38,6 +38,24 @@
 #include <cuda_fp16.h>
 #include "sm100_ptx.cuh"
 
+// Tuning knobs (compile-time; the defaults are the measured best on B200).
+// Pairs e (0..15) of a 32-column chunk whose exponentials go to the FMA pipe:
+// bit (e & 7) of this mask.
+#ifndef SDPA_POLY_MASK
+#define SDPA_POLY_MASK 0x88
+#endif
+// 1: the softmax signals each P tile once; 2: once per half of the keys.
+#ifndef SDPA_P_SPLIT
+#define SDPA_P_SPLIT 2
+#endif
+// K/V ring depth for d = 128 (16-bit) and d = 64.
+#ifndef SDPA_STAGES_D128
+#define SDPA_STAGES_D128 4
+#endif
+#ifndef SDPA_STAGES_D64
+#define SDPA_STAGES_D64 8
+#endif
+
 namespace sdpa {
 
 enum Kind { KIND_BF16 = 0, KIND_FP16 = 1, KIND_E4M3 = 2 };
@@ -46,8 +64,9 @@ constexpr int kBlockM = 128;        // query rows per tile (= TMEM lanes)
 constexpr int kBlockN = 128;        // keys per K/V tile
 constexpr int kQTiles = 2;          // query tiles per CTA
 constexpr int kThreads = 384;       // 3 warpgroups
-constexpr int kSoftmaxRegs = 200;   // per thread after setmaxnreg, warpgroups 0-1
-constexpr int kOtherRegs = 96;      // warpgroup 2 (TMA, MMA, two idle warps)
+constexpr int kSoftmaxRegs = 208;   // per thread after setmaxnreg, warpgroups 0-1
+constexpr int kOtherRegs = 88;      // warpgroup 2 (TMA, MMA, two idle warps)
+constexpr int kLaunchRegs = 168;    // registers per thread at launch (384 threads, 1 CTA/SM)
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
@@ -89,15 +108,16 @@ struct FwdCfg {
     static constexpr int kSmemQ = 0;
     static constexpr int kSmemKV = kQTiles * kTileBytes;
     static constexpr int kSmemBar = kSmemKV + NS * kTileBytes;
-    // barriers: q_full[2] kv_full[NS] kv_empty[NS] s_full[2] p_full[2] o_full[2] drain[1]
+    // barriers: q_full[2] kv_full[NS] kv_empty[NS] s_full[2] p_full[2 tiles][2 halves]
+    //           o_full[2] drain[1]
     static constexpr int kBarQFull = 0;
     static constexpr int kBarKVFull = 2;
     static constexpr int kBarKVEmpty = 2 + NS;
     static constexpr int kBarSFull = 2 + 2 * NS;
     static constexpr int kBarPFull = 4 + 2 * NS;
-    static constexpr int kBarOFull = 6 + 2 * NS;
-    static constexpr int kBarDrain = 8 + 2 * NS;
-    static constexpr int kNumBars = 9 + 2 * NS;
+    static constexpr int kBarOFull = 8 + 2 * NS;
+    static constexpr int kBarDrain = 10 + 2 * NS;
+    static constexpr int kNumBars = 11 + 2 * NS;
     static constexpr int kSmemTmemSlot = kSmemBar + 8 * kNumBars;
     static constexpr int kSmemAbort = kSmemTmemSlot + 4;
     static constexpr int kSmemUsed = kSmemAbort + 4;
@@ -148,6 +168,12 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, uint32_t
     return wait_bar_slow(bar, parity, abort_addr, where);
 }
 
+// Pairs of one 32-column chunk (e = 0..15) whose exponentials are evaluated
+// on the FMA pipe instead of the MUFU (SDPA_POLY_MASK).
+__device__ __forceinline__ constexpr bool poly_pair(int e) {
+    return ((SDPA_POLY_MASK >> (e & 7)) & 1) != 0;
+}
+
 // Row-tile key counts of one CTA: number of K/V tiles query tile w needs.
 __device__ __forceinline__ int tiles_for(int row0, int Sq, int Sk, int causal) {
     if (row0 >= Sq) return 0;
@@ -189,7 +215,8 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         for (int w = 0; w < kQTiles; ++w) {
             mbar_init(bar(C::kBarQFull + w), 1);
             mbar_init(bar(C::kBarSFull + w), 1);
-            mbar_init(bar(C::kBarPFull + w), kBlockM);
+            mbar_init(bar(C::kBarPFull + 2 * w), kBlockM);
+            mbar_init(bar(C::kBarPFull + 2 * w + 1), kBlockM);
             mbar_init(bar(C::kBarOFull + w), 1);
         }
         for (int s = 0; s < NS; ++s) {
@@ -213,8 +240,9 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ld_shared_u32(slot_addr);
-    // launch: 384 x 168 registers; split: 256 x 200 + 128 x 96 = 63488 <= 64512
-    static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * 168, "register split");
+    // launch: 384 x 168 registers; split: 256 x 208 + 128 x 88 = 64512 <= 64512 (the host
+    // checks the compiled register count before the first launch)
+    static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * kLaunchRegs, "register split");
 
     const uint32_t sQ = sbase + C::kSmemQ;
     const uint32_t sKV = sbase + C::kSmemKV;
@@ -293,13 +321,15 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             }
             __syncwarp();
         };
-        auto issue_pv = [&](int w, int slot, bool acc) {
+        // O_w (+)= P_w V over the keys of one half of the tile (K steps
+        // [h * kPvSteps / 2, (h + 1) * kPvSteps / 2)); P is read from TMEM.
+        auto issue_pv_half = [&](int w, int slot, bool acc, int h) {
             const uint32_t d_tmem = tmem + (w ? C::kColO1 : C::kColO0);
             const uint32_t a_tmem = tmem + (w ? C::kColS1 : C::kColS0) + C::kPOffset;
             const uint64_t dv = desc_v + (uint64_t)((slot * C::kTileBytes) >> 4);
             if (leader) {
 #pragma unroll
-                for (int kk = 0; kk < C::kPvSteps; ++kk) {
+                for (int kk = h * C::kPvSteps / 2; kk < (h + 1) * C::kPvSteps / 2; ++kk) {
                     const uint64_t off = (uint64_t)((kk * C::kPvKeysPerStep * 128) >> 4);
                     const uint32_t accum = (acc || kk > 0) ? 1u : 0u;
                     if constexpr (KIND == KIND_E4M3)
@@ -309,6 +339,22 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 }
             }
             __syncwarp();
+        };
+        // wait for each half of P_w(j) and issue its MMAs
+        auto pv = [&](int w, int slot, int j) -> bool {
+            for (int h = 0; h < SDPA_P_SPLIT; ++h) {
+                if (!wait_all(bar(C::kBarPFull + 2 * w + h), (uint32_t)j & 1u,
+                              0x22000u | (w << 11) | (h << 10) | (uint32_t)j))
+                    return false;
+                tc_fence_after();
+                if (SDPA_P_SPLIT == 1) {
+                    issue_pv_half(w, slot, j > 0, 0);
+                    issue_pv_half(w, slot, j > 0, 1);
+                } else {
+                    issue_pv_half(w, slot, j > 0, h);
+                }
+            }
+            return true;
         };
 
         if (nt0 > 0) ok = wait_all(bar(C::kBarQFull + 0), 0, 0x20000u);
@@ -320,7 +366,6 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             if (i < n) {
                 ok = wait_all(bar(C::kBarKVFull + slotK), (uint32_t)(tK / NS) & 1u, 0x21000u | (uint32_t)i);
                 if (!ok) break;
-                tc_fence_after();
                 if (i < nt0) {
                     issue_qk(0, slotK);
                     commit(bar(C::kBarSFull + 0));
@@ -329,10 +374,8 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             if (i >= 1) {
                 const int j = i - 1;
                 if (j < nt1) {
-                    ok = wait_all(bar(C::kBarPFull + 1), (uint32_t)j & 1u, 0x22000u | (uint32_t)j);
+                    ok = pv(1, (2 * j + 1) % NS, j);
                     if (!ok) break;
-                    tc_fence_after();
-                    issue_pv(1, (2 * j + 1) % NS, j > 0);
                     if (j == nt1 - 1) commit(bar(C::kBarOFull + 1));
                 }
                 commit(bar(C::kBarKVEmpty + (2 * j + 1) % NS));   // V_(i-1) free
@@ -345,12 +388,9 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 commit(bar(C::kBarKVEmpty + slotK));               // K_i free
                 ok = wait_all(bar(C::kBarKVFull + slotV), (uint32_t)(tV / NS) & 1u, 0x23000u | (uint32_t)i);
                 if (!ok) break;
-                tc_fence_after();
                 if (i < nt0) {
-                    ok = wait_all(bar(C::kBarPFull + 0), (uint32_t)i & 1u, 0x24000u | (uint32_t)i);
+                    ok = pv(0, slotV, i);
                     if (!ok) break;
-                    tc_fence_after();
-                    issue_pv(0, slotV, i > 0);
                     if (i == nt0 - 1) commit(bar(C::kBarOFull + 0));
                 }
             }
@@ -446,10 +486,26 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 m_run = tile_max;
             }
             l_run *= alpha;
+            // O_w (quiescent: its last update is covered by the S_w(i) commit)
+            // takes the same factor as l before any of P_w(i) V_i is added.
+            if (i > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    float o[32];
+                    tmem_ld32(tO + 32 * c, o);
+                    tmem_wait_ld();
+                    reg_fence32(o);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] *= alpha;
+                    tmem_st32(tO + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(o));
+                }
+            }
 
-            // weights p = 2^(s*sl - m [+ log2 of the P scale]): three pairs in
-            // four on the MUFU, the fourth on the FMA pipe (exp2_poly_x2);
-            // row sums from the fp32 values, P rounded for the PV product
+            // weights p = 2^(s*sl - m [+ log2 of the P scale]): most pairs on
+            // the MUFU, kPolyPairs in every 8 on the FMA pipe
+            // (exp2_poly_x2); row sums from the fp32 values, P rounded for the
+            // PV product and stored to TMEM one half of the keys at a time so
+            // the MMA warp can start on the first half.
             const float neg_m = C::kPLog2 - m_run;
             const uint64_t nm2 = f2_pack(neg_m, neg_m);
             uint64_t sum2[2] = {0ull, 0ull};
@@ -462,7 +518,7 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                     float x0, x1;
                     f2_unpack(x2, x0, x1);
                     uint64_t p2;
-                    if ((e & 3) == 3) {
+                    if (poly_pair(e)) {
                         p2 = exp2_poly_x2(f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f)));
                     } else {
                         p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
@@ -477,34 +533,27 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                         pk[e] = (KIND == KIND_BF16) ? pack_bf16x2(q0, q1) : pack_f16x2(q0, q1);
                     }
                 }
+                // first half of the keys: its stores were issued one chunk ago,
+                // so this wait finds them done
+                if (SDPA_P_SPLIT == 2 && c == 2) {
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(bar(C::kBarPFull + 2 * w));
+                }
                 if constexpr (KIND == KIND_E4M3)
                     tmem_st8(tP + 8 * c, pk);
                 else
                     tmem_st16(tP + 16 * c, pk);
             }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(C::kBarPFull + 2 * w + (SDPA_P_SPLIT - 1)));
             {
                 float a0, a1, b0, b1;
                 f2_unpack(sum2[0], a0, a1);
                 f2_unpack(sum2[1], b0, b1);
                 l_run += (a0 + a1) + (b0 + b1);
             }
-            // O_w (quiescent: its last update is covered by the S_w(i) commit)
-            // takes the same factor as l before P_w(i) V_i is added to it.
-            if (i > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
-#pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    float o[32];
-                    tmem_ld32(tO + 32 * c, o);
-                    tmem_wait_ld();
-                    reg_fence32(o);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] *= alpha;
-                    tmem_st32(tO + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(o));
-                }
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(bar(C::kBarPFull + w));
         }
 
         // ---- epilogue: O / l -> 16-bit, LSE ---------------------------------
