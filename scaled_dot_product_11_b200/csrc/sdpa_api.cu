@@ -49,6 +49,20 @@ int check_device() {
     return ok ? SDPA_OK : SDPA_ERR_UNSUPPORTED;
 }
 
+// Streaming multiprocessors of the current device (cached; 148 on B200).
+int sm_count() {
+    static int cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Common argument checks of both entry points.
@@ -64,7 +78,7 @@ int check_args(const void* q, const void* k, const void* v, const void* o, const
     // addressing limits: head counts and row indices fit the 32-bit TMA
     // coordinates and the grid, element offsets fit 64-bit size_t trivially
     const long long bhq = (long long)B * Hq, bhk = (long long)B * Hkv;
-    const long long qblocks = (Sq + 255) / 256;
+    const long long qblocks = (Sq + 127) / 128;
     if (bhq > INT32_MAX || bhk > INT32_MAX || bhq * qblocks > INT32_MAX) return SDPA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return SDPA_ERR_UNSUPPORTED;
     if (causal && Sq != Sk) return SDPA_ERR_UNSUPPORTED;
@@ -100,18 +114,12 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& prm, cu
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-        // The kernel moves registers between warpgroups with setmaxnreg; that
-        // split is sized for exactly kLaunchRegs per thread at launch, so a
-        // build that allocated a different count must not run.
-        cudaFuncAttributes fa;
-        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return SDPA_ERR_CUDA;
-        if (fa.numRegs != sdpa::kLaunchRegs) return SDPA_ERR_UNSUPPORTED;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
             cudaSuccess)
             return SDPA_ERR_CUDA;
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
-    const unsigned grid = (unsigned)((long long)prm.n_qblocks * prm.B * prm.Hq);
+    const unsigned grid = (unsigned)((long long)prm.n_qtiles * prm.B * prm.Hq);
     kern<<<grid, sdpa::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, prm);
     return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
 }
@@ -126,7 +134,11 @@ FwdParams make_params(void* o, float* lse, int B, int Hq, int Hkv, int Sq, int S
     prm.Sq = Sq;
     prm.Sk = Sk;
     prm.group = Hq / Hkv;
-    prm.n_qblocks = (Sq + 255) / 256;
+    prm.n_qtiles = (Sq + 127) / 128;
+    // about two waves of CTAs per group of (batch, head) pairs
+    prm.group_heads = (2 * sm_count() + prm.n_qtiles - 1) / prm.n_qtiles;
+    if (prm.group_heads < 1) prm.group_heads = 1;
+    if (prm.group_heads > B * Hq) prm.group_heads = B * Hq;
     prm.causal = causal;
     prm.score_log2 = 0.f;
     prm.out_mul = 1.f;
@@ -166,7 +178,7 @@ extern "C" int sdpa_fwd_fp8(const void* q8, const void* k8, const void* v8, floa
     FwdParams prm = make_params(o, lse, B, Hq, Hkv, Sq, Sk, causal);
     prm.score_log2 = scale * descale_q * descale_k * sdpa::kLog2e;
     prm.out_mul = descale_v;
-    return launch<128, sdpa::KIND_E4M3, 8>(q8, k8, v8, prm, reinterpret_cast<cudaStream_t>(stream));
+    return launch<128, sdpa::KIND_E4M3, SDPA_STAGES_FP8>(q8, k8, v8, prm, reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" const char* sdpa_strerror(int status) {

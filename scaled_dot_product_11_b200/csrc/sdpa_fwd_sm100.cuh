@@ -12,25 +12,26 @@
 // Lab 5: attention on GPU", section 1; causal mask section 7; MHA/GQA/MQA
 // section 9; FP8 E4M3 forward section 10.
 //
-// One CTA owns 2 x 128 query rows of one (batch, query head) and walks the
-// K/V tiles of that head's KV head.  Warp roles (384 threads):
-//   warps 0-3  softmax group 0: query tile 0, thread = row = TMEM lane
-//   warps 4-7  softmax group 1: query tile 1
-//   warp  8    TMA producer: Q tiles once, then K_0, V_0, K_1, V_1, ...
+// One CTA owns 128 query rows of one (batch, query head) and walks the K/V
+// tiles (128 keys each) of that head's KV head.  Warp roles (320 threads):
+//   warps 0-3  softmax group 0: keys 0-63 of every tile, thread = row = lane
+//   warps 4-7  softmax group 1: keys 64-127 of every tile
+//   warp  8    TMA producer: Q once, then K/V tiles in MMA consumption order
 //   warp  9    MMA issuer (one elected lane) and TMEM owner
-//   warps 10-11 idle (they complete warpgroup 2 for the register split)
-// Registers are moved with setmaxnreg from warpgroup 2 to the softmax groups.
 // Tensor memory (512 columns x 128 lanes, fp32):
-//   [0,128) S0   [128,256) S1   [256,256+d) O0   [384,384+d) O1
-//   P_w (the weights, packed 2 x 16-bit or 4 x e4m3 per column) overwrites
-//   the upper half of S_w once the softmax group has read S_w.
-// MMA issue order per K/V tile i: S0=Q0 K_i^T, O1+=P1(i-1) V_(i-1),
-// S1=Q1 K_i^T, O0+=P0(i) V_i -- while one softmax group works, the tensor
-// pipe always has the other group's products queued.  tcgen05 MMAs from one
-// thread execute in issue order, so an S_w write queued after the P_w read
-// of the previous tile cannot overtake it, and the commit that signals S_w(i)
-// also covers O_w += P_w(i-1) V_(i-1): when a softmax group sees S_w(i) its
-// O_w is quiescent and may be rescaled in place.
+//   [0,128) S_a  [128,256) S_b  [256,256+d) O_0  [384,384+d) O_1
+// S is double-buffered: S(i) lives in S_(i&1), and Q K_(i+2)^T is issued as
+// soon as O += P(i) V_i has been issued, so the scores of the next tile are
+// ready when the softmax finishes the current one and the tensor pipe works
+// while the softmax does.  Each softmax group keeps its own running max m_h,
+// sum l_h and output O_h over its half of the keys; the halves never
+// exchange data inside the loop and are merged once at the end:
+//   O = (2^(m_0-m) O_0 + 2^(m_1-m) O_1) / (2^(m_0-m) l_0 + 2^(m_1-m) l_1),
+//   m = max(m_0, m_1),  LSE = (m + log2(2^(m_0-m) l_0 + 2^(m_1-m) l_1)) ln 2.
+// P_h(i) (the weights, packed 2 x 16-bit or 4 x e4m3 per column) overwrites
+// group h's own columns of S_(i&1) once the group has read them.
+// tcgen05 MMAs from one thread execute in issue order, so the S write of
+// Q K_(i+2)^T queued after the P(i) reads cannot overtake them.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -42,31 +43,28 @@
 // Pairs e (0..15) of a 32-column chunk whose exponentials go to the FMA pipe:
 // bit (e & 7) of this mask.
 #ifndef SDPA_POLY_MASK
-#define SDPA_POLY_MASK 0x88
+#define SDPA_POLY_MASK 0x00
 #endif
-// 1: the softmax signals each P tile once; 2: once per half of the keys.
-#ifndef SDPA_P_SPLIT
-#define SDPA_P_SPLIT 2
-#endif
-// K/V ring depth for d = 128 (16-bit) and d = 64.
+// K/V ring depth for 16-bit d = 128, 16-bit d = 64 and e4m3 d = 128.
 #ifndef SDPA_STAGES_D128
-#define SDPA_STAGES_D128 4
+#define SDPA_STAGES_D128 6
 #endif
 #ifndef SDPA_STAGES_D64
 #define SDPA_STAGES_D64 8
+#endif
+#ifndef SDPA_STAGES_FP8
+#define SDPA_STAGES_FP8 10
 #endif
 
 namespace sdpa {
 
 enum Kind { KIND_BF16 = 0, KIND_FP16 = 1, KIND_E4M3 = 2 };
 
-constexpr int kBlockM = 128;        // query rows per tile (= TMEM lanes)
+constexpr int kBlockM = 128;        // query rows per CTA (= TMEM lanes)
 constexpr int kBlockN = 128;        // keys per K/V tile
-constexpr int kQTiles = 2;          // query tiles per CTA
-constexpr int kThreads = 384;       // 3 warpgroups
-constexpr int kSoftmaxRegs = 208;   // per thread after setmaxnreg, warpgroups 0-1
-constexpr int kOtherRegs = 88;      // warpgroup 2 (TMA, MMA, two idle warps)
-constexpr int kLaunchRegs = 168;    // registers per thread at launch (384 threads, 1 CTA/SM)
+constexpr int kHalfN = 64;          // keys per softmax group
+constexpr int kThreads = 320;       // 10 warps
+constexpr int kLaunchRegs = 168;    // registers per thread (10 warps: 3 on some sub-partitions)
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
@@ -82,7 +80,8 @@ struct FwdParams {
     float* lse;         // [B,Hq,Sq] or null
     int B, Hq, Hkv, Sq, Sk;
     int group;          // Hq / Hkv
-    int n_qblocks;      // ceil(Sq / 256)
+    int n_qtiles;       // ceil(Sq / 128)
+    int group_heads;    // (batch, head) pairs per CTA group
     int causal;
     float score_log2;   // multiplier from raw MMA score to log2 units
     float out_mul;      // multiplier on (sum_j p_j v_j) / l: the V descale for FP8, else 1
@@ -98,35 +97,41 @@ struct FwdCfg {
     static constexpr int kTileBytes = 128 * kRowBytes;
     static constexpr int kQkSteps = kRowBytes / 32;      // every MMA consumes 32 bytes of K
     static constexpr int kPvKeysPerStep = 32 / kElem;
-    static constexpr int kPvSteps = kBlockN / kPvKeysPerStep;
-    static constexpr int kPCols = kBlockN * kElem / 4;   // TMEM columns of one P row
+    static constexpr int kPvStepsHalf = kHalfN / kPvKeysPerStep;
+    static constexpr int kPWordsPer32 = 32 * kElem / 4;  // TMEM columns of P per 32 keys
     static constexpr float kRescaleThreshold = (KIND == KIND_E4M3) ? 0.0f : 8.0f;
     // log2 of the factor applied to p before it is rounded for the PV MMA:
     // 448 (the e4m3 maximum) for FP8, so that p in (0, 1] fills the format
     static constexpr float kPLog2 = (KIND == KIND_E4M3) ? 8.807354922057604f : 0.0f;
     // shared memory map (offsets from a 1024-byte aligned base)
     static constexpr int kSmemQ = 0;
-    static constexpr int kSmemKV = kQTiles * kTileBytes;
+    static constexpr int kSmemKV = kTileBytes;
     static constexpr int kSmemBar = kSmemKV + NS * kTileBytes;
-    // barriers: q_full[2] kv_full[NS] kv_empty[NS] s_full[2] p_full[2 tiles][2 halves]
-    //           o_full[2] drain[1]
+    // barriers: q_full, kv_full[NS], kv_empty[NS], s_full[2], p_full[2 buffers][2 groups],
+    //           o_done[2 groups] (once per tile), o_full (once per CTA), xchg, drain
     static constexpr int kBarQFull = 0;
-    static constexpr int kBarKVFull = 2;
-    static constexpr int kBarKVEmpty = 2 + NS;
-    static constexpr int kBarSFull = 2 + 2 * NS;
-    static constexpr int kBarPFull = 4 + 2 * NS;
-    static constexpr int kBarOFull = 8 + 2 * NS;
-    static constexpr int kBarDrain = 10 + 2 * NS;
-    static constexpr int kNumBars = 11 + 2 * NS;
+    static constexpr int kBarKVFull = 1;
+    static constexpr int kBarKVEmpty = 1 + NS;
+    static constexpr int kBarSFull = 1 + 2 * NS;
+    static constexpr int kBarPFull = 3 + 2 * NS;
+    static constexpr int kBarODone = 7 + 2 * NS;
+    static constexpr int kBarOFull = 9 + 2 * NS;
+    static constexpr int kBarXchg = 10 + 2 * NS;
+    static constexpr int kBarDrain = 11 + 2 * NS;
+    static constexpr int kNumBars = 12 + 2 * NS;
     static constexpr int kSmemTmemSlot = kSmemBar + 8 * kNumBars;
     static constexpr int kSmemAbort = kSmemTmemSlot + 4;
+    // the epilogue exchanges [2 groups][m, l][128] fp32 through the Q tile
+    // (every QK MMA has completed by then)
+    static constexpr int kSmemStats = kSmemQ;
     static constexpr int kSmemUsed = kSmemAbort + 4;
+    static_assert(2 * 2 * 128 * 4 <= kTileBytes, "stats fit in the Q tile");
     static constexpr int kSmemBytes = kSmemUsed + 1024;  // slack for the 1024-byte alignment
     // TMEM columns
     static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
-    static constexpr uint32_t kPOffset = 64;
     static_assert(kRowBytes % 128 == 0, "rows must fill whole 128-byte swizzle rows");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
+    static_assert(kSmemBytes > 116 * 1024, "one CTA per SM (each allocates all of TMEM)");
     static_assert(D <= 128, "O tile must fit its 128 TMEM columns");
 };
 
@@ -174,11 +179,46 @@ __device__ __forceinline__ constexpr bool poly_pair(int e) {
     return ((SDPA_POLY_MASK >> (e & 7)) & 1) != 0;
 }
 
-// Row-tile key counts of one CTA: number of K/V tiles query tile w needs.
+// Maximum of 32 consecutive registers (3-input max, two chains).
+__device__ __forceinline__ float chunk_max32(const float* s) {
+    float a = s[0], b = s[1];
+#pragma unroll
+    for (int c = 2; c + 4 <= 30; c += 4) {
+        a = fmax3(a, s[c], s[c + 1]);
+        b = fmax3(b, s[c + 2], s[c + 3]);
+    }
+    a = fmax3(a, s[30], s[31]);
+    return fmaxf(a, b);
+}
+
+// Number of K/V tiles the query rows [row0, row0 + 128) need.
 __device__ __forceinline__ int tiles_for(int row0, int Sq, int Sk, int causal) {
     if (row0 >= Sq) return 0;
     const int kend = causal ? min(Sk, row0 + kBlockM) : Sk;
     return (kend + kBlockN - 1) / kBlockN;
+}
+
+// The t-th K/V tile the MMA warp consumes (and the producer loads):
+// K_0, K_1, V_0, K_2, V_1, K_3, ..., V_(n-3), K_(n-1), V_(n-2), V_(n-1).
+__device__ __forceinline__ void kv_item(int t, int n, bool& is_v, int& tile) {
+    if (n == 1) {
+        is_v = (t == 1);
+        tile = 0;
+        return;
+    }
+    if (t < 2) {
+        is_v = false;
+        tile = t;
+        return;
+    }
+    const int r = t - 2;
+    if (r < 2 * (n - 2)) {
+        is_v = (r & 1) == 0;
+        tile = is_v ? (r >> 1) : (r >> 1) + 2;
+    } else {
+        is_v = true;
+        tile = (n - 2) + (r - 2 * (n - 2));
+    }
 }
 
 template <int D, int KIND, int NS>
@@ -191,38 +231,46 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
+    float* const stats = reinterpret_cast<float*>(smem_raw + (sbase - raw) + C::kSmemStats);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // ---- work unit: longest (last) query blocks first --------------------
+    // ---- work unit ------------------------------------------------------
+    // CTAs come in groups of p.group_heads (batch, head) pairs, every query
+    // tile of a group before the next group, so the K/V a group reads stay in
+    // L2; inside a group the longest (last, for causal) query tiles go first.
     const int n_bh = p.B * p.Hq;
-    const int qblk = p.n_qblocks - 1 - (int)(blockIdx.x / (unsigned)n_bh);
-    const int bh = (int)(blockIdx.x % (unsigned)n_bh);
+    const int per_group = p.group_heads * p.n_qtiles;
+    const int grp = (int)(blockIdx.x / (unsigned)per_group);
+    const int within = (int)blockIdx.x - grp * per_group;
+    const int gsize = min(p.group_heads, n_bh - grp * p.group_heads);
+    const int qtile = p.n_qtiles - 1 - within / gsize;
+    const int bh = grp * p.group_heads + within % gsize;
     const int b = bh / p.Hq;
     const int hq = bh - b * p.Hq;
     const int kvh = b * p.Hkv + hq / p.group;
-    const int m0 = qblk * (kQTiles * kBlockM);
-    const int nt0 = tiles_for(m0, p.Sq, p.Sk, p.causal);
-    const int nt1 = tiles_for(m0 + kBlockM, p.Sq, p.Sk, p.causal);
-    const int n = max(nt0, nt1);
+    const int m0 = qtile * kBlockM;
+    const int n = tiles_for(m0, p.Sq, p.Sk, p.causal);   // >= 1
 
     auto bar = [&](int i) -> uint32_t { return sbase + C::kSmemBar + 8u * (uint32_t)i; };
     const uint32_t abort_addr = sbase + C::kSmemAbort;
     const uint32_t slot_addr = sbase + C::kSmemTmemSlot;
 
     if (threadIdx.x == 0) {
-        for (int w = 0; w < kQTiles; ++w) {
-            mbar_init(bar(C::kBarQFull + w), 1);
-            mbar_init(bar(C::kBarSFull + w), 1);
-            mbar_init(bar(C::kBarPFull + 2 * w), kBlockM);
-            mbar_init(bar(C::kBarPFull + 2 * w + 1), kBlockM);
-            mbar_init(bar(C::kBarOFull + w), 1);
-        }
+        mbar_init(bar(C::kBarQFull), 1);
         for (int s = 0; s < NS; ++s) {
             mbar_init(bar(C::kBarKVFull + s), 1);
             mbar_init(bar(C::kBarKVEmpty + s), 1);
         }
+        for (int j = 0; j < 2; ++j) {
+            mbar_init(bar(C::kBarSFull + j), 1);
+            mbar_init(bar(C::kBarODone + j), 1);
+            mbar_init(bar(C::kBarPFull + 2 * j), kBlockM);
+            mbar_init(bar(C::kBarPFull + 2 * j + 1), kBlockM);
+        }
+        mbar_init(bar(C::kBarOFull), 1);
+        mbar_init(bar(C::kBarXchg), 2 * kBlockM);
         mbar_init(bar(C::kBarDrain), 1);
         st_shared_u32(abort_addr, 0u);
         fence_barrier_init();
@@ -240,38 +288,32 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ld_shared_u32(slot_addr);
-    // launch: 384 x 168 registers; split: 256 x 208 + 128 x 88 = 64512 <= 64512 (the host
-    // checks the compiled register count before the first launch)
-    static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * kLaunchRegs, "register split");
-
     const uint32_t sQ = sbase + C::kSmemQ;
     const uint32_t sKV = sbase + C::kSmemKV;
 
-    if (warp >= 8) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
     if (warp == kLoadWarp) {
         // ================= TMA producer =================================
         if (lane == 0) {
             bool ok = true;
-            for (int w = 0; w < kQTiles; ++w) {
-                if ((w ? nt1 : nt0) == 0) continue;
-                const uint32_t qb = bar(C::kBarQFull + w);
-                mbar_arrive_expect_tx(qb, C::kTileBytes);
-                for (int kb = 0; kb < C::kSwBlocks; ++kb)
-                    tma_load_3d(sQ + w * C::kTileBytes + kb * C::kSwBlockBytes, &tmQ, qb,
-                                kb * C::kElemsPerSw, m0 + w * kBlockM, bh);
-            }
+            mbar_arrive_expect_tx(bar(C::kBarQFull), C::kTileBytes);
+            for (int kb = 0; kb < C::kSwBlocks; ++kb)
+                tma_load_3d(sQ + kb * C::kSwBlockBytes, &tmQ, bar(C::kBarQFull),
+                            kb * C::kElemsPerSw, m0, bh);
             int t = 0;
             for (; t < 2 * n && ok; ++t) {
                 const int slot = t % NS;
                 const uint32_t par = ((uint32_t)(t / NS) & 1u) ^ 1u;
                 ok = wait_bar(bar(C::kBarKVEmpty + slot), par, abort_addr, 0x10000u | (uint32_t)t);
                 if (!ok) break;
+                bool is_v;
+                int tile;
+                kv_item(t, n, is_v, tile);
                 const uint32_t fb = bar(C::kBarKVFull + slot);
                 mbar_arrive_expect_tx(fb, C::kTileBytes);
-                const CUtensorMap* m = (t & 1) ? &tmV : &tmK;
+                const CUtensorMap* m = is_v ? &tmV : &tmK;
                 for (int kb = 0; kb < C::kSwBlocks; ++kb)
                     tma_load_3d(sKV + slot * C::kTileBytes + kb * C::kSwBlockBytes, m, fb,
-                                kb * C::kElemsPerSw, (t >> 1) * kBlockN, kvh);
+                                kb * C::kElemsPerSw, tile * kBlockN, kvh);
             }
             if (!ok) {
                 // let the copies already issued land before the CTA exits
@@ -285,17 +327,17 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
     } else if (warp == kMmaWarp) {
         // ================= MMA issuer ===================================
-        // The whole warp runs the loop (so descriptors and addresses stay
-        // warp-uniform); one elected lane issues the MMAs and commits.
+        // The whole warp runs the loop (descriptors stay warp-uniform); one
+        // elected lane issues the MMAs and commits.
         const bool leader = elect_one();
         constexpr uint32_t fmt = (KIND == KIND_BF16) ? 1u : 0u;
         constexpr uint32_t idesc_qk = make_idesc(fmt, false, kBlockM, kBlockN);
         constexpr uint32_t idesc_pv = make_idesc(fmt, true, kBlockM, D);
-        const uint64_t desc_q0 = make_smem_desc(sQ, 16, 1024);
-        const uint64_t desc_q1 = make_smem_desc(sQ + C::kTileBytes, 16, 1024);
+        const uint64_t desc_q = make_smem_desc(sQ, 16, 1024);
         const uint64_t desc_k = make_smem_desc(sKV, 16, 1024);
         const uint64_t desc_v = make_smem_desc(sKV, C::kSwBlockBytes, 1024);
         bool ok = true;
+        int t = 0;   // K/V tiles consumed
 
         auto wait_all = [&](uint32_t b_, uint32_t par, uint32_t where) {
             const bool r_ = wait_bar(b_, par, abort_addr, where);
@@ -305,31 +347,31 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             if (leader) mma_commit(b_);
             __syncwarp();
         };
-        auto issue_qk = [&](int w, int slot) {
-            const uint32_t d_tmem = tmem + (w ? C::kColS1 : C::kColS0);
-            const uint64_t dq = w ? desc_q1 : desc_q0;
+        // S_buf = Q K^T for the K tile in `slot`
+        auto issue_qk = [&](int buf, int slot) {
+            const uint32_t d_tmem = tmem + (buf ? C::kColS1 : C::kColS0);
             const uint64_t dk = desc_k + (uint64_t)((slot * C::kTileBytes) >> 4);
             if (leader) {
 #pragma unroll
                 for (int kk = 0; kk < C::kQkSteps; ++kk) {
                     const uint64_t off = (uint64_t)(((kk >> 2) * C::kSwBlockBytes + (kk & 3) * 32) >> 4);
                     if constexpr (KIND == KIND_E4M3)
-                        mma_f8_ss(d_tmem, dq + off, dk + off, idesc_qk, kk > 0);
+                        mma_f8_ss(d_tmem, desc_q + off, dk + off, idesc_qk, kk > 0);
                     else
-                        mma_f16_ss(d_tmem, dq + off, dk + off, idesc_qk, kk > 0);
+                        mma_f16_ss(d_tmem, desc_q + off, dk + off, idesc_qk, kk > 0);
                 }
             }
             __syncwarp();
         };
-        // O_w (+)= P_w V over the keys of one half of the tile (K steps
-        // [h * kPvSteps / 2, (h + 1) * kPvSteps / 2)); P is read from TMEM.
-        auto issue_pv_half = [&](int w, int slot, bool acc, int h) {
-            const uint32_t d_tmem = tmem + (w ? C::kColO1 : C::kColO0);
-            const uint32_t a_tmem = tmem + (w ? C::kColS1 : C::kColS0) + C::kPOffset;
-            const uint64_t dv = desc_v + (uint64_t)((slot * C::kTileBytes) >> 4);
+        // O_h (+)= P_h V[keys of half h]; P_h is in TMEM over group h's
+        // columns of S_buf
+        auto issue_pv = [&](int h, int buf, int slot, bool acc) {
+            const uint32_t d_tmem = tmem + (h ? C::kColO1 : C::kColO0);
+            const uint32_t a_tmem = tmem + (buf ? C::kColS1 : C::kColS0) + h * kHalfN;
+            const uint64_t dv = desc_v + (uint64_t)((slot * C::kTileBytes + h * kHalfN * 128) >> 4);
             if (leader) {
 #pragma unroll
-                for (int kk = h * C::kPvSteps / 2; kk < (h + 1) * C::kPvSteps / 2; ++kk) {
+                for (int kk = 0; kk < C::kPvStepsHalf; ++kk) {
                     const uint64_t off = (uint64_t)((kk * C::kPvKeysPerStep * 128) >> 4);
                     const uint32_t accum = (acc || kk > 0) ? 1u : 0u;
                     if constexpr (KIND == KIND_E4M3)
@@ -340,59 +382,44 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             }
             __syncwarp();
         };
-        // wait for each half of P_w(j) and issue its MMAs
-        auto pv = [&](int w, int slot, int j) -> bool {
-            for (int h = 0; h < SDPA_P_SPLIT; ++h) {
-                if (!wait_all(bar(C::kBarPFull + 2 * w + h), (uint32_t)j & 1u,
-                              0x22000u | (w << 11) | (h << 10) | (uint32_t)j))
-                    return false;
-                tc_fence_after();
-                if (SDPA_P_SPLIT == 1) {
-                    issue_pv_half(w, slot, j > 0, 0);
-                    issue_pv_half(w, slot, j > 0, 1);
-                } else {
-                    issue_pv_half(w, slot, j > 0, h);
-                }
-            }
-            return true;
+        auto next_kv = [&](uint32_t where) -> int {
+            const int slot = t % NS;
+            ok = wait_all(bar(C::kBarKVFull + slot), (uint32_t)(t / NS) & 1u, where | (uint32_t)t);
+            return slot;
         };
 
-        if (nt0 > 0) ok = wait_all(bar(C::kBarQFull + 0), 0, 0x20000u);
-        if (ok && nt1 > 0) ok = wait_all(bar(C::kBarQFull + 1), 0, 0x20001u);
-
-        for (int i = 0; i <= n && ok; ++i) {
-            const int tK = 2 * i, tV = 2 * i + 1;
-            const int slotK = tK % NS, slotV = tV % NS;
-            if (i < n) {
-                ok = wait_all(bar(C::kBarKVFull + slotK), (uint32_t)(tK / NS) & 1u, 0x21000u | (uint32_t)i);
+        ok = wait_all(bar(C::kBarQFull), 0, 0x20000u);
+        for (int j = 0; j < min(n, 2) && ok; ++j) {
+            const int slot = next_kv(0x21000u);
+            if (!ok) break;
+            issue_qk(j, slot);
+            commit(bar(C::kBarSFull + j));
+            commit(bar(C::kBarKVEmpty + slot));
+            ++t;
+        }
+        for (int i = 0; i < n && ok; ++i) {
+            const int buf = i & 1;
+            const int slotV = next_kv(0x22000u);
+            if (!ok) break;
+            for (int h = 0; h < 2 && ok; ++h) {
+                ok = wait_all(bar(C::kBarPFull + 2 * buf + h), (uint32_t)(i >> 1) & 1u,
+                              0x23000u | (h << 11) | (uint32_t)i);
                 if (!ok) break;
-                if (i < nt0) {
-                    issue_qk(0, slotK);
-                    commit(bar(C::kBarSFull + 0));
-                }
+                tc_fence_after();
+                issue_pv(h, buf, slotV, i > 0);
+                commit(bar(C::kBarODone + h));
             }
-            if (i >= 1) {
-                const int j = i - 1;
-                if (j < nt1) {
-                    ok = pv(1, (2 * j + 1) % NS, j);
-                    if (!ok) break;
-                    if (j == nt1 - 1) commit(bar(C::kBarOFull + 1));
-                }
-                commit(bar(C::kBarKVEmpty + (2 * j + 1) % NS));   // V_(i-1) free
-            }
-            if (i < n) {
-                if (i < nt1) {
-                    issue_qk(1, slotK);
-                    commit(bar(C::kBarSFull + 1));
-                }
-                commit(bar(C::kBarKVEmpty + slotK));               // K_i free
-                ok = wait_all(bar(C::kBarKVFull + slotV), (uint32_t)(tV / NS) & 1u, 0x23000u | (uint32_t)i);
+            if (!ok) break;
+            if (i == n - 1) commit(bar(C::kBarOFull));
+            commit(bar(C::kBarKVEmpty + slotV));
+            ++t;
+            if (i + 2 < n) {
+                const int slotK = next_kv(0x24000u);
                 if (!ok) break;
-                if (i < nt0) {
-                    ok = pv(0, slotV, i);
-                    if (!ok) break;
-                    if (i == nt0 - 1) commit(bar(C::kBarOFull + 0));
-                }
+                issue_qk(buf, slotK);
+                commit(bar(C::kBarSFull + buf));
+                commit(bar(C::kBarKVEmpty + slotK));
+                ++t;
             }
         }
         if (!ok) {
@@ -409,175 +436,192 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         tmem_dealloc(tmem, kTmemCols);
     } else if (warp < 8) {
         // ================= softmax groups (warps 0-7) ====================
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
-        const int w = warp >> 2;                 // query tile
+        const int h = warp >> 2;                 // key half of every tile
         const int quarter = warp & 3;            // TMEM lane quarter of this warp
         const int r = (int)(threadIdx.x & 127);  // row within the tile
-        const int row = m0 + w * kBlockM + r;
-        const int nw = w ? nt1 : nt0;
+        const int row = m0 + r;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-        const uint32_t tS = tmem + lane_base + (w ? C::kColS1 : C::kColS0);
-        const uint32_t tP = tS + C::kPOffset;
-        const uint32_t tO = tmem + lane_base + (w ? C::kColO1 : C::kColO0);
+        const uint32_t tO = tmem + lane_base + (h ? C::kColO1 : C::kColO0);
         const float sl = p.score_log2;
         const uint64_t sl2 = f2_pack(sl, sl);
-        float m_run = -INFINITY;   // running max of the scaled scores (log2 units)
+        float m_run = -INFINITY;   // running max of this half's scaled scores (log2 units)
         float l_run = 0.0f;        // running sum of 2^(s*sl - m_run + kPLog2)
         bool ok = true;
 
-        for (int i = 0; i < nw; ++i) {
-            ok = wait_bar(bar(C::kBarSFull + w), (uint32_t)i & 1u, abort_addr, 0x30000u | (w << 12) | i);
+        // -m [+ log2 of the P scale] as a pair; a row whose keys of this half
+        // have all been masked so far keeps m = -inf and gets p = 0
+        auto neg_m_of = [&](float m) -> uint64_t {
+            const float nm = (m == -INFINITY) ? 0.0f : C::kPLog2 - m;
+            return f2_pack(nm, nm);
+        };
+        // Weights p = 2^(s*sl + nm) of 32 scores: pairs on the MUFU, or on the
+        // FMA pipe for the pairs SDPA_POLY_MASK selects; P rounded for the PV
+        // product and stored into chunk c of this group's columns of S.
+        // Returns the fp32 sum of the weights as a pair.
+        auto exp_chunk = [&](const float* sc, uint64_t sl2_, uint64_t nm2, uint32_t tS_,
+                             int c) -> uint64_t {
+            uint64_t sum2[2] = {0ull, 0ull};
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const uint64_t x2 = f2_fma(f2_pack(sc[2 * e], sc[2 * e + 1]), sl2_, nm2);
+                float x0, x1;
+                f2_unpack(x2, x0, x1);
+                uint64_t p2;
+                if (poly_pair(e)) {
+                    p2 = exp2_poly_x2(f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f)));
+                } else {
+                    p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+                }
+                sum2[e & 1] = f2_add(sum2[e & 1], p2);
+                float q0, q1;
+                f2_unpack(p2, q0, q1);
+                if constexpr (KIND == KIND_E4M3) {
+                    if (e & 1) pk[e >> 1] |= pack_e4m3x4(0.f, 0.f, q0, q1) & 0xFFFF0000u;
+                    else pk[e >> 1] = pack_e4m3x4(q0, q1, 0.f, 0.f) & 0x0000FFFFu;
+                } else {
+                    pk[e] = (KIND == KIND_BF16) ? pack_bf16x2(q0, q1) : pack_f16x2(q0, q1);
+                }
+            }
+            if constexpr (KIND == KIND_E4M3)
+                tmem_st8(tS_ + C::kPWordsPer32 * c, pk);
+            else
+                tmem_st16(tS_ + C::kPWordsPer32 * c, pk);
+            return f2_add(sum2[0], sum2[1]);
+        };
+
+        for (int i = 0; i < n; ++i) {
+            const int buf = i & 1;
+            ok = wait_bar(bar(C::kBarSFull + buf), (uint32_t)(i >> 1) & 1u, abort_addr,
+                          0x30000u | (h << 12) | i);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
+            const uint32_t tS = tmem + lane_base + (buf ? C::kColS1 : C::kColS0) + h * kHalfN;
 
-            // S row in two halves: the second half's load overlaps the first
-            // half's masking and max
-            float s[kBlockN];
+            float s[kHalfN];
+            // chunk 0 (keys 0-31 of this half); chunk 1 is loaded while the
+            // exponentials of chunk 0 run
             tmem_ld32(tS + 0, *reinterpret_cast<float(*)[32]>(&s[0]));
-            tmem_ld32(tS + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
             tmem_wait_ld();
             reg_fence32(&s[0]);
-            reg_fence32(&s[32]);
-            tmem_ld32(tS + 64, *reinterpret_cast<float(*)[32]>(&s[64]));
-            tmem_ld32(tS + 96, *reinterpret_cast<float(*)[32]>(&s[96]));
+            tmem_ld32(tS + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
 
             // mask: keys past Sk, and (causal) keys after the row
-            const int key0 = i * kBlockN;
-            const bool edge = (key0 + kBlockN > p.Sk) ||
-                              (p.causal && key0 + kBlockN - 1 > m0 + w * kBlockM);
-            int lim = p.Sk - key0;
-            if (p.causal) lim = min(lim, row - key0 + 1);
+            const int key0 = i * kBlockN + h * kHalfN;
+            const bool edge = (key0 + kHalfN > p.Sk) || (p.causal && key0 + kHalfN - 1 > m0);
+            int lim = kHalfN;
             if (edge) {
+                lim = p.Sk - key0;
+                if (p.causal) lim = min(lim, row - key0 + 1);
 #pragma unroll
-                for (int c = 0; c < kBlockN / 2; ++c)
+                for (int c = 0; c < 32; ++c)
                     if (c >= lim) s[c] = -INFINITY;
             }
-            // first half only: columns 0..63 (64..127 are still in flight)
-            float mx0 = s[0], mx1 = s[1];
-#pragma unroll
-            for (int c = 2; c + 4 <= kBlockN / 2 - 2; c += 4) {
-                mx0 = fmax3(mx0, s[c], s[c + 1]);
-                mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
-            }
-            mx0 = fmax3(mx0, s[kBlockN / 2 - 2], s[kBlockN / 2 - 1]);
+            const float cmax0 = chunk_max32(&s[0]) * sl;
+
+            // Fast path: while a chunk's maximum stays within the rescale
+            // threshold of the running max m_run, its weights are computed
+            // against m_run at once.  Otherwise (always on the first tile)
+            // the tile takes the full path: maximum of both chunks, new m_run,
+            // l and O rescaled, chunk 0 recomputed.
+            const bool fast0 = !__any_sync(0xffffffffu, cmax0 > m_run + C::kRescaleThreshold);
+            uint64_t sum0 = 0ull, sum1 = 0ull;
+            if (fast0) sum0 = exp_chunk(&s[0], sl2, neg_m_of(m_run), tS, 0);
+
             tmem_wait_ld();
-            reg_fence32(&s[64]);
-            reg_fence32(&s[96]);
+            reg_fence32(&s[32]);
             if (edge) {
 #pragma unroll
-                for (int c = kBlockN / 2; c < kBlockN; ++c)
+                for (int c = 32; c < kHalfN; ++c)
                     if (c >= lim) s[c] = -INFINITY;
             }
-#pragma unroll
-            for (int c = kBlockN / 2; c < kBlockN; c += 4) {
-                mx0 = fmax3(mx0, s[c], s[c + 1]);
-                mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
-            }
-            const float tile_max = fmaxf(mx0, mx1) * sl;
-
-            // The running max only moves when the new one exceeds it by more
-            // than the threshold; weights computed against a stale max are
-            // bounded by 2^threshold and the final O / l and LSE are exact
-            // for any reference value as long as O and l share it.
-            float alpha = 1.0f;
-            if (tile_max > m_run + C::kRescaleThreshold) {
-                alpha = ex2_approx(m_run - tile_max);   // 0 on the first tile
-                m_run = tile_max;
-            }
-            l_run *= alpha;
-            // O_w (quiescent: its last update is covered by the S_w(i) commit)
-            // takes the same factor as l before any of P_w(i) V_i is added.
-            if (i > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+            const float cmax1 = chunk_max32(&s[32]) * sl;
+            if (!fast0 || __any_sync(0xffffffffu, cmax1 > m_run + C::kRescaleThreshold)) {
+                const float tile_max = fmaxf(cmax0, cmax1);
+                float alpha = 1.0f;
+                if (tile_max > m_run + C::kRescaleThreshold) {
+                    alpha = ex2_approx(m_run - tile_max);   // 0 on the first live tile
+                    m_run = tile_max;
+                }
+                l_run *= alpha;
+                // O_h takes the same factor before P_h(i) V_i is added; its
+                // last update, O_h += P_h(i-1) V_(i-1), must have completed.
+                // o_done[h] completes once per tile; this parity wait is exact
+                // because the barrier is within one phase of tile i-1: the
+                // S(i) commit covered tile i-2's product and tile i's cannot
+                // exist yet.
+                if (i > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+                    ok = wait_bar(bar(C::kBarODone + h), (uint32_t)(i - 1) & 1u, abort_addr,
+                                  0x31000u | (h << 12) | i);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                    tc_fence_after();
 #pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    float o[32];
-                    tmem_ld32(tO + 32 * c, o);
-                    tmem_wait_ld();
-                    reg_fence32(o);
+                    for (int c = 0; c < D / 32; ++c) {
+                        float o[32];
+                        tmem_ld32(tO + 32 * c, o);
+                        tmem_wait_ld();
+                        reg_fence32(o);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] *= alpha;
-                    tmem_st32(tO + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(o));
+                        for (int e = 0; e < 32; ++e) o[e] *= alpha;
+                        tmem_st32(tO + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(o));
+                    }
                 }
+                sum0 = exp_chunk(&s[0], sl2, neg_m_of(m_run), tS, 0);
             }
-
-            // weights p = 2^(s*sl - m [+ log2 of the P scale]): most pairs on
-            // the MUFU, kPolyPairs in every 8 on the FMA pipe
-            // (exp2_poly_x2); row sums from the fp32 values, P rounded for the
-            // PV product and stored to TMEM one half of the keys at a time so
-            // the MMA warp can start on the first half.
-            const float neg_m = C::kPLog2 - m_run;
-            const uint64_t nm2 = f2_pack(neg_m, neg_m);
-            uint64_t sum2[2] = {0ull, 0ull};
-#pragma unroll
-            for (int c = 0; c < kBlockN / 32; ++c) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const uint64_t x2 = f2_fma(f2_pack(s[32 * c + 2 * e], s[32 * c + 2 * e + 1]), sl2, nm2);
-                    float x0, x1;
-                    f2_unpack(x2, x0, x1);
-                    uint64_t p2;
-                    if (poly_pair(e)) {
-                        p2 = exp2_poly_x2(f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f)));
-                    } else {
-                        p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
-                    }
-                    sum2[e & 1] = f2_add(sum2[e & 1], p2);
-                    float q0, q1;
-                    f2_unpack(p2, q0, q1);
-                    if constexpr (KIND == KIND_E4M3) {
-                        if (e & 1) pk[e >> 1] |= pack_e4m3x4(0.f, 0.f, q0, q1) & 0xFFFF0000u;
-                        else pk[e >> 1] = pack_e4m3x4(q0, q1, 0.f, 0.f) & 0x0000FFFFu;
-                    } else {
-                        pk[e] = (KIND == KIND_BF16) ? pack_bf16x2(q0, q1) : pack_f16x2(q0, q1);
-                    }
-                }
-                // first half of the keys: its stores were issued one chunk ago,
-                // so this wait finds them done
-                if (SDPA_P_SPLIT == 2 && c == 2) {
-                    tmem_wait_st();
-                    tc_fence_before();
-                    mbar_arrive(bar(C::kBarPFull + 2 * w));
-                }
-                if constexpr (KIND == KIND_E4M3)
-                    tmem_st8(tP + 8 * c, pk);
-                else
-                    tmem_st16(tP + 16 * c, pk);
+            sum1 = exp_chunk(&s[32], sl2, neg_m_of(m_run), tS, 1);
+            {
+                float a0, a1, b0, b1;
+                f2_unpack(sum0, a0, a1);
+                f2_unpack(sum1, b0, b1);
+                l_run += (a0 + a1) + (b0 + b1);
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(C::kBarPFull + 2 * w + (SDPA_P_SPLIT - 1)));
-            {
-                float a0, a1, b0, b1;
-                f2_unpack(sum2[0], a0, a1);
-                f2_unpack(sum2[1], b0, b1);
-                l_run += (a0 + a1) + (b0 + b1);
-            }
+            mbar_arrive(bar(C::kBarPFull + 2 * buf + h));
         }
 
-        // ---- epilogue: O / l -> 16-bit, LSE ---------------------------------
-        if (ok && nw > 0) {
-            ok = wait_bar(bar(C::kBarOFull + w), 0, abort_addr, 0x40000u | w);
+        // ---- epilogue: merge the two halves, O -> 16-bit, LSE --------------
+        // stats[g][0][r] = m_g, stats[g][1][r] = l_g
+        if (ok) {
+            stats[(h * 2 + 0) * 128 + r] = m_run;
+            stats[(h * 2 + 1) * 128 + r] = l_run;
+            mbar_arrive(bar(C::kBarXchg));
+            ok = wait_bar(bar(C::kBarXchg), 0, abort_addr, 0x40000u | h);
+            // o_full completes once per CTA, after the last O_0 and O_1 updates
+            ok = ok && wait_bar(bar(C::kBarOFull), 0, abort_addr, 0x41000u | h);
             ok = __all_sync(0xffffffffu, ok);
         }
-        if (ok && nw > 0) {
+        if (ok) {
             tc_fence_after();
-            const float inv_l = p.out_mul / l_run;
+            const float m_0 = stats[0 * 128 + r], l_0 = stats[1 * 128 + r];
+            const float m_1 = stats[2 * 128 + r], l_1 = stats[3 * 128 + r];
+            const float m = fmaxf(m_0, m_1);
+            const float a0 = (m_0 == -INFINITY) ? 0.0f : ex2_approx(m_0 - m);
+            const float a1 = (m_1 == -INFINITY) ? 0.0f : ex2_approx(m_1 - m);
+            const float l = l_0 * a0 + l_1 * a1;
+            const float c0 = a0 * (p.out_mul / l), c1 = a1 * (p.out_mul / l);
             const bool live = row < p.Sq;
             const size_t orow = ((size_t)bh * p.Sq + (size_t)(live ? row : 0)) * D;
             uint16_t* obase = reinterpret_cast<uint16_t*>(p.o) + orow;
+            const uint32_t tO0 = tmem + lane_base + C::kColO0, tO1 = tmem + lane_base + C::kColO1;
+            // group h writes output columns [h * D / 2, (h + 1) * D / 2)
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                float o[32];
-                tmem_ld32(tO + 32 * c, o);
+            for (int c = h * (D / 64); c < (h + 1) * (D / 64); ++c) {
+                float x[32], y[32];
+                tmem_ld32(tO0 + 32 * c, x);
+                tmem_ld32(tO1 + 32 * c, y);
                 tmem_wait_ld();
-                reg_fence32(o);
+                reg_fence32(x);
+                reg_fence32(y);
                 uint32_t u[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    u[e] = (KIND == KIND_FP16) ? pack_f16x2(o[2 * e] * inv_l, o[2 * e + 1] * inv_l)
-                                               : pack_bf16x2(o[2 * e] * inv_l, o[2 * e + 1] * inv_l);
+                for (int e = 0; e < 16; ++e) {
+                    const float v0 = x[2 * e] * c0 + y[2 * e] * c1;
+                    const float v1 = x[2 * e + 1] * c0 + y[2 * e + 1] * c1;
+                    u[e] = (KIND == KIND_FP16) ? pack_f16x2(v0, v1) : pack_bf16x2(v0, v1);
+                }
                 if (live) {
                     uint4* dst = reinterpret_cast<uint4*>(obase + 32 * c);
 #pragma unroll
@@ -585,13 +629,12 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                         dst[v4] = make_uint4(u[4 * v4], u[4 * v4 + 1], u[4 * v4 + 2], u[4 * v4 + 3]);
                 }
             }
-            if (p.lse != nullptr && live)
-                p.lse[(size_t)bh * p.Sq + row] = (m_run + __log2f(l_run) - C::kPLog2) * kLn2;
+            if (h == 0 && p.lse != nullptr && live)
+                p.lse[(size_t)bh * p.Sq + row] = (m + __log2f(l) - C::kPLog2) * kLn2;
         }
         tc_fence_before();
         named_bar_sync(1, 256 + 32);
     }
-
 }
 
 }  // namespace sdpa
