@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--ref-budget-s", type=float, default=90.0,
+                    help="host seconds the reference (oracle) arm spends over all its steps")
     return ap.parse_args()
 
 
@@ -64,6 +66,32 @@ def load_traffic(workload_name):
         d = json.load(f)
     e = d.get(workload_name)
     return None if e is None else e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# ranks: one process per GPU, each with its own copy of the workload
+# ---------------------------------------------------------------------------
+def rank_barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks_value(x, world, device):
+    """Max of a per-rank scalar over all ranks (the job's time is its slowest
+    rank's); a no-op for one rank."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, flops_per_rank_step, steps, ms_max):
+    """Whole-job TFLOP/s: the work of every rank over the slowest rank's time."""
+    return world * flops_per_rank_step * steps / (ms_max * 1e-3) / 1e12
 
 
 # ---------------------------------------------------------------------------
@@ -164,7 +192,7 @@ def run_reference(args, w):
     q, k, v, ds = cpu_inputs(w)
     t, _ = oracle_rows_tflops(w, q, k, v, 32, 7, nt, ds)
     per_row = t / 32
-    budget = 90.0
+    budget = args.ref_budget_s
     rows_per_step = int(max(1, min(4096, budget / max(1, args.steps + args.warmup) / per_row)))
     for s in range(args.warmup):
         oracle_rows_tflops(w, q, k, v, rows_per_step, 100 + s, nt, ds)
@@ -194,7 +222,7 @@ def run_reference(args, w):
 # ---------------------------------------------------------------------------
 def main():
     args = parse()
-    from sdpa_workloads import WORKLOADS, make_qkv, make_qkv_fp8, sample_rows
+    from sdpa_workloads import WORKLOADS, make_qkv, make_qkv_fp8, sample_rows, with_shape
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
@@ -217,26 +245,20 @@ def main():
 
     import scaled_dot_product_11_b200 as sdpa
     fp8 = w.dtype == "e4m3"
+    # every rank draws its own batch of the same shape (weak scaling)
+    w_rank = with_shape(w, seed=w.seed + 1000 * rank)
     if fp8:
-        q, k, v, ds, _ = make_qkv_fp8(w, dev)
+        q, k, v, ds, _ = make_qkv_fp8(w_rank, dev)
         run = lambda: sdpa.attention_fp8(q, k, v, ds, causal=w.causal, scale=w.scale, out=o, lse=lse)
     else:
-        q, k, v = make_qkv(w, dev)
+        q, k, v = make_qkv(w_rank, dev)
         run = lambda: sdpa.attention(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse)
     o = torch.empty((w.B, w.Hq, w.Sq, w.d), dtype=torch.bfloat16 if fp8 or w.dtype == "bf16"
                     else torch.float16, device=dev)
     lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device=dev)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier = lambda: rank_barrier(world)
+    max_over_ranks = lambda x: max_over_ranks_value(x, world, dev)
 
     # warm-up (also the parity spot check of this exact launch configuration)
     for _ in range(args.warmup):
@@ -279,7 +301,7 @@ def main():
     if st != 0:
         raise SystemExit("device status %d (%#x) after timing" % (st, detail))
     ms_per_step = ms_total / args.steps
-    value = world * w.flops * args.steps / (ms_total * 1e-3) / 1e12
+    value = job_throughput(world, w.flops, args.steps, ms_total)
 
     # end to end through the public API: pinned host inputs -> device -> fused
     # forward -> O and LSE back to pinned host memory, all inside the region
@@ -314,7 +336,7 @@ def main():
         e1.synchronize()
         barrier()
         ms_e2e = max_over_ranks(e0.elapsed_time(e1))
-        e2e_value = world * w.flops * e2e_steps / (ms_e2e * 1e-3) / 1e12
+        e2e_value = job_throughput(world, w.flops, e2e_steps, ms_e2e)
 
     if rank == 0:
         peaks, src = load_peaks()

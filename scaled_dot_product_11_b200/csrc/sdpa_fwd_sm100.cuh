@@ -45,6 +45,10 @@
 #ifndef SDPA_POLY_MASK
 #define SDPA_POLY_MASK 0x00
 #endif
+// 1: the two softmax groups run staggered by part of a tile.
+#ifndef SDPA_STAGGER
+#define SDPA_STAGGER 0
+#endif
 // K/V ring depth for 16-bit d = 128, 16-bit d = 64 and e4m3 d = 128.
 #ifndef SDPA_STAGES_D128
 #define SDPA_STAGES_D128 6
@@ -118,7 +122,8 @@ struct FwdCfg {
     static constexpr int kBarOFull = 9 + 2 * NS;
     static constexpr int kBarXchg = 10 + 2 * NS;
     static constexpr int kBarDrain = 11 + 2 * NS;
-    static constexpr int kNumBars = 12 + 2 * NS;
+    static constexpr int kBarStagger = 12 + 2 * NS;
+    static constexpr int kNumBars = 13 + 2 * NS;
     static constexpr int kSmemTmemSlot = kSmemBar + 8 * kNumBars;
     static constexpr int kSmemAbort = kSmemTmemSlot + 4;
     // the epilogue exchanges [2 groups][m, l][128] fp32 through the Q tile
@@ -271,6 +276,7 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
         mbar_init(bar(C::kBarOFull), 1);
         mbar_init(bar(C::kBarXchg), 2 * kBlockM);
+        mbar_init(bar(C::kBarStagger), kBlockM);
         mbar_init(bar(C::kBarDrain), 1);
         st_shared_u32(abort_addr, 0u);
         fence_barrier_init();
@@ -490,7 +496,16 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             return f2_add(sum2[0], sum2[1]);
         };
 
-        for (int i = 0; i < n; ++i) {
+#if SDPA_STAGGER
+        // Group 1 starts once group 0 has produced the first chunk of its
+        // first tile, so the two groups run half a tile apart: one group's
+        // exponentials overlap the other's score load and maximum.
+        if (h == 1) {
+            ok = wait_bar(bar(C::kBarStagger), 0, abort_addr, 0x32000u);
+            ok = __all_sync(0xffffffffu, ok);
+        }
+#endif
+        for (int i = 0; i < n && ok; ++i) {
             const int buf = i & 1;
             ok = wait_bar(bar(C::kBarSFull + buf), (uint32_t)(i >> 1) & 1u, abort_addr,
                           0x30000u | (h << 12) | i);
@@ -570,6 +585,9 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 }
                 sum0 = exp_chunk(&s[0], sl2, neg_m_of(m_run), tS, 0);
             }
+#if SDPA_STAGGER
+            if (h == 0 && i == 0) mbar_arrive(bar(C::kBarStagger));
+#endif
             sum1 = exp_chunk(&s[32], sl2, neg_m_of(m_run), tS, 1);
             {
                 float a0, a1, b0, b1;
