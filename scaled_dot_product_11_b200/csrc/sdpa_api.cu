@@ -98,9 +98,9 @@ bool encode_3d(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const voi
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int KIND, int NS>
+template <int D, int KIND, int NS, int QB>
 int launch(const void* q, const void* k, const void* v, const FwdParams& prm, cudaStream_t stream) {
-    using C = FwdCfg<D, KIND, NS>;
+    using C = FwdCfg<D, KIND, NS, QB>;
     const CUtensorMapDataType dt = KIND == sdpa::KIND_BF16   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                    : KIND == sdpa::KIND_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                              : CU_TENSOR_MAP_DATA_TYPE_UINT8;
@@ -109,7 +109,7 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& prm, cu
         !encode_3d(&tk, dt, C::kElem, k, D, prm.Sk, (long long)prm.B * prm.Hkv, C::kElemsPerSw) ||
         !encode_3d(&tv, dt, C::kElem, v, D, prm.Sk, (long long)prm.B * prm.Hkv, C::kElemsPerSw))
         return SDPA_ERR_CUDA;
-    auto kern = sdpa::sdpa_fwd_sm100_kernel<D, KIND, NS>;
+    auto kern = sdpa::sdpa_fwd_sm100_kernel<D, KIND, NS, QB>;
     static bool attr_set[64];
     int dev = 0;
     cudaGetDevice(&dev);
@@ -119,7 +119,8 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& prm, cu
             return SDPA_ERR_CUDA;
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
-    const unsigned grid = (unsigned)((long long)prm.n_qtiles * prm.B * prm.Hq);
+    // persistent: one CTA per SM (fewer when there are fewer items)
+    const unsigned grid = (unsigned)(prm.n_items < sm_count() ? prm.n_items : sm_count());
     kern<<<grid, sdpa::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, prm);
     return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
 }
@@ -135,8 +136,11 @@ FwdParams make_params(void* o, float* lse, int B, int Hq, int Hkv, int Sq, int S
     prm.Sk = Sk;
     prm.group = Hq / Hkv;
     prm.n_qtiles = (Sq + 127) / 128;
-    // about two waves of CTAs per group of (batch, head) pairs
-    prm.group_heads = (2 * sm_count() + prm.n_qtiles - 1) / prm.n_qtiles;
+    // schedule items: causal pairs query tiles j and nq-1-j of a head
+    prm.items_per_head = causal ? (prm.n_qtiles + 1) / 2 : prm.n_qtiles;
+    prm.n_items = B * Hq * prm.items_per_head;
+    // about two waves of items per group of (batch, head) pairs
+    prm.group_heads = (2 * sm_count() + prm.items_per_head - 1) / prm.items_per_head;
     if (prm.group_heads < 1) prm.group_heads = 1;
     if (prm.group_heads > B * Hq) prm.group_heads = B * Hq;
     prm.causal = causal;
@@ -159,10 +163,10 @@ extern "C" int sdpa_fwd(const void* q, const void* k, const void* v, void* o, fl
     prm.score_log2 = scale * sdpa::kLog2e;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (dtype == SDPA_BF16)
-        return d == 128 ? launch<128, sdpa::KIND_BF16, SDPA_STAGES_D128>(q, k, v, prm, s)
-                        : launch<64, sdpa::KIND_BF16, SDPA_STAGES_D64>(q, k, v, prm, s);
-    return d == 128 ? launch<128, sdpa::KIND_FP16, SDPA_STAGES_D128>(q, k, v, prm, s)
-                    : launch<64, sdpa::KIND_FP16, SDPA_STAGES_D64>(q, k, v, prm, s);
+        return d == 64 ? launch<64, sdpa::KIND_BF16, SDPA_STAGES_D64, 2>(q, k, v, prm, s)
+                       : launch<128, sdpa::KIND_BF16, SDPA_STAGES_D128, 1>(q, k, v, prm, s);
+    return d == 64 ? launch<64, sdpa::KIND_FP16, SDPA_STAGES_D64, 2>(q, k, v, prm, s)
+                   : launch<128, sdpa::KIND_FP16, SDPA_STAGES_D128, 1>(q, k, v, prm, s);
 }
 
 extern "C" int sdpa_fwd_fp8(const void* q8, const void* k8, const void* v8, float descale_q,
@@ -178,7 +182,8 @@ extern "C" int sdpa_fwd_fp8(const void* q8, const void* k8, const void* v8, floa
     FwdParams prm = make_params(o, lse, B, Hq, Hkv, Sq, Sk, causal);
     prm.score_log2 = scale * descale_q * descale_k * sdpa::kLog2e;
     prm.out_mul = descale_v;
-    return launch<128, sdpa::KIND_E4M3, SDPA_STAGES_FP8>(q8, k8, v8, prm, reinterpret_cast<cudaStream_t>(stream));
+    return launch<128, sdpa::KIND_E4M3, SDPA_STAGES_FP8, 2>(q8, k8, v8, prm,
+                                                            reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" const char* sdpa_strerror(int status) {

@@ -1,7 +1,7 @@
 // sdpa_fwd_sm100.cuh -- fused scaled-dot-product attention forward for
 // sm_100a (B200): TMA-fed K/V ring, tcgen05 MMAs with accumulators in tensor
 // memory, warp-specialised roles, exp2 online softmax, causal tile skipping,
-// GQA/MQA K/V heads shared by index.
+// GQA/MQA K/V heads shared by index, persistent CTAs.
 //
 // Method (article "Self-attention, CUDA kernels and FlashAttention", section
 // 3): Q, K, V are cut into on-chip tiles, scores of a tile are turned into
@@ -12,26 +12,32 @@
 // Lab 5: attention on GPU", section 1; causal mask section 7; MHA/GQA/MQA
 // section 9; FP8 E4M3 forward section 10.
 //
-// One CTA owns 128 query rows of one (batch, query head) and walks the K/V
-// tiles (128 keys each) of that head's KV head.  Warp roles (320 threads):
+// Work units are 128 query rows of one (batch, query head).  One CTA runs
+// per SM and walks a static list of schedule items: for causal attention an
+// item pairs query tile j with tile nq-1-j of the same head (together always
+// nq+1 K/V tiles), so a round-robin assignment of items balances the SMs;
+// items come in groups of heads so their K/V stay in L2.  The CTA treats the
+// K/V tiles of all its units as one stream, so the scores of the next unit
+// are computed while the current one finishes.  Warp roles (320 threads):
 //   warps 0-3  softmax group 0: keys 0-63 of every tile, thread = row = lane
 //   warps 4-7  softmax group 1: keys 64-127 of every tile
-//   warp  8    TMA producer: Q once, then K/V tiles in MMA consumption order
+//   warp  8    TMA producer: Q per unit (double-buffered), K/V tiles in MMA
+//              consumption order K_0, K_1, V_0, K_2, V_1, ... over the stream
 //   warp  9    MMA issuer (one elected lane) and TMEM owner
 // Tensor memory (512 columns x 128 lanes, fp32):
 //   [0,128) S_a  [128,256) S_b  [256,256+d) O_0  [384,384+d) O_1
-// S is double-buffered: S(i) lives in S_(i&1), and Q K_(i+2)^T is issued as
-// soon as O += P(i) V_i has been issued, so the scores of the next tile are
-// ready when the softmax finishes the current one and the tensor pipe works
-// while the softmax does.  Each softmax group keeps its own running max m_h,
-// sum l_h and output O_h over its half of the keys; the halves never
-// exchange data inside the loop and are merged once at the end:
+// S is double-buffered: S(g) of stream tile g lives in S_(g&1), and
+// Q K_(g+2)^T is issued as soon as O += P(g) V_g has been issued, so the
+// next scores are ready when the softmax finishes a tile and the tensor pipe
+// works while the softmax does.  Each softmax group keeps its own running max
+// m_h, sum l_h and output O_h over its half of the keys; the halves never
+// exchange data inside the loop and are merged once per unit:
 //   O = (2^(m_0-m) O_0 + 2^(m_1-m) O_1) / (2^(m_0-m) l_0 + 2^(m_1-m) l_1),
 //   m = max(m_0, m_1),  LSE = (m + log2(2^(m_0-m) l_0 + 2^(m_1-m) l_1)) ln 2.
-// P_h(i) (the weights, packed 2 x 16-bit or 4 x e4m3 per column) overwrites
-// group h's own columns of S_(i&1) once the group has read them.
+// P_h(g) (the weights, packed 2 x 16-bit or 4 x e4m3 per column) overwrites
+// group h's own columns of S_(g&1) once the group has read them.
 // tcgen05 MMAs from one thread execute in issue order, so the S write of
-// Q K_(i+2)^T queued after the P(i) reads cannot overtake them.
+// Q K_(g+2)^T queued after the P(g) reads cannot overtake them.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -45,11 +51,9 @@
 #ifndef SDPA_POLY_MASK
 #define SDPA_POLY_MASK 0x00
 #endif
-// 1: the two softmax groups run staggered by part of a tile.
-#ifndef SDPA_STAGGER
-#define SDPA_STAGGER 0
-#endif
-// K/V ring depth for 16-bit d = 128, 16-bit d = 64 and e4m3 d = 128.
+// K/V ring depth for 16-bit d = 128 (with one Q buffer: the next unit's Q is
+// loaded once the current unit's last QK has completed, one tile ahead),
+// 16-bit d = 64 and e4m3 d = 128 (two Q buffers each).
 #ifndef SDPA_STAGES_D128
 #define SDPA_STAGES_D128 6
 #endif
@@ -64,11 +68,10 @@ namespace sdpa {
 
 enum Kind { KIND_BF16 = 0, KIND_FP16 = 1, KIND_E4M3 = 2 };
 
-constexpr int kBlockM = 128;        // query rows per CTA (= TMEM lanes)
+constexpr int kBlockM = 128;        // query rows per unit (= TMEM lanes)
 constexpr int kBlockN = 128;        // keys per K/V tile
 constexpr int kHalfN = 64;          // keys per softmax group
 constexpr int kThreads = 320;       // 10 warps
-constexpr int kLaunchRegs = 168;    // registers per thread (10 warps: 3 on some sub-partitions)
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
@@ -85,13 +88,15 @@ struct FwdParams {
     int B, Hq, Hkv, Sq, Sk;
     int group;          // Hq / Hkv
     int n_qtiles;       // ceil(Sq / 128)
-    int group_heads;    // (batch, head) pairs per CTA group
+    int items_per_head; // schedule items per (batch, head): causal ceil(nq/2), else nq
+    int n_items;        // B * Hq * items_per_head
+    int group_heads;    // (batch, head) pairs per schedule group
     int causal;
     float score_log2;   // multiplier from raw MMA score to log2 units
     float out_mul;      // multiplier on (sum_j p_j v_j) / l: the V descale for FP8, else 1
 };
 
-template <int D, int KIND, int NS>
+template <int D, int KIND, int NS, int QB>
 struct FwdCfg {
     static constexpr int kElem = (KIND == KIND_E4M3) ? 1 : 2;
     static constexpr int kRowBytes = D * kElem;
@@ -108,29 +113,27 @@ struct FwdCfg {
     // 448 (the e4m3 maximum) for FP8, so that p in (0, 1] fills the format
     static constexpr float kPLog2 = (KIND == KIND_E4M3) ? 8.807354922057604f : 0.0f;
     // shared memory map (offsets from a 1024-byte aligned base)
-    static constexpr int kSmemQ = 0;
-    static constexpr int kSmemKV = kTileBytes;
-    static constexpr int kSmemBar = kSmemKV + NS * kTileBytes;
-    // barriers: q_full, kv_full[NS], kv_empty[NS], s_full[2], p_full[2 buffers][2 groups],
-    //           o_done[2 groups] (once per tile), o_full (once per CTA), xchg, drain
+    static constexpr int kSmemQ = 0;                      // QB Q tiles
+    static constexpr int kSmemKV = QB * kTileBytes;
+    static constexpr int kSmemStats = kSmemKV + NS * kTileBytes;   // [128 rows][2] fp32
+    static constexpr int kSmemBar = kSmemStats + 128 * 2 * 4;
+    // barriers (Q ones: [QB buffers], QB <= 2)
     static constexpr int kBarQFull = 0;
-    static constexpr int kBarKVFull = 1;
-    static constexpr int kBarKVEmpty = 1 + NS;
-    static constexpr int kBarSFull = 1 + 2 * NS;
-    static constexpr int kBarPFull = 3 + 2 * NS;
-    static constexpr int kBarODone = 7 + 2 * NS;
-    static constexpr int kBarOFull = 9 + 2 * NS;
-    static constexpr int kBarXchg = 10 + 2 * NS;
-    static constexpr int kBarDrain = 11 + 2 * NS;
-    static constexpr int kBarStagger = 12 + 2 * NS;
-    static constexpr int kNumBars = 13 + 2 * NS;
+    static constexpr int kBarQEmpty = 2;
+    static constexpr int kBarKVFull = 4;                  // [NS]
+    static constexpr int kBarKVEmpty = 4 + NS;            // [NS]
+    static constexpr int kBarSFull = 4 + 2 * NS;          // [2 S buffers]
+    static constexpr int kBarPFull = 6 + 2 * NS;          // [2 S buffers][2 groups]
+    static constexpr int kBarODone = 10 + 2 * NS;         // [2 groups], once per tile
+    static constexpr int kBarOFull = 12 + 2 * NS;         // once per unit
+    static constexpr int kBarOEmpty = 13 + 2 * NS;        // once per unit
+    static constexpr int kBarXchg1 = 14 + 2 * NS;         // group 1 -> group 0, once per unit
+    static constexpr int kBarXchg2 = 15 + 2 * NS;         // group 0 -> group 1, once per unit
+    static constexpr int kBarDrain = 16 + 2 * NS;
+    static constexpr int kNumBars = 17 + 2 * NS;
     static constexpr int kSmemTmemSlot = kSmemBar + 8 * kNumBars;
     static constexpr int kSmemAbort = kSmemTmemSlot + 4;
-    // the epilogue exchanges [2 groups][m, l][128] fp32 through the Q tile
-    // (every QK MMA has completed by then)
-    static constexpr int kSmemStats = kSmemQ;
     static constexpr int kSmemUsed = kSmemAbort + 4;
-    static_assert(2 * 2 * 128 * 4 <= kTileBytes, "stats fit in the Q tile");
     static constexpr int kSmemBytes = kSmemUsed + 1024;  // slack for the 1024-byte alignment
     // TMEM columns
     static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
@@ -138,7 +141,9 @@ struct FwdCfg {
     static_assert(kSmemBytes <= 232448, "shared memory budget");
     static_assert(kSmemBytes > 116 * 1024, "one CTA per SM (each allocates all of TMEM)");
     static_assert(D <= 128, "O tile must fit its 128 TMEM columns");
+    static_assert(QB == 1 || QB == 2, "one or two Q buffers");
 };
+
 
 // ---------------------------------------------------------------------------
 // bounded waiting
@@ -203,36 +208,91 @@ __device__ __forceinline__ int tiles_for(int row0, int Sq, int Sk, int causal) {
     return (kend + kBlockN - 1) / kBlockN;
 }
 
-// The t-th K/V tile the MMA warp consumes (and the producer loads):
-// K_0, K_1, V_0, K_2, V_1, K_3, ..., V_(n-3), K_(n-1), V_(n-2), V_(n-1).
-__device__ __forceinline__ void kv_item(int t, int n, bool& is_v, int& tile) {
-    if (n == 1) {
-        is_v = (t == 1);
-        tile = 0;
-        return;
+
+// ---------------------------------------------------------------------------
+// schedule: the units (128 query rows of one (batch, head)) a CTA processes
+// ---------------------------------------------------------------------------
+// Unit `sub` (0 or 1) of this CTA's k-th schedule item.  Item index
+// blockIdx.x + k * gridDim.x; items come in groups of p.group_heads heads;
+// within a group, item j of a head holds query tile nq-1-j (and, for causal
+// attention, also tile j: long and short tiles of the same head paired).
+__device__ __forceinline__ bool sched_unit(const FwdParams& p, int k, int sub, int& bh,
+                                           int& qtile) {
+    const long long item = (long long)blockIdx.x + (long long)k * gridDim.x;
+    if (item >= p.n_items) return false;
+    const int n_bh = p.B * p.Hq;
+    const int per_group = p.group_heads * p.items_per_head;
+    const int grp = (int)(item / per_group);
+    const int within = (int)(item - (long long)grp * per_group);
+    const int gsize = min(p.group_heads, n_bh - grp * p.group_heads);
+    const int j = within / gsize;
+    bh = grp * p.group_heads + within % gsize;
+    const int hi = p.n_qtiles - 1 - j;
+    if (sub == 0) {
+        qtile = hi;
+        return true;
     }
-    if (t < 2) {
-        is_v = false;
-        tile = t;
-        return;
+    if (!p.causal || j == hi) return false;
+    qtile = j;
+    return true;
+}
+
+struct UnitCursor {
+    int k, sub;      // schedule position
+    int bh, qtile;   // the unit
+    int n;           // its K/V tiles
+    int ku;          // units of this CTA before it
+    bool valid;
+};
+
+__device__ __forceinline__ void unit_load(const FwdParams& p, UnitCursor& u) {
+    u.valid = sched_unit(p, u.k, u.sub, u.bh, u.qtile);
+    u.n = u.valid ? tiles_for(u.qtile * kBlockM, p.Sq, p.Sk, p.causal) : 0;
+}
+__device__ __forceinline__ void unit_first(const FwdParams& p, UnitCursor& u) {
+    u.k = 0;
+    u.sub = 0;
+    u.ku = 0;
+    unit_load(p, u);
+}
+__device__ __forceinline__ void unit_next(const FwdParams& p, UnitCursor& u) {
+    ++u.ku;
+    if (u.sub == 0) {
+        u.sub = 1;
+        unit_load(p, u);
+        if (u.valid) return;
     }
-    const int r = t - 2;
-    if (r < 2 * (n - 2)) {
-        is_v = (r & 1) == 0;
-        tile = is_v ? (r >> 1) : (r >> 1) + 2;
-    } else {
-        is_v = true;
-        tile = (n - 2) + (r - 2 * (n - 2));
+    ++u.k;
+    u.sub = 0;
+    unit_load(p, u);
+}
+
+// One position in the CTA's stream of K/V tiles.
+struct TileCursor {
+    UnitCursor u;
+    int i;           // tile within the unit
+    int g;           // tile within the stream
+};
+__device__ __forceinline__ void tile_first(const FwdParams& p, TileCursor& c) {
+    unit_first(p, c.u);
+    c.i = 0;
+    c.g = 0;
+}
+__device__ __forceinline__ void tile_next(const FwdParams& p, TileCursor& c) {
+    ++c.g;
+    if (++c.i == c.u.n) {
+        unit_next(p, c.u);
+        c.i = 0;
     }
 }
 
-template <int D, int KIND, int NS>
+template <int D, int KIND, int NS, int QB>
 __global__ void __launch_bounds__(kThreads, 1)
 sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV,
                       const FwdParams p) {
-    using C = FwdCfg<D, KIND, NS>;
+    using C = FwdCfg<D, KIND, NS, QB>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -241,42 +301,27 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // ---- work unit ------------------------------------------------------
-    // CTAs come in groups of p.group_heads (batch, head) pairs, every query
-    // tile of a group before the next group, so the K/V a group reads stay in
-    // L2; inside a group the longest (last, for causal) query tiles go first.
-    const int n_bh = p.B * p.Hq;
-    const int per_group = p.group_heads * p.n_qtiles;
-    const int grp = (int)(blockIdx.x / (unsigned)per_group);
-    const int within = (int)blockIdx.x - grp * per_group;
-    const int gsize = min(p.group_heads, n_bh - grp * p.group_heads);
-    const int qtile = p.n_qtiles - 1 - within / gsize;
-    const int bh = grp * p.group_heads + within % gsize;
-    const int b = bh / p.Hq;
-    const int hq = bh - b * p.Hq;
-    const int kvh = b * p.Hkv + hq / p.group;
-    const int m0 = qtile * kBlockM;
-    const int n = tiles_for(m0, p.Sq, p.Sk, p.causal);   // >= 1
-
     auto bar = [&](int i) -> uint32_t { return sbase + C::kSmemBar + 8u * (uint32_t)i; };
     const uint32_t abort_addr = sbase + C::kSmemAbort;
     const uint32_t slot_addr = sbase + C::kSmemTmemSlot;
 
     if (threadIdx.x == 0) {
-        mbar_init(bar(C::kBarQFull), 1);
-        for (int s = 0; s < NS; ++s) {
-            mbar_init(bar(C::kBarKVFull + s), 1);
-            mbar_init(bar(C::kBarKVEmpty + s), 1);
-        }
         for (int j = 0; j < 2; ++j) {
+            mbar_init(bar(C::kBarQFull + j), 1);
+            mbar_init(bar(C::kBarQEmpty + j), 1);
             mbar_init(bar(C::kBarSFull + j), 1);
             mbar_init(bar(C::kBarODone + j), 1);
             mbar_init(bar(C::kBarPFull + 2 * j), kBlockM);
             mbar_init(bar(C::kBarPFull + 2 * j + 1), kBlockM);
         }
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(bar(C::kBarKVFull + s), 1);
+            mbar_init(bar(C::kBarKVEmpty + s), 1);
+        }
         mbar_init(bar(C::kBarOFull), 1);
-        mbar_init(bar(C::kBarXchg), 2 * kBlockM);
-        mbar_init(bar(C::kBarStagger), kBlockM);
+        mbar_init(bar(C::kBarOEmpty), 2 * kBlockM);
+        mbar_init(bar(C::kBarXchg1), kBlockM);
+        mbar_init(bar(C::kBarXchg2), kBlockM);
         mbar_init(bar(C::kBarDrain), 1);
         st_shared_u32(abort_addr, 0u);
         fence_barrier_init();
@@ -301,31 +346,66 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         // ================= TMA producer =================================
         if (lane == 0) {
             bool ok = true;
-            mbar_arrive_expect_tx(bar(C::kBarQFull), C::kTileBytes);
-            for (int kb = 0; kb < C::kSwBlocks; ++kb)
-                tma_load_3d(sQ + kb * C::kSwBlockBytes, &tmQ, bar(C::kBarQFull),
-                            kb * C::kElemsPerSw, m0, bh);
-            int t = 0;
-            for (; t < 2 * n && ok; ++t) {
+            int t = 0;        // K/V tiles issued
+            int q_last = -1;  // last unit whose Q was issued
+            TileCursor kc, vc;
+            tile_first(p, kc);
+            tile_first(p, vc);
+            // Issue the K (or V) tile of stream position c into the ring; a
+            // unit's Q goes in right before its first K tile.
+            auto emit = [&](const TileCursor& c, bool is_v) -> bool {
+                if (!is_v && c.i == 0) {
+                    const int qb = c.u.ku % QB, qm = c.u.ku / QB;
+                    if (qm >= 1 &&
+                        !wait_bar(bar(C::kBarQEmpty + qb), (uint32_t)(qm - 1) & 1u,
+                                  abort_addr, 0x11000u | (uint32_t)c.u.ku))
+                        return false;
+                    mbar_arrive_expect_tx(bar(C::kBarQFull + qb), C::kTileBytes);
+                    for (int kb = 0; kb < C::kSwBlocks; ++kb)
+                        tma_load_3d(sQ + qb * C::kTileBytes + kb * C::kSwBlockBytes, &tmQ,
+                                    bar(C::kBarQFull + qb), kb * C::kElemsPerSw,
+                                    c.u.qtile * kBlockM, c.u.bh);
+                    q_last = c.u.ku;
+                }
                 const int slot = t % NS;
-                const uint32_t par = ((uint32_t)(t / NS) & 1u) ^ 1u;
-                ok = wait_bar(bar(C::kBarKVEmpty + slot), par, abort_addr, 0x10000u | (uint32_t)t);
-                if (!ok) break;
-                bool is_v;
-                int tile;
-                kv_item(t, n, is_v, tile);
+                if (!wait_bar(bar(C::kBarKVEmpty + slot), ((uint32_t)(t / NS) & 1u) ^ 1u, abort_addr,
+                              0x10000u | (uint32_t)t))
+                    return false;
+                const int b = c.u.bh / p.Hq;
+                const int kvh = b * p.Hkv + (c.u.bh - b * p.Hq) / p.group;
                 const uint32_t fb = bar(C::kBarKVFull + slot);
                 mbar_arrive_expect_tx(fb, C::kTileBytes);
-                const CUtensorMap* m = is_v ? &tmV : &tmK;
                 for (int kb = 0; kb < C::kSwBlocks; ++kb)
-                    tma_load_3d(sKV + slot * C::kTileBytes + kb * C::kSwBlockBytes, m, fb,
-                                kb * C::kElemsPerSw, tile * kBlockN, kvh);
+                    tma_load_3d(sKV + slot * C::kTileBytes + kb * C::kSwBlockBytes,
+                                is_v ? &tmV : &tmK, fb, kb * C::kElemsPerSw, c.i * kBlockN, kvh);
+                ++t;
+                return true;
+            };
+            // MMA consumption order: K(0), K(1), then V(g), K(g+2), ..., then
+            // the last V tiles
+            for (int j = 0; j < 2 && ok && kc.u.valid; ++j) {
+                ok = emit(kc, false);
+                tile_next(p, kc);
+            }
+            while (ok && vc.u.valid) {
+                ok = emit(vc, true);
+                tile_next(p, vc);
+                if (ok && kc.u.valid) {
+                    ok = emit(kc, false);
+                    tile_next(p, kc);
+                }
             }
             if (!ok) {
                 // let the copies already issued land before the CTA exits
                 for (int u = max(0, t - NS); u < t; ++u) {
                     const uint64_t t0 = global_timer_ns();
                     while (!mbar_try_wait(bar(C::kBarKVFull + u % NS), (uint32_t)(u / NS) & 1u) &&
+                           global_timer_ns() - t0 < 100000000ull) {
+                    }
+                }
+                for (int u = max(0, q_last - QB + 1); u <= q_last; ++u) {
+                    const uint64_t t0 = global_timer_ns();
+                    while (!mbar_try_wait(bar(C::kBarQFull + u % QB), (uint32_t)(u / QB) & 1u) &&
                            global_timer_ns() - t0 < 100000000ull) {
                     }
                 }
@@ -353,18 +433,24 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             if (leader) mma_commit(b_);
             __syncwarp();
         };
-        // S_buf = Q K^T for the K tile in `slot`
-        auto issue_qk = [&](int buf, int slot) {
+        auto next_kv = [&](uint32_t where) -> int {
+            const int slot = t % NS;
+            ok = wait_all(bar(C::kBarKVFull + slot), (uint32_t)(t / NS) & 1u, where | (uint32_t)(t & 0xfff));
+            return slot;
+        };
+        // S_buf = Q_qb K^T for the K tile in `slot`
+        auto issue_qk = [&](int buf, int qb, int slot) {
             const uint32_t d_tmem = tmem + (buf ? C::kColS1 : C::kColS0);
+            const uint64_t dq = desc_q + (uint64_t)((qb * C::kTileBytes) >> 4);
             const uint64_t dk = desc_k + (uint64_t)((slot * C::kTileBytes) >> 4);
             if (leader) {
 #pragma unroll
                 for (int kk = 0; kk < C::kQkSteps; ++kk) {
                     const uint64_t off = (uint64_t)(((kk >> 2) * C::kSwBlockBytes + (kk & 3) * 32) >> 4);
                     if constexpr (KIND == KIND_E4M3)
-                        mma_f8_ss(d_tmem, desc_q + off, dk + off, idesc_qk, kk > 0);
+                        mma_f8_ss(d_tmem, dq + off, dk + off, idesc_qk, kk > 0);
                     else
-                        mma_f16_ss(d_tmem, desc_q + off, dk + off, idesc_qk, kk > 0);
+                        mma_f16_ss(d_tmem, dq + off, dk + off, idesc_qk, kk > 0);
                 }
             }
             __syncwarp();
@@ -388,45 +474,52 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             }
             __syncwarp();
         };
-        auto next_kv = [&](uint32_t where) -> int {
-            const int slot = t % NS;
-            ok = wait_all(bar(C::kBarKVFull + slot), (uint32_t)(t / NS) & 1u, where | (uint32_t)t);
-            return slot;
+
+        TileCursor kc, vc;
+        tile_first(p, kc);
+        tile_first(p, vc);
+        // S_(g&1) = Q K^T for stream tile kc (g = kc.g)
+        auto qk_tile = [&]() -> bool {
+            const int qb = kc.u.ku % QB;
+            if (kc.i == 0 &&
+                !wait_all(bar(C::kBarQFull + qb), (uint32_t)(kc.u.ku / QB) & 1u, 0x20000u | (uint32_t)kc.u.ku))
+                return false;
+            const int slot = next_kv(0x21000u);
+            if (!ok) return false;
+            issue_qk(kc.g & 1, qb, slot);
+            commit(bar(C::kBarSFull + (kc.g & 1)));
+            commit(bar(C::kBarKVEmpty + slot));
+            if (kc.i == kc.u.n - 1) commit(bar(C::kBarQEmpty + qb));   // Q_qb free
+            ++t;
+            tile_next(p, kc);
+            return true;
         };
 
-        ok = wait_all(bar(C::kBarQFull), 0, 0x20000u);
-        for (int j = 0; j < min(n, 2) && ok; ++j) {
-            const int slot = next_kv(0x21000u);
-            if (!ok) break;
-            issue_qk(j, slot);
-            commit(bar(C::kBarSFull + j));
-            commit(bar(C::kBarKVEmpty + slot));
-            ++t;
-        }
-        for (int i = 0; i < n && ok; ++i) {
-            const int buf = i & 1;
+        for (int j = 0; j < 2 && ok && kc.u.valid; ++j) ok = qk_tile();
+        while (ok && vc.u.valid) {
+            const int buf = vc.g & 1;
             const int slotV = next_kv(0x22000u);
             if (!ok) break;
+            // the first product of a unit overwrites O: the previous unit's
+            // epilogue must have read it
+            if (vc.i == 0 && vc.u.ku > 0) {
+                ok = wait_all(bar(C::kBarOEmpty), (uint32_t)(vc.u.ku - 1) & 1u, 0x25000u | (uint32_t)vc.u.ku);
+                if (!ok) break;
+            }
             for (int h = 0; h < 2 && ok; ++h) {
-                ok = wait_all(bar(C::kBarPFull + 2 * buf + h), (uint32_t)(i >> 1) & 1u,
-                              0x23000u | (h << 11) | (uint32_t)i);
+                ok = wait_all(bar(C::kBarPFull + 2 * buf + h), (uint32_t)(vc.g >> 1) & 1u,
+                              0x23000u | (h << 11) | (uint32_t)(vc.g & 0x7ff));
                 if (!ok) break;
                 tc_fence_after();
-                issue_pv(h, buf, slotV, i > 0);
+                issue_pv(h, buf, slotV, vc.i > 0);
                 commit(bar(C::kBarODone + h));
             }
             if (!ok) break;
-            if (i == n - 1) commit(bar(C::kBarOFull));
+            if (vc.i == vc.u.n - 1) commit(bar(C::kBarOFull));
             commit(bar(C::kBarKVEmpty + slotV));
             ++t;
-            if (i + 2 < n) {
-                const int slotK = next_kv(0x24000u);
-                if (!ok) break;
-                issue_qk(buf, slotK);
-                commit(bar(C::kBarSFull + buf));
-                commit(bar(C::kBarKVEmpty + slotK));
-                ++t;
-            }
+            tile_next(p, vc);
+            if (kc.u.valid) ok = qk_tile();
         }
         if (!ok) {
             // make sure no MMA is still writing tensor memory at exit
@@ -444,14 +537,11 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         // ================= softmax groups (warps 0-7) ====================
         const int h = warp >> 2;                 // key half of every tile
         const int quarter = warp & 3;            // TMEM lane quarter of this warp
-        const int r = (int)(threadIdx.x & 127);  // row within the tile
-        const int row = m0 + r;
+        const int r = (int)(threadIdx.x & 127);  // row within the unit
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         const uint32_t tO = tmem + lane_base + (h ? C::kColO1 : C::kColO0);
         const float sl = p.score_log2;
         const uint64_t sl2 = f2_pack(sl, sl);
-        float m_run = -INFINITY;   // running max of this half's scaled scores (log2 units)
-        float l_run = 0.0f;        // running sum of 2^(s*sl - m_run + kPLog2)
         bool ok = true;
 
         // -m [+ log2 of the P scale] as a pair; a row whose keys of this half
@@ -496,159 +586,177 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             return f2_add(sum2[0], sum2[1]);
         };
 
-#if SDPA_STAGGER
-        // Group 1 starts once group 0 has produced the first chunk of its
-        // first tile, so the two groups run half a tile apart: one group's
-        // exponentials overlap the other's score load and maximum.
-        if (h == 1) {
-            ok = wait_bar(bar(C::kBarStagger), 0, abort_addr, 0x32000u);
-            ok = __all_sync(0xffffffffu, ok);
-        }
-#endif
-        for (int i = 0; i < n && ok; ++i) {
-            const int buf = i & 1;
-            ok = wait_bar(bar(C::kBarSFull + buf), (uint32_t)(i >> 1) & 1u, abort_addr,
-                          0x30000u | (h << 12) | i);
-            ok = __all_sync(0xffffffffu, ok);
+        UnitCursor u;
+        unit_first(p, u);
+        int g = 0;   // stream tile
+        while (ok && u.valid) {
+            const int m0 = u.qtile * kBlockM;
+            const int row = m0 + r;
+            const int n = u.n;
+            float m_run = -INFINITY;   // running max of this half's scaled scores (log2 units)
+            float l_run = 0.0f;        // running sum of 2^(s*sl - m_run + kPLog2)
+
+            for (int i = 0; i < n && ok; ++i, ++g) {
+                const int buf = g & 1;
+                ok = wait_bar(bar(C::kBarSFull + buf), (uint32_t)(g >> 1) & 1u, abort_addr,
+                              0x30000u | (h << 12) | (uint32_t)(g & 0xfff));
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t tS = tmem + lane_base + (buf ? C::kColS1 : C::kColS0) + h * kHalfN;
+
+                float s[kHalfN];
+                // chunk 0 (keys 0-31 of this half); chunk 1 is loaded while the
+                // exponentials of chunk 0 run
+                tmem_ld32(tS + 0, *reinterpret_cast<float(*)[32]>(&s[0]));
+                tmem_wait_ld();
+                reg_fence32(&s[0]);
+                tmem_ld32(tS + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
+
+                // mask: keys past Sk, and (causal) keys after the row
+                const int key0 = i * kBlockN + h * kHalfN;
+                const bool edge = (key0 + kHalfN > p.Sk) || (p.causal && key0 + kHalfN - 1 > m0);
+                int lim = kHalfN;
+                if (edge) {
+                    lim = p.Sk - key0;
+                    if (p.causal) lim = min(lim, row - key0 + 1);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        if (c >= lim) s[c] = -INFINITY;
+                }
+                const float cmax0 = chunk_max32(&s[0]) * sl;
+
+                // Fast path: while a chunk's maximum stays within the rescale
+                // threshold of the running max m_run, its weights are computed
+                // against m_run at once.  Otherwise (always on the first tile)
+                // the tile takes the full path: maximum of both chunks, new
+                // m_run, l and O rescaled, chunk 0 recomputed.
+                const bool fast0 = !__any_sync(0xffffffffu, cmax0 > m_run + C::kRescaleThreshold);
+                uint64_t sum0 = 0ull, sum1 = 0ull;
+                if (fast0) sum0 = exp_chunk(&s[0], sl2, neg_m_of(m_run), tS, 0);
+
+                tmem_wait_ld();
+                reg_fence32(&s[32]);
+                if (edge) {
+#pragma unroll
+                    for (int c = 32; c < kHalfN; ++c)
+                        if (c >= lim) s[c] = -INFINITY;
+                }
+                const float cmax1 = chunk_max32(&s[32]) * sl;
+                if (!fast0 || __any_sync(0xffffffffu, cmax1 > m_run + C::kRescaleThreshold)) {
+                    const float tile_max = fmaxf(cmax0, cmax1);
+                    float alpha = 1.0f;
+                    if (tile_max > m_run + C::kRescaleThreshold) {
+                        alpha = ex2_approx(m_run - tile_max);   // 0 on the first live tile
+                        m_run = tile_max;
+                    }
+                    l_run *= alpha;
+                    // O_h takes the same factor before P_h V is added; its last
+                    // update (stream tile g-1, same unit since i > 0) must have
+                    // completed.  o_done[h] completes once per tile; this
+                    // parity wait is exact because the barrier is within one
+                    // phase of tile g-1: the S(g) commit covered tile g-2's
+                    // product and tile g's cannot exist yet.
+                    if (i > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+                        ok = wait_bar(bar(C::kBarODone + h), (uint32_t)(g - 1) & 1u, abort_addr,
+                                      0x31000u | (h << 12) | (uint32_t)(g & 0xfff));
+                        ok = __all_sync(0xffffffffu, ok);
+                        if (!ok) break;
+                        tc_fence_after();
+#pragma unroll 1
+                        for (int c = 0; c < D / 32; ++c) {
+                            float o[32];
+                            tmem_ld32(tO + 32 * c, o);
+                            tmem_wait_ld();
+                            reg_fence32(o);
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+                            tmem_st32(tO + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(o));
+                        }
+                    }
+                    sum0 = exp_chunk(&s[0], sl2, neg_m_of(m_run), tS, 0);
+                }
+                sum1 = exp_chunk(&s[32], sl2, neg_m_of(m_run), tS, 1);
+                {
+                    float a0, a1, b0, b1;
+                    f2_unpack(sum0, a0, a1);
+                    f2_unpack(sum1, b0, b1);
+                    l_run += (a0 + a1) + (b0 + b1);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(C::kBarPFull + 2 * buf + h));
+            }
+            if (!ok) break;
+
+            // ---- epilogue of the unit: merge the halves, O -> 16-bit, LSE ----
+            // Group 1 hands (m_1, l_1) to group 0 through `stats`; group 0
+            // computes the merge factors c_0, c_1 and hands them back.
+            const uint32_t xpar = (uint32_t)u.ku & 1u;
+            float c0 = 0.f, c1 = 0.f;
+            if (h == 1) {
+                stats[2 * r] = m_run;
+                stats[2 * r + 1] = l_run;
+                mbar_arrive(bar(C::kBarXchg1));
+                ok = wait_bar(bar(C::kBarXchg2), xpar, abort_addr, 0x40000u | (uint32_t)u.ku);
+                ok = __all_sync(0xffffffffu, ok);
+                c0 = stats[2 * r];
+                c1 = stats[2 * r + 1];
+            } else {
+                ok = wait_bar(bar(C::kBarXchg1), xpar, abort_addr, 0x41000u | (uint32_t)u.ku);
+                ok = __all_sync(0xffffffffu, ok);
+                const float m_1 = stats[2 * r], l_1 = stats[2 * r + 1];
+                const float m = fmaxf(m_run, m_1);
+                const float a0 = (m_run == -INFINITY) ? 0.0f : ex2_approx(m_run - m);
+                const float a1 = (m_1 == -INFINITY) ? 0.0f : ex2_approx(m_1 - m);
+                const float l = l_run * a0 + l_1 * a1;
+                c0 = a0 * (p.out_mul / l);
+                c1 = a1 * (p.out_mul / l);
+                stats[2 * r] = c0;
+                stats[2 * r + 1] = c1;
+                mbar_arrive(bar(C::kBarXchg2));
+                if (ok && p.lse != nullptr && row < p.Sq)
+                    p.lse[(size_t)u.bh * p.Sq + row] = (m + __log2f(l) - C::kPLog2) * kLn2;
+            }
+            if (ok) {
+                ok = wait_bar(bar(C::kBarOFull), xpar, abort_addr, 0x42000u | (uint32_t)u.ku);
+                ok = __all_sync(0xffffffffu, ok);
+            }
             if (!ok) break;
             tc_fence_after();
-            const uint32_t tS = tmem + lane_base + (buf ? C::kColS1 : C::kColS0) + h * kHalfN;
-
-            float s[kHalfN];
-            // chunk 0 (keys 0-31 of this half); chunk 1 is loaded while the
-            // exponentials of chunk 0 run
-            tmem_ld32(tS + 0, *reinterpret_cast<float(*)[32]>(&s[0]));
-            tmem_wait_ld();
-            reg_fence32(&s[0]);
-            tmem_ld32(tS + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
-
-            // mask: keys past Sk, and (causal) keys after the row
-            const int key0 = i * kBlockN + h * kHalfN;
-            const bool edge = (key0 + kHalfN > p.Sk) || (p.causal && key0 + kHalfN - 1 > m0);
-            int lim = kHalfN;
-            if (edge) {
-                lim = p.Sk - key0;
-                if (p.causal) lim = min(lim, row - key0 + 1);
-#pragma unroll
-                for (int c = 0; c < 32; ++c)
-                    if (c >= lim) s[c] = -INFINITY;
-            }
-            const float cmax0 = chunk_max32(&s[0]) * sl;
-
-            // Fast path: while a chunk's maximum stays within the rescale
-            // threshold of the running max m_run, its weights are computed
-            // against m_run at once.  Otherwise (always on the first tile)
-            // the tile takes the full path: maximum of both chunks, new m_run,
-            // l and O rescaled, chunk 0 recomputed.
-            const bool fast0 = !__any_sync(0xffffffffu, cmax0 > m_run + C::kRescaleThreshold);
-            uint64_t sum0 = 0ull, sum1 = 0ull;
-            if (fast0) sum0 = exp_chunk(&s[0], sl2, neg_m_of(m_run), tS, 0);
-
-            tmem_wait_ld();
-            reg_fence32(&s[32]);
-            if (edge) {
-#pragma unroll
-                for (int c = 32; c < kHalfN; ++c)
-                    if (c >= lim) s[c] = -INFINITY;
-            }
-            const float cmax1 = chunk_max32(&s[32]) * sl;
-            if (!fast0 || __any_sync(0xffffffffu, cmax1 > m_run + C::kRescaleThreshold)) {
-                const float tile_max = fmaxf(cmax0, cmax1);
-                float alpha = 1.0f;
-                if (tile_max > m_run + C::kRescaleThreshold) {
-                    alpha = ex2_approx(m_run - tile_max);   // 0 on the first live tile
-                    m_run = tile_max;
-                }
-                l_run *= alpha;
-                // O_h takes the same factor before P_h(i) V_i is added; its
-                // last update, O_h += P_h(i-1) V_(i-1), must have completed.
-                // o_done[h] completes once per tile; this parity wait is exact
-                // because the barrier is within one phase of tile i-1: the
-                // S(i) commit covered tile i-2's product and tile i's cannot
-                // exist yet.
-                if (i > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
-                    ok = wait_bar(bar(C::kBarODone + h), (uint32_t)(i - 1) & 1u, abort_addr,
-                                  0x31000u | (h << 12) | i);
-                    ok = __all_sync(0xffffffffu, ok);
-                    if (!ok) break;
-                    tc_fence_after();
+            {
+                const bool live = row < p.Sq;
+                const size_t orow = ((size_t)u.bh * p.Sq + (size_t)(live ? row : 0)) * D;
+                uint16_t* obase = reinterpret_cast<uint16_t*>(p.o) + orow;
+                const uint32_t tO0 = tmem + lane_base + C::kColO0, tO1 = tmem + lane_base + C::kColO1;
+                // group h writes output columns [h * D / 2, (h + 1) * D / 2)
 #pragma unroll 1
-                    for (int c = 0; c < D / 32; ++c) {
-                        float o[32];
-                        tmem_ld32(tO + 32 * c, o);
-                        tmem_wait_ld();
-                        reg_fence32(o);
+                for (int c = h * (D / 64); c < (h + 1) * (D / 64); ++c) {
+                    float x[32], y[32];
+                    tmem_ld32(tO0 + 32 * c, x);
+                    tmem_ld32(tO1 + 32 * c, y);
+                    tmem_wait_ld();
+                    reg_fence32(x);
+                    reg_fence32(y);
+                    uint32_t w4[16];
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] *= alpha;
-                        tmem_st32(tO + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(o));
+                    for (int e = 0; e < 16; ++e) {
+                        const float v0 = x[2 * e] * c0 + y[2 * e] * c1;
+                        const float v1 = x[2 * e + 1] * c0 + y[2 * e + 1] * c1;
+                        w4[e] = (KIND == KIND_FP16) ? pack_f16x2(v0, v1) : pack_bf16x2(v0, v1);
+                    }
+                    if (live) {
+                        uint4* dst = reinterpret_cast<uint4*>(obase + 32 * c);
+#pragma unroll
+                        for (int v4 = 0; v4 < 4; ++v4)
+                            dst[v4] = make_uint4(w4[4 * v4], w4[4 * v4 + 1], w4[4 * v4 + 2], w4[4 * v4 + 3]);
                     }
                 }
-                sum0 = exp_chunk(&s[0], sl2, neg_m_of(m_run), tS, 0);
             }
-#if SDPA_STAGGER
-            if (h == 0 && i == 0) mbar_arrive(bar(C::kBarStagger));
-#endif
-            sum1 = exp_chunk(&s[32], sl2, neg_m_of(m_run), tS, 1);
-            {
-                float a0, a1, b0, b1;
-                f2_unpack(sum0, a0, a1);
-                f2_unpack(sum1, b0, b1);
-                l_run += (a0 + a1) + (b0 + b1);
-            }
-            tmem_wait_st();
+            // O may now be overwritten by the next unit's first product
             tc_fence_before();
-            mbar_arrive(bar(C::kBarPFull + 2 * buf + h));
-        }
-
-        // ---- epilogue: merge the two halves, O -> 16-bit, LSE --------------
-        // stats[g][0][r] = m_g, stats[g][1][r] = l_g
-        if (ok) {
-            stats[(h * 2 + 0) * 128 + r] = m_run;
-            stats[(h * 2 + 1) * 128 + r] = l_run;
-            mbar_arrive(bar(C::kBarXchg));
-            ok = wait_bar(bar(C::kBarXchg), 0, abort_addr, 0x40000u | h);
-            // o_full completes once per CTA, after the last O_0 and O_1 updates
-            ok = ok && wait_bar(bar(C::kBarOFull), 0, abort_addr, 0x41000u | h);
-            ok = __all_sync(0xffffffffu, ok);
-        }
-        if (ok) {
-            tc_fence_after();
-            const float m_0 = stats[0 * 128 + r], l_0 = stats[1 * 128 + r];
-            const float m_1 = stats[2 * 128 + r], l_1 = stats[3 * 128 + r];
-            const float m = fmaxf(m_0, m_1);
-            const float a0 = (m_0 == -INFINITY) ? 0.0f : ex2_approx(m_0 - m);
-            const float a1 = (m_1 == -INFINITY) ? 0.0f : ex2_approx(m_1 - m);
-            const float l = l_0 * a0 + l_1 * a1;
-            const float c0 = a0 * (p.out_mul / l), c1 = a1 * (p.out_mul / l);
-            const bool live = row < p.Sq;
-            const size_t orow = ((size_t)bh * p.Sq + (size_t)(live ? row : 0)) * D;
-            uint16_t* obase = reinterpret_cast<uint16_t*>(p.o) + orow;
-            const uint32_t tO0 = tmem + lane_base + C::kColO0, tO1 = tmem + lane_base + C::kColO1;
-            // group h writes output columns [h * D / 2, (h + 1) * D / 2)
-#pragma unroll 1
-            for (int c = h * (D / 64); c < (h + 1) * (D / 64); ++c) {
-                float x[32], y[32];
-                tmem_ld32(tO0 + 32 * c, x);
-                tmem_ld32(tO1 + 32 * c, y);
-                tmem_wait_ld();
-                reg_fence32(x);
-                reg_fence32(y);
-                uint32_t u[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float v0 = x[2 * e] * c0 + y[2 * e] * c1;
-                    const float v1 = x[2 * e + 1] * c0 + y[2 * e + 1] * c1;
-                    u[e] = (KIND == KIND_FP16) ? pack_f16x2(v0, v1) : pack_bf16x2(v0, v1);
-                }
-                if (live) {
-                    uint4* dst = reinterpret_cast<uint4*>(obase + 32 * c);
-#pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4)
-                        dst[v4] = make_uint4(u[4 * v4], u[4 * v4 + 1], u[4 * v4 + 2], u[4 * v4 + 3]);
-                }
-            }
-            if (h == 0 && p.lse != nullptr && live)
-                p.lse[(size_t)bh * p.Sq + row] = (m + __log2f(l) - C::kPLog2) * kLn2;
+            mbar_arrive(bar(C::kBarOEmpty));
+            unit_next(p, u);
         }
         tc_fence_before();
         named_bar_sync(1, 256 + 32);
