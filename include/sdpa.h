@@ -65,8 +65,12 @@ typedef enum {
                                     unknown dtype, device not sm_100 */
     SDPA_ERR_CUDA = 3,           /* the CUDA runtime or driver reported an
                                     error while preparing or launching */
-    SDPA_ERR_DEVICE_TIMEOUT = 4  /* a kernel's bounded wait expired (reported
+    SDPA_ERR_DEVICE_TIMEOUT = 4, /* a kernel's bounded wait expired (reported
                                     by sdpa_device_status only) */
+    SDPA_ERR_DEVICE_LAYOUT = 5   /* the kernel's shared-memory layout did not
+                                    fit its allocation at the base address the
+                                    device gave it; nothing was computed
+                                    (reported by sdpa_device_status only) */
 } sdpa_status;
 
 /*
@@ -123,7 +127,9 @@ SDPA_API const char* sdpa_strerror(int status);
  * sdpa_device_status -- read (and with clear != 0, reset) the device status
  * word of the current device.  The kernels never trap: a wait that does not
  * complete within about one second stops the kernel and records
- * SDPA_ERR_DEVICE_TIMEOUT here.  *status receives SDPA_OK or that code and
+ * SDPA_ERR_DEVICE_TIMEOUT here; a kernel whose shared-memory layout does not
+ * fit at the base address it was given computes nothing and records
+ * SDPA_ERR_DEVICE_LAYOUT.  *status receives SDPA_OK or one of those codes and
  * *detail a kernel-specific location code (0 when none).  This call
  * synchronises the current device.  Returns SDPA_OK or SDPA_ERR_CUDA.
  */

@@ -16,7 +16,7 @@ import os
 
 __all__ = [
     "SDPA_BF16", "SDPA_FP16", "SDPA_OK", "SDPA_ERR_INVALID_ARG", "SDPA_ERR_UNSUPPORTED",
-    "SDPA_ERR_CUDA", "SDPA_ERR_DEVICE_TIMEOUT", "SdpaError", "LIB_PATH",
+    "SDPA_ERR_CUDA", "SDPA_ERR_DEVICE_TIMEOUT", "SDPA_ERR_DEVICE_LAYOUT", "SdpaError", "LIB_PATH",
     "sdpa_fwd", "sdpa_fwd_fp8", "sdpa_strerror", "sdpa_device_status",
     "sdpa_launches_per_call", "attention", "attention_fp8",
 ]
@@ -25,7 +25,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsdpa_b200.so")
 
 SDPA_BF16, SDPA_FP16 = 0, 1
-SDPA_OK, SDPA_ERR_INVALID_ARG, SDPA_ERR_UNSUPPORTED, SDPA_ERR_CUDA, SDPA_ERR_DEVICE_TIMEOUT = range(5)
+(SDPA_OK, SDPA_ERR_INVALID_ARG, SDPA_ERR_UNSUPPORTED, SDPA_ERR_CUDA, SDPA_ERR_DEVICE_TIMEOUT,
+ SDPA_ERR_DEVICE_LAYOUT) = range(6)
 
 
 class SdpaError(RuntimeError):

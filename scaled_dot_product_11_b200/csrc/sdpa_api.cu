@@ -98,9 +98,9 @@ bool encode_3d(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const voi
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int KIND, int NS, int QB>
-int launch(const void* q, const void* k, const void* v, const FwdParams& prm, cudaStream_t stream) {
-    using C = FwdCfg<D, KIND, NS, QB>;
+template <int D, int KIND, int NS, int QB, bool EPI>
+int launch_cfg(const void* q, const void* k, const void* v, const FwdParams& prm, cudaStream_t stream) {
+    using C = FwdCfg<D, KIND, NS, QB, EPI>;
     const CUtensorMapDataType dt = KIND == sdpa::KIND_BF16   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                    : KIND == sdpa::KIND_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                              : CU_TENSOR_MAP_DATA_TYPE_UINT8;
@@ -109,7 +109,7 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& prm, cu
         !encode_3d(&tk, dt, C::kElem, k, D, prm.Sk, (long long)prm.B * prm.Hkv, C::kElemsPerSw) ||
         !encode_3d(&tv, dt, C::kElem, v, D, prm.Sk, (long long)prm.B * prm.Hkv, C::kElemsPerSw))
         return SDPA_ERR_CUDA;
-    auto kern = sdpa::sdpa_fwd_sm100_kernel<D, KIND, NS, QB>;
+    auto kern = sdpa::sdpa_fwd_sm100_kernel<D, KIND, NS, QB, EPI>;
     static bool attr_set[64];
     int dev = 0;
     cudaGetDevice(&dev);
@@ -121,8 +121,30 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& prm, cu
     }
     // persistent: one CTA per SM (fewer when there are fewer items)
     const unsigned grid = (unsigned)(prm.n_items < sm_count() ? prm.n_items : sm_count());
-    kern<<<grid, sdpa::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, prm);
+    kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, prm);
     return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
+// The separate epilogue warps take the per-unit epilogue off the softmax
+// warps' critical path: measured on B200 this pays when a unit (128 query
+// rows of one head) averages 3 to 24 K/V tiles, and costs a few percent on
+// longer units (and on units of one or two tiles).
+#ifndef SDPA_EPI_MIN_AVG_TILES
+#define SDPA_EPI_MIN_AVG_TILES 3
+#endif
+#ifndef SDPA_EPI_MAX_AVG_TILES
+#define SDPA_EPI_MAX_AVG_TILES 24
+#endif
+bool use_epilogue_warps(const FwdParams& prm) {
+    const int nk = (prm.Sk + 127) / 128;
+    const double avg = prm.causal ? 0.5 * (prm.n_qtiles + 1) : (double)nk;
+    return avg >= SDPA_EPI_MIN_AVG_TILES && avg <= SDPA_EPI_MAX_AVG_TILES;
+}
+
+template <int D, int KIND, int NS, int QB>
+int launch(const void* q, const void* k, const void* v, const FwdParams& prm, cudaStream_t stream) {
+    return use_epilogue_warps(prm) ? launch_cfg<D, KIND, NS, QB, true>(q, k, v, prm, stream)
+                                   : launch_cfg<D, KIND, NS, QB, false>(q, k, v, prm, stream);
 }
 
 FwdParams make_params(void* o, float* lse, int B, int Hq, int Hkv, int Sq, int Sk, int causal) {
@@ -193,6 +215,7 @@ extern "C" const char* sdpa_strerror(int status) {
     case SDPA_ERR_UNSUPPORTED: return "unsupported configuration";
     case SDPA_ERR_CUDA: return "CUDA runtime or driver error";
     case SDPA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case SDPA_ERR_DEVICE_LAYOUT: return "shared-memory layout did not fit at the device's base address";
     default: return "unknown status";
     }
 }

@@ -19,11 +19,18 @@
 // items come in groups of heads so their K/V stay in L2.  The CTA treats the
 // K/V tiles of all its units as one stream, so the scores of the next unit
 // are computed while the current one finishes.  Warp roles (320 threads):
-//   warps 0-3  softmax group 0: keys 0-63 of every tile, thread = row = lane
-//   warps 4-7  softmax group 1: keys 64-127 of every tile
-//   warp  8    TMA producer: Q per unit (double-buffered), K/V tiles in MMA
-//              consumption order K_0, K_1, V_0, K_2, V_1, ... over the stream
-//   warp  9    MMA issuer (one elected lane) and TMEM owner
+//   warps 0-3    softmax group 0: keys 0-63 of every tile, thread = row = lane
+//   warps 4-7    softmax group 1: keys 64-127 of every tile
+//   warps 8-11   (EPI) epilogue: merge the halves of a finished unit,
+//                O -> 16-bit, LSE, while the softmax groups go on with the
+//                next unit; without EPI the softmax groups do it themselves
+//   next warp    TMA producer: Q per unit, K/V tiles in MMA consumption
+//                order K_0, K_1, V_0, K_2, V_1, ... over the stream
+//   last warp    MMA issuer (one elected lane) and TMEM owner
+// With EPI the roles follow warp groups, so that the softmax warp groups can
+// take registers from the epilogue one (setmaxnreg).  EPI pays when units
+// are short (the epilogue leaves the softmax critical path once per unit)
+// and costs a few percent on long ones.
 // Tensor memory (512 columns x 128 lanes, fp32):
 //   [0,128) S_a  [128,256) S_b  [256,256+d) O_0  [384,384+d) O_1
 // S is double-buffered: S(g) of stream tile g lives in S_(g&1), and
@@ -31,7 +38,8 @@
 // next scores are ready when the softmax finishes a tile and the tensor pipe
 // works while the softmax does.  Each softmax group keeps its own running max
 // m_h, sum l_h and output O_h over its half of the keys; the halves never
-// exchange data inside the loop and are merged once per unit:
+// exchange data inside the loop and are merged once per unit, by the
+// epilogue warps:
 //   O = (2^(m_0-m) O_0 + 2^(m_1-m) O_1) / (2^(m_0-m) l_0 + 2^(m_1-m) l_1),
 //   m = max(m_0, m_1),  LSE = (m + log2(2^(m_0-m) l_0 + 2^(m_1-m) l_1)) ln 2.
 // P_h(g) (the weights, packed 2 x 16-bit or 4 x e4m3 per column) overwrites
@@ -71,15 +79,14 @@ enum Kind { KIND_BF16 = 0, KIND_FP16 = 1, KIND_E4M3 = 2 };
 constexpr int kBlockM = 128;        // query rows per unit (= TMEM lanes)
 constexpr int kBlockN = 128;        // keys per K/V tile
 constexpr int kHalfN = 64;          // keys per softmax group
-constexpr int kThreads = 320;       // 10 warps
-constexpr int kLoadWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kEpiWarp0 = 8;        // EPI: warps 8-11, TMEM lane quarters 0-3
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // bounded waits: 1 s
 
-// Device status word: [0] status (0 ok, 4 = device timeout), [1] location.
+// Device status word: [0] status (0 ok, 4 = device timeout, 5 = shared
+// memory layout does not fit the allocation), [1] location.
 __device__ unsigned int g_sdpa_status[2];
 
 struct FwdParams {
@@ -96,8 +103,12 @@ struct FwdParams {
     float out_mul;      // multiplier on (sum_j p_j v_j) / l: the V descale for FP8, else 1
 };
 
-template <int D, int KIND, int NS, int QB>
+template <int D, int KIND, int NS, int QB, bool EPI>
 struct FwdCfg {
+    static constexpr int kThreads = EPI ? 448 : 320;     // 14 or 10 warps
+    static constexpr int kLoadWarp = EPI ? 12 : 8;
+    static constexpr int kMmaWarp = EPI ? 13 : 9;
+    static constexpr int kTmemUsers = 256 + 32 + (EPI ? 128 : 0);   // softmax, MMA, epilogue threads
     static constexpr int kElem = (KIND == KIND_E4M3) ? 1 : 2;
     static constexpr int kRowBytes = D * kElem;
     static constexpr int kElemsPerSw = 128 / kElem;      // elements in one 128-byte swizzle row
@@ -115,8 +126,8 @@ struct FwdCfg {
     // shared memory map (offsets from a 1024-byte aligned base)
     static constexpr int kSmemQ = 0;                      // QB Q tiles
     static constexpr int kSmemKV = QB * kTileBytes;
-    static constexpr int kSmemStats = kSmemKV + NS * kTileBytes;   // [128 rows][2] fp32
-    static constexpr int kSmemBar = kSmemStats + 128 * 2 * 4;
+    static constexpr int kSmemStats = kSmemKV + NS * kTileBytes;   // [2 groups][128 rows][m, l] fp32
+    static constexpr int kSmemBar = kSmemStats + 2 * 128 * 2 * 4;
     // barriers (Q ones: [QB buffers], QB <= 2)
     static constexpr int kBarQFull = 0;
     static constexpr int kBarQEmpty = 2;
@@ -127,18 +138,22 @@ struct FwdCfg {
     static constexpr int kBarODone = 10 + 2 * NS;         // [2 groups], once per tile
     static constexpr int kBarOFull = 12 + 2 * NS;         // once per unit
     static constexpr int kBarOEmpty = 13 + 2 * NS;        // once per unit
-    static constexpr int kBarXchg1 = 14 + 2 * NS;         // group 1 -> group 0, once per unit
-    static constexpr int kBarXchg2 = 15 + 2 * NS;         // group 0 -> group 1, once per unit
-    static constexpr int kBarDrain = 16 + 2 * NS;
-    static constexpr int kNumBars = 17 + 2 * NS;
+    static constexpr int kBarStatsFull = 14 + 2 * NS;     // softmax -> epilogue, once per unit
+    static constexpr int kBarStatsEmpty = 15 + 2 * NS;    // epilogue -> softmax, once per unit
+    static constexpr int kBarXchg1 = 16 + 2 * NS;         // no EPI: group 1 -> group 0, once per unit
+    static constexpr int kBarXchg2 = 17 + 2 * NS;         // no EPI: group 0 -> group 1, once per unit
+    static constexpr int kBarDrain = 18 + 2 * NS;
+    static constexpr int kNumBars = 19 + 2 * NS;
     static constexpr int kSmemTmemSlot = kSmemBar + 8 * kNumBars;
     static constexpr int kSmemAbort = kSmemTmemSlot + 4;
     static constexpr int kSmemUsed = kSmemAbort + 4;
-    static constexpr int kSmemBytes = kSmemUsed + 1024;  // slack for the 1024-byte alignment
+    // slack for the 1024-byte alignment of the tiles, as far as the budget
+    // allows; the kernel checks at entry that its layout fits
+    static constexpr int kSmemBytes = (kSmemUsed + 1024 <= 232448) ? kSmemUsed + 1024 : 232448;
     // TMEM columns
     static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
     static_assert(kRowBytes % 128 == 0, "rows must fill whole 128-byte swizzle rows");
-    static_assert(kSmemBytes <= 232448, "shared memory budget");
+    static_assert(kSmemUsed <= 232448, "shared memory budget");
     static_assert(kSmemBytes > 116 * 1024, "one CTA per SM (each allocates all of TMEM)");
     static_assert(D <= 128, "O tile must fit its 128 TMEM columns");
     static_assert(QB == 1 || QB == 2, "one or two Q buffers");
@@ -181,6 +196,42 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, uint32_t
                                          uint32_t where) {
     if (mbar_try_wait(bar, parity)) return true;
     return wait_bar_slow(bar, parity, abort_addr, where);
+}
+
+// Registers per thread of the softmax and epilogue warp groups (0: leave
+// the launch budget of 65536 / 448 -> 128 each).  The producer and MMA warps
+// keep the launch budget; the sum must stay within the launch allocation.
+#ifndef SDPA_REGS_SOFTMAX
+#define SDPA_REGS_SOFTMAX 152
+#endif
+#ifndef SDPA_REGS_EPILOGUE
+#define SDPA_REGS_EPILOGUE 80
+#endif
+static_assert(SDPA_REGS_SOFTMAX == 0 || 8 * SDPA_REGS_SOFTMAX + 4 * SDPA_REGS_EPILOGUE + 2 * 128 <= 14 * 128,
+              "register split exceeds the launch allocation");
+
+#ifndef SDPA_EPI_SLEEP_NS
+#define SDPA_EPI_SLEEP_NS 256
+#endif
+// As wait_bar, for warps off the critical path: sleeps between polls so that
+// the waiting warp takes no issue slots from the softmax warps.
+__device__ __forceinline__ bool wait_bar_sleep(uint32_t bar, uint32_t parity, uint32_t abort_addr,
+                                               uint32_t where) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t k = 1;; ++k) {
+        __nanosleep(SDPA_EPI_SLEEP_NS);
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((k & 15u) == 0) {
+            if (ld_shared_u32(abort_addr) != 0u) return false;
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                st_shared_u32(abort_addr, 1u);
+                if (atomicCAS(&g_sdpa_status[0], 0u, 4u) == 0u)
+                    atomicExch(&g_sdpa_status[1], where);
+                return false;
+            }
+        }
+    }
 }
 
 // Pairs of one 32-column chunk (e = 0..15) whose exponentials are evaluated
@@ -286,17 +337,25 @@ __device__ __forceinline__ void tile_next(const FwdParams& p, TileCursor& c) {
     }
 }
 
-template <int D, int KIND, int NS, int QB>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, int KIND, int NS, int QB, bool EPI>
+__global__ void __launch_bounds__(FwdCfg<D, KIND, NS, QB, EPI>::kThreads, 1)
 sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV,
                       const FwdParams p) {
-    using C = FwdCfg<D, KIND, NS, QB>;
+    using C = FwdCfg<D, KIND, NS, QB, EPI>;
+    constexpr int kLoadWarp = C::kLoadWarp;
+    constexpr int kMmaWarp = C::kMmaWarp;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
     float* const stats = reinterpret_cast<float*>(smem_raw + (sbase - raw) + C::kSmemStats);
+    // the aligned layout must end inside the allocation (uniform exit)
+    if (sbase - raw + (uint32_t)C::kSmemUsed > (uint32_t)C::kSmemBytes) {
+        if (threadIdx.x == 0 && atomicCAS(&g_sdpa_status[0], 0u, 5u) == 0u)
+            atomicExch(&g_sdpa_status[1], sbase - raw);
+        return;
+    }
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -319,9 +378,11 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             mbar_init(bar(C::kBarKVEmpty + s), 1);
         }
         mbar_init(bar(C::kBarOFull), 1);
-        mbar_init(bar(C::kBarOEmpty), 2 * kBlockM);
+        mbar_init(bar(C::kBarOEmpty), EPI ? kBlockM : 2 * kBlockM);
         mbar_init(bar(C::kBarXchg1), kBlockM);
         mbar_init(bar(C::kBarXchg2), kBlockM);
+        mbar_init(bar(C::kBarStatsFull), 2 * kBlockM);
+        mbar_init(bar(C::kBarStatsEmpty), kBlockM);
         mbar_init(bar(C::kBarDrain), 1);
         st_shared_u32(abort_addr, 0u);
         fence_barrier_init();
@@ -528,13 +589,14 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             while (!mbar_try_wait(bar(C::kBarDrain), 0) && global_timer_ns() - t0 < 100000000ull) {
             }
         }
-        // teardown: the softmax groups have read O for the last time
-        named_bar_sync(1, 256 + 32);
+        // teardown: the softmax and epilogue warps are done with TMEM
+        named_bar_sync(1, C::kTmemUsers);
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     } else if (warp < 8) {
         // ================= softmax groups (warps 0-7) ====================
+        if constexpr (EPI && SDPA_REGS_SOFTMAX > 0) regs_inc<(SDPA_REGS_SOFTMAX > 0 ? SDPA_REGS_SOFTMAX : 128)>();
         const int h = warp >> 2;                 // key half of every tile
         const int quarter = warp & 3;            // TMEM lane quarter of this warp
         const int r = (int)(threadIdx.x & 127);  // row within the unit
@@ -689,42 +751,55 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             }
             if (!ok) break;
 
-            // ---- epilogue of the unit: merge the halves, O -> 16-bit, LSE ----
-            // Group 1 hands (m_1, l_1) to group 0 through `stats`; group 0
-            // computes the merge factors c_0, c_1 and hands them back.
-            const uint32_t xpar = (uint32_t)u.ku & 1u;
-            float c0 = 0.f, c1 = 0.f;
-            if (h == 1) {
-                stats[2 * r] = m_run;
-                stats[2 * r + 1] = l_run;
-                mbar_arrive(bar(C::kBarXchg1));
-                ok = wait_bar(bar(C::kBarXchg2), xpar, abort_addr, 0x40000u | (uint32_t)u.ku);
-                ok = __all_sync(0xffffffffu, ok);
-                c0 = stats[2 * r];
-                c1 = stats[2 * r + 1];
+            if constexpr (EPI) {
+                // ---- end of the unit: hand (m_h, l_h) of every row to the
+                // epilogue warps and go on with the next unit ----
+                if (u.ku > 0) {
+                    ok = wait_bar(bar(C::kBarStatsEmpty), (uint32_t)(u.ku - 1) & 1u, abort_addr,
+                                  0x40000u | (h << 12) | (uint32_t)(u.ku & 0xfff));
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                }
+                stats[(h * kBlockM + r) * 2] = m_run;
+                stats[(h * kBlockM + r) * 2 + 1] = l_run;
+                mbar_arrive(bar(C::kBarStatsFull));
             } else {
-                ok = wait_bar(bar(C::kBarXchg1), xpar, abort_addr, 0x41000u | (uint32_t)u.ku);
-                ok = __all_sync(0xffffffffu, ok);
-                const float m_1 = stats[2 * r], l_1 = stats[2 * r + 1];
-                const float m = fmaxf(m_run, m_1);
-                const float a0 = (m_run == -INFINITY) ? 0.0f : ex2_approx(m_run - m);
-                const float a1 = (m_1 == -INFINITY) ? 0.0f : ex2_approx(m_1 - m);
-                const float l = l_run * a0 + l_1 * a1;
-                c0 = a0 * (p.out_mul / l);
-                c1 = a1 * (p.out_mul / l);
-                stats[2 * r] = c0;
-                stats[2 * r + 1] = c1;
-                mbar_arrive(bar(C::kBarXchg2));
-                if (ok && p.lse != nullptr && row < p.Sq)
-                    p.lse[(size_t)u.bh * p.Sq + row] = (m + __log2f(l) - C::kPLog2) * kLn2;
-            }
-            if (ok) {
-                ok = wait_bar(bar(C::kBarOFull), xpar, abort_addr, 0x42000u | (uint32_t)u.ku);
-                ok = __all_sync(0xffffffffu, ok);
-            }
-            if (!ok) break;
-            tc_fence_after();
-            {
+                // ---- epilogue of the unit: merge the halves, O -> 16-bit,
+                // LSE.  Group 1 hands (m_1, l_1) to group 0 through `stats`;
+                // group 0 computes the merge factors c_0, c_1 and hands them
+                // back; each group writes half of O's columns. ----
+                const uint32_t xpar = (uint32_t)u.ku & 1u;
+                float c0 = 0.f, c1 = 0.f;
+                if (h == 1) {
+                    stats[2 * r] = m_run;
+                    stats[2 * r + 1] = l_run;
+                    mbar_arrive(bar(C::kBarXchg1));
+                    ok = wait_bar(bar(C::kBarXchg2), xpar, abort_addr, 0x43000u | (uint32_t)(u.ku & 0xfff));
+                    ok = __all_sync(0xffffffffu, ok);
+                    c0 = stats[2 * r];
+                    c1 = stats[2 * r + 1];
+                } else {
+                    ok = wait_bar(bar(C::kBarXchg1), xpar, abort_addr, 0x44000u | (uint32_t)(u.ku & 0xfff));
+                    ok = __all_sync(0xffffffffu, ok);
+                    const float m_1 = stats[2 * r], l_1 = stats[2 * r + 1];
+                    const float m = fmaxf(m_run, m_1);
+                    const float a0 = (m_run == -INFINITY) ? 0.0f : ex2_approx(m_run - m);
+                    const float a1 = (m_1 == -INFINITY) ? 0.0f : ex2_approx(m_1 - m);
+                    const float l = l_run * a0 + l_1 * a1;
+                    c0 = a0 * (p.out_mul / l);
+                    c1 = a1 * (p.out_mul / l);
+                    stats[2 * r] = c0;
+                    stats[2 * r + 1] = c1;
+                    mbar_arrive(bar(C::kBarXchg2));
+                    if (ok && p.lse != nullptr && row < p.Sq)
+                        p.lse[(size_t)u.bh * p.Sq + row] = (m + __log2f(l) - C::kPLog2) * kLn2;
+                }
+                if (ok) {
+                    ok = wait_bar(bar(C::kBarOFull), xpar, abort_addr, 0x45000u | (uint32_t)(u.ku & 0xfff));
+                    ok = __all_sync(0xffffffffu, ok);
+                }
+                if (!ok) break;
+                tc_fence_after();
                 const bool live = row < p.Sq;
                 const size_t orow = ((size_t)u.bh * p.Sq + (size_t)(live ? row : 0)) * D;
                 uint16_t* obase = reinterpret_cast<uint16_t*>(p.o) + orow;
@@ -752,15 +827,83 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                             dst[v4] = make_uint4(w4[4 * v4], w4[4 * v4 + 1], w4[4 * v4 + 2], w4[4 * v4 + 3]);
                     }
                 }
+                // O may now be overwritten by the next unit's first product
+                tc_fence_before();
+                mbar_arrive(bar(C::kBarOEmpty));
             }
-            // O may now be overwritten by the next unit's first product
-            tc_fence_before();
-            mbar_arrive(bar(C::kBarOEmpty));
             unit_next(p, u);
         }
         tc_fence_before();
-        named_bar_sync(1, 256 + 32);
+        named_bar_sync(1, C::kTmemUsers);
+    } else if (EPI && warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
+        // ================= epilogue (warps 8-11) =========================
+        if constexpr (EPI && SDPA_REGS_SOFTMAX > 0) regs_dec<(SDPA_REGS_SOFTMAX > 0 ? SDPA_REGS_EPILOGUE : 128)>();
+        // Per unit: O = (2^(m_0-m) O_0 + 2^(m_1-m) O_1) / l with l the
+        // halves' sums on the common max m; O is read from this warp's TMEM
+        // lane quarter, rounded to 16 bits and stored, then LSE.
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;       // row within the unit = TMEM lane
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        const uint32_t tO0 = tmem + lane_base + C::kColO0, tO1 = tmem + lane_base + C::kColO1;
+        bool ok = true;
+        UnitCursor u;
+        unit_first(p, u);
+        while (ok && u.valid) {
+            const uint32_t par = (uint32_t)u.ku & 1u;
+            ok = wait_bar_sleep(bar(C::kBarStatsFull), par, abort_addr, 0x41000u | (uint32_t)(u.ku & 0xfff));
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            const float m_0 = stats[r * 2], l_0 = stats[r * 2 + 1];
+            const float m_1 = stats[(kBlockM + r) * 2], l_1 = stats[(kBlockM + r) * 2 + 1];
+            mbar_arrive(bar(C::kBarStatsEmpty));
+            const float m = fmaxf(m_0, m_1);
+            const float a0 = (m_0 == -INFINITY) ? 0.0f : ex2_approx(m_0 - m);
+            const float a1 = (m_1 == -INFINITY) ? 0.0f : ex2_approx(m_1 - m);
+            const float l = l_0 * a0 + l_1 * a1;
+            const float c0 = a0 * (p.out_mul / l);
+            const float c1 = a1 * (p.out_mul / l);
+            const int row = u.qtile * kBlockM + r;
+            const bool live = row < p.Sq;
+            if (live && p.lse != nullptr)
+                p.lse[(size_t)u.bh * p.Sq + row] = (m + __log2f(l) - C::kPLog2) * kLn2;
+            ok = wait_bar_sleep(bar(C::kBarOFull), par, abort_addr, 0x42000u | (uint32_t)(u.ku & 0xfff));
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            const size_t orow = ((size_t)u.bh * p.Sq + (size_t)(live ? row : 0)) * D;
+            uint16_t* obase = reinterpret_cast<uint16_t*>(p.o) + orow;
+#pragma unroll 1
+            for (int c = 0; c < D / 16; ++c) {
+                float x[16], y[16];
+                tmem_ld16(tO0 + 16 * c, x);
+                tmem_ld16(tO1 + 16 * c, y);
+                tmem_wait_ld();
+                reg_fence16(x);
+                reg_fence16(y);
+                if (c == D / 16 - 1) {
+                    // O is read: the next unit's first product may overwrite it
+                    tc_fence_before();
+                    mbar_arrive(bar(C::kBarOEmpty));
+                }
+                uint32_t w4[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float v0 = x[2 * e] * c0 + y[2 * e] * c1;
+                    const float v1 = x[2 * e + 1] * c0 + y[2 * e + 1] * c1;
+                    w4[e] = (KIND == KIND_FP16) ? pack_f16x2(v0, v1) : pack_bf16x2(v0, v1);
+                }
+                if (live) {
+                    uint4* dst = reinterpret_cast<uint4*>(obase + 16 * c);
+                    dst[0] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    dst[1] = make_uint4(w4[4], w4[5], w4[6], w4[7]);
+                }
+            }
+            unit_next(p, u);
+        }
+        tc_fence_before();
+        named_bar_sync(1, C::kTmemUsers);
     }
 }
+
 
 }  // namespace sdpa

@@ -117,6 +117,12 @@ SMALL = [
     (1, 2, 2, 100, 300, 128, False),
     (1, 2, 2, 300, 77, 64, False),
     (1, 1, 1, 513, 1000, 128, False),
+    # units of 128 query rows averaging 3-24 K/V tiles run the kernel form
+    # with separate epilogue warps; shorter and longer ones (such as these
+    # three) the form whose softmax warps write O themselves
+    (1, 2, 2, 200, 3200, 128, False),
+    (1, 4, 2, 130, 3329, 128, False),
+    (1, 2, 2, 100, 3100, 64, False),
 ]
 
 
@@ -252,7 +258,7 @@ def run_fp8(lib, w):
 
 
 @pytest.mark.parametrize("shape", [(1, 2, 2, 256, 256, True), (1, 2, 1, 333, 333, True),
-                                   (2, 4, 2, 200, 500, False)])
+                                   (2, 4, 2, 200, 500, False), (1, 2, 2, 150, 3300, False)])
 def test_fp8_small(sdpa, shape):
     B, Hq, Hkv, Sq, Sk, causal = shape
     w = Workload("f8", B, Hq, Hkv, Sq, Sk, 128, causal, dtype="e4m3", seed=Sq + Sk)
