@@ -96,6 +96,30 @@ SDPA_API int sdpa_fwd(const void* q, const void* k, const void* v, void* o, floa
              float scale, int causal, int dtype, void* stream);
 
 /*
+ * sdpa_fwd_strided -- sdpa_fwd on strided views, so that the codelab's
+ * [batch, time, heads, head_dim] layout (the layout JAX expects; codelab
+ * "JAX on GPU, Lab 5: attention on GPU", section 3, the table of array
+ * dimensions) or any other layout whose head_dim elements are contiguous is
+ * read and written in place, with no transpose copy.
+ *
+ *   q_strides, k_strides, v_strides, o_strides
+ *       host arrays of three element strides each: {batch, head, row} of
+ *       the [B,H,S,d] view (d contiguous).  For BTNH data [B,T,N,d] they
+ *       are {T*N*d, d, N*d}.  Every stride is positive and its byte size a
+ *       multiple of 16, else SDPA_ERR_INVALID_ARG.  The library reads the
+ *       arrays during the call only.
+ *   lse  stays contiguous [B,Hq,Sq] float32 (or NULL).
+ *
+ * The other arguments, results and errors are those of sdpa_fwd.  O must
+ * not overlap Q, K or V.
+ */
+SDPA_API int sdpa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
+                              int B, int Hq, int Hkv, int Sq, int Sk, int d,
+                              const long long* q_strides, const long long* k_strides,
+                              const long long* v_strides, const long long* o_strides,
+                              float scale, int causal, int dtype, void* stream);
+
+/*
  * sdpa_fwd_fp8 -- the same forward with FP8 E4M3 ("fn", max 448) Q/K/V.
  *
  * The codelab runs attention in E4M3 for the forward pass with per-tensor

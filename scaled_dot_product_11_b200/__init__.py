@@ -17,7 +17,7 @@ import os
 __all__ = [
     "SDPA_BF16", "SDPA_FP16", "SDPA_OK", "SDPA_ERR_INVALID_ARG", "SDPA_ERR_UNSUPPORTED",
     "SDPA_ERR_CUDA", "SDPA_ERR_DEVICE_TIMEOUT", "SDPA_ERR_DEVICE_LAYOUT", "SdpaError", "LIB_PATH",
-    "sdpa_fwd", "sdpa_fwd_fp8", "sdpa_strerror", "sdpa_device_status",
+    "sdpa_fwd", "sdpa_fwd_strided", "sdpa_fwd_fp8", "sdpa_strerror", "sdpa_device_status",
     "sdpa_launches_per_call", "attention", "attention_fp8",
 ]
 
@@ -44,6 +44,10 @@ _lib = ctypes.CDLL(LIB_PATH)
 _vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 _lib.sdpa_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _vp]
 _lib.sdpa_fwd.restype = _i
+_ll3 = ctypes.c_longlong * 3
+_lib.sdpa_fwd_strided.argtypes = ([_vp] * 5 + [_i] * 6 + [ctypes.POINTER(ctypes.c_longlong)] * 4
+                                  + [_f, _i, _i, _vp])
+_lib.sdpa_fwd_strided.restype = _i
 _lib.sdpa_fwd_fp8.argtypes = [_vp, _vp, _vp, _f, _f, _f, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]
 _lib.sdpa_fwd_fp8.restype = _i
 _lib.sdpa_strerror.argtypes = [_i]
@@ -61,6 +65,15 @@ def sdpa_fwd(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal, dtype, strea
     stream an int cudaStream_t (0 = default stream).  Returns the status."""
     return int(_lib.sdpa_fwd(q, k, v, o, lse or None, B, Hq, Hkv, Sq, Sk, d, float(scale),
                              int(causal), int(dtype), stream or None))
+
+
+def sdpa_fwd_strided(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, q_strides, k_strides, v_strides,
+                     o_strides, scale, causal, dtype, stream) -> int:
+    """Raw call with element strides (batch, head, row) per tensor, each a
+    sequence of three ints."""
+    st = [_ll3(*[int(x) for x in t]) for t in (q_strides, k_strides, v_strides, o_strides)]
+    return int(_lib.sdpa_fwd_strided(q, k, v, o, lse or None, B, Hq, Hkv, Sq, Sk, d, *st,
+                                     float(scale), int(causal), int(dtype), stream or None))
 
 
 def sdpa_fwd_fp8(q8, k8, v8, descale_q, descale_k, descale_v, o, lse, B, Hq, Hkv, Sq, Sk, d,
@@ -89,7 +102,7 @@ def sdpa_launches_per_call() -> int:
 
 # ---- torch conveniences -------------------------------------------------------
 
-def _dims(q, k, v):
+def _dims(q, k, v, allow_views=False):
     if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
         raise ValueError("q, k, v must be 4-D [B, H, S, d]")
     B, Hq, Sq, d = q.shape
@@ -98,8 +111,11 @@ def _dims(q, k, v):
         raise ValueError("shape mismatch: q %s k %s v %s" % (tuple(q.shape), tuple(k.shape),
                                                               tuple(v.shape)))
     for t in (q, k, v):
-        if not t.is_cuda or not t.is_contiguous():
-            raise ValueError("q, k, v must be contiguous CUDA tensors")
+        if not t.is_cuda:
+            raise ValueError("q, k, v must be CUDA tensors")
+        if not (t.is_contiguous() or (allow_views and t.stride(3) == 1)):
+            raise ValueError("q, k, v must be contiguous CUDA tensors%s" % (
+                " or views whose last dimension is contiguous" if allow_views else ""))
     return int(B), int(Hq), int(Hkv), int(Sq), int(Sk), int(d)
 
 
@@ -112,10 +128,13 @@ def _stream_handle(stream):
 def attention(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
               return_lse: bool = True, stream=None):
     """O (and LSE) = softmax(q k^T * scale [causal]) v for bf16 / fp16 CUDA
-    tensors q [B,Hq,Sq,d], k/v [B,Hkv,Sk,d].  Enqueued on `stream` (default:
+    tensors q [B,Hq,Sq,d], k/v [B,Hkv,Sk,d].  They may be strided views
+    whose last dimension is contiguous, e.g. BTNH data passed as
+    x.transpose(1, 2): those go through sdpa_fwd_strided, in place.  `out`
+    defaults to a tensor laid out like q.  Enqueued on `stream` (default:
     torch's current stream); raises SdpaError on a refused call."""
     import torch
-    B, Hq, Hkv, Sq, Sk, d = _dims(q, k, v)
+    B, Hq, Hkv, Sq, Sk, d = _dims(q, k, v, allow_views=True)
     if q.dtype not in (torch.bfloat16, torch.float16) or k.dtype != q.dtype or v.dtype != q.dtype:
         raise ValueError("q, k, v must share dtype bfloat16 or float16")
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
@@ -124,12 +143,22 @@ def attention(q, k, v, causal: bool = False, scale: float | None = None, out=Non
             out = torch.empty_like(q)
         if lse is None and return_lse:
             lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
-        rc = sdpa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                      lse.data_ptr() if lse is not None else 0, B, Hq, Hkv, Sq, Sk, d, scale,
-                      causal, SDPA_BF16 if q.dtype == torch.bfloat16 else SDPA_FP16,
-                      _stream_handle(stream))
+        dt = SDPA_BF16 if q.dtype == torch.bfloat16 else SDPA_FP16
+        lp = lse.data_ptr() if lse is not None else 0
+        if all(t.is_contiguous() for t in (q, k, v, out)):
+            what = "sdpa_fwd"
+            rc = sdpa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lp,
+                          B, Hq, Hkv, Sq, Sk, d, scale, causal, dt, _stream_handle(stream))
+        else:
+            what = "sdpa_fwd_strided"
+            if tuple(out.shape) != (B, Hq, Sq, d) or out.stride(3) != 1:
+                raise ValueError("out must be [B, Hq, Sq, d] with a contiguous last dimension")
+            rc = sdpa_fwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lp,
+                                  B, Hq, Hkv, Sq, Sk, d, q.stride()[:3], k.stride()[:3],
+                                  v.stride()[:3], out.stride()[:3], scale, causal, dt,
+                                  _stream_handle(stream))
     if rc != SDPA_OK:
-        raise SdpaError(rc, "sdpa_fwd")
+        raise SdpaError(rc, what)
     return (out, lse) if return_lse else out
 
 

@@ -85,31 +85,59 @@ int check_args(const void* q, const void* k, const void* v, const void* o, const
     return SDPA_OK;
 }
 
-bool encode_3d(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* base, int d,
-               int rows, long long heads, int box_inner) {
+// Element strides (batch, head, row) of a [B, H, S, d] view, d contiguous.
+struct View {
+    long long sb, sh, ss;
+};
+View bhsd(int H, int S, int d) {
+    return View{(long long)H * S * d, (long long)S * d, (long long)d};
+}
+
+bool same(const View& a, const View& b) { return a.sb == b.sb && a.sh == b.sh && a.ss == b.ss; }
+
+// Tiled map over (d, S, H, B) with the view's strides -- 3-D (d, S, B*H) for
+// contiguous [B,H,S,d] data (`rank3`); boxes of box_inner x 128 rows of one
+// (head, batch), 128-byte swizzle.
+bool encode_view(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* base, int d,
+                 int rows, int heads, int batch, const View& v, int box_inner, bool rank3) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
-    const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)heads};
-    const cuuint64_t strides[2] = {(cuuint64_t)d * elem_bytes, (cuuint64_t)d * elem_bytes * rows};
-    const cuuint32_t box[3] = {(cuuint32_t)box_inner, 128u, 1u};
-    const cuuint32_t estr[3] = {1u, 1u, 1u};
-    return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+    const cuuint32_t rank = rank3 ? 3u : 4u;
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)heads, (cuuint64_t)batch};
+    cuuint64_t strides[3] = {(cuuint64_t)(v.ss * elem_bytes), (cuuint64_t)(v.sh * elem_bytes),
+                             (cuuint64_t)(v.sb * elem_bytes)};
+    if (rank == 3) dims[2] = (cuuint64_t)heads * (cuuint64_t)batch;
+    const cuuint32_t box[4] = {(cuuint32_t)box_inner, 128u, 1u, 1u};
+    const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    return fn(m, dt, rank, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int KIND, int NS, int QB, bool EPI>
-int launch_cfg(const void* q, const void* k, const void* v, const FwdParams& prm, cudaStream_t stream) {
+// A view the kernel can address: positive strides whose byte sizes are
+// multiples of 16 (TMA and the 16-byte output stores) and below 2^40.
+bool view_ok(const long long* st, int elem_bytes) {
+    if (!st) return false;
+    for (int i = 0; i < 3; ++i) {
+        if (st[i] <= 0 || st[i] > (1LL << 40) / elem_bytes) return false;
+        if ((st[i] * elem_bytes) % 16 != 0) return false;
+    }
+    return true;
+}
+
+template <int D, int KIND, int NS, int QB, bool EPI, bool STRIDED>
+int launch_cfg(const void* q, const void* k, const void* v, const View& vq, const View& vk,
+               const View& vv, const FwdParams& prm, cudaStream_t stream) {
     using C = FwdCfg<D, KIND, NS, QB, EPI>;
     const CUtensorMapDataType dt = KIND == sdpa::KIND_BF16   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                    : KIND == sdpa::KIND_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                              : CU_TENSOR_MAP_DATA_TYPE_UINT8;
     CUtensorMap tq, tk, tv;
-    if (!encode_3d(&tq, dt, C::kElem, q, D, prm.Sq, (long long)prm.B * prm.Hq, C::kElemsPerSw) ||
-        !encode_3d(&tk, dt, C::kElem, k, D, prm.Sk, (long long)prm.B * prm.Hkv, C::kElemsPerSw) ||
-        !encode_3d(&tv, dt, C::kElem, v, D, prm.Sk, (long long)prm.B * prm.Hkv, C::kElemsPerSw))
+    if (!encode_view(&tq, dt, C::kElem, q, D, prm.Sq, prm.Hq, prm.B, vq, C::kElemsPerSw, !STRIDED) ||
+        !encode_view(&tk, dt, C::kElem, k, D, prm.Sk, prm.Hkv, prm.B, vk, C::kElemsPerSw, !STRIDED) ||
+        !encode_view(&tv, dt, C::kElem, v, D, prm.Sk, prm.Hkv, prm.B, vv, C::kElemsPerSw, !STRIDED))
         return SDPA_ERR_CUDA;
-    auto kern = sdpa::sdpa_fwd_sm100_kernel<D, KIND, NS, QB, EPI>;
+    auto kern = sdpa::sdpa_fwd_sm100_kernel<D, KIND, NS, QB, EPI, STRIDED>;
     static bool attr_set[64];
     int dev = 0;
     cudaGetDevice(&dev);
@@ -141,15 +169,34 @@ bool use_epilogue_warps(const FwdParams& prm) {
     return avg >= SDPA_EPI_MIN_AVG_TILES && avg <= SDPA_EPI_MAX_AVG_TILES;
 }
 
-template <int D, int KIND, int NS, int QB>
-int launch(const void* q, const void* k, const void* v, const FwdParams& prm, cudaStream_t stream) {
-    return use_epilogue_warps(prm) ? launch_cfg<D, KIND, NS, QB, true>(q, k, v, prm, stream)
-                                   : launch_cfg<D, KIND, NS, QB, false>(q, k, v, prm, stream);
+// STRIDED kernels address Q/K/V through 4-D maps and O through its strides;
+// contiguous [B,H,S,d] data takes the 3-D form, measured ~5% faster.
+template <int D, int KIND, int NS, int QB, bool STRIDED>
+int launch_form(const void* q, const void* k, const void* v, const View& vq, const View& vk,
+                const View& vv, const FwdParams& prm, cudaStream_t stream) {
+    return use_epilogue_warps(prm)
+               ? launch_cfg<D, KIND, NS, QB, true, STRIDED>(q, k, v, vq, vk, vv, prm, stream)
+               : launch_cfg<D, KIND, NS, QB, false, STRIDED>(q, k, v, vq, vk, vv, prm, stream);
 }
 
-FwdParams make_params(void* o, float* lse, int B, int Hq, int Hkv, int Sq, int Sk, int causal) {
+template <int D, int KIND, int NS, int QB>
+int launch(const void* q, const void* k, const void* v, const View& vq, const View& vk, const View& vv,
+           const FwdParams& prm, cudaStream_t stream) {
+    const bool contiguous = same(vq, bhsd(prm.Hq, prm.Sq, D)) && same(vk, bhsd(prm.Hkv, prm.Sk, D)) &&
+                            same(vv, bhsd(prm.Hkv, prm.Sk, D)) &&
+                            prm.o_sb == (long long)prm.Hq * prm.Sq * D && prm.o_sh == (long long)prm.Sq * D &&
+                            prm.o_ss == D;
+    return contiguous ? launch_form<D, KIND, NS, QB, false>(q, k, v, vq, vk, vv, prm, stream)
+                      : launch_form<D, KIND, NS, QB, true>(q, k, v, vq, vk, vv, prm, stream);
+}
+
+FwdParams make_params(void* o, const View& vo, float* lse, int B, int Hq, int Hkv, int Sq, int Sk,
+                      int causal) {
     FwdParams prm;
     prm.o = o;
+    prm.o_sb = vo.sb;
+    prm.o_sh = vo.sh;
+    prm.o_ss = vo.ss;
     prm.lse = lse;
     prm.B = B;
     prm.Hq = Hq;
@@ -171,24 +218,46 @@ FwdParams make_params(void* o, float* lse, int B, int Hq, int Hkv, int Sq, int S
     return prm;
 }
 
+int fwd_16bit(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+              int Hkv, int Sq, int Sk, int d, const View& vq, const View& vk, const View& vv,
+              const View& vo, float scale, int causal, int dtype, void* stream) {
+    if (dtype != SDPA_BF16 && dtype != SDPA_FP16) return SDPA_ERR_UNSUPPORTED;
+    int rc = check_device();
+    if (rc != SDPA_OK) return rc;
+    FwdParams prm = make_params(o, vo, lse, B, Hq, Hkv, Sq, Sk, causal);
+    prm.score_log2 = scale * sdpa::kLog2e;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (dtype == SDPA_BF16)
+        return d == 64 ? launch<64, sdpa::KIND_BF16, SDPA_STAGES_D64, 2>(q, k, v, vq, vk, vv, prm, s)
+                       : launch<128, sdpa::KIND_BF16, SDPA_STAGES_D128, 1>(q, k, v, vq, vk, vv, prm, s);
+    return d == 64 ? launch<64, sdpa::KIND_FP16, SDPA_STAGES_D64, 2>(q, k, v, vq, vk, vv, prm, s)
+                   : launch<128, sdpa::KIND_FP16, SDPA_STAGES_D128, 1>(q, k, v, vq, vk, vv, prm, s);
+}
+
 }  // namespace
 
 extern "C" int sdpa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                         int Hq, int Hkv, int Sq, int Sk, int d, float scale, int causal, int dtype,
                         void* stream) {
-    int rc = check_args(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal);
+    const int rc = check_args(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal);
     if (rc != SDPA_OK) return rc;
-    if (dtype != SDPA_BF16 && dtype != SDPA_FP16) return SDPA_ERR_UNSUPPORTED;
-    rc = check_device();
+    return fwd_16bit(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, bhsd(Hq, Sq, d), bhsd(Hkv, Sk, d),
+                     bhsd(Hkv, Sk, d), bhsd(Hq, Sq, d), scale, causal, dtype, stream);
+}
+
+extern "C" int sdpa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
+                                int B, int Hq, int Hkv, int Sq, int Sk, int d,
+                                const long long* q_strides, const long long* k_strides,
+                                const long long* v_strides, const long long* o_strides, float scale,
+                                int causal, int dtype, void* stream) {
+    const int rc = check_args(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal);
     if (rc != SDPA_OK) return rc;
-    FwdParams prm = make_params(o, lse, B, Hq, Hkv, Sq, Sk, causal);
-    prm.score_log2 = scale * sdpa::kLog2e;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (dtype == SDPA_BF16)
-        return d == 64 ? launch<64, sdpa::KIND_BF16, SDPA_STAGES_D64, 2>(q, k, v, prm, s)
-                       : launch<128, sdpa::KIND_BF16, SDPA_STAGES_D128, 1>(q, k, v, prm, s);
-    return d == 64 ? launch<64, sdpa::KIND_FP16, SDPA_STAGES_D64, 2>(q, k, v, prm, s)
-                   : launch<128, sdpa::KIND_FP16, SDPA_STAGES_D128, 1>(q, k, v, prm, s);
+    if (!view_ok(q_strides, 2) || !view_ok(k_strides, 2) || !view_ok(v_strides, 2) ||
+        !view_ok(o_strides, 2))
+        return SDPA_ERR_INVALID_ARG;
+    auto view = [](const long long* st) { return View{st[0], st[1], st[2]}; };
+    return fwd_16bit(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, view(q_strides), view(k_strides),
+                     view(v_strides), view(o_strides), scale, causal, dtype, stream);
 }
 
 extern "C" int sdpa_fwd_fp8(const void* q8, const void* k8, const void* v8, float descale_q,
@@ -201,11 +270,12 @@ extern "C" int sdpa_fwd_fp8(const void* q8, const void* k8, const void* v8, floa
     if (d != 128) return SDPA_ERR_UNSUPPORTED;
     rc = check_device();
     if (rc != SDPA_OK) return rc;
-    FwdParams prm = make_params(o, lse, B, Hq, Hkv, Sq, Sk, causal);
+    FwdParams prm = make_params(o, bhsd(Hq, Sq, d), lse, B, Hq, Hkv, Sq, Sk, causal);
     prm.score_log2 = scale * descale_q * descale_k * sdpa::kLog2e;
     prm.out_mul = descale_v;
-    return launch<128, sdpa::KIND_E4M3, SDPA_STAGES_FP8, 2>(q8, k8, v8, prm,
-                                                            reinterpret_cast<cudaStream_t>(stream));
+    return launch<128, sdpa::KIND_E4M3, SDPA_STAGES_FP8, 2>(
+        q8, k8, v8, bhsd(Hq, Sq, d), bhsd(Hkv, Sk, d), bhsd(Hkv, Sk, d), prm,
+        reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" const char* sdpa_strerror(int status) {

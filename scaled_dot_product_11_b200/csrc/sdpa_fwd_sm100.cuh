@@ -90,8 +90,8 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // bounded waits: 1 s
 __device__ unsigned int g_sdpa_status[2];
 
 struct FwdParams {
-    void* o;            // [B,Hq,Sq,D] 16-bit
-    float* lse;         // [B,Hq,Sq] or null
+    void* o;            // [B,Hq,Sq,D] view, 16-bit, D contiguous (strides below)
+    float* lse;         // [B,Hq,Sq] contiguous, or null
     int B, Hq, Hkv, Sq, Sk;
     int group;          // Hq / Hkv
     int n_qtiles;       // ceil(Sq / 128)
@@ -101,6 +101,7 @@ struct FwdParams {
     int causal;
     float score_log2;   // multiplier from raw MMA score to log2 units
     float out_mul;      // multiplier on (sum_j p_j v_j) / l: the V descale for FP8, else 1
+    long long o_sb, o_sh, o_ss;   // O's batch, head, row strides in elements (STRIDED)
 };
 
 template <int D, int KIND, int NS, int QB, bool EPI>
@@ -252,6 +253,18 @@ __device__ __forceinline__ float chunk_max32(const float* s) {
     return fmaxf(a, b);
 }
 
+// Element offset of row `row` of (batch, head) pair bh in O: contiguous
+// [B,Hq,Sq,D], or the strided view.
+template <int D, bool STRIDED>
+__device__ __forceinline__ long long o_offset(const FwdParams& p, int bh, int row) {
+    if constexpr (STRIDED) {
+        const int b = bh / p.Hq;
+        return (long long)b * p.o_sb + (long long)(bh - b * p.Hq) * p.o_sh + (long long)row * p.o_ss;
+    } else {
+        return ((long long)bh * p.Sq + row) * D;
+    }
+}
+
 // Number of K/V tiles the query rows [row0, row0 + 128) need.
 __device__ __forceinline__ int tiles_for(int row0, int Sq, int Sk, int causal) {
     if (row0 >= Sq) return 0;
@@ -337,7 +350,7 @@ __device__ __forceinline__ void tile_next(const FwdParams& p, TileCursor& c) {
     }
 }
 
-template <int D, int KIND, int NS, int QB, bool EPI>
+template <int D, int KIND, int NS, int QB, bool EPI, bool STRIDED>
 __global__ void __launch_bounds__(FwdCfg<D, KIND, NS, QB, EPI>::kThreads, 1)
 sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
@@ -422,10 +435,17 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                                   abort_addr, 0x11000u | (uint32_t)c.u.ku))
                         return false;
                     mbar_arrive_expect_tx(bar(C::kBarQFull + qb), C::kTileBytes);
-                    for (int kb = 0; kb < C::kSwBlocks; ++kb)
-                        tma_load_3d(sQ + qb * C::kTileBytes + kb * C::kSwBlockBytes, &tmQ,
-                                    bar(C::kBarQFull + qb), kb * C::kElemsPerSw,
-                                    c.u.qtile * kBlockM, c.u.bh);
+                    for (int kb = 0; kb < C::kSwBlocks; ++kb) {
+                        const uint32_t dst = sQ + qb * C::kTileBytes + kb * C::kSwBlockBytes;
+                        if constexpr (STRIDED) {
+                            const int qbat = c.u.bh / p.Hq;
+                            tma_load_4d(dst, &tmQ, bar(C::kBarQFull + qb), kb * C::kElemsPerSw,
+                                        c.u.qtile * kBlockM, c.u.bh - qbat * p.Hq, qbat);
+                        } else {
+                            tma_load_3d(dst, &tmQ, bar(C::kBarQFull + qb), kb * C::kElemsPerSw,
+                                        c.u.qtile * kBlockM, c.u.bh);
+                        }
+                    }
                     q_last = c.u.ku;
                 }
                 const int slot = t % NS;
@@ -433,12 +453,18 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                               0x10000u | (uint32_t)t))
                     return false;
                 const int b = c.u.bh / p.Hq;
-                const int kvh = b * p.Hkv + (c.u.bh - b * p.Hq) / p.group;
+                const int kvh = (c.u.bh - b * p.Hq) / p.group;   // K/V head of the group
                 const uint32_t fb = bar(C::kBarKVFull + slot);
                 mbar_arrive_expect_tx(fb, C::kTileBytes);
-                for (int kb = 0; kb < C::kSwBlocks; ++kb)
-                    tma_load_3d(sKV + slot * C::kTileBytes + kb * C::kSwBlockBytes,
-                                is_v ? &tmV : &tmK, fb, kb * C::kElemsPerSw, c.i * kBlockN, kvh);
+                for (int kb = 0; kb < C::kSwBlocks; ++kb) {
+                    if constexpr (STRIDED)
+                        tma_load_4d(sKV + slot * C::kTileBytes + kb * C::kSwBlockBytes,
+                                    is_v ? &tmV : &tmK, fb, kb * C::kElemsPerSw, c.i * kBlockN, kvh, b);
+                    else
+                        tma_load_3d(sKV + slot * C::kTileBytes + kb * C::kSwBlockBytes,
+                                    is_v ? &tmV : &tmK, fb, kb * C::kElemsPerSw, c.i * kBlockN,
+                                    b * p.Hkv + kvh);
+                }
                 ++t;
                 return true;
             };
@@ -801,8 +827,7 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 if (!ok) break;
                 tc_fence_after();
                 const bool live = row < p.Sq;
-                const size_t orow = ((size_t)u.bh * p.Sq + (size_t)(live ? row : 0)) * D;
-                uint16_t* obase = reinterpret_cast<uint16_t*>(p.o) + orow;
+                uint16_t* obase = reinterpret_cast<uint16_t*>(p.o) + o_offset<D, STRIDED>(p, u.bh, live ? row : 0);
                 const uint32_t tO0 = tmem + lane_base + C::kColO0, tO1 = tmem + lane_base + C::kColO1;
                 // group h writes output columns [h * D / 2, (h + 1) * D / 2)
 #pragma unroll 1
@@ -870,8 +895,7 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-            const size_t orow = ((size_t)u.bh * p.Sq + (size_t)(live ? row : 0)) * D;
-            uint16_t* obase = reinterpret_cast<uint16_t*>(p.o) + orow;
+            uint16_t* obase = reinterpret_cast<uint16_t*>(p.o) + o_offset<D, STRIDED>(p, u.bh, live ? row : 0);
 #pragma unroll 1
             for (int c = 0; c < D / 16; ++c) {
                 float x[16], y[16];

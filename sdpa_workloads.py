@@ -113,6 +113,19 @@ def make_qkv(w: Workload, device="cpu"):
     return q.to(device), k.to(device), v.to(device)
 
 
+def make_qkv_btnh(w: Workload, device="cpu"):
+    """(q, k, v) in the codelab's [batch, time, heads, head_dim] layout
+    (q [B,Sq,Hq,d], k/v [B,Sk,Hkv,d]), drawn on the CPU from w.seed."""
+    if w.dtype not in _TORCH_DTYPES:
+        raise ValueError("make_qkv_btnh: bf16 / fp16 only, not %s" % w.dtype)
+    g = torch.Generator(device="cpu").manual_seed(w.seed)
+    dt = _TORCH_DTYPES[w.dtype]
+    q = torch.randn(w.B, w.Sq, w.Hq, w.d, generator=g, dtype=torch.float32).to(dt)
+    k = torch.randn(w.B, w.Sk, w.Hkv, w.d, generator=g, dtype=torch.float32).to(dt)
+    v = torch.randn(w.B, w.Sk, w.Hkv, w.d, generator=g, dtype=torch.float32).to(dt)
+    return q.to(device), k.to(device), v.to(device)
+
+
 E4M3_MAX = 448.0
 
 

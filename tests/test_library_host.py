@@ -18,8 +18,9 @@ def declared_symbols():
 
 
 def test_header_declares_the_entry_points():
-    assert set(declared_symbols()) == {"sdpa_fwd", "sdpa_fwd_fp8", "sdpa_strerror",
-                                       "sdpa_device_status", "sdpa_launches_per_call"}
+    assert set(declared_symbols()) == {"sdpa_fwd", "sdpa_fwd_strided", "sdpa_fwd_fp8",
+                                       "sdpa_strerror", "sdpa_device_status",
+                                       "sdpa_launches_per_call"}
 
 
 def test_library_exports_every_declared_symbol():
@@ -41,6 +42,7 @@ def test_strerror_and_launch_count():
     assert "invalid" in sdpa.sdpa_strerror(1)
     assert "unsupported" in sdpa.sdpa_strerror(2)
     assert "timed out" in sdpa.sdpa_strerror(4)
+    assert "layout" in sdpa.sdpa_strerror(5)
     assert sdpa.sdpa_strerror(99) == "unknown status"
     assert sdpa.sdpa_launches_per_call() == 1
 
@@ -98,3 +100,32 @@ def test_torch_wrapper_rejects_cpu_tensors():
     q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         sdpa.attention(q, q, q)
+
+
+def test_strided_argument_checks():
+    """sdpa_fwd_strided refuses views the kernel cannot address: strides that
+    are not positive or whose byte size is not a multiple of 16."""
+    import scaled_dot_product_11_b200 as sdpa
+    B, H, S, d = 2, 4, 256, 128
+    btnh = (S * H * d, d, H * d)            # [B, T, N, d] viewed as [B, N, T, d]
+
+    def strided(qs=btnh, ks=btnh, vs=btnh, os_=btnh, d=d, dtype=0):
+        return sdpa.sdpa_fwd_strided(P, P + 0x1000, P + 0x2000, P + 0x3000, P + 0x4000,
+                                     B, H, H, S, S, d, qs, ks, vs, os_, 0.088, 0, dtype, 0)
+    for bad in ((0, d, H * d), (S * H * d, -d, H * d), (S * H * d, d, H * d + 4),
+                (S * H * d + 2, d, H * d), (1 << 41, d, H * d)):
+        assert strided(qs=bad) == 1, bad
+        assert strided(os_=bad) == 1, bad
+    assert strided(ks=(S * H * d, d, 100)) == 1
+    assert strided(d=96) == 2          # unsupported head dim before the strides
+    assert strided(dtype=3) == 2
+    assert sdpa.sdpa_fwd_strided(P, P, P, 0, 0, B, H, H, S, S, d, btnh, btnh, btnh, btnh,
+                                 0.088, 0, 0, 0) == 1
+
+
+def test_torch_wrapper_rejects_views_with_strided_last_dim():
+    import torch
+    import scaled_dot_product_11_b200 as sdpa
+    x = torch.zeros(1, 2, 8, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        sdpa.attention(x[..., ::2], x[..., ::2], x[..., ::2])

@@ -21,8 +21,8 @@ import pytest
 import torch
 
 import oracle
-from sdpa_workloads import (WORKLOADS, Workload, make_qkv, make_qkv_fp8, sample_rows, sweep,
-                            with_shape)
+from sdpa_workloads import (WORKLOADS, Workload, make_qkv, make_qkv_btnh, make_qkv_fp8,
+                            sample_rows, sweep, with_shape)
 
 pytestmark = pytest.mark.gpu
 
@@ -244,6 +244,57 @@ def test_tile_varying_score_scale(sdpa, causal, pattern):
     o_tol = O_TOL + half_ulp(ro, "bf16") + 2.0 ** -9 * vmax
     assert (np.abs(o.double().cpu().numpy() - ro) <= o_tol).all()
     assert np.abs(lse.double().cpu().numpy() - rl).max() <= LSE_TOL * max(1.0, np.abs(rl).max() / 16)
+
+
+# ---- strided views (sdpa_fwd_strided) ---------------------------------------------
+
+BTNH = [
+    # (B, Hq, Hkv, Sq, Sk, d, causal): the codelab's [batch, time, heads, dim]
+    (2, 4, 4, 256, 256, 64, False),
+    (1, 8, 2, 300, 300, 128, True),
+    (2, 4, 4, 640, 640, 128, True),
+    (1, 4, 1, 130, 3329, 128, False),   # long units: the form without epilogue warps
+]
+
+
+@pytest.mark.parametrize("shape", BTNH, ids=lambda s: "b%d_hq%d_hkv%d_sq%d_sk%d_d%d_%s" % (
+    *s[:6], "causal" if s[6] else "full"))
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_btnh_views_in_place(sdpa, shape, dtype):
+    """BTNH data read and written in place through transposed views."""
+    B, Hq, Hkv, Sq, Sk, d, causal = shape
+    w = Workload("btnh", B, Hq, Hkv, Sq, Sk, d, causal, dtype=dtype, seed=3 * Sq + Sk)
+    qb, kb, vb = make_qkv_btnh(w, "cuda")
+    ob = torch.full_like(qb, float("nan"))
+    o, lse = sdpa.attention(qb.transpose(1, 2), kb.transpose(1, 2), vb.transpose(1, 2),
+                            causal=causal, out=ob.transpose(1, 2))
+    torch.cuda.synchronize()
+    st, detail = sdpa.sdpa_device_status(clear=True)
+    assert st == 0, "device status %d detail %#x" % (st, detail)
+    assert o.data_ptr() == ob.data_ptr()
+    ro, rl = oracle.sdpa_fwd(*(t.transpose(1, 2).contiguous().cpu() for t in (qb, kb, vb)),
+                             w.scale, causal)
+    check_o(ob.transpose(1, 2).double().cpu().numpy(), ro, O_TOL, dtype, "btnh")
+    assert np.abs(lse.double().cpu().numpy() - rl).max() <= LSE_TOL
+
+
+def test_padded_rows_and_mixed_layouts(sdpa):
+    """Rows padded to 192 elements (Q, O) next to a BHSD K and a BTNH V: every
+    tensor has its own strides, and O's padding is never written."""
+    B, Hq, Hkv, S, d = 2, 4, 2, 333, 128
+    w = Workload("pad", B, Hq, Hkv, S, S, d, True, seed=77)
+    q, k, v = make_qkv(w, "cuda")
+    qpad = torch.zeros(B, Hq, S, 192, dtype=q.dtype, device="cuda")
+    qpad[..., :d] = q
+    vb = v.transpose(1, 2).contiguous()                    # [B, S, Hkv, d]
+    opad = torch.full((B, Hq, S, 192), 7.0, dtype=q.dtype, device="cuda")
+    o, lse = sdpa.attention(qpad[..., :d], k, vb.transpose(1, 2), causal=True, out=opad[..., :d])
+    torch.cuda.synchronize()
+    assert sdpa.sdpa_device_status(clear=True)[0] == 0
+    assert bool((opad[..., d:] == 7.0).all())
+    ro, rl = oracle.sdpa_fwd(q.cpu(), k.cpu(), v.cpu(), w.scale, True)
+    check_o(opad[..., :d].double().cpu().numpy(), ro, O_TOL, "bf16", "padded")
+    assert np.abs(lse.double().cpu().numpy() - rl).max() <= LSE_TOL
 
 
 # ---- FP8 ----------------------------------------------------------------------
