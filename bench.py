@@ -163,11 +163,11 @@ def oracle_rows_tflops(w, q, k, v, nrows, seed, nthreads, descales=(1.0, 1.0, 1.
 
 
 def cpu_inputs(w):
-    from sdpa_workloads import make_qkv, make_qkv_fp8
+    from sdpa_workloads import make_inputs, make_qkv_fp8
     if w.dtype == "e4m3":
         q8, k8, v8, ds, _ = make_qkv_fp8(w)
         return q8, k8, v8, ds
-    q, k, v = make_qkv(w)
+    q, k, v = (t.contiguous() for t in make_inputs(w))
     return q, k, v, (1.0, 1.0, 1.0)
 
 
@@ -222,7 +222,7 @@ def run_reference(args, w):
 # ---------------------------------------------------------------------------
 def main():
     args = parse()
-    from sdpa_workloads import WORKLOADS, make_qkv, make_qkv_fp8, sample_rows, with_shape
+    from sdpa_workloads import WORKLOADS, make_inputs, make_qkv_fp8, sample_rows, with_shape
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
@@ -251,10 +251,13 @@ def main():
         q, k, v, ds, _ = make_qkv_fp8(w_rank, dev)
         run = lambda: sdpa.attention_fp8(q, k, v, ds, causal=w.causal, scale=w.scale, out=o, lse=lse)
     else:
-        q, k, v = make_qkv(w_rank, dev)
+        # "btnh" workloads: [B,S,H,d] data as views, through sdpa_fwd_strided
+        q, k, v = make_inputs(w_rank, dev)
         run = lambda: sdpa.attention(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse)
     o = torch.empty((w.B, w.Hq, w.Sq, w.d), dtype=torch.bfloat16 if fp8 or w.dtype == "bf16"
                     else torch.float16, device=dev)
+    if w.layout == "btnh":
+        o = torch.empty_like(q)             # laid out like q: [B,S,H,d] memory
     lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device=dev)
 
     barrier = lambda: rank_barrier(world)
@@ -271,7 +274,7 @@ def main():
     if rank == 0:
         import oracle
         rows = sample_rows(w, n_random=32)[:: max(1, len(sample_rows(w, n_random=32)) // 96)]
-        qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
+        qc, kc, vc = (t.contiguous().cpu() for t in (q, k, v))
         ro, rl = oracle.sdpa_rows(qc, kc, vc, rows, w.scale, w.causal,
                                   descales=ds if fp8 else (1.0, 1.0, 1.0))
         idx = torch.tensor(rows, device=dev)

@@ -32,6 +32,7 @@ class Workload:
     causal: bool
     dtype: str = "bf16"     # "bf16", "fp16" or "e4m3"
     seed: int = 0
+    layout: str = "bhsd"    # "bhsd": [B,H,S,d] tensors; "btnh": [B,S,H,d] data passed as views
 
     @property
     def scale(self) -> float:
@@ -93,6 +94,17 @@ def sweep(causal: bool, tokens: int = 32768, heads: int = 16, d: int = 128):
     return out
 
 
+def batch_sweep():
+    """The codelab's batch-size sweep (section 8): B in {1, 2, 4, 8, 16},
+    T = S = 256, N = 8 heads, head dim 64, no mask, seed B + 100, inputs in
+    its [batch, time, heads, head_dim] layout."""
+    return [Workload("bsweep_b%d_t256_n8_h64" % b, b, 8, 8, 256, 256, 64, False, seed=b + 100,
+                     layout="btnh") for b in (1, 2, 4, 8, 16)]
+
+
+WORKLOADS.update({"bsweep_b%d" % w.B: w for w in batch_sweep()})
+
+
 def with_shape(w: Workload, **kw) -> Workload:
     return replace(w, **kw)
 
@@ -111,6 +123,14 @@ def make_qkv(w: Workload, device="cpu"):
     k = torch.randn(w.B, w.Hkv, w.Sk, w.d, generator=g, dtype=torch.float32).to(dt)
     v = torch.randn(w.B, w.Hkv, w.Sk, w.d, generator=g, dtype=torch.float32).to(dt)
     return q.to(device), k.to(device), v.to(device)
+
+
+def make_inputs(w: Workload, device="cpu"):
+    """(q, k, v) as [B,H,S,d] tensors for a bf16/fp16 workload: contiguous
+    for layout "bhsd", transposed views of [B,S,H,d] data for "btnh"."""
+    if w.layout == "btnh":
+        return tuple(t.transpose(1, 2) for t in make_qkv_btnh(w, device))
+    return make_qkv(w, device)
 
 
 def make_qkv_btnh(w: Workload, device="cpu"):
