@@ -13,7 +13,11 @@ Parity status of each function (what pins it, in ``tests/test_oracle.py``):
                    row), invariants (rows of weights sum to 1, constant V,
                    affine V, key permutation, LSE shift, GQA == repeated-KV
                    MHA, causal prefix independence), a dominant key, and a
-                   40-digit mpmath evaluation on tiny inputs.
+                   40-digit mpmath evaluation on tiny inputs.  The mask
+                   aligned to the end of the keys (causal=2) is pinned by
+                   equality with the causal mask when Sq == Sk, with no mask
+                   when Sq == 1, and row by row with unmasked attention over
+                   the visible key prefix.
   sdpa_rows        pinned: equals sdpa_fwd on the same rows (same per-row code
                    reached through a different index path) and the pins above.
   sdpa_bruteforce  pinned: mpmath evaluation, weights-sum, V = identity.
@@ -110,9 +114,17 @@ def _check(rc):
     if rc == 1:
         raise ValueError("oracle: invalid arguments")
     if rc == 2:
-        raise ValueError("oracle: causal attention needs Sq == Sk")
+        raise ValueError("oracle: causal attention needs Sq == Sk (bottom-right: Sq <= Sk)")
     if rc != 0:
         raise MemoryError("oracle: allocation failed")
+
+
+def _mask(causal) -> int:
+    """0 no mask, 1 causal (key j <= query i, Sq == Sk), 2 causal aligned to
+    the end of the keys (j <= i + Sk - Sq, Sq <= Sk).  True means 1."""
+    if causal in ("bottom_right", 2):
+        return 2
+    return 1 if causal else 0
 
 
 def _prep(q, k, v):
@@ -138,7 +150,7 @@ def sdpa_fwd(q, k, v, scale: float, causal: bool = False, descales=(1.0, 1.0, 1.
     _check(lib.oracle_sdpa_fwd(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, t,
                                float(descales[0]), float(descales[1]), float(descales[2]),
                                o.ctypes.data, lse.ctypes.data,
-                               B, Hq, Hkv, Sq, Sk, d, float(scale), int(bool(causal)), nt))
+                               B, Hq, Hkv, Sq, Sk, d, float(scale), _mask(causal), nt))
     return o, lse
 
 
@@ -156,7 +168,7 @@ def sdpa_rows(q, k, v, rows, scale: float, causal: bool = False, descales=(1.0, 
     _check(lib.oracle_sdpa_rows(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, t,
                                 float(descales[0]), float(descales[1]), float(descales[2]),
                                 r.ctypes.data, r.size, o.ctypes.data, lse.ctypes.data,
-                                B, Hq, Hkv, Sq, Sk, d, float(scale), int(bool(causal)), nt))
+                                B, Hq, Hkv, Sq, Sk, d, float(scale), _mask(causal), nt))
     return o, lse
 
 
@@ -174,7 +186,7 @@ def sdpa_bruteforce(q, k, v, scale: float, causal: bool = False, descales=(1.0, 
                                       float(descales[0]), float(descales[1]), float(descales[2]),
                                       o.ctypes.data, lse.ctypes.data,
                                       None if w is None else w.ctypes.data,
-                                      B, Hq, Hkv, Sq, Sk, d, float(scale), int(bool(causal))))
+                                      B, Hq, Hkv, Sq, Sk, d, float(scale), _mask(causal)))
     return (o, lse, w) if return_weights else (o, lse)
 
 

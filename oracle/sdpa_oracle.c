@@ -16,6 +16,11 @@
  *                                                    query heads; contiguous groups)
  *     J_i = {0 .. Sk-1}, or {0 .. i} when causal     (codelab section 7: each
  *                                                    position sees earlier ones)
+ *           or {0 .. i + Sk - Sq} when causal is 2   (the Sq queries are the last
+ *                                                    Sq positions of a sequence of
+ *                                                    Sk, as with a KV cache: codelab
+ *                                                    section 9 and its closing
+ *                                                    suggestions; Sq <= Sk)
  *     s_j = scale * sum_c Q[b,hq,i,c] * K[b,hk,j,c]  for j in J_i
  *     m   = max_j s_j ;  l = sum_j exp(s_j - m)
  *     O[b,hq,i,:] = sum_j exp(s_j - m) / l * V[b,hk,j,:]
@@ -109,7 +114,9 @@ static int check_problem(const problem_t* p) {
     if (!p->q || !p->k || !p->v) return 1;
     if (p->B <= 0 || p->Hq <= 0 || p->Hkv <= 0 || p->Sq <= 0 || p->Sk <= 0 || p->d <= 0) return 1;
     if (p->Hq % p->Hkv != 0) return 1;
-    if (p->causal && p->Sq != p->Sk) return 2;
+    if (p->causal < 0 || p->causal > 2) return 1;
+    if (p->causal == 1 && p->Sq != p->Sk) return 2;
+    if (p->causal == 2 && p->Sq > p->Sk) return 2;
     if (p->dtype < ORC_F64 || p->dtype > ORC_E4M3) return 1;
     return 0;
 }
@@ -121,7 +128,9 @@ static void one_row(const problem_t* p, int b, int hq, int i, double* work,
     const int hk = hq / group;
     const size_t qoff = (((size_t)b * p->Hq + hq) * p->Sq + i) * p->d;
     const size_t kvhead = ((size_t)b * p->Hkv + hk) * p->Sk;
-    const int nkeys = p->causal ? i + 1 : p->Sk;
+    /* keys 0 .. last visible: all, the diagonal, or the diagonal shifted by
+       Sk - Sq (queries aligned to the end of the key sequence) */
+    const int nkeys = p->causal == 1 ? i + 1 : p->causal == 2 ? i + 1 + (p->Sk - p->Sq) : p->Sk;
 
     /* score step: s_j = scale * q_i . k_j */
     double m = -INFINITY;
@@ -150,7 +159,8 @@ static void one_row(const problem_t* p, int b, int hq, int i, double* work,
 
 /*
  * Full forward.  o: [B,Hq,Sq,d] doubles, lse: [B,Hq,Sq] doubles.
- * Returns 0 on success, 1 for invalid arguments, 2 for causal with Sq != Sk.
+ * Returns 0 on success, 1 for invalid arguments, 2 for causal 1 with Sq != Sk
+ * or causal 2 with Sq > Sk.
  */
 int oracle_sdpa_fwd(const void* q, const void* k, const void* v, int dtype,
                     double dq, double dk, double dv, double* o, double* lse,
@@ -247,14 +257,16 @@ int oracle_sdpa_bruteforce(const void* q, const void* k, const void* v, int dtyp
             const int hk = hq / group;
             const size_t qh = ((size_t)b * Hq + hq) * Sq;
             const size_t kh = ((size_t)b * Hkv + hk) * Sk;
-            /* scores = (Q K^T) * scale, causal entries above the diagonal -inf */
+            /* scores = (Q K^T) * scale; masked entries (above the diagonal,
+               shifted by Sk - Sq when causal is 2) -inf */
             for (int i = 0; i < Sq; ++i)
                 for (int j = 0; j < Sk; ++j) {
                     double acc = 0.0;
                     for (int c = 0; c < d; ++c)
                         acc += load_elem(q, dtype, (qh + i) * d + c, dq) *
                                load_elem(k, dtype, (kh + j) * d + c, dk);
-                    S[(size_t)i * Sk + j] = (causal && j > i) ? -INFINITY : acc * scale;
+                    const int last = causal == 2 ? i + Sk - Sq : i;
+                    S[(size_t)i * Sk + j] = (causal && j > last) ? -INFINITY : acc * scale;
                 }
             /* row softmax in place; keep each row's log normaliser */
             for (int i = 0; i < Sq; ++i) {

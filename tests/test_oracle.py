@@ -323,3 +323,60 @@ def test_rejects_bad_arguments():
 def test_page_tolerance_precedents_recorded():
     g = json.load(open(os.path.join(GOLDEN, "codelab_tolerances.json")))
     assert g["f32_atol"] == 1e-3 and g["bf16_atol"] == 1e-2 and g["bf16_rtol"] == 1e-2
+
+
+# --------------------------------------------------------------------------
+# causal mask aligned to the end of the keys (causal=2): query i of Sq is
+# position Sk - Sq + i of the sequence and sees keys 0 .. i + Sk - Sq
+# --------------------------------------------------------------------------
+
+def test_bottom_right_equal_lengths_is_the_causal_mask():
+    q, k, v = rand(1, 2, 9, 8), rand(1, 2, 9, 8), rand(1, 2, 9, 8)
+    o1, l1 = oracle.sdpa_fwd(q, k, v, 0.5, causal=True)
+    o2, l2 = oracle.sdpa_fwd(q, k, v, 0.5, causal="bottom_right")
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+
+
+def test_bottom_right_single_query_sees_every_key():
+    """Sq = 1 (one new token against a cache of Sk keys): no key is masked."""
+    q, k, v = rand(2, 4, 1, 8), rand(2, 2, 13, 8), rand(2, 2, 13, 8)
+    o1, l1 = oracle.sdpa_fwd(q, k, v, 0.4, causal=False)
+    o2, l2 = oracle.sdpa_fwd(q, k, v, 0.4, causal=2)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+
+
+def test_bottom_right_rows_are_unmasked_attention_over_a_key_prefix():
+    """Row i equals unmasked attention of that one query over keys
+    0 .. i + Sk - Sq (sliced K, V), so the offset and its off-by-one are
+    pinned by the (independently pinned) unmasked path."""
+    Sq, Sk = 5, 12
+    q, k, v = rand(1, 2, Sq, 8), rand(1, 1, Sk, 8), rand(1, 1, Sk, 8)
+    o, l = oracle.sdpa_fwd(q, k, v, 0.45, causal=2)
+    for i in range(Sq):
+        n = i + 1 + Sk - Sq
+        oi, li = oracle.sdpa_fwd(q[:, :, i:i + 1].copy(), k[:, :, :n].copy(), v[:, :, :n].copy(), 0.45)
+        np.testing.assert_allclose(o[:, :, i], oi[:, :, 0], rtol=0, atol=1e-14)
+        np.testing.assert_allclose(l[:, :, i], li[:, :, 0], rtol=0, atol=1e-14)
+    # and it differs from the top-left reading, under which row 0 sees key 0
+    # only and returns V[0]
+    assert np.abs(o[:, :, 0] - v[:, :, 0]).max() > 1e-3
+
+
+def test_bottom_right_bruteforce_and_rows_agree():
+    q, k, v = rand(2, 4, 7, 8), rand(2, 2, 11, 8), rand(2, 2, 11, 8)
+    o1, l1 = oracle.sdpa_fwd(q, k, v, 0.37, 2)
+    o2, l2 = oracle.sdpa_bruteforce(q, k, v, 0.37, 2)
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l1, l2, rtol=0, atol=1e-13)
+    rows = [0, 6, 7, 20, 2 * 4 * 7 - 1]
+    orow, lrow = oracle.sdpa_rows(q, k, v, rows, 0.37, 2)
+    np.testing.assert_array_equal(orow, o1.reshape(-1, 8)[rows])
+    np.testing.assert_array_equal(lrow, l1.reshape(-1)[rows])
+
+
+def test_bottom_right_rejects_more_queries_than_keys():
+    q, k, v = rand(1, 2, 6, 8), rand(1, 2, 5, 8), rand(1, 2, 5, 8)
+    with pytest.raises(ValueError):
+        oracle.sdpa_fwd(q, k, v, 1.0, causal=2)
