@@ -55,13 +55,26 @@ typedef enum {
     SDPA_FP16 = 1    /* float16  Q/K/V/O */
 } sdpa_dtype;
 
+/* Values of the `causal` argument. */
+typedef enum {
+    SDPA_NO_MASK = 0,              /* every query sees every key */
+    SDPA_CAUSAL = 1,               /* query i sees keys 0..i (codelab section 7);
+                                      needs Sq == Sk */
+    SDPA_CAUSAL_BOTTOM_RIGHT = 2   /* the queries are the last Sq positions of the
+                                      Sk-long sequence (a KV cache): query i
+                                      sees keys 0..i+Sk-Sq; needs Sq <= Sk and
+                                      equals SDPA_CAUSAL when Sq == Sk */
+} sdpa_causal;
+
 typedef enum {
     SDPA_OK = 0,
     SDPA_ERR_INVALID_ARG = 1,    /* null pointer, a size <= 0, Hq % Hkv != 0,
+                                    causal not an sdpa_causal value,
                                     non-finite or non-positive scale, a pointer
                                     not 16-byte aligned, sizes whose element
                                     counts overflow the addressing limits */
-    SDPA_ERR_UNSUPPORTED = 2,    /* d not 64 or 128, causal with Sq != Sk,
+    SDPA_ERR_UNSUPPORTED = 2,    /* d not 64 or 128, SDPA_CAUSAL with Sq != Sk,
+                                    SDPA_CAUSAL_BOTTOM_RIGHT with Sq > Sk,
                                     unknown dtype, device not sm_100 */
     SDPA_ERR_CUDA = 3,           /* the CUDA runtime or driver reported an
                                     error while preparing or launching */
@@ -83,8 +96,9 @@ typedef enum {
  *                     scores of each row (may be NULL to skip it)
  *   scale            applied to Q K^T as given; pass 1/sqrt(d) for the
  *                    codelab's default (section 4, scale = 1/sqrt(H))
- *   causal           0: every key; 1: key j only for query i >= j (needs
- *                    Sq == Sk)
+ *   causal           an sdpa_causal: 0 every key; 1 key j only for query
+ *                    i >= j (needs Sq == Sk); 2 key j only for query
+ *                    i >= j - (Sk - Sq) (needs Sq <= Sk)
  *   dtype            an sdpa_dtype
  *   stream           cudaStream_t to enqueue on
  *

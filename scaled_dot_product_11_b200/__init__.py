@@ -17,6 +17,7 @@ import os
 __all__ = [
     "SDPA_BF16", "SDPA_FP16", "SDPA_OK", "SDPA_ERR_INVALID_ARG", "SDPA_ERR_UNSUPPORTED",
     "SDPA_ERR_CUDA", "SDPA_ERR_DEVICE_TIMEOUT", "SDPA_ERR_DEVICE_LAYOUT", "SdpaError", "LIB_PATH",
+    "SDPA_NO_MASK", "SDPA_CAUSAL", "SDPA_CAUSAL_BOTTOM_RIGHT",
     "sdpa_fwd", "sdpa_fwd_strided", "sdpa_fwd_fp8", "sdpa_strerror", "sdpa_device_status",
     "sdpa_launches_per_call", "attention", "attention_fp8",
 ]
@@ -102,6 +103,18 @@ def sdpa_launches_per_call() -> int:
 
 # ---- torch conveniences -------------------------------------------------------
 
+SDPA_NO_MASK, SDPA_CAUSAL, SDPA_CAUSAL_BOTTOM_RIGHT = 0, 1, 2
+
+
+def _causal_code(causal) -> int:
+    """False/0: no mask; True/1: key j <= query i (Sq == Sk); 2 or
+    "bottom_right": key j <= i + Sk - Sq (Sq <= Sk, queries at the end)."""
+    if causal in (2, "bottom_right"):
+        return SDPA_CAUSAL_BOTTOM_RIGHT
+    if causal in (True, False, 0, 1):
+        return int(bool(causal))
+    raise ValueError("causal must be False, True, 2 or 'bottom_right'")
+
 def _dims(q, k, v, allow_views=False):
     if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
         raise ValueError("q, k, v must be 4-D [B, H, S, d]")
@@ -125,7 +138,7 @@ def _stream_handle(stream):
     return int(s.cuda_stream)
 
 
-def attention(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
+def attention(q, k, v, causal=False, scale: float | None = None, out=None, lse=None,
               return_lse: bool = True, stream=None):
     """O (and LSE) = softmax(q k^T * scale [causal]) v for bf16 / fp16 CUDA
     tensors q [B,Hq,Sq,d], k/v [B,Hkv,Sk,d].  They may be strided views
@@ -135,6 +148,7 @@ def attention(q, k, v, causal: bool = False, scale: float | None = None, out=Non
     torch's current stream); raises SdpaError on a refused call."""
     import torch
     B, Hq, Hkv, Sq, Sk, d = _dims(q, k, v, allow_views=True)
+    causal = _causal_code(causal)
     if q.dtype not in (torch.bfloat16, torch.float16) or k.dtype != q.dtype or v.dtype != q.dtype:
         raise ValueError("q, k, v must share dtype bfloat16 or float16")
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
@@ -162,13 +176,14 @@ def attention(q, k, v, causal: bool = False, scale: float | None = None, out=Non
     return (out, lse) if return_lse else out
 
 
-def attention_fp8(q8, k8, v8, descales, causal: bool = False, scale: float | None = None,
+def attention_fp8(q8, k8, v8, descales, causal=False, scale: float | None = None,
                   out=None, lse=None, stream=None):
     """FP8 E4M3 forward: q8/k8/v8 torch.float8_e4m3fn CUDA tensors holding
     codes, descales = (dq, dk, dv) so that value = code * descale.  Returns
     (O bf16, LSE fp32)."""
     import torch
     B, Hq, Hkv, Sq, Sk, d = _dims(q8, k8, v8)
+    causal = _causal_code(causal)
     for t in (q8, k8, v8):
         if t.dtype != torch.float8_e4m3fn:
             raise ValueError("q8, k8, v8 must be float8_e4m3fn")

@@ -74,14 +74,15 @@ int check_args(const void* q, const void* k, const void* v, const void* o, const
     if (!std::isfinite(scale) || !(scale > 0.0f)) return SDPA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SDPA_ERR_INVALID_ARG;
     if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return SDPA_ERR_INVALID_ARG;
-    if (causal != 0 && causal != 1) return SDPA_ERR_INVALID_ARG;
+    if (causal < 0 || causal > 2) return SDPA_ERR_INVALID_ARG;
     // addressing limits: head counts and row indices fit the 32-bit TMA
     // coordinates and the grid, element offsets fit 64-bit size_t trivially
     const long long bhq = (long long)B * Hq, bhk = (long long)B * Hkv;
     const long long qblocks = (Sq + 127) / 128;
     if (bhq > INT32_MAX || bhk > INT32_MAX || bhq * qblocks > INT32_MAX) return SDPA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return SDPA_ERR_UNSUPPORTED;
-    if (causal && Sq != Sk) return SDPA_ERR_UNSUPPORTED;
+    if (causal == SDPA_CAUSAL && Sq != Sk) return SDPA_ERR_UNSUPPORTED;
+    if (causal == SDPA_CAUSAL_BOTTOM_RIGHT && Sq > Sk) return SDPA_ERR_UNSUPPORTED;
     return SDPA_OK;
 }
 
@@ -165,7 +166,7 @@ int launch_cfg(const void* q, const void* k, const void* v, const View& vq, cons
 #endif
 bool use_epilogue_warps(const FwdParams& prm) {
     const int nk = (prm.Sk + 127) / 128;
-    const double avg = prm.causal ? 0.5 * (prm.n_qtiles + 1) : (double)nk;
+    const double avg = prm.causal ? 0.5 * (prm.n_qtiles + 1) + prm.causal_off / 128.0 : (double)nk;
     return avg >= SDPA_EPI_MIN_AVG_TILES && avg <= SDPA_EPI_MAX_AVG_TILES;
 }
 
@@ -212,7 +213,8 @@ FwdParams make_params(void* o, const View& vo, float* lse, int B, int Hq, int Hk
     prm.group_heads = (2 * sm_count() + prm.items_per_head - 1) / prm.items_per_head;
     if (prm.group_heads < 1) prm.group_heads = 1;
     if (prm.group_heads > B * Hq) prm.group_heads = B * Hq;
-    prm.causal = causal;
+    prm.causal = causal != 0 ? 1 : 0;
+    prm.causal_off = causal == SDPA_CAUSAL_BOTTOM_RIGHT ? Sk - Sq : 0;
     prm.score_log2 = 0.f;
     prm.out_mul = 1.f;
     return prm;

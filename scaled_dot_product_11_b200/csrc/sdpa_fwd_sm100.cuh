@@ -102,6 +102,8 @@ struct FwdParams {
     float score_log2;   // multiplier from raw MMA score to log2 units
     float out_mul;      // multiplier on (sum_j p_j v_j) / l: the V descale for FP8, else 1
     long long o_sb, o_sh, o_ss;   // O's batch, head, row strides in elements (STRIDED)
+    int causal_off;     // causal: query row i sees keys 0 .. i + causal_off (0, or Sk - Sq
+                        // when the queries are aligned to the end of the keys)
 };
 
 template <int D, int KIND, int NS, int QB, bool EPI>
@@ -266,9 +268,9 @@ __device__ __forceinline__ long long o_offset(const FwdParams& p, int bh, int ro
 }
 
 // Number of K/V tiles the query rows [row0, row0 + 128) need.
-__device__ __forceinline__ int tiles_for(int row0, int Sq, int Sk, int causal) {
+__device__ __forceinline__ int tiles_for(int row0, int Sq, int Sk, int causal, int off) {
     if (row0 >= Sq) return 0;
-    const int kend = causal ? min(Sk, row0 + kBlockM) : Sk;
+    const int kend = causal ? min(Sk, row0 + kBlockM + off) : Sk;
     return (kend + kBlockN - 1) / kBlockN;
 }
 
@@ -311,7 +313,7 @@ struct UnitCursor {
 
 __device__ __forceinline__ void unit_load(const FwdParams& p, UnitCursor& u) {
     u.valid = sched_unit(p, u.k, u.sub, u.bh, u.qtile);
-    u.n = u.valid ? tiles_for(u.qtile * kBlockM, p.Sq, p.Sk, p.causal) : 0;
+    u.n = u.valid ? tiles_for(u.qtile * kBlockM, p.Sq, p.Sk, p.causal, p.causal_off) : 0;
 }
 __device__ __forceinline__ void unit_first(const FwdParams& p, UnitCursor& u) {
     u.k = 0;
@@ -701,13 +703,15 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 reg_fence32(&s[0]);
                 tmem_ld32(tS + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
 
-                // mask: keys past Sk, and (causal) keys after the row
+                // mask: keys past Sk, and (causal) keys after the row's last
+                // visible key row + causal_off
                 const int key0 = i * kBlockN + h * kHalfN;
-                const bool edge = (key0 + kHalfN > p.Sk) || (p.causal && key0 + kHalfN - 1 > m0);
+                const bool edge = (key0 + kHalfN > p.Sk) ||
+                                  (p.causal && key0 + kHalfN - 1 > m0 + p.causal_off);
                 int lim = kHalfN;
                 if (edge) {
                     lim = p.Sk - key0;
-                    if (p.causal) lim = min(lim, row - key0 + 1);
+                    if (p.causal) lim = min(lim, row + p.causal_off - key0 + 1);
 #pragma unroll
                     for (int c = 0; c < 32; ++c)
                         if (c >= lim) s[c] = -INFINITY;

@@ -246,6 +246,48 @@ def test_tile_varying_score_scale(sdpa, causal, pattern):
     assert np.abs(lse.double().cpu().numpy() - rl).max() <= LSE_TOL * max(1.0, np.abs(rl).max() / 16)
 
 
+# ---- causal mask aligned to the end of the keys (causal=2) -------------------------
+
+BOTTOM_RIGHT = [
+    # (B, Hq, Hkv, Sq, Sk, d)
+    (1, 2, 2, 100, 300, 128),
+    (1, 4, 1, 1, 1000, 128),     # one new token against a 1000-key cache
+    (2, 4, 2, 16, 777, 64),      # a few new tokens, ragged cache
+    (1, 2, 2, 300, 300, 128),    # Sq == Sk: the causal mask
+    (2, 4, 1, 257, 640, 64),
+    (1, 2, 2, 130, 4000, 128),   # long units: the form without epilogue warps
+]
+
+
+@pytest.mark.parametrize("shape", BOTTOM_RIGHT, ids=lambda s: "b%d_hq%d_hkv%d_sq%d_sk%d_d%d" % s)
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_bottom_right_causal(sdpa, shape, dtype):
+    B, Hq, Hkv, Sq, Sk, d = shape
+    w = Workload("br", B, Hq, Hkv, Sq, Sk, d, False, dtype=dtype, seed=5 * Sq + Sk)
+    q, k, v = make_qkv(w, "cuda")
+    o, lse = sdpa.attention(q, k, v, causal="bottom_right", scale=w.scale)
+    torch.cuda.synchronize()
+    st, detail = sdpa.sdpa_device_status(clear=True)
+    assert st == 0, "device status %d detail %#x" % (st, detail)
+    ro, rl = oracle.sdpa_fwd(q.cpu(), k.cpu(), v.cpu(), w.scale, causal="bottom_right")
+    check_o(o.double().cpu().numpy(), ro, O_TOL, dtype, "bottom-right")
+    assert np.abs(lse.double().cpu().numpy() - rl).max() <= LSE_TOL
+
+
+def test_bottom_right_decode_batch_sampled(sdpa):
+    """16 new tokens per sequence against an 8192-key cache, GQA 32/8."""
+    w = Workload("decode", 4, 32, 8, 16, 8192, 128, False, seed=16)
+    q, k, v = make_qkv(w, "cuda")
+    o, lse = sdpa.attention(q, k, v, causal=2, scale=w.scale)
+    torch.cuda.synchronize()
+    assert sdpa.sdpa_device_status(clear=True)[0] == 0
+    rows = list(range(0, w.B * w.Hq * w.Sq, 7)) + [w.B * w.Hq * w.Sq - 1]
+    ro, rl = oracle.sdpa_rows(q.cpu(), k.cpu(), v.cpu(), rows, w.scale, causal=2)
+    idx = torch.tensor(rows, device="cuda")
+    check_o(o.reshape(-1, w.d).index_select(0, idx).double().cpu().numpy(), ro, O_TOL, "bf16", "decode")
+    assert np.abs(lse.reshape(-1).index_select(0, idx).double().cpu().numpy() - rl).max() <= LSE_TOL
+
+
 # ---- strided views (sdpa_fwd_strided) ---------------------------------------------
 
 BTNH = [
@@ -309,7 +351,8 @@ def run_fp8(lib, w):
 
 
 @pytest.mark.parametrize("shape", [(1, 2, 2, 256, 256, True), (1, 2, 1, 333, 333, True),
-                                   (2, 4, 2, 200, 500, False), (1, 2, 2, 150, 3300, False)])
+                                   (2, 4, 2, 200, 500, False), (1, 2, 2, 150, 3300, False),
+                                   (1, 2, 2, 100, 500, "bottom_right")])
 def test_fp8_small(sdpa, shape):
     B, Hq, Hkv, Sq, Sk, causal = shape
     w = Workload("f8", B, Hq, Hkv, Sq, Sk, 128, causal, dtype="e4m3", seed=Sq + Sk)
