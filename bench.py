@@ -352,6 +352,22 @@ def main():
         peak = float(peaks["bf16_tflops"]) * ratio
         achieved = w.flops / (ms_per_step * 1e-3) / 1e12
         traffic = load_traffic(w.name)
+        # the bound: tensor peak when the arithmetic intensity (algorithmic
+        # flops per algorithmic byte) is above the ridge, HBM otherwise
+        ridge = peak * 1e12 / (float(peaks["hbm_gbs"]) * 1e9)
+        hbm_bound = w.flops / w.min_hbm_bytes < ridge
+        if hbm_bound:
+            roofline = {"bound": "hbm", "achieved": w.min_hbm_bytes / (ms_per_step * 1e-3) / 1e9,
+                        "peak": float(peaks["hbm_gbs"]), "unit": "GB/s", "traffic": traffic,
+                        "peak_source": "%s hbm_gbs (copy)" % src,
+                        "arithmetic_intensity": w.flops / w.min_hbm_bytes, "ridge": ridge}
+            roofline["frac"] = roofline["achieved"] / roofline["peak"]
+        else:
+            roofline = {"bound": "tensor", "achieved": achieved, "peak": peak,
+                        "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                        "peak_source": "%s bf16_tflops (burst)%s; frac of sustained %.3f" % (
+                            src, " x 2 (nominal fp8/bf16)" if fp8 else "",
+                            achieved / (float(peaks["bf16_tflops_sustained"]) * ratio))}
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -360,11 +376,7 @@ def main():
             "config": dict(w.describe(), global_batch=w.B * world,
                            parallelism="dp%d (independent batches per GPU)" % world,
                            l2=l2_note),
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
-                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                         "peak_source": "%s bf16_tflops (burst)%s; frac of sustained %.3f" % (
-                             src, " x 2 (nominal fp8/bf16)" if fp8 else "",
-                             achieved / (float(peaks["bf16_tflops_sustained"]) * ratio))},
+            "roofline": roofline,
             "clocks": clk,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},

@@ -100,7 +100,8 @@ bool same(const View& a, const View& b) { return a.sb == b.sb && a.sh == b.sh &&
 // contiguous [B,H,S,d] data (`rank3`); boxes of box_inner x 128 rows of one
 // (head, batch), 128-byte swizzle.
 bool encode_view(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* base, int d,
-                 int rows, int heads, int batch, const View& v, int box_inner, bool rank3) {
+                 int rows, int heads, int batch, const View& v, int box_inner, bool rank3,
+                 int box_rows = 128, int box_heads = 1) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint32_t rank = rank3 ? 3u : 4u;
@@ -108,7 +109,7 @@ bool encode_view(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const v
     cuuint64_t strides[3] = {(cuuint64_t)(v.ss * elem_bytes), (cuuint64_t)(v.sh * elem_bytes),
                              (cuuint64_t)(v.sb * elem_bytes)};
     if (rank == 3) dims[2] = (cuuint64_t)heads * (cuuint64_t)batch;
-    const cuuint32_t box[4] = {(cuuint32_t)box_inner, 128u, 1u, 1u};
+    const cuuint32_t box[4] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, (cuuint32_t)box_heads, 1u};
     const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
     return fn(m, dt, rank, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -126,7 +127,7 @@ bool view_ok(const long long* st, int elem_bytes) {
     return true;
 }
 
-template <int D, int KIND, int NS, int QB, bool EPI, bool STRIDED>
+template <int D, int KIND, int NS, int QB, bool EPI, bool STRIDED, bool PACK = false>
 int launch_cfg(const void* q, const void* k, const void* v, const View& vq, const View& vk,
                const View& vv, const FwdParams& prm, cudaStream_t stream) {
     using C = FwdCfg<D, KIND, NS, QB, EPI>;
@@ -134,11 +135,16 @@ int launch_cfg(const void* q, const void* k, const void* v, const View& vq, cons
                                    : KIND == sdpa::KIND_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                              : CU_TENSOR_MAP_DATA_TYPE_UINT8;
     CUtensorMap tq, tk, tv;
-    if (!encode_view(&tq, dt, C::kElem, q, D, prm.Sq, prm.Hq, prm.B, vq, C::kElemsPerSw, !STRIDED) ||
+    // PACK: Q boxes hold all Sq rows of the pk_group query heads of a K/V head
+    const bool qok = PACK ? encode_view(&tq, dt, C::kElem, q, D, prm.Sq, prm.pk_hq, prm.B, vq,
+                                        C::kElemsPerSw, false, prm.Sq, prm.pk_group)
+                          : encode_view(&tq, dt, C::kElem, q, D, prm.Sq, prm.Hq, prm.B, vq,
+                                        C::kElemsPerSw, !STRIDED);
+    if (!qok ||
         !encode_view(&tk, dt, C::kElem, k, D, prm.Sk, prm.Hkv, prm.B, vk, C::kElemsPerSw, !STRIDED) ||
         !encode_view(&tv, dt, C::kElem, v, D, prm.Sk, prm.Hkv, prm.B, vv, C::kElemsPerSw, !STRIDED))
         return SDPA_ERR_CUDA;
-    auto kern = sdpa::sdpa_fwd_sm100_kernel<D, KIND, NS, QB, EPI, STRIDED>;
+    auto kern = sdpa::sdpa_fwd_sm100_kernel<D, KIND, NS, QB, EPI, STRIDED, PACK>;
     static bool attr_set[64];
     int dev = 0;
     cudaGetDevice(&dev);
@@ -180,9 +186,40 @@ int launch_form(const void* q, const void* k, const void* v, const View& vq, con
                : launch_cfg<D, KIND, NS, QB, false, STRIDED>(q, k, v, vq, vk, vv, prm, stream);
 }
 
+// Decode-shaped GQA/MQA: when the Sq rows of all query heads sharing a K/V
+// head fit one 128-row tile (group >= 2), one unit holds them all, so each
+// K/V tile is streamed and multiplied once per K/V head instead of once per
+// query head.
+#ifndef SDPA_PACK_MAX_ROWS
+#define SDPA_PACK_MAX_ROWS 128
+#endif
+bool use_packed_units(const FwdParams& prm) {
+    return prm.group >= 2 && (long long)prm.group * prm.Sq <= SDPA_PACK_MAX_ROWS;
+}
+
+template <int D, int KIND, int NS, int QB>
+int launch_packed(const void* q, const void* k, const void* v, const View& vq, const View& vk,
+                  const View& vv, const FwdParams& prm, cudaStream_t stream) {
+    using C = FwdCfg<D, KIND, NS, QB, false>;
+    FwdParams pk = prm;
+    pk.pk_hq = prm.Hq;
+    pk.pk_group = prm.group;
+    pk.pk_rows = prm.group * prm.Sq;
+    pk.pk_qbytes = pk.pk_rows * C::kRowBytes;
+    // units are (batch, K/V head) pairs of one tile each
+    pk.Hq = prm.Hkv;
+    pk.group = 1;
+    pk.n_qtiles = 1;
+    pk.items_per_head = 1;
+    pk.n_items = prm.B * prm.Hkv;
+    pk.group_heads = pk.n_items < 2 * sm_count() ? pk.n_items : 2 * sm_count();
+    return launch_cfg<D, KIND, NS, QB, false, true, true>(q, k, v, vq, vk, vv, pk, stream);
+}
+
 template <int D, int KIND, int NS, int QB>
 int launch(const void* q, const void* k, const void* v, const View& vq, const View& vk, const View& vv,
            const FwdParams& prm, cudaStream_t stream) {
+    if (use_packed_units(prm)) return launch_packed<D, KIND, NS, QB>(q, k, v, vq, vk, vv, prm, stream);
     const bool contiguous = same(vq, bhsd(prm.Hq, prm.Sq, D)) && same(vk, bhsd(prm.Hkv, prm.Sk, D)) &&
                             same(vv, bhsd(prm.Hkv, prm.Sk, D)) &&
                             prm.o_sb == (long long)prm.Hq * prm.Sq * D && prm.o_sh == (long long)prm.Sq * D &&
@@ -215,6 +252,10 @@ FwdParams make_params(void* o, const View& vo, float* lse, int B, int Hq, int Hk
     if (prm.group_heads > B * Hq) prm.group_heads = B * Hq;
     prm.causal = causal != 0 ? 1 : 0;
     prm.causal_off = causal == SDPA_CAUSAL_BOTTOM_RIGHT ? Sk - Sq : 0;
+    prm.pk_hq = Hq;
+    prm.pk_group = 1;
+    prm.pk_rows = 0;
+    prm.pk_qbytes = 0;
     prm.score_log2 = 0.f;
     prm.out_mul = 1.f;
     return prm;

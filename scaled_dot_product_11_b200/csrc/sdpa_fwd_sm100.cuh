@@ -104,6 +104,11 @@ struct FwdParams {
     long long o_sb, o_sh, o_ss;   // O's batch, head, row strides in elements (STRIDED)
     int causal_off;     // causal: query row i sees keys 0 .. i + causal_off (0, or Sk - Sq
                         // when the queries are aligned to the end of the keys)
+    // PACK form: a unit holds the Sq rows of all pk_group query heads of one
+    // K/V head (pk_rows = pk_group * Sq <= 128 TMEM lanes, row r = head
+    // r / Sq, position r % Sq); Hq and group above then describe units
+    // (Hq = Hkv, group = 1) and these the query heads.
+    int pk_hq, pk_group, pk_rows, pk_qbytes;
 };
 
 template <int D, int KIND, int NS, int QB, bool EPI>
@@ -258,13 +263,21 @@ __device__ __forceinline__ float chunk_max32(const float* s) {
 // Element offset of row `row` of (batch, head) pair bh in O: contiguous
 // [B,Hq,Sq,D], or the strided view.
 template <int D, bool STRIDED>
-__device__ __forceinline__ long long o_offset(const FwdParams& p, int bh, int row) {
+__device__ __forceinline__ long long o_offset(const FwdParams& p, int bh, int row, int heads = 0) {
     if constexpr (STRIDED) {
-        const int b = bh / p.Hq;
-        return (long long)b * p.o_sb + (long long)(bh - b * p.Hq) * p.o_sh + (long long)row * p.o_ss;
+        const int h_n = heads > 0 ? heads : p.Hq;
+        const int b = bh / h_n;
+        return (long long)b * p.o_sb + (long long)(bh - b * h_n) * p.o_sh + (long long)row * p.o_ss;
     } else {
         return ((long long)bh * p.Sq + row) * D;
     }
+}
+
+// PACK form: (batch, query head) index b * pk_hq + hq of lane r of the unit
+// of (batch, K/V head) pair ubh.
+__device__ __forceinline__ int packed_qhead(const FwdParams& p, int ubh, int r) {
+    const int b = ubh / p.Hq;                       // p.Hq = K/V heads here
+    return b * p.pk_hq + (ubh - b * p.Hq) * p.pk_group + r / p.Sq;
 }
 
 // Number of K/V tiles the query rows [row0, row0 + 128) need.
@@ -352,13 +365,14 @@ __device__ __forceinline__ void tile_next(const FwdParams& p, TileCursor& c) {
     }
 }
 
-template <int D, int KIND, int NS, int QB, bool EPI, bool STRIDED>
+template <int D, int KIND, int NS, int QB, bool EPI, bool STRIDED, bool PACK>
 __global__ void __launch_bounds__(FwdCfg<D, KIND, NS, QB, EPI>::kThreads, 1)
 sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV,
                       const FwdParams p) {
     using C = FwdCfg<D, KIND, NS, QB, EPI>;
+    static_assert(!PACK || (STRIDED && !EPI), "packed units use the strided form without epilogue warps");
     constexpr int kLoadWarp = C::kLoadWarp;
     constexpr int kMmaWarp = C::kMmaWarp;
     extern __shared__ uint8_t smem_raw[];
@@ -402,6 +416,19 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         st_shared_u32(abort_addr, 0u);
         fence_barrier_init();
     }
+    if constexpr (PACK) {
+        // rows pk_rows..127 of every Q buffer stay zero: the packed Q box
+        // never writes them, and their scores are then finite
+        const int dead = (kBlockM - p.pk_rows) * 128;   // bytes per column block
+        for (int qb = 0; qb < QB; ++qb)
+            for (int kb = 0; kb < C::kSwBlocks; ++kb) {
+                uint8_t* blk = smem_raw + (sbase - raw) + C::kSmemQ + qb * C::kTileBytes +
+                               kb * C::kSwBlockBytes + p.pk_rows * 128;
+                for (int i = threadIdx.x * 16; i < dead; i += C::kThreads * 16)
+                    *reinterpret_cast<uint4*>(blk + i) = make_uint4(0u, 0u, 0u, 0u);
+            }
+        fence_proxy_async_smem();
+    }
     if (warp == kMmaWarp) {
         tmem_alloc(slot_addr, kTmemCols);
         tmem_relinquish();
@@ -436,10 +463,15 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                         !wait_bar(bar(C::kBarQEmpty + qb), (uint32_t)(qm - 1) & 1u,
                                   abort_addr, 0x11000u | (uint32_t)c.u.ku))
                         return false;
-                    mbar_arrive_expect_tx(bar(C::kBarQFull + qb), C::kTileBytes);
+                    mbar_arrive_expect_tx(bar(C::kBarQFull + qb), PACK ? p.pk_qbytes : C::kTileBytes);
                     for (int kb = 0; kb < C::kSwBlocks; ++kb) {
                         const uint32_t dst = sQ + qb * C::kTileBytes + kb * C::kSwBlockBytes;
-                        if constexpr (STRIDED) {
+                        if constexpr (PACK) {
+                            // box: all Sq rows of the group's pk_group query heads
+                            const int qbat = c.u.bh / p.Hq;
+                            tma_load_4d(dst, &tmQ, bar(C::kBarQFull + qb), kb * C::kElemsPerSw, 0,
+                                        (c.u.bh - qbat * p.Hq) * p.pk_group, qbat);
+                        } else if constexpr (STRIDED) {
                             const int qbat = c.u.bh / p.Hq;
                             tma_load_4d(dst, &tmQ, bar(C::kBarQFull + qb), kb * C::kElemsPerSw,
                                         c.u.qtile * kBlockM, c.u.bh - qbat * p.Hq, qbat);
@@ -681,7 +713,8 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         int g = 0;   // stream tile
         while (ok && u.valid) {
             const int m0 = u.qtile * kBlockM;
-            const int row = m0 + r;
+            // a packed unit's lane r is position r % Sq of query head r / Sq
+            const int row = PACK ? r % p.Sq : m0 + r;
             const int n = u.n;
             float m_run = -INFINITY;   // running max of this half's scaled scores (log2 units)
             float l_run = 0.0f;        // running sum of 2^(s*sl - m_run + kPLog2)
@@ -821,8 +854,14 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                     stats[2 * r] = c0;
                     stats[2 * r + 1] = c1;
                     mbar_arrive(bar(C::kBarXchg2));
-                    if (ok && p.lse != nullptr && row < p.Sq)
-                        p.lse[(size_t)u.bh * p.Sq + row] = (m + __log2f(l) - C::kPLog2) * kLn2;
+                    if constexpr (PACK) {
+                        if (ok && p.lse != nullptr && r < p.pk_rows)
+                            p.lse[(size_t)packed_qhead(p, u.bh, r) * p.Sq + row] =
+                                (m + __log2f(l) - C::kPLog2) * kLn2;
+                    } else {
+                        if (ok && p.lse != nullptr && row < p.Sq)
+                            p.lse[(size_t)u.bh * p.Sq + row] = (m + __log2f(l) - C::kPLog2) * kLn2;
+                    }
                 }
                 if (ok) {
                     ok = wait_bar(bar(C::kBarOFull), xpar, abort_addr, 0x45000u | (uint32_t)(u.ku & 0xfff));
@@ -830,8 +869,13 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 }
                 if (!ok) break;
                 tc_fence_after();
-                const bool live = row < p.Sq;
-                uint16_t* obase = reinterpret_cast<uint16_t*>(p.o) + o_offset<D, STRIDED>(p, u.bh, live ? row : 0);
+                const bool live = PACK ? r < p.pk_rows : row < p.Sq;
+                uint16_t* obase = reinterpret_cast<uint16_t*>(p.o);
+                if constexpr (PACK)
+                    obase += o_offset<D, true>(p, live ? packed_qhead(p, u.bh, r) : 0, live ? row : 0,
+                                               p.pk_hq);
+                else
+                    obase += o_offset<D, STRIDED>(p, u.bh, live ? row : 0);
                 const uint32_t tO0 = tmem + lane_base + C::kColO0, tO1 = tmem + lane_base + C::kColO1;
                 // group h writes output columns [h * D / 2, (h + 1) * D / 2)
 #pragma unroll 1

@@ -29,7 +29,7 @@ class Workload:
     Sq: int
     Sk: int
     d: int
-    causal: bool
+    causal: int             # 0 none, 1 causal (Sq == Sk), 2 aligned to the end of the keys
     dtype: str = "bf16"     # "bf16", "fp16" or "e4m3"
     seed: int = 0
     layout: str = "bhsd"    # "bhsd": [B,H,S,d] tensors; "btnh": [B,S,H,d] data passed as views
@@ -41,7 +41,12 @@ class Workload:
     @property
     def flops(self) -> float:
         """Algorithmic FLOPs of the two contractions, 4*B*Hq*Sq*Sk*d, halved
-        when causal (the masked half of the score matrix is not work)."""
+        when causal (the masked half of the score matrix is not work); for
+        the mask aligned to the end of the keys (causal == 2) the visible
+        (query, key) pairs are counted exactly."""
+        if self.causal == 2:
+            pairs = self.Sq * (self.Sk - self.Sq) + self.Sq * (self.Sq + 1) / 2.0
+            return 4.0 * self.B * self.Hq * pairs * self.d
         f = 4.0 * self.B * self.Hq * self.Sq * self.Sk * self.d
         return f / 2.0 if self.causal else f
 
@@ -76,6 +81,10 @@ WORKLOADS = {
                     seed=42),
     "fp8": Workload("fp8_b2_h32_s16384_d128_causal", 2, 32, 32, 16384, 16384, 128, True,
                     dtype="e4m3", seed=9000),
+    # decode-shaped GQA: one new token per sequence against an 8192-key cache
+    # (the codelab's KV-cache motivation, section 9); query heads packed
+    "decode_gqa": Workload("decode_gqa_b64_hq32_hkv8_sq1_sk8192_d128", 64, 32, 8, 1, 8192, 128, 2,
+                           seed=8192),
     # profiling-sized cases: inputs above the 126 MB L2, a few hundred MB in all
     "lm_causal_b4": Workload("lm_causal_b4_h16_s4096_d128", 4, 16, 16, 4096, 4096, 128, True,
                              seed=4096),

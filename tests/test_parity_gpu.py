@@ -288,6 +288,52 @@ def test_bottom_right_decode_batch_sampled(sdpa):
     assert np.abs(lse.reshape(-1).index_select(0, idx).double().cpu().numpy() - rl).max() <= LSE_TOL
 
 
+# ---- decode-shaped GQA / MQA: the query heads of a K/V head share one tile ---------
+
+PACKED = [
+    # (B, Hq, Hkv, Sq, Sk, d, causal): group * Sq <= 128 rows in one unit
+    (2, 8, 2, 1, 1000, 128, 0),
+    (2, 8, 2, 1, 1000, 128, 2),
+    (3, 32, 1, 4, 2000, 128, 2),      # MQA, 128 rows exactly
+    (2, 16, 4, 16, 777, 64, 2),
+    (1, 6, 2, 5, 300, 64, 0),         # group of 3, 15 rows
+    (2, 4, 2, 40, 40, 128, 1),        # causal Sq == Sk inside a packed tile
+    (1, 8, 1, 9, 4100, 128, 2),       # long cache
+]
+
+
+@pytest.mark.parametrize("shape", PACKED, ids=lambda s: "b%d_hq%d_hkv%d_sq%d_sk%d_d%d_c%d" % s)
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_packed_query_heads(sdpa, shape, dtype):
+    B, Hq, Hkv, Sq, Sk, d, causal = shape
+    w = Workload("pk", B, Hq, Hkv, Sq, Sk, d, False, dtype=dtype, seed=11 * Sq + Sk)
+    q, k, v = make_qkv(w, "cuda")
+    lse = torch.full((B, Hq, Sq), float("nan"), device="cuda")
+    o, lse = sdpa.attention(q, k, v, causal=causal, scale=w.scale, lse=lse)
+    torch.cuda.synchronize()
+    st, detail = sdpa.sdpa_device_status(clear=True)
+    assert st == 0, "device status %d detail %#x" % (st, detail)
+    ro, rl = oracle.sdpa_fwd(q.cpu(), k.cpu(), v.cpu(), w.scale, causal=causal)
+    check_o(o.double().cpu().numpy(), ro, O_TOL, dtype, "packed")
+    assert np.abs(lse.double().cpu().numpy() - rl).max() <= LSE_TOL
+
+
+def test_packed_btnh_decode_views(sdpa):
+    """One new token per sequence in the codelab's layout: Q [B,1,N,d] and a
+    [B,S,K,d] cache as views, packed 8 query heads per K/V head."""
+    w = Workload("pkv", 4, 16, 2, 1, 1500, 128, False, seed=99)
+    qb, kb, vb = make_qkv_btnh(w, "cuda")
+    ob = torch.zeros_like(qb)
+    o, lse = sdpa.attention(qb.transpose(1, 2), kb.transpose(1, 2), vb.transpose(1, 2),
+                            causal="bottom_right", out=ob.transpose(1, 2))
+    torch.cuda.synchronize()
+    assert sdpa.sdpa_device_status(clear=True)[0] == 0
+    ro, rl = oracle.sdpa_fwd(*(t.transpose(1, 2).contiguous().cpu() for t in (qb, kb, vb)),
+                             w.scale, causal=2)
+    check_o(ob.transpose(1, 2).double().cpu().numpy(), ro, O_TOL, "bf16", "packed btnh")
+    assert np.abs(lse.double().cpu().numpy() - rl).max() <= LSE_TOL
+
+
 # ---- strided views (sdpa_fwd_strided) ---------------------------------------------
 
 BTNH = [
@@ -352,7 +398,8 @@ def run_fp8(lib, w):
 
 @pytest.mark.parametrize("shape", [(1, 2, 2, 256, 256, True), (1, 2, 1, 333, 333, True),
                                    (2, 4, 2, 200, 500, False), (1, 2, 2, 150, 3300, False),
-                                   (1, 2, 2, 100, 500, "bottom_right")])
+                                   (1, 2, 2, 100, 500, "bottom_right"),
+                                   (2, 8, 1, 2, 1500, "bottom_right")])   # packed query heads
 def test_fp8_small(sdpa, shape):
     B, Hq, Hkv, Sq, Sk, causal = shape
     w = Workload("f8", B, Hq, Hkv, Sq, Sk, 128, causal, dtype="e4m3", seed=Sq + Sk)
