@@ -73,7 +73,8 @@ typedef enum {
                                     non-finite or non-positive scale, a pointer
                                     not 16-byte aligned, sizes whose element
                                     counts overflow the addressing limits */
-    SDPA_ERR_UNSUPPORTED = 2,    /* d not 64 or 128, SDPA_CAUSAL with Sq != Sk,
+    SDPA_ERR_UNSUPPORTED = 2,    /* d not 32, 64 or 128 (FP8: not 128),
+                                    SDPA_CAUSAL with Sq != Sk,
                                     SDPA_CAUSAL_BOTTOM_RIGHT with Sq > Sk,
                                     unknown dtype, device not sm_100 */
     SDPA_ERR_CUDA = 3,           /* the CUDA runtime or driver reported an
@@ -89,6 +90,7 @@ typedef enum {
 /*
  * sdpa_fwd -- fused attention forward, bf16 or fp16.
  *
+ *   d                head dim: 32, 64 or 128
  *   q    [B,Hq,Sq,d]  in,  dtype
  *   k, v [B,Hkv,Sk,d] in,  dtype
  *   o    [B,Hq,Sq,d]  out, dtype (rounded to nearest even from fp32)

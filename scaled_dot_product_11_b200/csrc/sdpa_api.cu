@@ -80,7 +80,7 @@ int check_args(const void* q, const void* k, const void* v, const void* o, const
     const long long bhq = (long long)B * Hq, bhk = (long long)B * Hkv;
     const long long qblocks = (Sq + 127) / 128;
     if (bhq > INT32_MAX || bhk > INT32_MAX || bhq * qblocks > INT32_MAX) return SDPA_ERR_INVALID_ARG;
-    if (d != 64 && d != 128) return SDPA_ERR_UNSUPPORTED;
+    if (d != 32 && d != 64 && d != 128) return SDPA_ERR_UNSUPPORTED;
     if (causal == SDPA_CAUSAL && Sq != Sk) return SDPA_ERR_UNSUPPORTED;
     if (causal == SDPA_CAUSAL_BOTTOM_RIGHT && Sq > Sk) return SDPA_ERR_UNSUPPORTED;
     return SDPA_OK;
@@ -102,6 +102,9 @@ bool same(const View& a, const View& b) { return a.sb == b.sb && a.sh == b.sh &&
 bool encode_view(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* base, int d,
                  int rows, int heads, int batch, const View& v, int box_inner, bool rank3,
                  int box_rows = 128, int box_heads = 1) {
+    // swizzle rows of box_inner elements: 128 bytes, or 64 (head dim 32, 16-bit)
+    const CUtensorMapSwizzle swz =
+        box_inner * elem_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint32_t rank = rank3 ? 3u : 4u;
@@ -112,7 +115,7 @@ bool encode_view(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const v
     const cuuint32_t box[4] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, (cuuint32_t)box_heads, 1u};
     const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
     return fn(m, dt, rank, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -271,10 +274,12 @@ int fwd_16bit(const void* q, const void* k, const void* v, void* o, float* lse, 
     prm.score_log2 = scale * sdpa::kLog2e;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (dtype == SDPA_BF16)
-        return d == 64 ? launch<64, sdpa::KIND_BF16, SDPA_STAGES_D64, 2>(q, k, v, vq, vk, vv, prm, s)
-                       : launch<128, sdpa::KIND_BF16, SDPA_STAGES_D128, 1>(q, k, v, vq, vk, vv, prm, s);
-    return d == 64 ? launch<64, sdpa::KIND_FP16, SDPA_STAGES_D64, 2>(q, k, v, vq, vk, vv, prm, s)
-                   : launch<128, sdpa::KIND_FP16, SDPA_STAGES_D128, 1>(q, k, v, vq, vk, vv, prm, s);
+        return d == 32   ? launch<32, sdpa::KIND_BF16, SDPA_STAGES_D32, 2>(q, k, v, vq, vk, vv, prm, s)
+               : d == 64 ? launch<64, sdpa::KIND_BF16, SDPA_STAGES_D64, 2>(q, k, v, vq, vk, vv, prm, s)
+                         : launch<128, sdpa::KIND_BF16, SDPA_STAGES_D128, 1>(q, k, v, vq, vk, vv, prm, s);
+    return d == 32   ? launch<32, sdpa::KIND_FP16, SDPA_STAGES_D32, 2>(q, k, v, vq, vk, vv, prm, s)
+           : d == 64 ? launch<64, sdpa::KIND_FP16, SDPA_STAGES_D64, 2>(q, k, v, vq, vk, vv, prm, s)
+                     : launch<128, sdpa::KIND_FP16, SDPA_STAGES_D128, 1>(q, k, v, vq, vk, vv, prm, s);
 }
 
 }  // namespace

@@ -68,6 +68,9 @@
 #ifndef SDPA_STAGES_D64
 #define SDPA_STAGES_D64 8
 #endif
+#ifndef SDPA_STAGES_D32
+#define SDPA_STAGES_D32 16
+#endif
 #ifndef SDPA_STAGES_FP8
 #define SDPA_STAGES_FP8 10
 #endif
@@ -119,9 +122,14 @@ struct FwdCfg {
     static constexpr int kTmemUsers = 256 + 32 + (EPI ? 128 : 0);   // softmax, MMA, epilogue threads
     static constexpr int kElem = (KIND == KIND_E4M3) ? 1 : 2;
     static constexpr int kRowBytes = D * kElem;
-    static constexpr int kElemsPerSw = 128 / kElem;      // elements in one 128-byte swizzle row
-    static constexpr int kSwBlocks = kRowBytes / 128;    // 128-byte column blocks per row
-    static constexpr int kSwBlockBytes = 128 * 128;      // one column block of a 128-row tile
+    // swizzle rows of 128 bytes (64 when a whole row is 64 bytes: d = 32)
+    static constexpr int kSwBytes = kRowBytes >= 128 ? 128 : kRowBytes;
+    static constexpr uint32_t kSwLayout = kSwBytes == 128 ? 2u : 4u;   // descriptor swizzle field
+    static constexpr int kSbo = 8 * kSwBytes;            // 8-row core-matrix group stride
+    static constexpr int kElemsPerSw = kSwBytes / kElem; // elements in one swizzle row
+    static constexpr int kSwBlocks = kRowBytes / kSwBytes;   // swizzle column blocks per row
+    static constexpr int kSwBlockBytes = 128 * kSwBytes; // one column block of a 128-row tile
+    static constexpr int kStepsPerBlock = kSwBytes / 32; // MMA K steps (32 bytes) per block
     static constexpr int kTileBytes = 128 * kRowBytes;
     static constexpr int kQkSteps = kRowBytes / 32;      // every MMA consumes 32 bytes of K
     static constexpr int kPvKeysPerStep = 32 / kElem;
@@ -160,7 +168,8 @@ struct FwdCfg {
     static constexpr int kSmemBytes = (kSmemUsed + 1024 <= 232448) ? kSmemUsed + 1024 : 232448;
     // TMEM columns
     static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
-    static_assert(kRowBytes % 128 == 0, "rows must fill whole 128-byte swizzle rows");
+    static_assert(kSwBytes == 128 || kSwBytes == 64, "rows of 64 bytes or whole 128-byte swizzle rows");
+    static_assert(kRowBytes % kSwBytes == 0, "rows must fill whole swizzle rows");
     static_assert(kSmemUsed <= 232448, "shared memory budget");
     static_assert(kSmemBytes > 116 * 1024, "one CTA per SM (each allocates all of TMEM)");
     static_assert(D <= 128, "O tile must fit its 128 TMEM columns");
@@ -419,11 +428,11 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     if constexpr (PACK) {
         // rows pk_rows..127 of every Q buffer stay zero: the packed Q box
         // never writes them, and their scores are then finite
-        const int dead = (kBlockM - p.pk_rows) * 128;   // bytes per column block
+        const int dead = (kBlockM - p.pk_rows) * C::kSwBytes;   // bytes per column block
         for (int qb = 0; qb < QB; ++qb)
             for (int kb = 0; kb < C::kSwBlocks; ++kb) {
                 uint8_t* blk = smem_raw + (sbase - raw) + C::kSmemQ + qb * C::kTileBytes +
-                               kb * C::kSwBlockBytes + p.pk_rows * 128;
+                               kb * C::kSwBlockBytes + p.pk_rows * C::kSwBytes;
                 for (int i = threadIdx.x * 16; i < dead; i += C::kThreads * 16)
                     *reinterpret_cast<uint4*>(blk + i) = make_uint4(0u, 0u, 0u, 0u);
             }
@@ -540,9 +549,9 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         constexpr uint32_t fmt = (KIND == KIND_BF16) ? 1u : 0u;
         constexpr uint32_t idesc_qk = make_idesc(fmt, false, kBlockM, kBlockN);
         constexpr uint32_t idesc_pv = make_idesc(fmt, true, kBlockM, D);
-        const uint64_t desc_q = make_smem_desc(sQ, 16, 1024);
-        const uint64_t desc_k = make_smem_desc(sKV, 16, 1024);
-        const uint64_t desc_v = make_smem_desc(sKV, C::kSwBlockBytes, 1024);
+        const uint64_t desc_q = make_smem_desc(sQ, 16, C::kSbo, C::kSwLayout);
+        const uint64_t desc_k = make_smem_desc(sKV, 16, C::kSbo, C::kSwLayout);
+        const uint64_t desc_v = make_smem_desc(sKV, C::kSwBlockBytes, C::kSbo, C::kSwLayout);
         bool ok = true;
         int t = 0;   // K/V tiles consumed
 
@@ -567,7 +576,8 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             if (leader) {
 #pragma unroll
                 for (int kk = 0; kk < C::kQkSteps; ++kk) {
-                    const uint64_t off = (uint64_t)(((kk >> 2) * C::kSwBlockBytes + (kk & 3) * 32) >> 4);
+                    const uint64_t off = (uint64_t)(((kk / C::kStepsPerBlock) * C::kSwBlockBytes +
+                                                     (kk % C::kStepsPerBlock) * 32) >> 4);
                     if constexpr (KIND == KIND_E4M3)
                         mma_f8_ss(d_tmem, dq + off, dk + off, idesc_qk, kk > 0);
                     else
@@ -581,11 +591,11 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         auto issue_pv = [&](int h, int buf, int slot, bool acc) {
             const uint32_t d_tmem = tmem + (h ? C::kColO1 : C::kColO0);
             const uint32_t a_tmem = tmem + (buf ? C::kColS1 : C::kColS0) + h * kHalfN;
-            const uint64_t dv = desc_v + (uint64_t)((slot * C::kTileBytes + h * kHalfN * 128) >> 4);
+            const uint64_t dv = desc_v + (uint64_t)((slot * C::kTileBytes + h * kHalfN * C::kSwBytes) >> 4);
             if (leader) {
 #pragma unroll
                 for (int kk = 0; kk < C::kPvStepsHalf; ++kk) {
-                    const uint64_t off = (uint64_t)((kk * C::kPvKeysPerStep * 128) >> 4);
+                    const uint64_t off = (uint64_t)((kk * C::kPvKeysPerStep * C::kSwBytes) >> 4);
                     const uint32_t accum = (acc || kk > 0) ? 1u : 0u;
                     if constexpr (KIND == KIND_E4M3)
                         mma_f8_ts(d_tmem, a_tmem + kk * 8, dv + off, idesc_pv, accum);
@@ -878,6 +888,26 @@ sdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                     obase += o_offset<D, STRIDED>(p, u.bh, live ? row : 0);
                 const uint32_t tO0 = tmem + lane_base + C::kColO0, tO1 = tmem + lane_base + C::kColO1;
                 // group h writes output columns [h * D / 2, (h + 1) * D / 2)
+                if constexpr (D == 32) {
+                    float x[16], y[16];
+                    tmem_ld16(tO0 + 16 * h, x);
+                    tmem_ld16(tO1 + 16 * h, y);
+                    tmem_wait_ld();
+                    reg_fence16(x);
+                    reg_fence16(y);
+                    uint32_t w4[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float v0 = x[2 * e] * c0 + y[2 * e] * c1;
+                        const float v1 = x[2 * e + 1] * c0 + y[2 * e + 1] * c1;
+                        w4[e] = (KIND == KIND_FP16) ? pack_f16x2(v0, v1) : pack_bf16x2(v0, v1);
+                    }
+                    if (live) {
+                        uint4* dst = reinterpret_cast<uint4*>(obase + 16 * h);
+                        dst[0] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                        dst[1] = make_uint4(w4[4], w4[5], w4[6], w4[7]);
+                    }
+                }
 #pragma unroll 1
                 for (int c = h * (D / 64); c < (h + 1) * (D / 64); ++c) {
                     float x[32], y[32];

@@ -263,14 +263,15 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* u) {
 //   bit  52    leading-offset mode (0: relative)
 //   bits 61-63 swizzle: 0 none, 2 = 128B, 4 = 64B, 6 = 32B
 // ---------------------------------------------------------------------------
+// `layout`: the swizzle field, 2 = 128-byte swizzle, 4 = 64-byte swizzle.
 __device__ __forceinline__ uint64_t make_smem_desc(uint32_t saddr, uint32_t lbo_bytes,
-                                                   uint32_t sbo_bytes) {
+                                                   uint32_t sbo_bytes, uint32_t layout = 2) {
     uint64_t desc = 0;
     desc |= (uint64_t)((saddr >> 4) & 0x3FFF);
     desc |= (uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16;
     desc |= (uint64_t)((sbo_bytes >> 4) & 0x3FFF) << 32;
     desc |= (uint64_t)1 << 46;
-    desc |= (uint64_t)2 << 61;   // 128-byte swizzle
+    desc |= (uint64_t)(layout & 7u) << 61;
     return desc;
 }
 

@@ -74,7 +74,7 @@ def call(**kw):
     (dict(ptrs=(P, P, P, P, P + 2)), 1),
     (dict(causal=3), 1), (dict(causal=-1), 1),
     (dict(B=1 << 16, Hq=1 << 16, Hkv=1 << 16), 1),
-    (dict(d=96), 2), (dict(d=256), 2), (dict(d=32), 2),
+    (dict(d=96), 2), (dict(d=256), 2), (dict(d=16), 2), (dict(d=48), 2),
     (dict(causal=1, Sq=128, Sk=256), 2),
     (dict(causal=2, Sq=257, Sk=256), 2),
     (dict(dtype=2), 2), (dict(dtype=-1), 2),

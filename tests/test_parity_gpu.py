@@ -123,6 +123,11 @@ SMALL = [
     (1, 2, 2, 200, 3200, 128, False),
     (1, 4, 2, 130, 3329, 128, False),
     (1, 2, 2, 100, 3100, 64, False),
+    # head dim 32 (64-byte rows, 64-byte swizzle)
+    (1, 2, 2, 256, 256, 32, False),
+    (1, 3, 3, 300, 300, 32, True),
+    (2, 4, 2, 100, 700, 32, False),
+    (1, 2, 2, 130, 3329, 32, False),
 ]
 
 
@@ -299,6 +304,7 @@ PACKED = [
     (1, 6, 2, 5, 300, 64, 0),         # group of 3, 15 rows
     (2, 4, 2, 40, 40, 128, 1),        # causal Sq == Sk inside a packed tile
     (1, 8, 1, 9, 4100, 128, 2),       # long cache
+    (2, 8, 2, 3, 900, 32, 2),         # head dim 32
 ]
 
 
@@ -342,6 +348,7 @@ BTNH = [
     (1, 8, 2, 300, 300, 128, True),
     (2, 4, 4, 640, 640, 128, True),
     (1, 4, 1, 130, 3329, 128, False),   # long units: the form without epilogue warps
+    (2, 4, 4, 256, 256, 32, True),      # head dim 32, the codelab's suggested variant
 ]
 
 
