@@ -18,6 +18,10 @@ Parity status of each function (what pins it, in ``tests/test_oracle.py``):
                    equality with the causal mask when Sq == Sk, with no mask
                    when Sq == 1, and row by row with unmasked attention over
                    the visible key prefix.
+  sdpa_bwd         pinned: central differences of sdpa_fwd (no mask, causal,
+                   end-aligned causal, GQA) to 1e-8, the single-key closed
+                   form, invariance to a common key shift, GQA == summed
+                   repeated-KV MHA.
   sdpa_rows        pinned: equals sdpa_fwd on the same rows (same per-row code
                    reached through a different index path) and the pins above.
   sdpa_bruteforce  pinned: mpmath evaluation, weights-sum, V = identity.
@@ -64,6 +68,9 @@ def _load():
                                          vp, vp, i32, i32, i32, i32, i32, i32, f64, i32, i32]
         lib.oracle_sdpa_bruteforce.argtypes = [vp, vp, vp, i32, f64, f64, f64, vp, vp, vp,
                                                i32, i32, i32, i32, i32, i32, f64, i32]
+        lib.oracle_sdpa_bwd.argtypes = [vp, vp, vp, vp, i32, vp, vp, vp,
+                                        i32, i32, i32, i32, i32, i32, f64, i32, i32]
+        lib.oracle_sdpa_bwd.restype = i32
         lib.oracle_decode_bf16.argtypes = [ctypes.c_uint16]
         lib.oracle_decode_bf16.restype = f64
         lib.oracle_decode_f16.argtypes = [ctypes.c_uint16]
@@ -170,6 +177,28 @@ def sdpa_rows(q, k, v, rows, scale: float, causal: bool = False, descales=(1.0, 
                                 r.ctypes.data, r.size, o.ctypes.data, lse.ctypes.data,
                                 B, Hq, Hkv, Sq, Sk, d, float(scale), _mask(causal), nt))
     return o, lse
+
+
+def sdpa_bwd(q, k, v, dout, scale: float, causal=False, nthreads: int | None = None):
+    """Gradients (dQ, dK, dV) as float64 arrays of q's, k's and v's shapes
+    for the loss whose gradient with respect to O is `dout` (q's shape and
+    storage type; bf16, fp16 or float)."""
+    lib = _load()
+    qa, ka, va, t = _prep(q, k, v)
+    da, td = _raw(dout)
+    if td != t:
+        raise ValueError("dout must share q's storage type")
+    B, Hq, Hkv, Sq, Sk, d = _shape(q, k)
+    if tuple(da.shape) != (B, Hq, Sq, d):
+        raise ValueError("dout must have q's shape")
+    dq = np.empty((B, Hq, Sq, d), np.float64)
+    dk = np.empty((B, Hkv, Sk, d), np.float64)
+    dv = np.empty((B, Hkv, Sk, d), np.float64)
+    nt = nthreads or max_threads()
+    _check(lib.oracle_sdpa_bwd(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, da.ctypes.data, t,
+                               dq.ctypes.data, dk.ctypes.data, dv.ctypes.data,
+                               B, Hq, Hkv, Sq, Sk, d, float(scale), _mask(causal), nt))
+    return dq, dk, dv
 
 
 def sdpa_bruteforce(q, k, v, scale: float, causal: bool = False, descales=(1.0, 1.0, 1.0),

@@ -301,3 +301,93 @@ int oracle_max_threads(void) {
     return 1;
 #endif
 }
+
+/*
+ * Backward of the same forward: given dO = dL/dO for a loss L, the gradients
+ * dL/dQ, dL/dK, dL/dV (codelab section 12 suggests training with these
+ * kernels; the article's section 3 keeps the per-row statistics so that the
+ * backward can recompute the weights).  For every (b, hq, i), with the
+ * weights p_j of the forward (recomputed here in fp64, two-pass):
+ *
+ *   dp_j = dO_i . V_j                      (gradient of the weights)
+ *   D_i  = sum_j p_j dp_j                  (= dO_i . O_i)
+ *   ds_j = p_j (dp_j - D_i)                (softmax Jacobian applied to dp)
+ *   dQ_i   = scale * sum_j ds_j K_j
+ *   dK_j  += scale * ds_j Q_i              (summed over the rows and over the
+ *   dV_j  += p_j dO_i                       query heads sharing K/V head hk)
+ *
+ * dout has Q's shape and storage type.  dq: [B,Hq,Sq,d], dk, dv: [B,Hkv,Sk,d]
+ * doubles.  Work is split by (b, hk), so every dK/dV row has one writer.
+ */
+int oracle_sdpa_bwd(const void* q, const void* k, const void* v, const void* dout, int dtype,
+                    double* dq_out, double* dk_out, double* dv_out,
+                    int B, int Hq, int Hkv, int Sq, int Sk, int d,
+                    double scale, int causal, int nthreads) {
+    problem_t p = {q, k, v, dtype, 1.0, 1.0, 1.0, B, Hq, Hkv, Sq, Sk, d, scale, causal};
+    int rc = check_problem(&p);
+    if (rc) return rc;
+    if (!dout || !dq_out || !dk_out || !dv_out || dtype == ORC_E4M3) return 1;
+    memset(dk_out, 0, sizeof(double) * (size_t)B * Hkv * Sk * d);
+    memset(dv_out, 0, sizeof(double) * (size_t)B * Hkv * Sk * d);
+    const int group = Hq / Hkv;
+    if (nthreads <= 0) nthreads = 1;
+    int failed = 0;
+#pragma omp parallel num_threads(nthreads)
+    {
+        double* s = (double*)malloc(sizeof(double) * (size_t)Sk * 2);
+        if (!s) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+            double* dp = s + Sk;
+#pragma omp for schedule(dynamic, 1)
+            for (long long bk = 0; bk < (long long)B * Hkv; ++bk) {
+                const int b = (int)(bk / Hkv), hk = (int)(bk % Hkv);
+                const size_t kvhead = ((size_t)b * Hkv + hk) * Sk;
+                for (int hq = hk * group; hq < (hk + 1) * group; ++hq) {
+                    for (int i = 0; i < Sq; ++i) {
+                        const size_t qoff = (((size_t)b * Hq + hq) * Sq + i) * d;
+                        const int nkeys = causal == 1 ? i + 1 : causal == 2 ? i + 1 + (Sk - Sq) : Sk;
+                        double m = -INFINITY;
+                        for (int j = 0; j < nkeys; ++j) {
+                            double acc = 0.0, accd = 0.0;
+                            for (int c = 0; c < d; ++c) {
+                                acc += load_elem(q, dtype, qoff + c, 1.0) *
+                                       load_elem(k, dtype, (kvhead + j) * d + c, 1.0);
+                                accd += load_elem(dout, dtype, qoff + c, 1.0) *
+                                        load_elem(v, dtype, (kvhead + j) * d + c, 1.0);
+                            }
+                            s[j] = scale * acc;
+                            dp[j] = accd;
+                            if (s[j] > m) m = s[j];
+                        }
+                        double l = 0.0;
+                        for (int j = 0; j < nkeys; ++j) {
+                            s[j] = exp(s[j] - m);
+                            l += s[j];
+                        }
+                        double Di = 0.0;
+                        for (int j = 0; j < nkeys; ++j) {
+                            s[j] /= l;                 /* p_j */
+                            Di += s[j] * dp[j];
+                        }
+                        double* dqi = dq_out + qoff;
+                        for (int c = 0; c < d; ++c) dqi[c] = 0.0;
+                        for (int j = 0; j < nkeys; ++j) {
+                            const double ds = s[j] * (dp[j] - Di);
+                            double* dkj = dk_out + (kvhead + j) * d;
+                            double* dvj = dv_out + (kvhead + j) * d;
+                            for (int c = 0; c < d; ++c) {
+                                dqi[c] += scale * ds * load_elem(k, dtype, (kvhead + j) * d + c, 1.0);
+                                dkj[c] += scale * ds * load_elem(q, dtype, qoff + c, 1.0);
+                                dvj[c] += s[j] * load_elem(dout, dtype, qoff + c, 1.0);
+                            }
+                        }
+                    }
+                }
+            }
+            free(s);
+        }
+    }
+    return failed ? 3 : 0;
+}

@@ -380,3 +380,77 @@ def test_bottom_right_rejects_more_queries_than_keys():
     q, k, v = rand(1, 2, 6, 8), rand(1, 2, 5, 8), rand(1, 2, 5, 8)
     with pytest.raises(ValueError):
         oracle.sdpa_fwd(q, k, v, 1.0, causal=2)
+
+
+# --------------------------------------------------------------------------
+# backward: dQ, dK, dV of the loss L = sum(dO * O)
+# --------------------------------------------------------------------------
+
+def _loss(q, k, v, dout, scale, causal):
+    o, _ = oracle.sdpa_fwd(q, k, v, scale, causal)
+    return float((o * dout).sum())
+
+
+@pytest.mark.parametrize("causal", [0, 1, 2])
+def test_backward_matches_finite_differences_of_the_forward(causal):
+    """Central differences of the (independently pinned) forward oracle:
+    every sampled coordinate of dQ, dK, dV agrees to 1e-8."""
+    B, Hq, Hkv, d = 1, 4, 2, 6
+    Sq, Sk = (7, 7) if causal != 2 else (5, 9)
+    q, k, v = rand(B, Hq, Sq, d), rand(B, Hkv, Sk, d), rand(B, Hkv, Sk, d)
+    dout = rand(B, Hq, Sq, d)
+    sc = 0.43
+    dq, dk, dv = oracle.sdpa_bwd(q, k, v, dout, sc, causal)
+    h = 1e-5
+    pick = np.random.default_rng(causal + 7)
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for _ in range(12):
+            idx = tuple(int(pick.integers(0, n)) for n in x.shape)
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = {"q": q, "k": k, "v": v}
+            args_m = dict(args_p)
+            args_p[name], args_m[name] = xp, xm
+            fd = (_loss(args_p["q"], args_p["k"], args_p["v"], dout, sc, causal) -
+                  _loss(args_m["q"], args_m["k"], args_m["v"], dout, sc, causal)) / (2 * h)
+            assert abs(fd - g[idx]) < 1e-8 * max(1.0, abs(fd)), (name, idx, fd, g[idx])
+
+
+def test_backward_single_key_closed_form():
+    """One key: the weights are all 1, so dQ = dK = 0 and dV is the sum of
+    dO over the rows and query heads sharing the key."""
+    q, k, v = rand(2, 4, 5, 3), rand(2, 2, 1, 3), rand(2, 2, 1, 3)
+    dout = rand(2, 4, 5, 3)
+    dq, dk, dv = oracle.sdpa_bwd(q, k, v, dout, 0.7)
+    assert np.abs(dq).max() < 1e-14 and np.abs(dk).max() < 1e-14
+    expect = dout.reshape(2, 2, 2, 5, 3).sum(axis=(2, 3))[:, :, None, :]
+    np.testing.assert_allclose(dv, expect, rtol=0, atol=1e-13)
+
+
+def test_backward_dq_invariant_to_a_common_key_shift():
+    """Adding one vector to every key shifts each row's scores by a constant:
+    the weights, dS and hence dK and dV are unchanged, and dQ too because
+    sum_j ds_j = 0 per row."""
+    q, k, v = rand(1, 2, 6, 5), rand(1, 2, 6, 5), rand(1, 2, 6, 5)
+    dout = rand(1, 2, 6, 5)
+    dq1, dk1, dv1 = oracle.sdpa_bwd(q, k, v, dout, 0.5)
+    shift = rand(5)
+    # the shift changes the scores by q . shift, constant per row: same weights
+    dq2, dk2, dv2 = oracle.sdpa_bwd(q, k + shift, v, dout, 0.5)
+    np.testing.assert_allclose(dq1, dq2, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dk1, dk2, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dv1, dv2, rtol=0, atol=1e-12)
+
+
+def test_backward_gqa_equals_summed_repeated_kv_mha():
+    B, Hq, Hkv, S, d = 1, 6, 2, 5, 4
+    q, k, v = rand(B, Hq, S, d), rand(B, Hkv, S, d), rand(B, Hkv, S, d)
+    dout = rand(B, Hq, S, d)
+    dq, dk, dv = oracle.sdpa_bwd(q, k, v, dout, 0.6, True)
+    g = Hq // Hkv
+    kr, vr = np.repeat(k, g, axis=1), np.repeat(v, g, axis=1)
+    dq2, dk2, dv2 = oracle.sdpa_bwd(q, kr, vr, dout, 0.6, True)
+    np.testing.assert_allclose(dq, dq2, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dk, dk2.reshape(B, Hkv, g, S, d).sum(axis=2), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dv, dv2.reshape(B, Hkv, g, S, d).sum(axis=2), rtol=0, atol=1e-13)
