@@ -160,6 +160,29 @@ SDPA_API int sdpa_fwd_fp8(const void* q8, const void* k8, const void* v8,
                  int B, int Hq, int Hkv, int Sq, int Sk, int d,
                  float scale, int causal, void* stream);
 
+/*
+ * sdpa_bwd -- gradients of sdpa_fwd: dQ, dK, dV for the loss whose gradient
+ * with respect to O is dout (article "Self-attention, CUDA kernels and
+ * FlashAttention", section 3: the weights are recomputed from the kept
+ * per-row statistics instead of being stored).
+ *
+ *   q, o, dout, dq  [B,Hq,Sq,d]  dtype, contiguous (dq written)
+ *   k, v, dk, dv    [B,Hkv,Sk,d] dtype, contiguous (dk, dv written; for GQA
+ *                   summed over the query heads sharing each K/V head)
+ *   lse             [B,Hq,Sq] float32 as written by sdpa_fwd for the same
+ *                   q, k, v, scale and causal (required)
+ *   other arguments as sdpa_fwd.
+ *
+ * Two kernel launches (keys-major for dK/dV, rows-major for dQ), each output
+ * element written once: deterministic, no scratch memory.  Arithmetic is
+ * fp32.  Errors as sdpa_fwd, plus SDPA_ERR_INVALID_ARG for a null dout, lse,
+ * dq, dk or dv, and for B*Hq above 65535.
+ */
+SDPA_API int sdpa_bwd(const void* q, const void* k, const void* v, const void* o,
+                      const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                      int B, int Hq, int Hkv, int Sq, int Sk, int d,
+                      float scale, int causal, int dtype, void* stream);
+
 /* Static, NUL-terminated description of a status code. */
 SDPA_API const char* sdpa_strerror(int status);
 

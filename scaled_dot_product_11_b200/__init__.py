@@ -18,7 +18,7 @@ __all__ = [
     "SDPA_BF16", "SDPA_FP16", "SDPA_OK", "SDPA_ERR_INVALID_ARG", "SDPA_ERR_UNSUPPORTED",
     "SDPA_ERR_CUDA", "SDPA_ERR_DEVICE_TIMEOUT", "SDPA_ERR_DEVICE_LAYOUT", "SdpaError", "LIB_PATH",
     "SDPA_NO_MASK", "SDPA_CAUSAL", "SDPA_CAUSAL_BOTTOM_RIGHT",
-    "sdpa_fwd", "sdpa_fwd_strided", "sdpa_fwd_fp8", "sdpa_strerror", "sdpa_device_status",
+    "sdpa_fwd", "sdpa_fwd_strided", "sdpa_fwd_fp8", "sdpa_bwd", "attention_backward", "sdpa_strerror", "sdpa_device_status",
     "sdpa_launches_per_call", "attention", "attention_fp8",
 ]
 
@@ -49,6 +49,8 @@ _ll3 = ctypes.c_longlong * 3
 _lib.sdpa_fwd_strided.argtypes = ([_vp] * 5 + [_i] * 6 + [ctypes.POINTER(ctypes.c_longlong)] * 4
                                   + [_f, _i, _i, _vp])
 _lib.sdpa_fwd_strided.restype = _i
+_lib.sdpa_bwd.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _i, _i, _vp]
+_lib.sdpa_bwd.restype = _i
 _lib.sdpa_fwd_fp8.argtypes = [_vp, _vp, _vp, _f, _f, _f, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]
 _lib.sdpa_fwd_fp8.restype = _i
 _lib.sdpa_strerror.argtypes = [_i]
@@ -82,6 +84,13 @@ def sdpa_fwd_fp8(q8, k8, v8, descale_q, descale_k, descale_v, o, lse, B, Hq, Hkv
     return int(_lib.sdpa_fwd_fp8(q8, k8, v8, float(descale_q), float(descale_k), float(descale_v),
                                  o, lse or None, B, Hq, Hkv, Sq, Sk, d, float(scale), int(causal),
                                  stream or None))
+
+
+def sdpa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Sq, Sk, d, scale, causal, dtype,
+             stream) -> int:
+    """Raw backward call: device addresses as ints, stream an int."""
+    return int(_lib.sdpa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Sq, Sk, d,
+                             float(scale), int(causal), int(dtype), stream or None))
 
 
 def sdpa_strerror(status: int) -> str:
@@ -199,3 +208,28 @@ def attention_fp8(q8, k8, v8, descales, causal=False, scale: float | None = None
     if rc != SDPA_OK:
         raise SdpaError(rc, "sdpa_fwd_fp8")
     return out, lse
+
+
+def attention_backward(q, k, v, o, lse, dout, causal=False, scale: float | None = None,
+                       stream=None):
+    """(dQ, dK, dV) for contiguous bf16 / fp16 CUDA tensors: q, o, dout
+    [B,Hq,Sq,d], k, v [B,Hkv,Sk,d], lse [B,Hq,Sq] float32 from attention()
+    with the same causal and scale."""
+    import torch
+    B, Hq, Hkv, Sq, Sk, d = _dims(q, k, v)
+    causal = _causal_code(causal)
+    for t in (o, dout):
+        if tuple(t.shape) != (B, Hq, Sq, d) or t.dtype != q.dtype or not t.is_contiguous():
+            raise ValueError("o and dout must be contiguous, q's shape and dtype")
+    if tuple(lse.shape) != (B, Hq, Sq) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be contiguous float32 [B, Hq, Sq]")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    with torch.cuda.device(q.device):
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        rc = sdpa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                      lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                      B, Hq, Hkv, Sq, Sk, d, scale, causal,
+                      SDPA_BF16 if q.dtype == torch.bfloat16 else SDPA_FP16, _stream_handle(stream))
+    if rc != SDPA_OK:
+        raise SdpaError(rc, "sdpa_bwd")
+    return dq, dk, dv

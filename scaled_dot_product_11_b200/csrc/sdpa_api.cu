@@ -9,6 +9,7 @@
 
 #include "sdpa.h"
 #include "sdpa_fwd_sm100.cuh"
+#include "sdpa_bwd_sm100.cuh"
 
 namespace {
 
@@ -324,6 +325,61 @@ extern "C" int sdpa_fwd_fp8(const void* q8, const void* k8, const void* v8, floa
     return launch<128, sdpa::KIND_E4M3, SDPA_STAGES_FP8, 2>(
         q8, k8, v8, bhsd(Hq, Sq, d), bhsd(Hkv, Sk, d), bhsd(Hkv, Sk, d), prm,
         reinterpret_cast<cudaStream_t>(stream));
+}
+
+namespace {
+
+template <int D, bool BF16>
+int launch_bwd(const sdpa::BwdParams& bp, cudaStream_t stream) {
+    using C = sdpa::BwdCfg<D>;
+    auto kdkdv = sdpa::sdpa_bwd_dkdv_kernel<D, BF16>;
+    auto kdq = sdpa::sdpa_bwd_dq_kernel<D, BF16>;
+    static bool attr_set[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        if (cudaFuncSetAttribute(kdkdv, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+                cudaSuccess)
+            return SDPA_ERR_CUDA;
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+    const dim3 gkv((bp.Sk + sdpa::kBwdTile - 1) / sdpa::kBwdTile, bp.B * bp.Hkv);
+    const dim3 gq((bp.Sq + sdpa::kBwdTile - 1) / sdpa::kBwdTile, bp.B * bp.Hq);
+    kdkdv<<<gkv, sdpa::kBwdThreads, C::kSmemBytes, stream>>>(bp);
+    if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
+    kdq<<<gq, sdpa::kBwdThreads, C::kSmemBytes, stream>>>(bp);
+    return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" int sdpa_bwd(const void* q, const void* k, const void* v, const void* o,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                        int Hq, int Hkv, int Sq, int Sk, int d, float scale, int causal, int dtype,
+                        void* stream) {
+    int rc = check_args(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal);
+    if (rc != SDPA_OK) return rc;
+    if (!dout || !lse || !dq || !dk || !dv) return SDPA_ERR_INVALID_ARG;
+    if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return SDPA_ERR_INVALID_ARG;
+    if ((long long)B * Hq > 65535) return SDPA_ERR_INVALID_ARG;   // grid rows
+    if (dtype != SDPA_BF16 && dtype != SDPA_FP16) return SDPA_ERR_UNSUPPORTED;
+    rc = check_device();
+    if (rc != SDPA_OK) return rc;
+    sdpa::BwdParams bp;
+    bp.q = q; bp.k = k; bp.v = v; bp.o = o; bp.dout = dout; bp.lse = lse;
+    bp.dq = dq; bp.dk = dk; bp.dv = dv;
+    bp.B = B; bp.Hq = Hq; bp.Hkv = Hkv; bp.Sq = Sq; bp.Sk = Sk; bp.group = Hq / Hkv;
+    bp.causal = causal != 0 ? 1 : 0;
+    bp.causal_off = causal == SDPA_CAUSAL_BOTTOM_RIGHT ? Sk - Sq : 0;
+    bp.scale = scale;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const bool bf = dtype == SDPA_BF16;
+    if (d == 32) return bf ? launch_bwd<32, true>(bp, s) : launch_bwd<32, false>(bp, s);
+    if (d == 64) return bf ? launch_bwd<64, true>(bp, s) : launch_bwd<64, false>(bp, s);
+    return bf ? launch_bwd<128, true>(bp, s) : launch_bwd<128, false>(bp, s);
 }
 
 extern "C" const char* sdpa_strerror(int status) {

@@ -19,7 +19,7 @@ def declared_symbols():
 
 def test_header_declares_the_entry_points():
     assert set(declared_symbols()) == {"sdpa_fwd", "sdpa_fwd_strided", "sdpa_fwd_fp8",
-                                       "sdpa_strerror", "sdpa_device_status",
+                                       "sdpa_bwd", "sdpa_strerror", "sdpa_device_status",
                                        "sdpa_launches_per_call"}
 
 
@@ -130,3 +130,24 @@ def test_torch_wrapper_rejects_views_with_strided_last_dim():
     x = torch.zeros(1, 2, 8, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         sdpa.attention(x[..., ::2], x[..., ::2], x[..., ::2])
+
+
+def test_backward_argument_checks():
+    import scaled_dot_product_11_b200 as sdpa
+
+    def bwd(ptrs=None, d=128, causal=0, dtype=0, B=1, Hq=2, Hkv=2, Sq=128, Sk=128):
+        ptrs = ptrs or tuple(P + 0x1000 * i for i in range(9))
+        return sdpa.sdpa_bwd(*ptrs, B, Hq, Hkv, Sq, Sk, d, 0.088, causal, dtype, 0)
+    good = tuple(P + 0x1000 * i for i in range(9))
+    for i in range(9):             # every pointer required, lse included
+        ptrs = list(good)
+        ptrs[i] = 0
+        assert bwd(tuple(ptrs)) == 1, i
+    ptrs = list(good)
+    ptrs[6] += 8                   # dq misaligned
+    assert bwd(tuple(ptrs)) == 1
+    assert bwd(d=96) == 2
+    assert bwd(dtype=2) == 2
+    assert bwd(causal=1, Sq=64) == 2
+    assert bwd(causal=3) == 1
+    assert bwd(B=300, Hq=256, Hkv=256) == 1   # grid rows
