@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd"],
+                    help="bwd: time sdpa_bwd (dQ, dK, dV) on the workload, one GPU")
     ap.add_argument("--ref-budget-s", type=float, default=90.0,
                     help="host seconds the reference (oracle) arm spends over all its steps")
     return ap.parse_args()
@@ -220,12 +222,62 @@ def run_reference(args, w):
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
+def run_backward(args, w):
+    """Device-timed sdpa_bwd on one GPU.  FLOPs are the five contractions of
+    the backward (S, dP, dV, dK, dQ: 2.5x the forward's); the kernels run on
+    the CUDA cores, so the roofline is the fp32 FMA rate of the SMs."""
+    import torch
+    import scaled_dot_product_11_b200 as sdpa
+    from sdpa_workloads import make_qkv
+    dev = torch.device("cuda", 0)
+    q, k, v = make_qkv(w, dev)
+    g = torch.Generator(device="cpu").manual_seed(w.seed + 1)
+    dout = torch.randn(q.shape, generator=g).to(q.dtype).to(dev)
+    o, lse = sdpa.attention(q, k, v, causal=w.causal, scale=w.scale)
+    run = lambda: sdpa.attention_backward(q, k, v, o, lse, dout, causal=w.causal, scale=w.scale)
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+    st, detail = sdpa.sdpa_device_status(clear=True)
+    if st != 0:
+        raise SystemExit("device status %d (%#x) after warm-up" % (st, detail))
+    clocks = ClockSampler(0)
+    clocks.start()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        run()
+    e1.record(stream)
+    e1.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    flops = 2.5 * w.flops
+    value = flops / (ms * 1e-3) / 1e12
+    props = torch.cuda.get_device_properties(dev)
+    max_mhz = float((clk or {}).get("sm_max_mhz") or 1965.0)
+    peak = props.multi_processor_count * 128 * 2 * max_mhz * 1e6 / 1e12   # fp32 FMA lanes
+    print(json.dumps({
+        "metric": "attention bwd (dQ, dK, dV) TFLOP/s on 1 B200", "value": value, "unit": "TFLOP/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic", "config": dict(w.describe(), pass_="bwd"),
+        "roofline": {"bound": "alu", "achieved": value, "peak": peak, "unit": "TFLOP/s",
+                     "frac": value / peak, "traffic": None,
+                     "peak_source": "%d SMs x 128 fp32 FMA lanes x 2 flop x %.0f MHz" % (
+                         props.multi_processor_count, max_mhz)},
+        "clocks": clk, "gpu_launches": 2 * args.steps}))
+
+
 def main():
     args = parse()
     from sdpa_workloads import WORKLOADS, make_inputs, make_qkv_fp8, sample_rows, with_shape
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.pass_ == "bwd":
+        assert args.warmup >= 3, "at least 3 warm-up steps"
+        return run_backward(args, w)
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
     import numpy as np
