@@ -224,8 +224,9 @@ def run_reference(args, w):
 # ---------------------------------------------------------------------------
 def run_backward(args, w):
     """Device-timed sdpa_bwd on one GPU.  FLOPs are the five contractions of
-    the backward (S, dP, dV, dK, dQ: 2.5x the forward's); the kernels run on
-    the CUDA cores, so the roofline is the fp32 FMA rate of the SMs."""
+    the backward (S, dP, dV, dK, dQ: 2.5x the forward's).  Head dims 64 and
+    128 run on the tensor cores (roofline: the dense bf16 peak); head dim 32
+    on the CUDA cores (roofline: their fp32 FMA rate)."""
     import torch
     import scaled_dot_product_11_b200 as sdpa
     from sdpa_workloads import make_qkv
@@ -256,16 +257,22 @@ def run_backward(args, w):
     value = flops / (ms * 1e-3) / 1e12
     props = torch.cuda.get_device_properties(dev)
     max_mhz = float((clk or {}).get("sm_max_mhz") or 1965.0)
-    peak = props.multi_processor_count * 128 * 2 * max_mhz * 1e6 / 1e12   # fp32 FMA lanes
+    if w.d == 32:
+        # head dim 32 runs on the CUDA cores
+        bound = "alu"
+        peak = props.multi_processor_count * 128 * 2 * max_mhz * 1e6 / 1e12   # fp32 FMA lanes
+        peak_source = "%d SMs x 128 fp32 FMA lanes x 2 flop x %.0f MHz" % (props.multi_processor_count, max_mhz)
+    else:
+        peaks, src = load_peaks()
+        bound, peak = "tensor", float(peaks["bf16_tflops"])
+        peak_source = "%s bf16_tflops (burst)" % src
     print(json.dumps({
         "metric": "attention bwd (dQ, dK, dV) TFLOP/s on 1 B200", "value": value, "unit": "TFLOP/s",
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic", "config": dict(w.describe(), pass_="bwd"),
-        "roofline": {"bound": "alu", "achieved": value, "peak": peak, "unit": "TFLOP/s",
-                     "frac": value / peak, "traffic": None,
-                     "peak_source": "%d SMs x 128 fp32 FMA lanes x 2 flop x %.0f MHz" % (
-                         props.multi_processor_count, max_mhz)},
+        "roofline": {"bound": bound, "achieved": value, "peak": peak, "unit": "TFLOP/s",
+                     "frac": value / peak, "traffic": None, "peak_source": peak_source},
         "clocks": clk, "gpu_launches": 2 * args.steps}))
 
 

@@ -10,6 +10,7 @@
 #include "sdpa.h"
 #include "sdpa_fwd_sm100.cuh"
 #include "sdpa_bwd_sm100.cuh"
+#include "sdpa_bwd_tc_sm100.cuh"
 
 namespace {
 
@@ -353,6 +354,49 @@ int launch_bwd(const sdpa::BwdParams& bp, cudaStream_t stream) {
     return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
 }
 
+// Tensor-core backward (head dims 64, 128): 3-D maps over (d, S, B*H) of
+// Q, K, V, dO, then the dK/dV and dQ kernels.
+#ifndef SDPA_BWD_TC
+#define SDPA_BWD_TC 1
+#endif
+template <int D, bool BF16>
+int launch_bwd_tc(const void* q, const void* k, const void* v, const sdpa::BwdParams& bp,
+                  cudaStream_t stream) {
+    using C = sdpa::BtCfg<D>;
+    const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    CUtensorMap tq, tk, tv, tdo;
+    const View vq = bhsd(bp.Hq, bp.Sq, D), vk = bhsd(bp.Hkv, bp.Sk, D);
+    if (!encode_view(&tq, dt, 2, q, D, bp.Sq, bp.Hq, bp.B, vq, C::kElemsPerSw, true) ||
+        !encode_view(&tk, dt, 2, k, D, bp.Sk, bp.Hkv, bp.B, vk, C::kElemsPerSw, true) ||
+        !encode_view(&tv, dt, 2, v, D, bp.Sk, bp.Hkv, bp.B, vk, C::kElemsPerSw, true) ||
+        !encode_view(&tdo, dt, 2, bp.dout, D, bp.Sq, bp.Hq, bp.B, vq, C::kElemsPerSw, true))
+        return SDPA_ERR_CUDA;
+    sdpa::BwdTcParams tp;
+    tp.o = bp.o; tp.dout = bp.dout; tp.lse = bp.lse;
+    tp.dq = bp.dq; tp.dk = bp.dk; tp.dv = bp.dv;
+    tp.B = bp.B; tp.Hq = bp.Hq; tp.Hkv = bp.Hkv; tp.Sq = bp.Sq; tp.Sk = bp.Sk; tp.group = bp.group;
+    tp.causal = bp.causal; tp.causal_off = bp.causal_off; tp.scale = bp.scale;
+    auto kdkdv = sdpa::sdpa_bwd_dkdv_tc_kernel<D, BF16>;
+    auto kdq = sdpa::sdpa_bwd_dq_tc_kernel<D, BF16>;
+    static bool attr_set[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        if (cudaFuncSetAttribute(kdkdv, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+                cudaSuccess)
+            return SDPA_ERR_CUDA;
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+    const dim3 gkv((bp.Sk + 127) / 128, bp.B * bp.Hkv);
+    const dim3 gq((bp.Sq + 127) / 128, bp.B * bp.Hq);
+    kdkdv<<<gkv, sdpa::kBtThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, tp);
+    if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
+    kdq<<<gq, sdpa::kBtThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, tp);
+    return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" int sdpa_bwd(const void* q, const void* k, const void* v, const void* o,
@@ -378,6 +422,10 @@ extern "C" int sdpa_bwd(const void* q, const void* k, const void* v, const void*
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool bf = dtype == SDPA_BF16;
     if (d == 32) return bf ? launch_bwd<32, true>(bp, s) : launch_bwd<32, false>(bp, s);
+    if (SDPA_BWD_TC) {
+        if (d == 64) return bf ? launch_bwd_tc<64, true>(q, k, v, bp, s) : launch_bwd_tc<64, false>(q, k, v, bp, s);
+        return bf ? launch_bwd_tc<128, true>(q, k, v, bp, s) : launch_bwd_tc<128, false>(q, k, v, bp, s);
+    }
     if (d == 64) return bf ? launch_bwd<64, true>(bp, s) : launch_bwd<64, false>(bp, s);
     return bf ? launch_bwd<128, true>(bp, s) : launch_bwd<128, false>(bp, s);
 }

@@ -1,0 +1,420 @@
+// sdpa_bwd_tc_sm100.cuh -- tensor-core form of the attention backward for
+// head dims 64 and 128 (tcgen05 MMAs, TMA tiles, TMEM accumulators).
+//
+// Same recomputation as sdpa_bwd_sm100.cuh (article "Self-attention, CUDA
+// kernels and FlashAttention", section 3), with every product on the tensor
+// cores and in the two operand forms of the forward kernel:
+//   QK form  D[M=128][N=128] = A[M][d] . B[N][d]^T, A and B K-major tiles
+//   PV form  D[M=128][N=d]  += A[M][128 (TMEM, bf16/fp16)] . B[128][d],
+//            B an MN-major tile (d contiguous)
+// dK/dV kernel, one CTA per 128 keys of one (batch, K/V head), TMEM lane =
+// key:  S^T = K Q^T, dP^T = V dO^T (QK form); P^T, dS^T computed per key row
+// and written over them; dV += P^T dO, dK += dS^T Q (PV form, Q and dO tiles
+// used MN-major).  dQ kernel, one CTA per 128 rows of one (batch, query
+// head), TMEM lane = row:  S = Q K^T, dP = dO V^T; dS; dQ += dS K.
+// One CTA of 128 threads runs each loop step in turn (TMA, MMAs, elementwise
+// work); every wait is bounded.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include "sm100_ptx.cuh"
+
+namespace sdpa {
+
+constexpr int kBtThreads = 128;
+
+struct BwdTcParams {
+    const void* o;                   // [B,Hq,Sq,D] (for D_i = dO_i . O_i)
+    const void* dout;                // [B,Hq,Sq,D]
+    const float* lse;                // [B,Hq,Sq]
+    void *dq, *dk, *dv;
+    int B, Hq, Hkv, Sq, Sk, group;
+    int causal, causal_off;
+    float scale;
+};
+
+template <int D>
+struct BtCfg {
+    static constexpr int kRowBytes = D * 2;
+    static constexpr int kElemsPerSw = 64;               // 128-byte swizzle rows of 16-bit data
+    static constexpr int kSwBlocks = kRowBytes / 128;
+    static constexpr int kSwBlockBytes = 128 * 128;
+    static constexpr int kTileBytes = 128 * kRowBytes;
+    static constexpr int kQkSteps = kRowBytes / 32;
+    // four tiles (K, V, Q, dO), barriers, TMEM slot, status flag
+    static constexpr int kSmemUsed = 4 * kTileBytes + 2 * 128 * 4 + 64;
+    // one CTA per SM: each allocates all 512 TMEM columns
+    static constexpr int kSmemBytes = kSmemUsed + 1024 > 120 * 1024 ? kSmemUsed + 1024 : 120 * 1024;
+    static_assert(D == 64 || D == 128, "tensor-core backward: head dims 64 and 128");
+};
+
+// Bounded wait (1 s) on `bar`'s phase `parity`; on expiry records a device
+// timeout at `where` and returns false.
+__device__ __forceinline__ bool bt_wait(uint32_t bar, uint32_t parity, uint32_t where) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > 1000000000ull) {
+            if (atomicCAS(&g_sdpa_status[0], 0u, 4u) == 0u) atomicExch(&g_sdpa_status[1], where);
+            return false;
+        }
+    }
+    return true;
+}
+
+template <bool BF16>
+__device__ __forceinline__ float bt_ld(const void* base, size_t i) {
+    if constexpr (BF16)
+        return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[i]);
+    else
+        return __half2float(reinterpret_cast<const __half*>(base)[i]);
+}
+
+template <bool BF16>
+__device__ __forceinline__ uint32_t bt_pack(float a, float b) {
+    return BF16 ? pack_bf16x2(a, b) : pack_f16x2(a, b);
+}
+
+// D_i = dO_i . O_i of row `row` (0 past the end)
+template <int D, bool BF16>
+__device__ __forceinline__ float bt_row_dot(const BwdTcParams& p, size_t head, int row) {
+    if (row >= p.Sq) return 0.0f;
+    float acc = 0.0f;
+    const size_t off = head + (size_t)row * D;
+    for (int c = 0; c < D; ++c) acc = fmaf(bt_ld<BF16>(p.dout, off + c), bt_ld<BF16>(p.o, off + c), acc);
+    return acc;
+}
+
+// QK form: d_tmem[128][128] = A_tile . B_tile^T over D (both K-major, SW128)
+template <int D, bool BF16>
+__device__ __forceinline__ void bt_mma_qk(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
+    using C = BtCfg<D>;
+    constexpr uint32_t idesc = make_idesc(BF16 ? 1u : 0u, false, 128, 128);
+    const uint64_t da = make_smem_desc(a_smem, 16, 1024), db = make_smem_desc(b_smem, 16, 1024);
+#pragma unroll
+    for (int kk = 0; kk < C::kQkSteps; ++kk) {
+        const uint64_t off = (uint64_t)(((kk >> 2) * C::kSwBlockBytes + (kk & 3) * 32) >> 4);
+        mma_f16_ss(d_tmem, da + off, db + off, idesc, kk > 0);
+    }
+}
+
+// PV form: d_tmem[128][D] (+)= A (TMEM, 128 x 128, 16-bit packed in 64
+// columns) . B_tile (128 x D, MN-major)
+template <int D, bool BF16>
+__device__ __forceinline__ void bt_mma_pv(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, bool acc) {
+    using C = BtCfg<D>;
+    constexpr uint32_t idesc = make_idesc(BF16 ? 1u : 0u, true, 128, D);
+    const uint64_t db = make_smem_desc(b_smem, C::kSwBlockBytes, 1024);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {    // 16 keys (or rows) per step
+        const uint64_t off = (uint64_t)((kk * 16 * 128) >> 4);
+        mma_f16_ts(d_tmem, a_tmem + kk * 8, db + off, idesc, (acc || kk > 0) ? 1u : 0u);
+    }
+}
+
+// Shared set-up of both kernels: barriers, TMEM.  Returns the TMEM base.
+struct BtSmem {
+    uint32_t bar_in, bar_kv, bar_mma, bar_drain, slot;
+};
+
+__device__ __forceinline__ uint32_t bt_setup(const BtSmem& sm) {
+    if (threadIdx.x == 0) {
+        mbar_init(sm.bar_in, 1);
+        mbar_init(sm.bar_kv, 1);
+        mbar_init(sm.bar_mma, 1);
+        mbar_init(sm.bar_drain, 1);
+        fence_barrier_init();
+    }
+    if (threadIdx.x < 32) {
+        tmem_alloc(sm.slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    uint32_t t;
+    asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(t) : "r"(sm.slot));
+    return t;
+}
+
+// End of both kernels: after a failed wait no MMA may still write TMEM
+__device__ __forceinline__ void bt_teardown(const BtSmem& sm, uint32_t tmem, bool ok) {
+    if (!ok && threadIdx.x == 0) {
+        mma_commit(sm.bar_drain);
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(sm.bar_drain, 0) && global_timer_ns() - t0 < 100000000ull) {
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (threadIdx.x < 32) tmem_dealloc(tmem, 512);
+}
+
+// dQ: one CTA per 128 query rows of one (batch, query head); TMEM lane = row.
+// Columns: S [0,128) (dS written over its first 64), dP [128,256), dQ [256,256+D).
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kBtThreads, 1)
+sdpa_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                      const BwdTcParams p) {
+    using C = BtCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    const uint32_t sQ = base, sdO = base + C::kTileBytes, sK = base + 2 * C::kTileBytes,
+                   sV = base + 3 * C::kTileBytes;
+    const uint32_t bars = base + 4 * C::kTileBytes + 2 * 128 * 4;
+    const BtSmem sm{bars, bars + 8, bars + 16, bars + 24, bars + 32};
+    const uint32_t tmem = bt_setup(sm);
+
+    const int i0 = blockIdx.x * 128;
+    const int bh = blockIdx.y;
+    const int b = bh / p.Hq, hq = bh - b * p.Hq;
+    const int kvrow = b * p.Hkv + hq / p.group;        // 3-D map index of the K/V head
+    const int r = threadIdx.x, row = i0 + r;
+    const uint32_t lane_base = (uint32_t)((threadIdx.x >> 5) * 32) << 16;
+    const float kL2e = 1.44269504088896340736f;
+    const float sl = p.scale * kL2e;
+
+    if (threadIdx.x == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        prefetch_tmap(&tmdO);
+        mbar_arrive_expect_tx(sm.bar_in, 2 * C::kTileBytes);
+        for (int kb = 0; kb < C::kSwBlocks; ++kb) {
+            tma_load_3d(sQ + kb * C::kSwBlockBytes, &tmQ, sm.bar_in, kb * C::kElemsPerSw, i0, bh);
+            tma_load_3d(sdO + kb * C::kSwBlockBytes, &tmdO, sm.bar_in, kb * C::kElemsPerSw, i0, bh);
+        }
+    }
+    const float lse_r = row < p.Sq ? p.lse[(size_t)bh * p.Sq + row] * kL2e : 0.0f;
+    const float d_r = bt_row_dot<D, BF16>(p, (size_t)bh * p.Sq * D, row);
+    bool ok = bt_wait(sm.bar_in, 0, 0x50000u);
+    ok = __syncthreads_and(ok);
+
+    const int kend = p.causal ? min(p.Sk, i0 + 128 + p.causal_off) : p.Sk;
+    const int ntiles = (kend + 127) / 128;
+    for (int jt = 0; jt < ntiles && ok; ++jt) {
+        const int j0 = jt * 128;
+        if (threadIdx.x == 0) {
+            mbar_arrive_expect_tx(sm.bar_kv, 2 * C::kTileBytes);
+            for (int kb = 0; kb < C::kSwBlocks; ++kb) {
+                tma_load_3d(sK + kb * C::kSwBlockBytes, &tmK, sm.bar_kv, kb * C::kElemsPerSw, j0, kvrow);
+                tma_load_3d(sV + kb * C::kSwBlockBytes, &tmV, sm.bar_kv, kb * C::kElemsPerSw, j0, kvrow);
+            }
+        }
+        ok = __syncthreads_and(bt_wait(sm.bar_kv, (uint32_t)jt & 1u, 0x51000u | (uint32_t)(jt & 0xfff)));
+        if (!ok) break;
+        if (threadIdx.x == 0) {
+            tc_fence_after();
+            bt_mma_qk<D, BF16>(tmem, sQ, sK);            // S = Q K^T
+            bt_mma_qk<D, BF16>(tmem + 128, sdO, sV);     // dP = dO V^T
+            mma_commit(sm.bar_mma);
+        }
+        ok = __syncthreads_and(bt_wait(sm.bar_mma, 0u, 0x52000u | (uint32_t)(jt & 0xfff)));
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+            float s[32], dp[32];
+            tmem_ld32(tmem + lane_base + 32 * c, s);
+            tmem_ld32(tmem + lane_base + 128 + 32 * c, dp);
+            tmem_wait_ld();
+            reg_fence32(s);
+            reg_fence32(dp);
+            uint32_t w[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                float ds2[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int key = j0 + 32 * c + 2 * e + u;
+                    const bool vis = row < p.Sq && key < p.Sk && (!p.causal || key <= row + p.causal_off);
+                    const float pv = vis ? exp2f(s[2 * e + u] * sl - lse_r) : 0.0f;
+                    ds2[u] = pv * (dp[2 * e + u] - d_r);
+                }
+                w[e] = bt_pack<BF16>(ds2[0], ds2[1]);
+            }
+            tmem_st16(tmem + lane_base + 16 * c, w);     // dS over S's first 64 columns
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            tc_fence_after();
+            bt_mma_pv<D, BF16>(tmem + 256, tmem, sK, jt > 0);   // dQ += dS K
+            mma_commit(sm.bar_mma);
+        }
+        ok = __syncthreads_and(bt_wait(sm.bar_mma, 1u, 0x53000u | (uint32_t)(jt & 0xfff)));
+        tc_fence_after();
+    }
+    if (ok) {
+        // dQ row: scale and round (every row sees key 0, so ntiles >= 1);
+        // the TMEM loads are warp-collective, the stores per row
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+            float x[32];
+            tmem_ld32(tmem + lane_base + 256 + 32 * c, x);
+            tmem_wait_ld();
+            reg_fence32(x);
+            if (row < p.Sq) {
+                uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.dq) +
+                                                      ((size_t)bh * p.Sq + row) * D + 32 * c);
+#pragma unroll
+                for (int v4 = 0; v4 < 4; ++v4)
+                    dst[v4] = make_uint4(bt_pack<BF16>(x[8 * v4] * p.scale, x[8 * v4 + 1] * p.scale),
+                                         bt_pack<BF16>(x[8 * v4 + 2] * p.scale, x[8 * v4 + 3] * p.scale),
+                                         bt_pack<BF16>(x[8 * v4 + 4] * p.scale, x[8 * v4 + 5] * p.scale),
+                                         bt_pack<BF16>(x[8 * v4 + 6] * p.scale, x[8 * v4 + 7] * p.scale));
+            }
+        }
+    }
+    bt_teardown(sm, tmem, ok);
+}
+
+// dK, dV: one CTA per 128 keys of one (batch, K/V head); TMEM lane = key.
+// Columns: S^T [0,128) (P^T over its first 64), dP^T [128,256) (dS^T over its
+// first 64), dV [256,256+D), dK [384,384+D).
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kBtThreads, 1)
+sdpa_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                        const BwdTcParams p) {
+    using C = BtCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    const uint32_t sK = base, sV = base + C::kTileBytes, sQ = base + 2 * C::kTileBytes,
+                   sdO = base + 3 * C::kTileBytes;
+    float* const lse_s = reinterpret_cast<float*>(smem_raw + (base - raw) + 4 * C::kTileBytes);
+    float* const d_s = lse_s + 128;
+    const uint32_t bars = base + 4 * C::kTileBytes + 2 * 128 * 4;
+    const BtSmem sm{bars, bars + 8, bars + 16, bars + 24, bars + 32};
+    const uint32_t tmem = bt_setup(sm);
+
+    const int j0 = blockIdx.x * 128;
+    const int bk = blockIdx.y;                         // b * Hkv + hk
+    const int b = bk / p.Hkv, hk = bk - b * p.Hkv;
+    const int key = j0 + (int)threadIdx.x;
+    const uint32_t lane_base = (uint32_t)((threadIdx.x >> 5) * 32) << 16;
+    const float kL2e = 1.44269504088896340736f;
+    const float sl = p.scale * kL2e;
+
+    if (threadIdx.x == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        prefetch_tmap(&tmdO);
+        mbar_arrive_expect_tx(sm.bar_kv, 2 * C::kTileBytes);
+        for (int kb = 0; kb < C::kSwBlocks; ++kb) {
+            tma_load_3d(sK + kb * C::kSwBlockBytes, &tmK, sm.bar_kv, kb * C::kElemsPerSw, j0, bk);
+            tma_load_3d(sV + kb * C::kSwBlockBytes, &tmV, sm.bar_kv, kb * C::kElemsPerSw, j0, bk);
+        }
+    }
+    bool ok = __syncthreads_and(bt_wait(sm.bar_kv, 0, 0x58000u));
+
+    // the first query row that sees key j0
+    const int i_first = p.causal ? max(0, j0 - p.causal_off) : 0;
+    int it = 0;
+    for (int hq = hk * p.group; hq < (hk + 1) * p.group && ok; ++hq) {
+        const int bh = b * p.Hq + hq;
+        for (int i0 = (i_first / 128) * 128; i0 < p.Sq && ok; i0 += 128, ++it) {
+            if (threadIdx.x == 0) {
+                mbar_arrive_expect_tx(sm.bar_in, 2 * C::kTileBytes);
+                for (int kb = 0; kb < C::kSwBlocks; ++kb) {
+                    tma_load_3d(sQ + kb * C::kSwBlockBytes, &tmQ, sm.bar_in, kb * C::kElemsPerSw, i0, bh);
+                    tma_load_3d(sdO + kb * C::kSwBlockBytes, &tmdO, sm.bar_in, kb * C::kElemsPerSw, i0, bh);
+                }
+            }
+            // the 128 query rows' LSE (log2 units) and D = dO . O
+            {
+                const int qi = i0 + (int)threadIdx.x;
+                lse_s[threadIdx.x] = qi < p.Sq ? p.lse[(size_t)bh * p.Sq + qi] * kL2e : 0.0f;
+                d_s[threadIdx.x] = bt_row_dot<D, BF16>(p, (size_t)bh * p.Sq * D, qi);
+            }
+            ok = __syncthreads_and(bt_wait(sm.bar_in, (uint32_t)it & 1u, 0x59000u | (uint32_t)(it & 0xfff)));
+            if (!ok) break;
+            if (threadIdx.x == 0) {
+                tc_fence_after();
+                bt_mma_qk<D, BF16>(tmem, sK, sQ);          // S^T = K Q^T
+                bt_mma_qk<D, BF16>(tmem + 128, sV, sdO);   // dP^T = V dO^T
+                mma_commit(sm.bar_mma);
+            }
+            ok = __syncthreads_and(bt_wait(sm.bar_mma, 0u, 0x5a000u | (uint32_t)(it & 0xfff)));
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                float s[32], dp[32];
+                tmem_ld32(tmem + lane_base + 32 * c, s);
+                tmem_ld32(tmem + lane_base + 128 + 32 * c, dp);
+                tmem_wait_ld();
+                reg_fence32(s);
+                reg_fence32(dp);
+                uint32_t wp[16], wd[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    float pv2[2], ds2[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int col = 32 * c + 2 * e + u;
+                        const int qi = i0 + col;
+                        const bool vis = key < p.Sk && qi < p.Sq && (!p.causal || key <= qi + p.causal_off);
+                        pv2[u] = vis ? exp2f(s[2 * e + u] * sl - lse_s[col]) : 0.0f;
+                        ds2[u] = pv2[u] * (dp[2 * e + u] - d_s[col]);
+                    }
+                    wp[e] = bt_pack<BF16>(pv2[0], pv2[1]);
+                    wd[e] = bt_pack<BF16>(ds2[0], ds2[1]);
+                }
+                tmem_st16(tmem + lane_base + 16 * c, wp);          // P^T
+                tmem_st16(tmem + lane_base + 128 + 16 * c, wd);    // dS^T
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                tc_fence_after();
+                bt_mma_pv<D, BF16>(tmem + 256, tmem, sdO, it > 0);         // dV += P^T dO
+                bt_mma_pv<D, BF16>(tmem + 384, tmem + 128, sQ, it > 0);    // dK += dS^T Q
+                mma_commit(sm.bar_mma);
+            }
+            ok = __syncthreads_and(bt_wait(sm.bar_mma, 1u, 0x5b000u | (uint32_t)(it & 0xfff)));
+            tc_fence_after();
+        }
+    }
+    if (ok) {
+        // dV and dK rows (zero when no query sees these keys); the TMEM loads
+        // are warp-collective, the stores per key
+        const size_t orow = ((size_t)bk * p.Sk + (size_t)key) * D;
+#pragma unroll 1
+        for (int t = 0; t < 2; ++t) {
+            void* out = t ? p.dk : p.dv;
+            const float mul = t ? p.scale : 1.0f;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                float x[32];
+                tmem_ld32(tmem + lane_base + (t ? 384 : 256) + 32 * c, x);
+                tmem_wait_ld();
+                reg_fence32(x);
+                if (key < p.Sk) {
+                    // with no step the accumulators were never written: zeros
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) x[e] = it > 0 ? x[e] * mul : 0.0f;
+                    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(out) + orow + 32 * c);
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4)
+                        dst[v4] = make_uint4(bt_pack<BF16>(x[8 * v4], x[8 * v4 + 1]),
+                                             bt_pack<BF16>(x[8 * v4 + 2], x[8 * v4 + 3]),
+                                             bt_pack<BF16>(x[8 * v4 + 4], x[8 * v4 + 5]),
+                                             bt_pack<BF16>(x[8 * v4 + 6], x[8 * v4 + 7]));
+                }
+            }
+        }
+    }
+    bt_teardown(sm, tmem, ok);
+}
+
+}  // namespace sdpa
