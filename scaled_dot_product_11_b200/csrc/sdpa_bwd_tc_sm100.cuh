@@ -43,8 +43,9 @@ struct BtCfg {
     static constexpr int kSwBlockBytes = 128 * 128;
     static constexpr int kTileBytes = 128 * kRowBytes;
     static constexpr int kQkSteps = kRowBytes / 32;
-    // four tiles (K, V, Q, dO), barriers, TMEM slot, status flag
-    static constexpr int kSmemUsed = 4 * kTileBytes + 2 * 128 * 4 + 64;
+    // six tiles (the streamed pair double-buffered), LSE/D rows, barriers,
+    // TMEM slot
+    static constexpr int kSmemUsed = 6 * kTileBytes + 2 * 128 * 4 + 64;
     // one CTA per SM: each allocates all 512 TMEM columns
     static constexpr int kSmemBytes = kSmemUsed + 1024 > 120 * 1024 ? kSmemUsed + 1024 : 120 * 1024;
     static_assert(D == 64 || D == 128, "tensor-core backward: head dims 64 and 128");
@@ -77,13 +78,38 @@ __device__ __forceinline__ uint32_t bt_pack(float a, float b) {
     return BF16 ? pack_bf16x2(a, b) : pack_f16x2(a, b);
 }
 
-// D_i = dO_i . O_i of row `row` (0 past the end)
+template <bool BF16>
+__device__ __forceinline__ float2 bt_unpack(uint32_t w) {
+    if constexpr (BF16)
+        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    else
+        return __half22float2(*reinterpret_cast<const __half2*>(&w));
+}
+
+// D_i = dO_i . O_i of row `row` (0 past the end); 16-byte loads
 template <int D, bool BF16>
 __device__ __forceinline__ float bt_row_dot(const BwdTcParams& p, size_t head, int row) {
     if (row >= p.Sq) return 0.0f;
-    float acc = 0.0f;
     const size_t off = head + (size_t)row * D;
-    for (int c = 0; c < D; ++c) acc = fmaf(bt_ld<BF16>(p.dout, off + c), bt_ld<BF16>(p.o, off + c), acc);
+    const uint4* g = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.dout) + off);
+    const uint4* o = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.o) + off);
+    uint4 gv[D / 8], ov[D / 8];
+#pragma unroll
+    for (int v = 0; v < D / 8; ++v) {
+        gv[v] = g[v];
+        ov[v] = o[v];
+    }
+    float acc = 0.0f;
+#pragma unroll
+    for (int v = 0; v < D / 8; ++v) {
+        const uint32_t gw[4] = {gv[v].x, gv[v].y, gv[v].z, gv[v].w};
+        const uint32_t ow[4] = {ov[v].x, ov[v].y, ov[v].z, ov[v].w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const float2 a = bt_unpack<BF16>(gw[u]), b = bt_unpack<BF16>(ow[u]);
+            acc = fmaf(a.x, b.x, fmaf(a.y, b.y, acc));
+        }
+    }
     return acc;
 }
 
@@ -116,13 +142,18 @@ __device__ __forceinline__ void bt_mma_pv(uint32_t d_tmem, uint32_t a_tmem, uint
 
 // Shared set-up of both kernels: barriers, TMEM.  Returns the TMEM base.
 struct BtSmem {
-    uint32_t bar_in, bar_kv, bar_mma, bar_drain, slot;
+    uint32_t bar_in[2], bar_kv[2], bar_mma, bar_drain, slot;
 };
+__device__ __forceinline__ BtSmem bt_layout(uint32_t bars) {
+    return BtSmem{{bars, bars + 8}, {bars + 16, bars + 24}, bars + 32, bars + 40, bars + 48};
+}
 
 __device__ __forceinline__ uint32_t bt_setup(const BtSmem& sm) {
     if (threadIdx.x == 0) {
-        mbar_init(sm.bar_in, 1);
-        mbar_init(sm.bar_kv, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(sm.bar_in[i], 1);
+            mbar_init(sm.bar_kv[i], 1);
+        }
         mbar_init(sm.bar_mma, 1);
         mbar_init(sm.bar_drain, 1);
         fence_barrier_init();
@@ -164,10 +195,11 @@ sdpa_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
-    const uint32_t sQ = base, sdO = base + C::kTileBytes, sK = base + 2 * C::kTileBytes,
-                   sV = base + 3 * C::kTileBytes;
-    const uint32_t bars = base + 4 * C::kTileBytes + 2 * 128 * 4;
-    const BtSmem sm{bars, bars + 8, bars + 16, bars + 24, bars + 32};
+    // Q, dO once; K/V tiles double-buffered: (sK(0), sV(0)), (sK(1), sV(1))
+    const uint32_t sQ = base, sdO = base + C::kTileBytes;
+    auto sK = [&](int buf) { return base + (uint32_t)(2 + 2 * buf) * C::kTileBytes; };
+    auto sV = [&](int buf) { return base + (uint32_t)(3 + 2 * buf) * C::kTileBytes; };
+    const BtSmem sm = bt_layout(base + 6 * C::kTileBytes + 2 * 128 * 4);
     const uint32_t tmem = bt_setup(sm);
 
     const int i0 = blockIdx.x * 128;
@@ -184,34 +216,42 @@ sdpa_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
         prefetch_tmap(&tmdO);
-        mbar_arrive_expect_tx(sm.bar_in, 2 * C::kTileBytes);
+        mbar_arrive_expect_tx(sm.bar_in[0], 2 * C::kTileBytes);
         for (int kb = 0; kb < C::kSwBlocks; ++kb) {
-            tma_load_3d(sQ + kb * C::kSwBlockBytes, &tmQ, sm.bar_in, kb * C::kElemsPerSw, i0, bh);
-            tma_load_3d(sdO + kb * C::kSwBlockBytes, &tmdO, sm.bar_in, kb * C::kElemsPerSw, i0, bh);
+            tma_load_3d(sQ + kb * C::kSwBlockBytes, &tmQ, sm.bar_in[0], kb * C::kElemsPerSw, i0, bh);
+            tma_load_3d(sdO + kb * C::kSwBlockBytes, &tmdO, sm.bar_in[0], kb * C::kElemsPerSw, i0, bh);
         }
     }
-    const float lse_r = row < p.Sq ? p.lse[(size_t)bh * p.Sq + row] * kL2e : 0.0f;
-    const float d_r = bt_row_dot<D, BF16>(p, (size_t)bh * p.Sq * D, row);
-    bool ok = bt_wait(sm.bar_in, 0, 0x50000u);
-    ok = __syncthreads_and(ok);
-
     const int kend = p.causal ? min(p.Sk, i0 + 128 + p.causal_off) : p.Sk;
     const int ntiles = (kend + 127) / 128;
-    for (int jt = 0; jt < ntiles && ok; ++jt) {
-        const int j0 = jt * 128;
-        if (threadIdx.x == 0) {
-            mbar_arrive_expect_tx(sm.bar_kv, 2 * C::kTileBytes);
-            for (int kb = 0; kb < C::kSwBlocks; ++kb) {
-                tma_load_3d(sK + kb * C::kSwBlockBytes, &tmK, sm.bar_kv, kb * C::kElemsPerSw, j0, kvrow);
-                tma_load_3d(sV + kb * C::kSwBlockBytes, &tmV, sm.bar_kv, kb * C::kElemsPerSw, j0, kvrow);
-            }
+    // K/V tile jt goes to buffer jt & 1, one tile ahead of its use
+    auto load_kv = [&](int jt) {
+        const int buf = jt & 1;
+        mbar_arrive_expect_tx((buf ? sm.bar_kv[1] : sm.bar_kv[0]), 2 * C::kTileBytes);
+        for (int kb = 0; kb < C::kSwBlocks; ++kb) {
+            tma_load_3d(sK(buf) + kb * C::kSwBlockBytes, &tmK, (buf ? sm.bar_kv[1] : sm.bar_kv[0]), kb * C::kElemsPerSw,
+                        jt * 128, kvrow);
+            tma_load_3d(sV(buf) + kb * C::kSwBlockBytes, &tmV, (buf ? sm.bar_kv[1] : sm.bar_kv[0]), kb * C::kElemsPerSw,
+                        jt * 128, kvrow);
         }
-        ok = __syncthreads_and(bt_wait(sm.bar_kv, (uint32_t)jt & 1u, 0x51000u | (uint32_t)(jt & 0xfff)));
+    };
+    if (threadIdx.x == 0 && ntiles > 0) load_kv(0);
+    const float lse_r = row < p.Sq ? p.lse[(size_t)bh * p.Sq + row] * kL2e : 0.0f;
+    const float d_r = bt_row_dot<D, BF16>(p, (size_t)bh * p.Sq * D, row);
+    bool ok = bt_wait(sm.bar_in[0], 0, 0x50000u);
+    ok = __syncthreads_and(ok);
+
+    for (int jt = 0; jt < ntiles && ok; ++jt) {
+        const int j0 = jt * 128, buf = jt & 1;
+        // the other buffer's last readers (tile jt-1's MMAs) have completed
+        if (threadIdx.x == 0 && jt + 1 < ntiles) load_kv(jt + 1);
+        ok = __syncthreads_and(bt_wait((buf ? sm.bar_kv[1] : sm.bar_kv[0]), (uint32_t)(jt >> 1) & 1u,
+                                       0x51000u | (uint32_t)(jt & 0xfff)));
         if (!ok) break;
         if (threadIdx.x == 0) {
             tc_fence_after();
-            bt_mma_qk<D, BF16>(tmem, sQ, sK);            // S = Q K^T
-            bt_mma_qk<D, BF16>(tmem + 128, sdO, sV);     // dP = dO V^T
+            bt_mma_qk<D, BF16>(tmem, sQ, sK(buf));            // S = Q K^T
+            bt_mma_qk<D, BF16>(tmem + 128, sdO, sV(buf));     // dP = dO V^T
             mma_commit(sm.bar_mma);
         }
         ok = __syncthreads_and(bt_wait(sm.bar_mma, 0u, 0x52000u | (uint32_t)(jt & 0xfff)));
@@ -245,7 +285,7 @@ sdpa_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         __syncthreads();
         if (threadIdx.x == 0) {
             tc_fence_after();
-            bt_mma_pv<D, BF16>(tmem + 256, tmem, sK, jt > 0);   // dQ += dS K
+            bt_mma_pv<D, BF16>(tmem + 256, tmem, sK(buf), jt > 0);   // dQ += dS K
             mma_commit(sm.bar_mma);
         }
         ok = __syncthreads_and(bt_wait(sm.bar_mma, 1u, 0x53000u | (uint32_t)(jt & 0xfff)));
@@ -287,12 +327,13 @@ sdpa_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
-    const uint32_t sK = base, sV = base + C::kTileBytes, sQ = base + 2 * C::kTileBytes,
-                   sdO = base + 3 * C::kTileBytes;
-    float* const lse_s = reinterpret_cast<float*>(smem_raw + (base - raw) + 4 * C::kTileBytes);
+    // K, V once; Q/dO tiles double-buffered: (sQ(0), sdO(0)), (sQ(1), sdO(1))
+    const uint32_t sK = base, sV = base + C::kTileBytes;
+    auto sQ = [&](int buf) { return base + (uint32_t)(2 + 2 * buf) * C::kTileBytes; };
+    auto sdO = [&](int buf) { return base + (uint32_t)(3 + 2 * buf) * C::kTileBytes; };
+    float* const lse_s = reinterpret_cast<float*>(smem_raw + (base - raw) + 6 * C::kTileBytes);
     float* const d_s = lse_s + 128;
-    const uint32_t bars = base + 4 * C::kTileBytes + 2 * 128 * 4;
-    const BtSmem sm{bars, bars + 8, bars + 16, bars + 24, bars + 32};
+    const BtSmem sm = bt_layout(base + 6 * C::kTileBytes + 2 * 128 * 4);
     const uint32_t tmem = bt_setup(sm);
 
     const int j0 = blockIdx.x * 128;
@@ -308,39 +349,50 @@ sdpa_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
         prefetch_tmap(&tmdO);
-        mbar_arrive_expect_tx(sm.bar_kv, 2 * C::kTileBytes);
+        mbar_arrive_expect_tx(sm.bar_kv[0], 2 * C::kTileBytes);
         for (int kb = 0; kb < C::kSwBlocks; ++kb) {
-            tma_load_3d(sK + kb * C::kSwBlockBytes, &tmK, sm.bar_kv, kb * C::kElemsPerSw, j0, bk);
-            tma_load_3d(sV + kb * C::kSwBlockBytes, &tmV, sm.bar_kv, kb * C::kElemsPerSw, j0, bk);
+            tma_load_3d(sK + kb * C::kSwBlockBytes, &tmK, sm.bar_kv[0], kb * C::kElemsPerSw, j0, bk);
+            tma_load_3d(sV + kb * C::kSwBlockBytes, &tmV, sm.bar_kv[0], kb * C::kElemsPerSw, j0, bk);
         }
     }
-    bool ok = __syncthreads_and(bt_wait(sm.bar_kv, 0, 0x58000u));
+    // steps: the (query head of the group, query tile) pairs that see these
+    // keys, query tiles from the first row that sees key j0
+    const int i_start = ((p.causal ? max(0, j0 - p.causal_off) : 0) / 128) * 128;
+    const int tiles_per_head = i_start < p.Sq ? (p.Sq - i_start + 127) / 128 : 0;
+    const int nsteps = tiles_per_head * p.group;
+    auto step_bh = [&](int st) { return b * p.Hq + hk * p.group + st / tiles_per_head; };
+    auto step_i0 = [&](int st) { return i_start + (st % tiles_per_head) * 128; };
+    // step st's Q/dO go to buffer st & 1, one step ahead of their use
+    auto load_q = [&](int st) {
+        const int buf = st & 1, bh = step_bh(st), i0 = step_i0(st);
+        mbar_arrive_expect_tx((buf ? sm.bar_in[1] : sm.bar_in[0]), 2 * C::kTileBytes);
+        for (int kb = 0; kb < C::kSwBlocks; ++kb) {
+            tma_load_3d(sQ(buf) + kb * C::kSwBlockBytes, &tmQ, (buf ? sm.bar_in[1] : sm.bar_in[0]), kb * C::kElemsPerSw, i0, bh);
+            tma_load_3d(sdO(buf) + kb * C::kSwBlockBytes, &tmdO, (buf ? sm.bar_in[1] : sm.bar_in[0]), kb * C::kElemsPerSw, i0, bh);
+        }
+    };
+    if (threadIdx.x == 0 && nsteps > 0) load_q(0);
+    bool ok = __syncthreads_and(bt_wait(sm.bar_kv[0], 0, 0x58000u));
 
-    // the first query row that sees key j0
-    const int i_first = p.causal ? max(0, j0 - p.causal_off) : 0;
     int it = 0;
-    for (int hq = hk * p.group; hq < (hk + 1) * p.group && ok; ++hq) {
-        const int bh = b * p.Hq + hq;
-        for (int i0 = (i_first / 128) * 128; i0 < p.Sq && ok; i0 += 128, ++it) {
-            if (threadIdx.x == 0) {
-                mbar_arrive_expect_tx(sm.bar_in, 2 * C::kTileBytes);
-                for (int kb = 0; kb < C::kSwBlocks; ++kb) {
-                    tma_load_3d(sQ + kb * C::kSwBlockBytes, &tmQ, sm.bar_in, kb * C::kElemsPerSw, i0, bh);
-                    tma_load_3d(sdO + kb * C::kSwBlockBytes, &tmdO, sm.bar_in, kb * C::kElemsPerSw, i0, bh);
-                }
-            }
+    for (; it < nsteps && ok; ++it) {
+        const int bh = step_bh(it), i0 = step_i0(it), buf = it & 1;
+        {
+            // the other buffer's last readers (step it-1's MMAs) have completed
+            if (threadIdx.x == 0 && it + 1 < nsteps) load_q(it + 1);
             // the 128 query rows' LSE (log2 units) and D = dO . O
             {
                 const int qi = i0 + (int)threadIdx.x;
                 lse_s[threadIdx.x] = qi < p.Sq ? p.lse[(size_t)bh * p.Sq + qi] * kL2e : 0.0f;
                 d_s[threadIdx.x] = bt_row_dot<D, BF16>(p, (size_t)bh * p.Sq * D, qi);
             }
-            ok = __syncthreads_and(bt_wait(sm.bar_in, (uint32_t)it & 1u, 0x59000u | (uint32_t)(it & 0xfff)));
+            ok = __syncthreads_and(bt_wait((buf ? sm.bar_in[1] : sm.bar_in[0]), (uint32_t)(it >> 1) & 1u,
+                                           0x59000u | (uint32_t)(it & 0xfff)));
             if (!ok) break;
             if (threadIdx.x == 0) {
                 tc_fence_after();
-                bt_mma_qk<D, BF16>(tmem, sK, sQ);          // S^T = K Q^T
-                bt_mma_qk<D, BF16>(tmem + 128, sV, sdO);   // dP^T = V dO^T
+                bt_mma_qk<D, BF16>(tmem, sK, sQ(buf));          // S^T = K Q^T
+                bt_mma_qk<D, BF16>(tmem + 128, sV, sdO(buf));   // dP^T = V dO^T
                 mma_commit(sm.bar_mma);
             }
             ok = __syncthreads_and(bt_wait(sm.bar_mma, 0u, 0x5a000u | (uint32_t)(it & 0xfff)));
@@ -377,8 +429,8 @@ sdpa_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             __syncthreads();
             if (threadIdx.x == 0) {
                 tc_fence_after();
-                bt_mma_pv<D, BF16>(tmem + 256, tmem, sdO, it > 0);         // dV += P^T dO
-                bt_mma_pv<D, BF16>(tmem + 384, tmem + 128, sQ, it > 0);    // dK += dS^T Q
+                bt_mma_pv<D, BF16>(tmem + 256, tmem, sdO(buf), it > 0);         // dV += P^T dO
+                bt_mma_pv<D, BF16>(tmem + 384, tmem + 128, sQ(buf), it > 0);    // dK += dS^T Q
                 mma_commit(sm.bar_mma);
             }
             ok = __syncthreads_and(bt_wait(sm.bar_mma, 1u, 0x5b000u | (uint32_t)(it & 0xfff)));
