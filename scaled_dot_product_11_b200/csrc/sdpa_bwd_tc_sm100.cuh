@@ -12,8 +12,10 @@
 // and written over them; dV += P^T dO, dK += dS^T Q (PV form, Q and dO tiles
 // used MN-major).  dQ kernel, one CTA per 128 rows of one (batch, query
 // head), TMEM lane = row:  S = Q K^T, dP = dO V^T; dS; dQ += dS K.
-// One CTA of 128 threads runs each loop step in turn (TMA, MMAs, elementwise
-// work); every wait is bounded.
+// One CTA of 256 threads per tile: thread 0 issues the TMA copies (the
+// streamed tile pair one step ahead, double-buffered) and the MMAs; all eight
+// warps do the elementwise work, two per TMEM lane quarter splitting the
+// columns; every wait is bounded.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -23,7 +25,9 @@
 
 namespace sdpa {
 
-constexpr int kBtThreads = 128;
+// 8 warps: warps w and w+4 share TMEM lane quarter w and split the 128
+// columns of every elementwise step; thread 0 issues TMA and MMAs
+constexpr int kBtThreads = 256;
 
 struct BwdTcParams {
     const void* o;                   // [B,Hq,Sq,D] (for D_i = dO_i . O_i)
@@ -43,9 +47,10 @@ struct BtCfg {
     static constexpr int kSwBlockBytes = 128 * 128;
     static constexpr int kTileBytes = 128 * kRowBytes;
     static constexpr int kQkSteps = kRowBytes / 32;
-    // six tiles (the streamed pair double-buffered), LSE/D rows, barriers,
-    // TMEM slot
-    static constexpr int kSmemUsed = 6 * kTileBytes + 2 * 128 * 4 + 64;
+    // six tiles (the streamed pair double-buffered), LSE rows, D partial
+    // sums of two halves, barriers, TMEM slot
+    static constexpr int kStatsBytes = 4 * 128 * 4;
+    static constexpr int kSmemUsed = 6 * kTileBytes + kStatsBytes + 64;
     // one CTA per SM: each allocates all 512 TMEM columns
     static constexpr int kSmemBytes = kSmemUsed + 1024 > 120 * 1024 ? kSmemUsed + 1024 : 120 * 1024;
     static_assert(D == 64 || D == 128, "tensor-core backward: head dims 64 and 128");
@@ -86,22 +91,23 @@ __device__ __forceinline__ float2 bt_unpack(uint32_t w) {
         return __half22float2(*reinterpret_cast<const __half2*>(&w));
 }
 
-// D_i = dO_i . O_i of row `row` (0 past the end); 16-byte loads
+// Half `half` (columns [half*D/2, (half+1)*D/2)) of D_i = dO_i . O_i of row
+// `row` (0 past the end); 16-byte loads
 template <int D, bool BF16>
-__device__ __forceinline__ float bt_row_dot(const BwdTcParams& p, size_t head, int row) {
+__device__ __forceinline__ float bt_row_dot(const BwdTcParams& p, size_t head, int row, int half) {
     if (row >= p.Sq) return 0.0f;
-    const size_t off = head + (size_t)row * D;
+    const size_t off = head + (size_t)row * D + (size_t)half * (D / 2);
     const uint4* g = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.dout) + off);
     const uint4* o = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.o) + off);
-    uint4 gv[D / 8], ov[D / 8];
+    uint4 gv[D / 16], ov[D / 16];
 #pragma unroll
-    for (int v = 0; v < D / 8; ++v) {
+    for (int v = 0; v < D / 16; ++v) {
         gv[v] = g[v];
         ov[v] = o[v];
     }
     float acc = 0.0f;
 #pragma unroll
-    for (int v = 0; v < D / 8; ++v) {
+    for (int v = 0; v < D / 16; ++v) {
         const uint32_t gw[4] = {gv[v].x, gv[v].y, gv[v].z, gv[v].w};
         const uint32_t ow[4] = {ov[v].x, ov[v].y, ov[v].z, ov[v].w};
 #pragma unroll
@@ -199,15 +205,16 @@ sdpa_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     const uint32_t sQ = base, sdO = base + C::kTileBytes;
     auto sK = [&](int buf) { return base + (uint32_t)(2 + 2 * buf) * C::kTileBytes; };
     auto sV = [&](int buf) { return base + (uint32_t)(3 + 2 * buf) * C::kTileBytes; };
-    const BtSmem sm = bt_layout(base + 6 * C::kTileBytes + 2 * 128 * 4);
+    float* const dpart = reinterpret_cast<float*>(smem_raw + (base - raw) + 6 * C::kTileBytes);
+    const BtSmem sm = bt_layout(base + 6 * C::kTileBytes + C::kStatsBytes);
     const uint32_t tmem = bt_setup(sm);
 
     const int i0 = blockIdx.x * 128;
     const int bh = blockIdx.y;
     const int b = bh / p.Hq, hq = bh - b * p.Hq;
     const int kvrow = b * p.Hkv + hq / p.group;        // 3-D map index of the K/V head
-    const int r = threadIdx.x, row = i0 + r;
-    const uint32_t lane_base = (uint32_t)((threadIdx.x >> 5) * 32) << 16;
+    const int r = threadIdx.x & 127, row = i0 + r, half = threadIdx.x >> 7;
+    const uint32_t lane_base = (uint32_t)(((threadIdx.x >> 5) & 3) * 32) << 16;
     const float kL2e = 1.44269504088896340736f;
     const float sl = p.scale * kL2e;
 
@@ -237,9 +244,10 @@ sdpa_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     };
     if (threadIdx.x == 0 && ntiles > 0) load_kv(0);
     const float lse_r = row < p.Sq ? p.lse[(size_t)bh * p.Sq + row] * kL2e : 0.0f;
-    const float d_r = bt_row_dot<D, BF16>(p, (size_t)bh * p.Sq * D, row);
+    dpart[threadIdx.x] = bt_row_dot<D, BF16>(p, (size_t)bh * p.Sq * D, row, half);
     bool ok = bt_wait(sm.bar_in[0], 0, 0x50000u);
     ok = __syncthreads_and(ok);
+    const float d_r = dpart[r] + dpart[r + 128];
 
     for (int jt = 0; jt < ntiles && ok; ++jt) {
         const int j0 = jt * 128, buf = jt & 1;
@@ -257,15 +265,18 @@ sdpa_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         ok = __syncthreads_and(bt_wait(sm.bar_mma, 0u, 0x52000u | (uint32_t)(jt & 0xfff)));
         if (!ok) break;
         tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        // this thread's half of the row: key chunks 2*half and 2*half+1; all
+        // reads of S finish before dS is written over its first 64 columns
+        uint32_t w[2][16];
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            const int c = 2 * half + cc;
             float s[32], dp[32];
             tmem_ld32(tmem + lane_base + 32 * c, s);
             tmem_ld32(tmem + lane_base + 128 + 32 * c, dp);
             tmem_wait_ld();
             reg_fence32(s);
             reg_fence32(dp);
-            uint32_t w[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 float ds2[2];
@@ -276,10 +287,14 @@ sdpa_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
                     const float pv = vis ? exp2f(s[2 * e + u] * sl - lse_r) : 0.0f;
                     ds2[u] = pv * (dp[2 * e + u] - d_r);
                 }
-                w[e] = bt_pack<BF16>(ds2[0], ds2[1]);
+                w[cc][e] = bt_pack<BF16>(ds2[0], ds2[1]);
             }
-            tmem_st16(tmem + lane_base + 16 * c, w);     // dS over S's first 64 columns
         }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        tmem_st16(tmem + lane_base + 16 * (2 * half), w[0]);      // dS
+        tmem_st16(tmem + lane_base + 16 * (2 * half + 1), w[1]);
         tmem_wait_st();
         tc_fence_before();
         __syncthreads();
@@ -295,7 +310,7 @@ sdpa_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         // dQ row: scale and round (every row sees key 0, so ntiles >= 1);
         // the TMEM loads are warp-collective, the stores per row
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
             float x[32];
             tmem_ld32(tmem + lane_base + 256 + 32 * c, x);
             tmem_wait_ld();
@@ -331,16 +346,18 @@ sdpa_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
     const uint32_t sK = base, sV = base + C::kTileBytes;
     auto sQ = [&](int buf) { return base + (uint32_t)(2 + 2 * buf) * C::kTileBytes; };
     auto sdO = [&](int buf) { return base + (uint32_t)(3 + 2 * buf) * C::kTileBytes; };
+    // lse_s[128]: LSE of the step's query rows (log2 units); dpart[256]: the
+    // two halves of their D = dO . O
     float* const lse_s = reinterpret_cast<float*>(smem_raw + (base - raw) + 6 * C::kTileBytes);
-    float* const d_s = lse_s + 128;
-    const BtSmem sm = bt_layout(base + 6 * C::kTileBytes + 2 * 128 * 4);
+    float* const dpart = lse_s + 128;
+    const BtSmem sm = bt_layout(base + 6 * C::kTileBytes + C::kStatsBytes);
     const uint32_t tmem = bt_setup(sm);
 
     const int j0 = blockIdx.x * 128;
     const int bk = blockIdx.y;                         // b * Hkv + hk
     const int b = bk / p.Hkv, hk = bk - b * p.Hkv;
-    const int key = j0 + (int)threadIdx.x;
-    const uint32_t lane_base = (uint32_t)((threadIdx.x >> 5) * 32) << 16;
+    const int key = j0 + (int)(threadIdx.x & 127), half = threadIdx.x >> 7;
+    const uint32_t lane_base = (uint32_t)(((threadIdx.x >> 5) & 3) * 32) << 16;
     const float kL2e = 1.44269504088896340736f;
     const float sl = p.scale * kL2e;
 
@@ -382,9 +399,9 @@ sdpa_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             if (threadIdx.x == 0 && it + 1 < nsteps) load_q(it + 1);
             // the 128 query rows' LSE (log2 units) and D = dO . O
             {
-                const int qi = i0 + (int)threadIdx.x;
-                lse_s[threadIdx.x] = qi < p.Sq ? p.lse[(size_t)bh * p.Sq + qi] * kL2e : 0.0f;
-                d_s[threadIdx.x] = bt_row_dot<D, BF16>(p, (size_t)bh * p.Sq * D, qi);
+                const int qr = i0 + (int)(threadIdx.x & 127);
+                if (half == 0) lse_s[threadIdx.x] = qr < p.Sq ? p.lse[(size_t)bh * p.Sq + qr] * kL2e : 0.0f;
+                dpart[threadIdx.x] = bt_row_dot<D, BF16>(p, (size_t)bh * p.Sq * D, qr, half);
             }
             ok = __syncthreads_and(bt_wait((buf ? sm.bar_in[1] : sm.bar_in[0]), (uint32_t)(it >> 1) & 1u,
                                            0x59000u | (uint32_t)(it & 0xfff)));
@@ -398,15 +415,19 @@ sdpa_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             ok = __syncthreads_and(bt_wait(sm.bar_mma, 0u, 0x5a000u | (uint32_t)(it & 0xfff)));
             if (!ok) break;
             tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            // this thread's half of the key row: query chunks 2*half and
+            // 2*half+1; all reads finish before P^T and dS^T are written over
+            // the first 64 columns of S^T and dP^T
+            uint32_t wp[2][16], wd[2][16];
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c = 2 * half + cc;
                 float s[32], dp[32];
                 tmem_ld32(tmem + lane_base + 32 * c, s);
                 tmem_ld32(tmem + lane_base + 128 + 32 * c, dp);
                 tmem_wait_ld();
                 reg_fence32(s);
                 reg_fence32(dp);
-                uint32_t wp[16], wd[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     float pv2[2], ds2[2];
@@ -416,13 +437,20 @@ sdpa_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                         const int qi = i0 + col;
                         const bool vis = key < p.Sk && qi < p.Sq && (!p.causal || key <= qi + p.causal_off);
                         pv2[u] = vis ? exp2f(s[2 * e + u] * sl - lse_s[col]) : 0.0f;
-                        ds2[u] = pv2[u] * (dp[2 * e + u] - d_s[col]);
+                        ds2[u] = pv2[u] * (dp[2 * e + u] - (dpart[col] + dpart[128 + col]));
                     }
-                    wp[e] = bt_pack<BF16>(pv2[0], pv2[1]);
-                    wd[e] = bt_pack<BF16>(ds2[0], ds2[1]);
+                    wp[cc][e] = bt_pack<BF16>(pv2[0], pv2[1]);
+                    wd[cc][e] = bt_pack<BF16>(ds2[0], ds2[1]);
                 }
-                tmem_st16(tmem + lane_base + 16 * c, wp);          // P^T
-                tmem_st16(tmem + lane_base + 128 + 16 * c, wd);    // dS^T
+            }
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c = 2 * half + cc;
+                tmem_st16(tmem + lane_base + 16 * c, wp[cc]);          // P^T
+                tmem_st16(tmem + lane_base + 128 + 16 * c, wd[cc]);    // dS^T
             }
             tmem_wait_st();
             tc_fence_before();
@@ -441,8 +469,9 @@ sdpa_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         // dV and dK rows (zero when no query sees these keys); the TMEM loads
         // are warp-collective, the stores per key
         const size_t orow = ((size_t)bk * p.Sk + (size_t)key) * D;
-#pragma unroll 1
-        for (int t = 0; t < 2; ++t) {
+        {
+            // warps 0-3 write dV, warps 4-7 dK
+            const int t = half;
             void* out = t ? p.dk : p.dv;
             const float mul = t ? p.scale : 1.0f;
 #pragma unroll 1
