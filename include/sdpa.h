@@ -171,16 +171,21 @@ SDPA_API int sdpa_fwd_fp8(const void* q8, const void* k8, const void* v8,
  *                   summed over the query heads sharing each K/V head)
  *   lse             [B,Hq,Sq] float32 as written by sdpa_fwd for the same
  *                   q, k, v, scale and causal (required)
+ *   delta           [B,Hq,Sq] float32 workspace, device memory owned by the
+ *                   caller, 4-byte aligned; the call overwrites it (for head
+ *                   dims 64 and 128 it holds D_i = dO_i . O_i on return, for
+ *                   32 its contents are unspecified)
  *   other arguments as sdpa_fwd.
  *
- * Two kernel launches (keys-major for dK/dV, rows-major for dQ), each output
- * element written once: deterministic, no scratch memory.  Arithmetic is
- * fp32.  Errors as sdpa_fwd, plus SDPA_ERR_INVALID_ARG for a null dout, lse,
- * dq, dk or dv, and for B*Hq above 65535.
+ * Two kernel launches (rows-major for dQ, which also writes D to delta, then
+ * keys-major for dK/dV, which reads it), each output element written once:
+ * deterministic.  The library allocates nothing.  Arithmetic is fp32.
+ * Errors as sdpa_fwd, plus SDPA_ERR_INVALID_ARG for a null dout, lse, dq,
+ * dk, dv or delta, a misaligned delta, and B*Hq above 65535.
  */
 SDPA_API int sdpa_bwd(const void* q, const void* k, const void* v, const void* o,
                       const void* dout, const float* lse, void* dq, void* dk, void* dv,
-                      int B, int Hq, int Hkv, int Sq, int Sk, int d,
+                      float* delta, int B, int Hq, int Hkv, int Sq, int Sk, int d,
                       float scale, int causal, int dtype, void* stream);
 
 /* Static, NUL-terminated description of a status code. */

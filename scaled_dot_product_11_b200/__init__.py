@@ -49,7 +49,7 @@ _ll3 = ctypes.c_longlong * 3
 _lib.sdpa_fwd_strided.argtypes = ([_vp] * 5 + [_i] * 6 + [ctypes.POINTER(ctypes.c_longlong)] * 4
                                   + [_f, _i, _i, _vp])
 _lib.sdpa_fwd_strided.restype = _i
-_lib.sdpa_bwd.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _i, _i, _vp]
+_lib.sdpa_bwd.argtypes = [_vp] * 10 + [_i] * 6 + [_f, _i, _i, _vp]
 _lib.sdpa_bwd.restype = _i
 _lib.sdpa_fwd_fp8.argtypes = [_vp, _vp, _vp, _f, _f, _f, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]
 _lib.sdpa_fwd_fp8.restype = _i
@@ -86,10 +86,11 @@ def sdpa_fwd_fp8(q8, k8, v8, descale_q, descale_k, descale_v, o, lse, B, Hq, Hkv
                                  stream or None))
 
 
-def sdpa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Sq, Sk, d, scale, causal, dtype,
-             stream) -> int:
-    """Raw backward call: device addresses as ints, stream an int."""
-    return int(_lib.sdpa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Sq, Sk, d,
+def sdpa_bwd(q, k, v, o, dout, lse, dq, dk, dv, delta, B, Hq, Hkv, Sq, Sk, d, scale, causal,
+             dtype, stream) -> int:
+    """Raw backward call: device addresses as ints (delta: a [B,Hq,Sq] float32
+    workspace), stream an int."""
+    return int(_lib.sdpa_bwd(q, k, v, o, dout, lse, dq, dk, dv, delta, B, Hq, Hkv, Sq, Sk, d,
                              float(scale), int(causal), int(dtype), stream or None))
 
 
@@ -226,8 +227,9 @@ def attention_backward(q, k, v, o, lse, dout, causal=False, scale: float | None 
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     with torch.cuda.device(q.device):
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        delta = torch.empty(B, Hq, Sq, dtype=torch.float32, device=q.device)   # workspace
         rc = sdpa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
-                      lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                      lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), delta.data_ptr(),
                       B, Hq, Hkv, Sq, Sk, d, scale, causal,
                       SDPA_BF16 if q.dtype == torch.bfloat16 else SDPA_FP16, _stream_handle(stream))
     if rc != SDPA_OK:

@@ -372,7 +372,7 @@ int launch_bwd_tc(const void* q, const void* k, const void* v, const sdpa::BwdPa
         !encode_view(&tdo, dt, 2, bp.dout, D, bp.Sq, bp.Hq, bp.B, vq, C::kElemsPerSw, true))
         return SDPA_ERR_CUDA;
     sdpa::BwdTcParams tp;
-    tp.o = bp.o; tp.dout = bp.dout; tp.lse = bp.lse;
+    tp.o = bp.o; tp.dout = bp.dout; tp.lse = bp.lse; tp.delta = bp.delta;
     tp.dq = bp.dq; tp.dk = bp.dk; tp.dv = bp.dv;
     tp.B = bp.B; tp.Hq = bp.Hq; tp.Hkv = bp.Hkv; tp.Sq = bp.Sq; tp.Sk = bp.Sk; tp.group = bp.group;
     tp.causal = bp.causal; tp.causal_off = bp.causal_off; tp.scale = bp.scale;
@@ -391,22 +391,24 @@ int launch_bwd_tc(const void* q, const void* k, const void* v, const sdpa::BwdPa
     }
     const dim3 gkv((bp.Sk + 127) / 128, bp.B * bp.Hkv);
     const dim3 gq((bp.Sq + 127) / 128, bp.B * bp.Hq);
-    kdkdv<<<gkv, sdpa::kBtThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, tp);
-    if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
+    // dQ first: it writes D of every row, which the dK/dV kernel reads
     kdq<<<gq, sdpa::kBtThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, tp);
+    if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
+    kdkdv<<<gkv, sdpa::kBtThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, tp);
     return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
 }
 
 }  // namespace
 
 extern "C" int sdpa_bwd(const void* q, const void* k, const void* v, const void* o,
-                        const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
-                        int Hq, int Hkv, int Sq, int Sk, int d, float scale, int causal, int dtype,
-                        void* stream) {
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                        float* delta, int B, int Hq, int Hkv, int Sq, int Sk, int d, float scale,
+                        int causal, int dtype, void* stream) {
     int rc = check_args(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal);
     if (rc != SDPA_OK) return rc;
-    if (!dout || !lse || !dq || !dk || !dv) return SDPA_ERR_INVALID_ARG;
-    if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    if (!dout || !lse || !dq || !dk || !dv || !delta) return SDPA_ERR_INVALID_ARG;
+    if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+        reinterpret_cast<uintptr_t>(delta) % 4 != 0)
         return SDPA_ERR_INVALID_ARG;
     if ((long long)B * Hq > 65535) return SDPA_ERR_INVALID_ARG;   // grid rows
     if (dtype != SDPA_BF16 && dtype != SDPA_FP16) return SDPA_ERR_UNSUPPORTED;
@@ -414,7 +416,7 @@ extern "C" int sdpa_bwd(const void* q, const void* k, const void* v, const void*
     if (rc != SDPA_OK) return rc;
     sdpa::BwdParams bp;
     bp.q = q; bp.k = k; bp.v = v; bp.o = o; bp.dout = dout; bp.lse = lse;
-    bp.dq = dq; bp.dk = dk; bp.dv = dv;
+    bp.dq = dq; bp.dk = dk; bp.dv = dv; bp.delta = delta;
     bp.B = B; bp.Hq = Hq; bp.Hkv = Hkv; bp.Sq = Sq; bp.Sk = Sk; bp.group = Hq / Hkv;
     bp.causal = causal != 0 ? 1 : 0;
     bp.causal_off = causal == SDPA_CAUSAL_BOTTOM_RIGHT ? Sk - Sq : 0;

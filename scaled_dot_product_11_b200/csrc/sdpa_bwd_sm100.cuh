@@ -31,6 +31,7 @@ constexpr int kBwdThreads = 256;
 struct BwdParams {
     const void *q, *k, *v, *o, *dout;
     const float* lse;                // [B, Hq, Sq], natural log, from the forward
+    float* delta;                    // [B, Hq, Sq] workspace (tensor-core kernels)
     void *dq, *dk, *dv;
     int B, Hq, Hkv, Sq, Sk, group;
     int causal, causal_off;          // key j visible to query i iff j <= i + causal_off

@@ -12,12 +12,20 @@
 // and written over them; dV += P^T dO, dK += dS^T Q (PV form, Q and dO tiles
 // used MN-major).  dQ kernel, one CTA per 128 rows of one (batch, query
 // head), TMEM lane = row:  S = Q K^T, dP = dO V^T; dS; dQ += dS K.
+// The dQ kernel runs first and also writes D_i = dO_i . O_i of every row to
+// the caller's workspace, from which the dK/dV kernel reads it per step.
 // One CTA of 256 threads per tile: thread 0 issues the TMA copies (the
-// streamed tile pair one step ahead, double-buffered) and the MMAs; all eight
-// warps do the elementwise work, two per TMEM lane quarter splitting the
-// columns; every wait is bounded.
+// streamed tile pair one step ahead, double-buffered) and the MMAs, and
+// queues the next step's S and dP products right behind the current step's
+// accumulating products under one commit (the tensor pipe runs them in issue
+// order, so the S/dP columns they overwrite have been read); all eight warps
+// do the elementwise work, two per TMEM lane quarter splitting the columns,
+// each half packing its results over columns that only it reads (no barrier
+// between reading S and writing P); tiles that need no mask skip it.  Every
+// wait is bounded.
 #pragma once
 #include <cstdint>
+#include <type_traits>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -33,6 +41,7 @@ struct BwdTcParams {
     const void* o;                   // [B,Hq,Sq,D] (for D_i = dO_i . O_i)
     const void* dout;                // [B,Hq,Sq,D]
     const float* lse;                // [B,Hq,Sq]
+    float* delta;                    // [B,Hq,Sq] D_i, written by the dQ kernel
     void *dq, *dk, *dv;
     int B, Hq, Hkv, Sq, Sk, group;
     int causal, causal_off;
@@ -47,8 +56,9 @@ struct BtCfg {
     static constexpr int kSwBlockBytes = 128 * 128;
     static constexpr int kTileBytes = 128 * kRowBytes;
     static constexpr int kQkSteps = kRowBytes / 32;
-    // six tiles (the streamed pair double-buffered), LSE rows, D partial
-    // sums of two halves, barriers, TMEM slot
+    // six tiles (the streamed pair double-buffered), per-row statistics
+    // (dQ: D partial sums of two halves; dK/dV: LSE and D of the step's
+    // rows), barriers, TMEM slot
     static constexpr int kStatsBytes = 4 * 128 * 4;
     static constexpr int kSmemUsed = 6 * kTileBytes + kStatsBytes + 64;
     // one CTA per SM: each allocates all 512 TMEM columns
@@ -132,8 +142,11 @@ __device__ __forceinline__ void bt_mma_qk(uint32_t d_tmem, uint32_t a_smem, uint
     }
 }
 
-// PV form: d_tmem[128][D] (+)= A (TMEM, 128 x 128, 16-bit packed in 64
-// columns) . B_tile (128 x D, MN-major)
+// PV form: d_tmem[128][D] (+)= A (TMEM, 128 x 128, 16-bit packed) . B_tile
+// (128 x D, MN-major).  A's keys (or rows) 0-63 are packed in columns
+// [0,32) and 64-127 in [64,96): each half of the threads writes its packed
+// results over the first of the two 32-column chunks it read, which no other
+// thread reads.
 template <int D, bool BF16>
 __device__ __forceinline__ void bt_mma_pv(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, bool acc) {
     using C = BtCfg<D>;
@@ -142,7 +155,7 @@ __device__ __forceinline__ void bt_mma_pv(uint32_t d_tmem, uint32_t a_tmem, uint
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {    // 16 keys (or rows) per step
         const uint64_t off = (uint64_t)((kk * 16 * 128) >> 4);
-        mma_f16_ts(d_tmem, a_tmem + kk * 8, db + off, idesc, (acc || kk > 0) ? 1u : 0u);
+        mma_f16_ts(d_tmem, a_tmem + kk * 8 + (kk >= 4 ? 32 : 0), db + off, idesc, (acc || kk > 0) ? 1u : 0u);
     }
 }
 
@@ -190,8 +203,15 @@ __device__ __forceinline__ void bt_teardown(const BtSmem& sm, uint32_t tmem, boo
     if (threadIdx.x < 32) tmem_dealloc(tmem, 512);
 }
 
+// Whether tile (rows [i0, i0+128), keys [j0, j0+128)) needs no mask: no row
+// or key past the end, and with causal every key visible to every row
+__device__ __forceinline__ bool bt_tile_full(const BwdTcParams& p, int i0, int j0) {
+    return i0 + 128 <= p.Sq && j0 + 128 <= p.Sk && (!p.causal || j0 + 127 <= i0 + p.causal_off);
+}
+
 // dQ: one CTA per 128 query rows of one (batch, query head); TMEM lane = row.
-// Columns: S [0,128) (dS written over its first 64), dP [128,256), dQ [256,256+D).
+// Columns: S [0,128) (dS packed over [0,32) and [64,96)), dP [128,256),
+// dQ [256,256+D).
 template <int D, bool BF16>
 __global__ void __launch_bounds__(kBtThreads, 1)
 sdpa_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -214,7 +234,8 @@ sdpa_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     const int b = bh / p.Hq, hq = bh - b * p.Hq;
     const int kvrow = b * p.Hkv + hq / p.group;        // 3-D map index of the K/V head
     const int r = threadIdx.x & 127, row = i0 + r, half = threadIdx.x >> 7;
-    const uint32_t lane_base = (uint32_t)(((threadIdx.x >> 5) & 3) * 32) << 16;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const float kL2e = 1.44269504088896340736f;
     const float sl = p.scale * kL2e;
 
@@ -242,71 +263,98 @@ sdpa_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
                         jt * 128, kvrow);
         }
     };
+    // S = Q K^T and dP = dO V^T of tile jt, after its K/V tiles landed; warp 0
+    // waits, lane 0 issues.  Returns the wait's result.
+    auto issue_qk = [&](int jt) {
+        const int buf = jt & 1;
+        const bool got = bt_wait((buf ? sm.bar_kv[1] : sm.bar_kv[0]), (uint32_t)(jt >> 1) & 1u,
+                                 0x51000u | (uint32_t)(jt & 0xfff));
+        if (got && lane == 0) {
+            tc_fence_after();
+            bt_mma_qk<D, BF16>(tmem, sQ, sK(buf));
+            bt_mma_qk<D, BF16>(tmem + 128, sdO, sV(buf));
+        }
+        return got;
+    };
     if (threadIdx.x == 0 && ntiles > 0) load_kv(0);
     const float lse_r = row < p.Sq ? p.lse[(size_t)bh * p.Sq + row] * kL2e : 0.0f;
     dpart[threadIdx.x] = bt_row_dot<D, BF16>(p, (size_t)bh * p.Sq * D, row, half);
-    bool ok = bt_wait(sm.bar_in[0], 0, 0x50000u);
-    ok = __syncthreads_and(ok);
+    bool ok = __syncthreads_and(bt_wait(sm.bar_in[0], 0, 0x50000u));
     const float d_r = dpart[r] + dpart[r + 128];
+    if (half == 0 && row < p.Sq) p.delta[(size_t)bh * p.Sq + row] = d_r;   // for the dK/dV kernel
 
-    for (int jt = 0; jt < ntiles && ok; ++jt) {
+    // this thread's own wait results since the last block-wide check
+    bool mine = true;
+    if (ok && ntiles > 0 && warp == 0) {
+        mine = issue_qk(0);
+        if (lane == 0) mma_commit(sm.bar_mma);
+        __syncwarp();
+    }
+    // commit jt (jt >= 1): dQ of tile jt-1, then S and dP of tile jt
+    int jt = 0;
+    for (; jt < ntiles && ok; ++jt) {
         const int j0 = jt * 128, buf = jt & 1;
-        // the other buffer's last readers (tile jt-1's MMAs) have completed
+        ok = __syncthreads_and(bt_wait(sm.bar_mma, (uint32_t)jt & 1u, 0x52000u | (uint32_t)(jt & 0xfff)) && mine);
+        if (!ok) break;
+        tc_fence_after();
+        // the other buffer's last readers (tile jt-1's dQ MMAs) have completed
         if (threadIdx.x == 0 && jt + 1 < ntiles) load_kv(jt + 1);
-        ok = __syncthreads_and(bt_wait((buf ? sm.bar_kv[1] : sm.bar_kv[0]), (uint32_t)(jt >> 1) & 1u,
-                                       0x51000u | (uint32_t)(jt & 0xfff)));
-        if (!ok) break;
-        if (threadIdx.x == 0) {
-            tc_fence_after();
-            bt_mma_qk<D, BF16>(tmem, sQ, sK(buf));            // S = Q K^T
-            bt_mma_qk<D, BF16>(tmem + 128, sdO, sV(buf));     // dP = dO V^T
-            mma_commit(sm.bar_mma);
-        }
-        ok = __syncthreads_and(bt_wait(sm.bar_mma, 0u, 0x52000u | (uint32_t)(jt & 0xfff)));
-        if (!ok) break;
-        tc_fence_after();
-        // this thread's half of the row: key chunks 2*half and 2*half+1; all
-        // reads of S finish before dS is written over its first 64 columns
-        uint32_t w[2][16];
+        // this thread's half of the row: key chunks 2*half and 2*half+1, each
+        // packed as soon as computed over the first of them (columns only
+        // this thread reads)
+        auto elementwise = [&](auto masked) {
+            constexpr bool kMask = decltype(masked)::value;
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-            const int c = 2 * half + cc;
-            float s[32], dp[32];
-            tmem_ld32(tmem + lane_base + 32 * c, s);
-            tmem_ld32(tmem + lane_base + 128 + 32 * c, dp);
-            tmem_wait_ld();
-            reg_fence32(s);
-            reg_fence32(dp);
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c = 2 * half + cc;
+                float s[32], dp[32];
+                uint32_t w[16];
+                tmem_ld32(tmem + lane_base + 32 * c, s);
+                tmem_ld32(tmem + lane_base + 128 + 32 * c, dp);
+                tmem_wait_ld();
+                reg_fence32(s);
+                reg_fence32(dp);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                float ds2[2];
+                for (int e = 0; e < 16; ++e) {
+                    float ds2[2];
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int key = j0 + 32 * c + 2 * e + u;
-                    const bool vis = row < p.Sq && key < p.Sk && (!p.causal || key <= row + p.causal_off);
-                    const float pv = vis ? exp2f(s[2 * e + u] * sl - lse_r) : 0.0f;
-                    ds2[u] = pv * (dp[2 * e + u] - d_r);
+                    for (int u = 0; u < 2; ++u) {
+                        float pv = ex2_approx(fmaf(s[2 * e + u], sl, -lse_r));
+                        if constexpr (kMask) {
+                            const int key = j0 + 32 * c + 2 * e + u;
+                            const bool vis = row < p.Sq && key < p.Sk && (!p.causal || key <= row + p.causal_off);
+                            pv = vis ? pv : 0.0f;
+                        }
+                        ds2[u] = pv * (dp[2 * e + u] - d_r);
+                    }
+                    w[e] = bt_pack<BF16>(ds2[0], ds2[1]);
                 }
-                w[cc][e] = bt_pack<BF16>(ds2[0], ds2[1]);
+                tmem_st16(tmem + lane_base + 64 * half + 16 * cc, w);    // dS
             }
-        }
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        tmem_st16(tmem + lane_base + 16 * (2 * half), w[0]);      // dS
-        tmem_st16(tmem + lane_base + 16 * (2 * half + 1), w[1]);
+        };
+        if (bt_tile_full(p, i0, j0))
+            elementwise(std::false_type{});
+        else
+            elementwise(std::true_type{});
         tmem_wait_st();
         tc_fence_before();
         __syncthreads();
-        if (threadIdx.x == 0) {
-            tc_fence_after();
-            bt_mma_pv<D, BF16>(tmem + 256, tmem, sK(buf), jt > 0);   // dQ += dS K
-            mma_commit(sm.bar_mma);
+        if (warp == 0) {
+            if (lane == 0) {
+                tc_fence_after();
+                bt_mma_pv<D, BF16>(tmem + 256, tmem, sK(buf), jt > 0);   // dQ += dS K
+            }
+            __syncwarp();
+            if (jt + 1 < ntiles) mine = issue_qk(jt + 1);
+            if (lane == 0) mma_commit(sm.bar_mma);
+            __syncwarp();
         }
-        ok = __syncthreads_and(bt_wait(sm.bar_mma, 1u, 0x53000u | (uint32_t)(jt & 0xfff)));
-        tc_fence_after();
     }
+    // the last commit: dQ of the last tile
+    if (ok && ntiles > 0)
+        ok = __syncthreads_and(bt_wait(sm.bar_mma, (uint32_t)ntiles & 1u, 0x53000u) && mine);
     if (ok) {
+        tc_fence_after();
         // dQ row: scale and round (every row sees key 0, so ntiles >= 1);
         // the TMEM loads are warp-collective, the stores per row
 #pragma unroll 1
@@ -331,8 +379,8 @@ sdpa_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
 }
 
 // dK, dV: one CTA per 128 keys of one (batch, K/V head); TMEM lane = key.
-// Columns: S^T [0,128) (P^T over its first 64), dP^T [128,256) (dS^T over its
-// first 64), dV [256,256+D), dK [384,384+D).
+// Columns: S^T [0,128) (P^T packed over [0,32) and [64,96)), dP^T [128,256)
+// (dS^T packed over [128,160) and [192,224)), dV [256,256+D), dK [384,384+D).
 template <int D, bool BF16>
 __global__ void __launch_bounds__(kBtThreads, 1)
 sdpa_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -346,18 +394,18 @@ sdpa_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
     const uint32_t sK = base, sV = base + C::kTileBytes;
     auto sQ = [&](int buf) { return base + (uint32_t)(2 + 2 * buf) * C::kTileBytes; };
     auto sdO = [&](int buf) { return base + (uint32_t)(3 + 2 * buf) * C::kTileBytes; };
-    // lse_s[128]: LSE of the step's query rows (log2 units); dpart[256]: the
-    // two halves of their D = dO . O
+    // lse_s[128]: LSE of the step's query rows (log2 units); dl_s[128]: their D
     float* const lse_s = reinterpret_cast<float*>(smem_raw + (base - raw) + 6 * C::kTileBytes);
-    float* const dpart = lse_s + 128;
+    float* const dl_s = lse_s + 128;
     const BtSmem sm = bt_layout(base + 6 * C::kTileBytes + C::kStatsBytes);
     const uint32_t tmem = bt_setup(sm);
 
     const int j0 = blockIdx.x * 128;
     const int bk = blockIdx.y;                         // b * Hkv + hk
     const int b = bk / p.Hkv, hk = bk - b * p.Hkv;
-    const int key = j0 + (int)(threadIdx.x & 127), half = threadIdx.x >> 7;
-    const uint32_t lane_base = (uint32_t)(((threadIdx.x >> 5) & 3) * 32) << 16;
+    const int r = threadIdx.x & 127, key = j0 + r, half = threadIdx.x >> 7;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const float kL2e = 1.44269504088896340736f;
     const float sl = p.scale * kL2e;
 
@@ -388,41 +436,60 @@ sdpa_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             tma_load_3d(sdO(buf) + kb * C::kSwBlockBytes, &tmdO, (buf ? sm.bar_in[1] : sm.bar_in[0]), kb * C::kElemsPerSw, i0, bh);
         }
     };
+    // LSE (log2 units) and D of step st's 128 query rows: warps 0-3 and 4-7
+    auto load_stats = [&](int st) {
+        const int qr = step_i0(st) + r;
+        const size_t idx = (size_t)step_bh(st) * p.Sq + qr;
+        if (half == 0)
+            lse_s[r] = qr < p.Sq ? p.lse[idx] * kL2e : 0.0f;
+        else
+            dl_s[r] = qr < p.Sq ? p.delta[idx] : 0.0f;
+    };
+    // S^T = K Q^T and dP^T = V dO^T of step st, after its Q/dO tiles landed;
+    // warp 0 waits, lane 0 issues.  Returns the wait's result.
+    auto issue_qk = [&](int st) {
+        const int buf = st & 1;
+        const bool got = bt_wait((buf ? sm.bar_in[1] : sm.bar_in[0]), (uint32_t)(st >> 1) & 1u,
+                                 0x59000u | (uint32_t)(st & 0xfff));
+        if (got && lane == 0) {
+            tc_fence_after();
+            bt_mma_qk<D, BF16>(tmem, sK, sQ(buf));
+            bt_mma_qk<D, BF16>(tmem + 128, sV, sdO(buf));
+        }
+        return got;
+    };
     if (threadIdx.x == 0 && nsteps > 0) load_q(0);
     bool ok = __syncthreads_and(bt_wait(sm.bar_kv[0], 0, 0x58000u));
+    // this thread's own wait results since the last block-wide check
+    bool mine = true;
+    if (ok && nsteps > 0) {
+        load_stats(0);
+        if (warp == 0) {
+            mine = issue_qk(0);
+            if (lane == 0) mma_commit(sm.bar_mma);
+            __syncwarp();
+        }
+    }
 
+    // commit it (it >= 1): dV, dK of step it-1, then S^T and dP^T of step it
     int it = 0;
     for (; it < nsteps && ok; ++it) {
-        const int bh = step_bh(it), i0 = step_i0(it), buf = it & 1;
-        {
-            // the other buffer's last readers (step it-1's MMAs) have completed
-            if (threadIdx.x == 0 && it + 1 < nsteps) load_q(it + 1);
-            // the 128 query rows' LSE (log2 units) and D = dO . O
-            {
-                const int qr = i0 + (int)(threadIdx.x & 127);
-                if (half == 0) lse_s[threadIdx.x] = qr < p.Sq ? p.lse[(size_t)bh * p.Sq + qr] * kL2e : 0.0f;
-                dpart[threadIdx.x] = bt_row_dot<D, BF16>(p, (size_t)bh * p.Sq * D, qr, half);
-            }
-            ok = __syncthreads_and(bt_wait((buf ? sm.bar_in[1] : sm.bar_in[0]), (uint32_t)(it >> 1) & 1u,
-                                           0x59000u | (uint32_t)(it & 0xfff)));
-            if (!ok) break;
-            if (threadIdx.x == 0) {
-                tc_fence_after();
-                bt_mma_qk<D, BF16>(tmem, sK, sQ(buf));          // S^T = K Q^T
-                bt_mma_qk<D, BF16>(tmem + 128, sV, sdO(buf));   // dP^T = V dO^T
-                mma_commit(sm.bar_mma);
-            }
-            ok = __syncthreads_and(bt_wait(sm.bar_mma, 0u, 0x5a000u | (uint32_t)(it & 0xfff)));
-            if (!ok) break;
-            tc_fence_after();
-            // this thread's half of the key row: query chunks 2*half and
-            // 2*half+1; all reads finish before P^T and dS^T are written over
-            // the first 64 columns of S^T and dP^T
-            uint32_t wp[2][16], wd[2][16];
+        const int i0 = step_i0(it), buf = it & 1;
+        ok = __syncthreads_and(bt_wait(sm.bar_mma, (uint32_t)it & 1u, 0x5a000u | (uint32_t)(it & 0xfff)) && mine);
+        if (!ok) break;
+        tc_fence_after();
+        // the other buffer's last readers (step it-1's MMAs) have completed
+        if (threadIdx.x == 0 && it + 1 < nsteps) load_q(it + 1);
+        // this thread's half of the key row: query chunks 2*half and
+        // 2*half+1, each packed as soon as computed over the first of them
+        // in S^T and dP^T (columns only this thread reads)
+        auto elementwise = [&](auto masked) {
+            constexpr bool kMask = decltype(masked)::value;
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
                 const int c = 2 * half + cc;
                 float s[32], dp[32];
+                uint32_t wp[16], wd[16];
                 tmem_ld32(tmem + lane_base + 32 * c, s);
                 tmem_ld32(tmem + lane_base + 128 + 32 * c, dp);
                 tmem_wait_ld();
@@ -434,64 +501,70 @@ sdpa_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
                         const int col = 32 * c + 2 * e + u;
-                        const int qi = i0 + col;
-                        const bool vis = key < p.Sk && qi < p.Sq && (!p.causal || key <= qi + p.causal_off);
-                        pv2[u] = vis ? exp2f(s[2 * e + u] * sl - lse_s[col]) : 0.0f;
-                        ds2[u] = pv2[u] * (dp[2 * e + u] - (dpart[col] + dpart[128 + col]));
+                        float pv = ex2_approx(fmaf(s[2 * e + u], sl, -lse_s[col]));
+                        if constexpr (kMask) {
+                            const int qi = i0 + col;
+                            const bool vis = key < p.Sk && qi < p.Sq && (!p.causal || key <= qi + p.causal_off);
+                            pv = vis ? pv : 0.0f;
+                        }
+                        pv2[u] = pv;
+                        ds2[u] = pv * (dp[2 * e + u] - dl_s[col]);
                     }
-                    wp[cc][e] = bt_pack<BF16>(pv2[0], pv2[1]);
-                    wd[cc][e] = bt_pack<BF16>(ds2[0], ds2[1]);
+                    wp[e] = bt_pack<BF16>(pv2[0], pv2[1]);
+                    wd[e] = bt_pack<BF16>(ds2[0], ds2[1]);
                 }
+                tmem_st16(tmem + lane_base + 64 * half + 16 * cc, wp);          // P^T
+                tmem_st16(tmem + lane_base + 128 + 64 * half + 16 * cc, wd);    // dS^T
             }
-            tc_fence_before();
-            __syncthreads();
-            tc_fence_after();
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                const int c = 2 * half + cc;
-                tmem_st16(tmem + lane_base + 16 * c, wp[cc]);          // P^T
-                tmem_st16(tmem + lane_base + 128 + 16 * c, wd[cc]);    // dS^T
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncthreads();
-            if (threadIdx.x == 0) {
+        };
+        if (bt_tile_full(p, i0, j0))
+            elementwise(std::false_type{});
+        else
+            elementwise(std::true_type{});
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 0) {
+            if (lane == 0) {
                 tc_fence_after();
                 bt_mma_pv<D, BF16>(tmem + 256, tmem, sdO(buf), it > 0);         // dV += P^T dO
                 bt_mma_pv<D, BF16>(tmem + 384, tmem + 128, sQ(buf), it > 0);    // dK += dS^T Q
-                mma_commit(sm.bar_mma);
             }
-            ok = __syncthreads_and(bt_wait(sm.bar_mma, 1u, 0x5b000u | (uint32_t)(it & 0xfff)));
-            tc_fence_after();
+            __syncwarp();
+            if (it + 1 < nsteps) mine = issue_qk(it + 1);
+            if (lane == 0) mma_commit(sm.bar_mma);
+            __syncwarp();
         }
+        // this step's reads of the statistics finished before the barrier above
+        if (it + 1 < nsteps) load_stats(it + 1);
     }
+    // the last commit: dV, dK of the last step
+    if (ok && nsteps > 0)
+        ok = __syncthreads_and(bt_wait(sm.bar_mma, (uint32_t)nsteps & 1u, 0x5b000u) && mine);
     if (ok) {
+        tc_fence_after();
         // dV and dK rows (zero when no query sees these keys); the TMEM loads
-        // are warp-collective, the stores per key
+        // are warp-collective, the stores per key.  Warps 0-3 write dV, 4-7 dK.
         const size_t orow = ((size_t)bk * p.Sk + (size_t)key) * D;
-        {
-            // warps 0-3 write dV, warps 4-7 dK
-            const int t = half;
-            void* out = t ? p.dk : p.dv;
-            const float mul = t ? p.scale : 1.0f;
+        void* out = half ? p.dk : p.dv;
+        const float mul = half ? p.scale : 1.0f;
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                float x[32];
-                tmem_ld32(tmem + lane_base + (t ? 384 : 256) + 32 * c, x);
-                tmem_wait_ld();
-                reg_fence32(x);
-                if (key < p.Sk) {
-                    // with no step the accumulators were never written: zeros
+        for (int c = 0; c < D / 32; ++c) {
+            float x[32];
+            tmem_ld32(tmem + lane_base + (half ? 384 : 256) + 32 * c, x);
+            tmem_wait_ld();
+            reg_fence32(x);
+            if (key < p.Sk) {
+                // with no step the accumulators were never written: zeros
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) x[e] = it > 0 ? x[e] * mul : 0.0f;
-                    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(out) + orow + 32 * c);
+                for (int e = 0; e < 32; ++e) x[e] = it > 0 ? x[e] * mul : 0.0f;
+                uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(out) + orow + 32 * c);
 #pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4)
-                        dst[v4] = make_uint4(bt_pack<BF16>(x[8 * v4], x[8 * v4 + 1]),
-                                             bt_pack<BF16>(x[8 * v4 + 2], x[8 * v4 + 3]),
-                                             bt_pack<BF16>(x[8 * v4 + 4], x[8 * v4 + 5]),
-                                             bt_pack<BF16>(x[8 * v4 + 6], x[8 * v4 + 7]));
-                }
+                for (int v4 = 0; v4 < 4; ++v4)
+                    dst[v4] = make_uint4(bt_pack<BF16>(x[8 * v4], x[8 * v4 + 1]),
+                                         bt_pack<BF16>(x[8 * v4 + 2], x[8 * v4 + 3]),
+                                         bt_pack<BF16>(x[8 * v4 + 4], x[8 * v4 + 5]),
+                                         bt_pack<BF16>(x[8 * v4 + 6], x[8 * v4 + 7]));
             }
         }
     }

@@ -84,3 +84,24 @@ def test_backward_is_deterministic(sdpa):
     b = sdpa.attention_backward(q, k, v, o, lse, dout, causal=True)
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+def test_backward_writes_row_statistic_to_workspace(sdpa):
+    """The raw call's workspace holds D_i = dO_i . O_i on return (head dims 64
+    and 128), computed here in fp64 from the same 16-bit O and dO."""
+    w = Workload("delta", 2, 4, 2, 200, 200, 128, 0, seed=11)
+    q, k, v = make_qkv(w, "cuda")
+    g = torch.Generator(device="cpu").manual_seed(12)
+    dout = torch.randn(q.shape, generator=g).to(q.dtype).cuda()
+    o, lse = sdpa.attention(q, k, v, scale=w.scale)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    delta = torch.full((2, 4, 200), float("nan"), device="cuda")
+    rc = sdpa.sdpa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                       lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), delta.data_ptr(),
+                       2, 4, 2, 200, 200, 128, w.scale, 0, sdpa.SDPA_BF16, 0)
+    assert rc == 0
+    torch.cuda.synchronize()
+    ref = (dout.double() * o.double()).sum(-1).cpu().numpy()
+    got = delta.double().cpu().numpy()
+    assert np.isfinite(got).all()
+    assert np.abs(got - ref).max() <= 1e-5 * max(1.0, float(np.abs(ref).max()))

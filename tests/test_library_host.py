@@ -136,15 +136,18 @@ def test_backward_argument_checks():
     import scaled_dot_product_11_b200 as sdpa
 
     def bwd(ptrs=None, d=128, causal=0, dtype=0, B=1, Hq=2, Hkv=2, Sq=128, Sk=128):
-        ptrs = ptrs or tuple(P + 0x1000 * i for i in range(9))
+        ptrs = ptrs or tuple(P + 0x1000 * i for i in range(10))
         return sdpa.sdpa_bwd(*ptrs, B, Hq, Hkv, Sq, Sk, d, 0.088, causal, dtype, 0)
-    good = tuple(P + 0x1000 * i for i in range(9))
-    for i in range(9):             # every pointer required, lse included
+    good = tuple(P + 0x1000 * i for i in range(10))
+    for i in range(10):            # every pointer required, lse and delta included
         ptrs = list(good)
         ptrs[i] = 0
         assert bwd(tuple(ptrs)) == 1, i
     ptrs = list(good)
     ptrs[6] += 8                   # dq misaligned
+    assert bwd(tuple(ptrs)) == 1
+    ptrs = list(good)
+    ptrs[9] += 2                   # delta not 4-byte aligned
     assert bwd(tuple(ptrs)) == 1
     assert bwd(d=96) == 2
     assert bwd(dtype=2) == 2
