@@ -37,6 +37,12 @@ class SdpaError(RuntimeError):
                                                 sdpa_strerror(self.status), self.status))
 
 
+from . import build as _build  # noqa: E402  (mtime checks; compiles nothing by itself)
+
+# A library missing or older than its sources (a new entry point, say) is
+# compiled first, when nvcc is here, so that what loads matches the header.
+if _build.needs_build() and _build.nvcc_available():
+    _build.build()
 if not os.path.exists(LIB_PATH):
     raise ImportError("libsdpa_b200.so is not built at %s; run "
                       "`python -m scaled_dot_product_11_b200.build` (nvcc, sm_100a)" % LIB_PATH)

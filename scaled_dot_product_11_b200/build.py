@@ -9,6 +9,7 @@ symbols) on machines without a GPU driver; it only needs one to run.
 from __future__ import annotations
 
 import os
+import shutil
 import subprocess
 import sys
 
@@ -35,6 +36,11 @@ def nvcc() -> str:
         if cand and (os.path.sep not in cand or os.path.exists(cand)):
             return cand
     return "nvcc"
+
+
+def nvcc_available() -> bool:
+    exe = nvcc()
+    return bool(shutil.which(exe)) or os.path.exists(exe)
 
 
 def needs_build() -> bool:

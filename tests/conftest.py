@@ -1,5 +1,4 @@
 import os
-import shutil
 import sys
 
 import pytest
@@ -20,7 +19,6 @@ def _built_libraries():
     import oracle
     oracle.build()
     from scaled_dot_product_11_b200 import build as lib_build
-    if lib_build.needs_build() and shutil.which(lib_build.nvcc()) or \
-            lib_build.needs_build() and os.path.exists(lib_build.nvcc()):
+    if lib_build.needs_build() and lib_build.nvcc_available():
         lib_build.build()
     yield
