@@ -81,10 +81,13 @@ typedef enum {
                                     error while preparing or launching */
     SDPA_ERR_DEVICE_TIMEOUT = 4, /* a kernel's bounded wait expired (reported
                                     by sdpa_device_status only) */
-    SDPA_ERR_DEVICE_LAYOUT = 5   /* the kernel's shared-memory layout did not
+    SDPA_ERR_DEVICE_LAYOUT = 5,  /* the kernel's shared-memory layout did not
                                     fit its allocation at the base address the
                                     device gave it; nothing was computed
                                     (reported by sdpa_device_status only) */
+    SDPA_ERR_SCRATCH_LIMIT = 6   /* sdpa_bwd_noalloc: B*Hq*Sq is above
+                                    SDPA_BWD_NOALLOC_MAX_ROWS; nothing was
+                                    launched */
 } sdpa_status;
 
 /*
@@ -187,6 +190,36 @@ SDPA_API int sdpa_bwd(const void* q, const void* k, const void* v, const void* o
                       const void* dout, const float* lse, void* dq, void* dk, void* dv,
                       float* delta, int B, int Hq, int Hkv, int Sq, int Sk, int d,
                       float scale, int causal, int dtype, void* stream);
+
+/*
+ * sdpa_bwd_noalloc -- sdpa_bwd without the delta argument, for callers that
+ * cannot allocate device memory: code running inside a host framework that
+ * owns every device allocation and lends none to its extensions, or code on
+ * a path that must not call cudaMalloc / cudaFree because those calls can
+ * synchronise the device.  The article and the codelab have no counterpart
+ * to it: it changes where the backward's workspace lives, not what it
+ * computes.
+ *
+ * The workspace (D_i = dO_i . O_i, one float per query row) is a static
+ * device array of SDPA_BWD_NOALLOC_MAX_ROWS floats (8 MiB), which every GPU
+ * that loads the library holds until the process exits.  Arguments, outputs
+ * and errors as sdpa_bwd, plus SDPA_ERR_SCRATCH_LIMIT, with nothing launched,
+ * when B*Hq*Sq is above SDPA_BWD_NOALLOC_MAX_ROWS.  The call allocates
+ * nothing.
+ *
+ * The first call on a device looks the array's device address up with that
+ * device current; make that first call before any stream capture begins.
+ * All calls on a device share the one array, which keeps the D values of the
+ * last call: nothing in it has to start at zero, since every call writes each
+ * row's D before reading it.  Calls whose kernels overlap on the GPU (on
+ * streams with no order between them) race on the array and give wrong
+ * gradients: order them on one stream, or with events.
+ */
+#define SDPA_BWD_NOALLOC_MAX_ROWS (1 << 21)
+SDPA_API int sdpa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                              const void* dout, const float* lse, void* dq, void* dk,
+                              void* dv, int B, int Hq, int Hkv, int Sq, int Sk, int d,
+                              float scale, int causal, int dtype, void* stream);
 
 /* Static, NUL-terminated description of a status code. */
 SDPA_API const char* sdpa_strerror(int status);

@@ -16,7 +16,8 @@ import os
 
 __all__ = [
     "SDPA_BF16", "SDPA_FP16", "SDPA_OK", "SDPA_ERR_INVALID_ARG", "SDPA_ERR_UNSUPPORTED",
-    "SDPA_ERR_CUDA", "SDPA_ERR_DEVICE_TIMEOUT", "SDPA_ERR_DEVICE_LAYOUT", "SdpaError", "LIB_PATH",
+    "SDPA_ERR_CUDA", "SDPA_ERR_DEVICE_TIMEOUT", "SDPA_ERR_DEVICE_LAYOUT", "SDPA_ERR_SCRATCH_LIMIT",
+    "SDPA_BWD_NOALLOC_MAX_ROWS", "sdpa_bwd_noalloc", "SdpaError", "LIB_PATH",
     "SDPA_NO_MASK", "SDPA_CAUSAL", "SDPA_CAUSAL_BOTTOM_RIGHT",
     "sdpa_fwd", "sdpa_fwd_strided", "sdpa_fwd_fp8", "sdpa_bwd", "attention_backward", "sdpa_strerror", "sdpa_device_status",
     "sdpa_launches_per_call", "attention", "attention_fp8",
@@ -27,7 +28,8 @@ LIB_PATH = os.path.join(_HERE, "libsdpa_b200.so")
 
 SDPA_BF16, SDPA_FP16 = 0, 1
 (SDPA_OK, SDPA_ERR_INVALID_ARG, SDPA_ERR_UNSUPPORTED, SDPA_ERR_CUDA, SDPA_ERR_DEVICE_TIMEOUT,
- SDPA_ERR_DEVICE_LAYOUT) = range(6)
+ SDPA_ERR_DEVICE_LAYOUT, SDPA_ERR_SCRATCH_LIMIT) = range(7)
+SDPA_BWD_NOALLOC_MAX_ROWS = 1 << 21    # B*Hq*Sq limit of sdpa_bwd_noalloc
 
 
 class SdpaError(RuntimeError):
@@ -57,6 +59,8 @@ _lib.sdpa_fwd_strided.argtypes = ([_vp] * 5 + [_i] * 6 + [ctypes.POINTER(ctypes.
 _lib.sdpa_fwd_strided.restype = _i
 _lib.sdpa_bwd.argtypes = [_vp] * 10 + [_i] * 6 + [_f, _i, _i, _vp]
 _lib.sdpa_bwd.restype = _i
+_lib.sdpa_bwd_noalloc.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _i, _i, _vp]
+_lib.sdpa_bwd_noalloc.restype = _i
 _lib.sdpa_fwd_fp8.argtypes = [_vp, _vp, _vp, _f, _f, _f, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]
 _lib.sdpa_fwd_fp8.restype = _i
 _lib.sdpa_strerror.argtypes = [_i]
@@ -98,6 +102,16 @@ def sdpa_bwd(q, k, v, o, dout, lse, dq, dk, dv, delta, B, Hq, Hkv, Sq, Sk, d, sc
     workspace), stream an int."""
     return int(_lib.sdpa_bwd(q, k, v, o, dout, lse, dq, dk, dv, delta, B, Hq, Hkv, Sq, Sk, d,
                              float(scale), int(causal), int(dtype), stream or None))
+
+
+def sdpa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Sq, Sk, d, scale, causal,
+                     dtype, stream) -> int:
+    """Raw call of the backward that allocates nothing (its workspace is a
+    static device array, B*Hq*Sq <= SDPA_BWD_NOALLOC_MAX_ROWS), for callers
+    that cannot allocate device memory.  Device addresses as ints, stream an
+    int; calls on one device must not overlap on the GPU."""
+    return int(_lib.sdpa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Sq, Sk, d,
+                                     float(scale), int(causal), int(dtype), stream or None))
 
 
 def sdpa_strerror(status: int) -> str:

@@ -3,6 +3,7 @@
 // synchronisation, no fallback path.
 #include <cmath>
 #include <cstdint>
+#include <atomic>
 #include <cstring>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -440,6 +441,7 @@ extern "C" const char* sdpa_strerror(int status) {
     case SDPA_ERR_CUDA: return "CUDA runtime or driver error";
     case SDPA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
     case SDPA_ERR_DEVICE_LAYOUT: return "shared-memory layout did not fit at the device's base address";
+    case SDPA_ERR_SCRATCH_LIMIT: return "B*Hq*Sq exceeds the no-alloc backward's static workspace";
     default: return "unknown status";
     }
 }
@@ -458,3 +460,61 @@ extern "C" int sdpa_device_status(int* status, int* detail, int clear) {
 }
 
 extern "C" int sdpa_launches_per_call(void) { return 1; }
+
+// ---------------------------------------------------------------------------
+// sdpa_bwd_noalloc: the backward for callers that cannot allocate device
+// memory (a host framework that owns every allocation, or a path on which
+// cudaMalloc's possible device synchronisation is not allowed).  Its
+// workspace -- one float of D_i = dO_i . O_i per query row -- lives in the
+// static array below instead of a caller buffer; the kernels are sdpa_bwd's.
+// The article and the codelab have no counterpart: only the workspace's home
+// differs.
+// ---------------------------------------------------------------------------
+namespace {
+
+// 8 MiB on every GPU that loads the library, held until the process exits.
+// Every call on a device shares it; no entry needs clearing, because the dQ
+// kernel writes each row's D before the dK/dV kernel reads it.  Calls whose
+// kernels overlap on the GPU race on it.
+static __device__ __align__(256) float g_bwd_noalloc_delta[SDPA_BWD_NOALLOC_MAX_ROWS];
+
+// Device address of the array on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up
+// once per device (that device current) and cached; cudaGetSymbolAddress
+// allocates nothing.
+float* noalloc_delta(int* rc) {
+    static std::atomic<float*> cached[64];
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        *rc = SDPA_ERR_CUDA;
+        return nullptr;
+    }
+    float* ptr = cached[dev].load(std::memory_order_acquire);
+    if (!ptr) {
+        void* addr = nullptr;
+        if (cudaGetSymbolAddress(&addr, g_bwd_noalloc_delta) != cudaSuccess || !addr) {
+            *rc = SDPA_ERR_CUDA;
+            return nullptr;
+        }
+        ptr = static_cast<float*>(addr);
+        cached[dev].store(ptr, std::memory_order_release);
+    }
+    *rc = SDPA_OK;
+    return ptr;
+}
+
+}  // namespace
+
+extern "C" int sdpa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                                int B, int Hq, int Hkv, int Sq, int Sk, int d, float scale,
+                                int causal, int dtype, void* stream) {
+    // the limit first: an oversized request launches nothing
+    if (B > 0 && Hq > 0 && Sq > 0 && (long long)B * Hq * Sq > SDPA_BWD_NOALLOC_MAX_ROWS)
+        return SDPA_ERR_SCRATCH_LIMIT;
+    int rc = SDPA_OK;
+    float* delta = noalloc_delta(&rc);
+    if (!delta) return rc;
+    return sdpa_bwd(q, k, v, o, dout, lse, dq, dk, dv, delta, B, Hq, Hkv, Sq, Sk, d, scale,
+                    causal, dtype, stream);
+}

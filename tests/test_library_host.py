@@ -19,8 +19,8 @@ def declared_symbols():
 
 def test_header_declares_the_entry_points():
     assert set(declared_symbols()) == {"sdpa_fwd", "sdpa_fwd_strided", "sdpa_fwd_fp8",
-                                       "sdpa_bwd", "sdpa_strerror", "sdpa_device_status",
-                                       "sdpa_launches_per_call"}
+                                       "sdpa_bwd", "sdpa_bwd_noalloc", "sdpa_strerror",
+                                       "sdpa_device_status", "sdpa_launches_per_call"}
 
 
 def test_library_exports_every_declared_symbol():
@@ -43,6 +43,7 @@ def test_strerror_and_launch_count():
     assert "unsupported" in sdpa.sdpa_strerror(2)
     assert "timed out" in sdpa.sdpa_strerror(4)
     assert "layout" in sdpa.sdpa_strerror(5)
+    assert "static workspace" in sdpa.sdpa_strerror(6)
     assert sdpa.sdpa_strerror(99) == "unknown status"
     assert sdpa.sdpa_launches_per_call() == 1
 
