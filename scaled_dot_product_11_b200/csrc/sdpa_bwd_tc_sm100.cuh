@@ -436,14 +436,20 @@ sdpa_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             tma_load_3d(sdO(buf) + kb * C::kSwBlockBytes, &tmdO, (buf ? sm.bar_in[1] : sm.bar_in[0]), kb * C::kElemsPerSw, i0, bh);
         }
     };
-    // LSE (log2 units) and D of step st's 128 query rows: warps 0-3 and 4-7
+    // LSE (log2 units) and D of step st's 128 query rows, loaded by warps
+    // 1-7: warp 0 issues the MMAs meanwhile, and its loads would land after
+    // them
     auto load_stats = [&](int st) {
-        const int qr = step_i0(st) + r;
-        const size_t idx = (size_t)step_bh(st) * p.Sq + qr;
-        if (half == 0)
-            lse_s[r] = qr < p.Sq ? p.lse[idx] * kL2e : 0.0f;
-        else
-            dl_s[r] = qr < p.Sq ? p.delta[idx] : 0.0f;
+        if (warp == 0) return;
+        const int si0 = step_i0(st);
+        const size_t rows = (size_t)step_bh(st) * p.Sq;
+        for (int i = (int)threadIdx.x - 32; i < 256; i += kBtThreads - 32) {
+            const int qr = si0 + (i & 127);
+            if (i < 128)
+                lse_s[i] = qr < p.Sq ? p.lse[rows + qr] * kL2e : 0.0f;
+            else
+                dl_s[i - 128] = qr < p.Sq ? p.delta[rows + qr] : 0.0f;
+        }
     };
     // S^T = K Q^T and dP^T = V dO^T of step st, after its Q/dO tiles landed;
     // warp 0 waits, lane 0 issues.  Returns the wait's result.
