@@ -154,12 +154,25 @@ def _dims(q, k, v, allow_views=False):
         raise ValueError("shape mismatch: q %s k %s v %s" % (tuple(q.shape), tuple(k.shape),
                                                               tuple(v.shape)))
     for t in (q, k, v):
-        if not t.is_cuda:
-            raise ValueError("q, k, v must be CUDA tensors")
+        if not t.is_cuda or t.device != q.device:
+            raise ValueError("q, k, v must be CUDA tensors on one device")
         if not (t.is_contiguous() or (allow_views and t.stride(3) == 1)):
             raise ValueError("q, k, v must be contiguous CUDA tensors%s" % (
                 " or views whose last dimension is contiguous" if allow_views else ""))
     return int(B), int(Hq), int(Hkv), int(Sq), int(Sk), int(d)
+
+
+def _check_buffer(t, name, shape, dtype, device, contiguous=True):
+    """A tensor the kernels read or write through a raw pointer, `shape`
+    elements of it: size, type, device and layout are checked here because
+    the C ABI cannot see them.  contiguous=False accepts any view whose last
+    dimension is contiguous."""
+    layout_ok = t.is_contiguous() if contiguous else t.stride(-1) == 1
+    if (tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_cuda or t.device != device
+            or not layout_ok):
+        raise ValueError("%s must be a %s CUDA tensor of shape %s on %s, %s" % (
+            name, dtype, tuple(shape), device,
+            "contiguous" if contiguous else "with a contiguous last dimension"))
 
 
 def _stream_handle(stream):
@@ -182,6 +195,10 @@ def attention(q, k, v, causal=False, scale: float | None = None, out=None, lse=N
     if q.dtype not in (torch.bfloat16, torch.float16) or k.dtype != q.dtype or v.dtype != q.dtype:
         raise ValueError("q, k, v must share dtype bfloat16 or float16")
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is not None:
+        _check_buffer(out, "out", (B, Hq, Sq, d), q.dtype, q.device, contiguous=False)
+    if lse is not None:
+        _check_buffer(lse, "lse", (B, Hq, Sq), torch.float32, q.device)
     with torch.cuda.device(q.device):
         if out is None:
             out = torch.empty_like(q)
@@ -218,6 +235,10 @@ def attention_fp8(q8, k8, v8, descales, causal=False, scale: float | None = None
         if t.dtype != torch.float8_e4m3fn:
             raise ValueError("q8, k8, v8 must be float8_e4m3fn")
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is not None:
+        _check_buffer(out, "out", (B, Hq, Sq, d), torch.bfloat16, q8.device)
+    if lse is not None:
+        _check_buffer(lse, "lse", (B, Hq, Sq), torch.float32, q8.device)
     with torch.cuda.device(q8.device):
         if out is None:
             out = torch.empty((B, Hq, Sq, d), dtype=torch.bfloat16, device=q8.device)
@@ -239,11 +260,9 @@ def attention_backward(q, k, v, o, lse, dout, causal=False, scale: float | None 
     import torch
     B, Hq, Hkv, Sq, Sk, d = _dims(q, k, v)
     causal = _causal_code(causal)
-    for t in (o, dout):
-        if tuple(t.shape) != (B, Hq, Sq, d) or t.dtype != q.dtype or not t.is_contiguous():
-            raise ValueError("o and dout must be contiguous, q's shape and dtype")
-    if tuple(lse.shape) != (B, Hq, Sq) or lse.dtype != torch.float32 or not lse.is_contiguous():
-        raise ValueError("lse must be contiguous float32 [B, Hq, Sq]")
+    _check_buffer(o, "o", (B, Hq, Sq, d), q.dtype, q.device)
+    _check_buffer(dout, "dout", (B, Hq, Sq, d), q.dtype, q.device)
+    _check_buffer(lse, "lse", (B, Hq, Sq), torch.float32, q.device)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     with torch.cuda.device(q.device):
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)

@@ -155,3 +155,66 @@ def test_backward_argument_checks():
     assert bwd(causal=1, Sq=64) == 2
     assert bwd(causal=3) == 1
     assert bwd(B=300, Hq=256, Hkv=256) == 1   # grid rows
+
+
+class _FakeCudaTensor:
+    """Duck-typed stand-in for a CUDA tensor (none can be made without a
+    GPU): just what the binding's buffer check looks at."""
+
+    def __init__(self, shape, dtype, device, strides=None, cuda=True):
+        import torch
+        self.shape, self.dtype, self.is_cuda = tuple(shape), dtype, cuda
+        self.device = torch.device(device)
+        if strides is None:
+            strides, acc = [], 1
+            for n in reversed(self.shape):
+                strides.insert(0, acc)
+                acc *= n
+        self._strides = tuple(strides)
+
+    def stride(self, i=None):
+        return self._strides if i is None else self._strides[i]
+
+    def is_contiguous(self):
+        acc = 1
+        for n, st in zip(reversed(self.shape), reversed(self._strides)):
+            if n != 1 and st != acc:
+                return False
+            acc *= n
+        return True
+
+
+def test_wrapper_buffer_check_accepts_matching_buffers():
+    import torch
+    from scaled_dot_product_11_b200 import _check_buffer
+    dev = torch.device("cuda", 0)
+    _check_buffer(_FakeCudaTensor((2, 4, 100, 64), torch.bfloat16, dev), "o", (2, 4, 100, 64),
+                  torch.bfloat16, dev)
+    # a BTNH view: contiguous last dimension only, accepted where views are
+    btnh = _FakeCudaTensor((2, 4, 100, 64), torch.bfloat16, dev, strides=(4 * 100 * 64, 64, 256, 1))
+    _check_buffer(btnh, "out", (2, 4, 100, 64), torch.bfloat16, dev, contiguous=False)
+    with pytest.raises(ValueError):
+        _check_buffer(btnh, "o", (2, 4, 100, 64), torch.bfloat16, dev)
+
+
+@pytest.mark.parametrize("bad", ["shape", "dtype", "device", "host", "last_stride"])
+def test_wrapper_buffer_check_refuses_mismatches(bad):
+    """Outputs and backward inputs reach the kernels as raw pointers: a short,
+    mistyped, host or other-device buffer is refused before any launch."""
+    import torch
+    from scaled_dot_product_11_b200 import _check_buffer
+    dev = torch.device("cuda", 0)
+    shape, dtype, device, strides, cuda = (2, 4, 100, 64), torch.bfloat16, dev, None, True
+    if bad == "shape":
+        shape = (2, 4, 99, 64)
+    elif bad == "dtype":
+        dtype = torch.float16
+    elif bad == "device":
+        device = torch.device("cuda", 1)
+    elif bad == "host":
+        cuda = False
+    else:
+        strides = (4 * 100 * 128, 100 * 128, 128, 2)
+    t = _FakeCudaTensor(shape, dtype, device, strides, cuda)
+    with pytest.raises(ValueError):
+        _check_buffer(t, "out", (2, 4, 100, 64), torch.bfloat16, dev, contiguous=False)
