@@ -1,6 +1,5 @@
 """The seeded input generators (no GPU): the recipe the parity tests and the
 benchmark rely on, checked against what it promises."""
-import numpy as np
 import pytest
 import torch
 
