@@ -237,7 +237,7 @@ SDPA_API const char* sdpa_strerror(int status);
 SDPA_API int sdpa_device_status(int* status, int* detail, int clear);
 
 /* Number of kernel launches sdpa_fwd / sdpa_fwd_strided / sdpa_fwd_fp8 issue
- * per call (1); sdpa_bwd issues 2. */
+ * per call (1); sdpa_bwd and sdpa_bwd_noalloc issue 2. */
 SDPA_API int sdpa_launches_per_call(void);
 
 #ifdef __cplusplus
