@@ -3,12 +3,12 @@
 // synchronisation, no fallback path.
 #include <cmath>
 #include <cstdint>
-#include <atomic>
 #include <cstring>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "sdpa.h"
+#include "sdpa_host.h"
 #include "sdpa_fwd_sm100.cuh"
 #include "sdpa_bwd_sm100.cuh"
 #include "sdpa_bwd_tc_sm100.cuh"
@@ -18,24 +18,11 @@ namespace {
 using sdpa::FwdCfg;
 using sdpa::FwdParams;
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (fn == nullptr) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
-                cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return nullptr;
-        fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
+using sdpa_host::View;
+using sdpa_host::bhsd;
+using sdpa_host::encode_view;
+using sdpa_host::same;
+using sdpa_host::sm_count;
 
 // 0 ok, else an sdpa_status.  Caches the answer per device.
 int check_device() {
@@ -50,20 +37,6 @@ int check_device() {
     const bool ok = (major == 10 && minor == 0);
     if (dev >= 0 && dev < 64) verdict[dev] = ok ? 1 : 2;
     return ok ? SDPA_OK : SDPA_ERR_UNSUPPORTED;
-}
-
-// Streaming multiprocessors of the current device (cached; 148 on B200).
-int sm_count() {
-    static int cache[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (cache[dev] == 0) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-            n = 148;
-        cache[dev] = n;
-    }
-    return cache[dev];
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -87,39 +60,6 @@ int check_args(const void* q, const void* k, const void* v, const void* o, const
     if (causal == SDPA_CAUSAL && Sq != Sk) return SDPA_ERR_UNSUPPORTED;
     if (causal == SDPA_CAUSAL_BOTTOM_RIGHT && Sq > Sk) return SDPA_ERR_UNSUPPORTED;
     return SDPA_OK;
-}
-
-// Element strides (batch, head, row) of a [B, H, S, d] view, d contiguous.
-struct View {
-    long long sb, sh, ss;
-};
-View bhsd(int H, int S, int d) {
-    return View{(long long)H * S * d, (long long)S * d, (long long)d};
-}
-
-bool same(const View& a, const View& b) { return a.sb == b.sb && a.sh == b.sh && a.ss == b.ss; }
-
-// Tiled map over (d, S, H, B) with the view's strides -- 3-D (d, S, B*H) for
-// contiguous [B,H,S,d] data (`rank3`); boxes of box_inner x 128 rows of one
-// (head, batch), 128-byte swizzle.
-bool encode_view(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* base, int d,
-                 int rows, int heads, int batch, const View& v, int box_inner, bool rank3,
-                 int box_rows = 128, int box_heads = 1) {
-    // swizzle rows of box_inner elements: 128 bytes, or 64 (head dim 32, 16-bit)
-    const CUtensorMapSwizzle swz =
-        box_inner * elem_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint32_t rank = rank3 ? 3u : 4u;
-    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)heads, (cuuint64_t)batch};
-    cuuint64_t strides[3] = {(cuuint64_t)(v.ss * elem_bytes), (cuuint64_t)(v.sh * elem_bytes),
-                             (cuuint64_t)(v.sb * elem_bytes)};
-    if (rank == 3) dims[2] = (cuuint64_t)heads * (cuuint64_t)batch;
-    const cuuint32_t box[4] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, (cuuint32_t)box_heads, 1u};
-    const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
-    return fn(m, dt, rank, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // A view the kernel can address: positive strides whose byte sizes are
@@ -222,6 +162,13 @@ int launch_packed(const void* q, const void* k, const void* v, const View& vq, c
     return launch_cfg<D, KIND, NS, QB, false, true, true>(q, k, v, vq, vk, vv, pk, stream);
 }
 
+// The two-query-tile kernel (sdpa_fwd2q.cu) serves head dims 64 and 128 in
+// every layout; this file's one-tile kernel serves head dim 32 and the
+// decode-shaped units with packed query heads.
+#ifndef SDPA_FWD2Q
+#define SDPA_FWD2Q 1
+#endif
+
 template <int D, int KIND, int NS, int QB>
 int launch(const void* q, const void* k, const void* v, const View& vq, const View& vk, const View& vv,
            const FwdParams& prm, cudaStream_t stream) {
@@ -230,8 +177,34 @@ int launch(const void* q, const void* k, const void* v, const View& vq, const Vi
                             same(vv, bhsd(prm.Hkv, prm.Sk, D)) &&
                             prm.o_sb == (long long)prm.Hq * prm.Sq * D && prm.o_sh == (long long)prm.Sq * D &&
                             prm.o_ss == D;
-    return contiguous ? launch_form<D, KIND, NS, QB, false>(q, k, v, vq, vk, vv, prm, stream)
-                      : launch_form<D, KIND, NS, QB, true>(q, k, v, vq, vk, vv, prm, stream);
+    if constexpr (SDPA_FWD2Q && D != 32) {
+        sdpa_host::Fwd2Request r;
+        r.q = q;
+        r.k = k;
+        r.v = v;
+        r.o = prm.o;
+        r.lse = prm.lse;
+        r.vq = vq;
+        r.vk = vk;
+        r.vv = vv;
+        r.vo = View{prm.o_sb, prm.o_sh, prm.o_ss};
+        r.B = prm.B;
+        r.Hq = prm.Hq;
+        r.Hkv = prm.Hkv;
+        r.Sq = prm.Sq;
+        r.Sk = prm.Sk;
+        r.d = D;
+        r.kind = KIND;
+        r.causal = prm.causal;
+        r.causal_off = prm.causal_off;
+        r.contiguous = contiguous;
+        r.score_log2 = prm.score_log2;
+        r.out_mul = prm.out_mul;
+        return sdpa_host::launch_fwd2q(r, stream);
+    } else {
+        return contiguous ? launch_form<D, KIND, NS, QB, false>(q, k, v, vq, vk, vv, prm, stream)
+                          : launch_form<D, KIND, NS, QB, true>(q, k, v, vq, vk, vv, prm, stream);
+    }
 }
 
 FwdParams make_params(void* o, const View& vo, float* lse, int B, int Hq, int Hkv, int Sq, int Sk,
@@ -447,9 +420,14 @@ extern "C" const char* sdpa_strerror(int status) {
 }
 
 extern "C" int sdpa_device_status(int* status, int* detail, int clear) {
-    unsigned int h[2] = {0u, 0u};
+    unsigned int h[2] = {0u, 0u}, h2[2] = {0u, 0u};
     if (cudaDeviceSynchronize() != cudaSuccess) return SDPA_ERR_CUDA;
     if (cudaMemcpyFromSymbol(h, sdpa::g_sdpa_status, sizeof h) != cudaSuccess) return SDPA_ERR_CUDA;
+    if (sdpa_host::fwd2q_status(h2, clear) != SDPA_OK) return SDPA_ERR_CUDA;
+    if (h[0] == 0u) {   // the first kernel that recorded a status wins
+        h[0] = h2[0];
+        h[1] = h2[1];
+    }
     if (status) *status = (int)h[0];
     if (detail) *detail = (int)h[1];
     if (clear) {
@@ -478,29 +456,20 @@ namespace {
 // kernels overlap on the GPU race on it.
 static __device__ __align__(256) float g_bwd_noalloc_delta[SDPA_BWD_NOALLOC_MAX_ROWS];
 
-// Device address of the array on the current device.  In host code the
-// array's name is only a host-side stand-in, so the address is looked up
-// once per device (that device current) and cached; cudaGetSymbolAddress
-// allocates nothing.
+// Device address of the array in the current context.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up on
+// every call, with the caller's device current: a cached address would go
+// stale when the context that holds the module is destroyed and recreated
+// (cudaDeviceReset) or when the caller switches to another context of the
+// same device.  cudaGetSymbolAddress allocates nothing.
 float* noalloc_delta(int* rc) {
-    static std::atomic<float*> cached[64];
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_bwd_noalloc_delta) != cudaSuccess || !addr) {
         *rc = SDPA_ERR_CUDA;
         return nullptr;
     }
-    float* ptr = cached[dev].load(std::memory_order_acquire);
-    if (!ptr) {
-        void* addr = nullptr;
-        if (cudaGetSymbolAddress(&addr, g_bwd_noalloc_delta) != cudaSuccess || !addr) {
-            *rc = SDPA_ERR_CUDA;
-            return nullptr;
-        }
-        ptr = static_cast<float*>(addr);
-        cached[dev].store(ptr, std::memory_order_release);
-    }
     *rc = SDPA_OK;
-    return ptr;
+    return static_cast<float*>(addr);
 }
 
 }  // namespace

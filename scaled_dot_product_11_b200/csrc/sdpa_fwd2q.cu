@@ -1,0 +1,116 @@
+// sdpa_fwd2q.cu -- host launch of the two-query-tile forward kernel
+// (sdpa_fwd2q_sm100.cuh): schedule parameters, TMA tensor maps, launch.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "sdpa.h"
+#include "sdpa_host.h"
+#include "sdpa_fwd2q_sm100.cuh"
+
+// K/V ring depth and Q buffers per stage: 16-bit head dim 128 (32 KB tiles:
+// 2 Q tiles + 5 ring slots fill the 227 KB), 16-bit head dim 64 and e4m3
+// head dim 128 (16 KB tiles: 2 x 2 Q tiles + 8 ring slots).
+#ifndef SDPA2_STAGES_D128
+#define SDPA2_STAGES_D128 5
+#endif
+#ifndef SDPA2_STAGES_16K
+#define SDPA2_STAGES_16K 8
+#endif
+
+namespace sdpa_host {
+namespace {
+
+using sdpa::fwd2::Cfg;
+using sdpa::fwd2::Params;
+
+template <int D, int KIND, int NS, int QB, bool STRIDED>
+int launch_cfg(const Fwd2Request& r, const Params& prm, cudaStream_t stream) {
+    using C = Cfg<D, KIND, NS, QB>;
+    const CUtensorMapDataType dt = KIND == sdpa::fwd2::K2_BF16   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                   : KIND == sdpa::fwd2::K2_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                                 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    CUtensorMap tq, tk, tv;
+    if (!encode_view(&tq, dt, C::kElem, r.q, D, r.Sq, r.Hq, r.B, r.vq, C::kElemsPerSw, !STRIDED) ||
+        !encode_view(&tk, dt, C::kElem, r.k, D, r.Sk, r.Hkv, r.B, r.vk, C::kElemsPerSw, !STRIDED) ||
+        !encode_view(&tv, dt, C::kElem, r.v, D, r.Sk, r.Hkv, r.B, r.vv, C::kElemsPerSw, !STRIDED))
+        return SDPA_ERR_CUDA;
+    auto kern = sdpa::fwd2::sdpa_fwd2q_sm100_kernel<D, KIND, NS, QB, STRIDED>;
+    static bool attr_set[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SDPA_ERR_CUDA;
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+            return SDPA_ERR_CUDA;
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+    // persistent: one CTA per SM (fewer when there are fewer items)
+    const unsigned grid = (unsigned)(prm.n_items < sm_count() ? prm.n_items : sm_count());
+    kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, prm);
+    return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
+template <int D, int KIND, int NS, int QB>
+int launch_form(const Fwd2Request& r, const Params& prm, cudaStream_t stream) {
+    return r.contiguous ? launch_cfg<D, KIND, NS, QB, false>(r, prm, stream)
+                        : launch_cfg<D, KIND, NS, QB, true>(r, prm, stream);
+}
+
+}  // namespace
+
+int launch_fwd2q(const Fwd2Request& r, cudaStream_t stream) {
+    Params prm;
+    prm.o = r.o;
+    prm.lse = r.lse;
+    prm.B = r.B;
+    prm.Hq = r.Hq;
+    prm.Hkv = r.Hkv;
+    prm.Sq = r.Sq;
+    prm.Sk = r.Sk;
+    prm.group = r.Hq / r.Hkv;
+    const int nq = (r.Sq + 127) / 128;
+    prm.n_pairs = (nq + 1) / 2;
+    // causal items pair unit m with unit n_pairs-1-m of the same head
+    prm.items_per_head = r.causal ? (prm.n_pairs + 1) / 2 : prm.n_pairs;
+    const long long n_items = (long long)r.B * r.Hq * prm.items_per_head;
+    if (n_items > INT32_MAX) return SDPA_ERR_INVALID_ARG;
+    prm.n_items = (int)n_items;
+    // about two waves of items per group of (batch, head) pairs
+    int gh = (2 * sm_count() + prm.items_per_head - 1) / prm.items_per_head;
+    if (gh < 1) gh = 1;
+    if (gh > r.B * r.Hq) gh = r.B * r.Hq;
+    prm.group_heads = gh;
+    prm.causal = r.causal ? 1 : 0;
+    prm.causal_off = r.causal_off;
+    prm.score_log2 = r.score_log2;
+    prm.out_mul = r.out_mul;
+    prm.o_sb = r.vo.sb;
+    prm.o_sh = r.vo.sh;
+    prm.o_ss = r.vo.ss;
+    using namespace sdpa::fwd2;
+    switch (r.kind) {
+    case K2_BF16:
+        return r.d == 64 ? launch_form<64, K2_BF16, SDPA2_STAGES_16K, 2>(r, prm, stream)
+                         : launch_form<128, K2_BF16, SDPA2_STAGES_D128, 1>(r, prm, stream);
+    case K2_FP16:
+        return r.d == 64 ? launch_form<64, K2_FP16, SDPA2_STAGES_16K, 2>(r, prm, stream)
+                         : launch_form<128, K2_FP16, SDPA2_STAGES_D128, 1>(r, prm, stream);
+    case K2_E4M3:
+        if (!r.contiguous || r.d != 128) return SDPA_ERR_UNSUPPORTED;
+        return launch_cfg<128, K2_E4M3, SDPA2_STAGES_16K, 2, false>(r, prm, stream);
+    default:
+        return SDPA_ERR_UNSUPPORTED;
+    }
+}
+
+int fwd2q_status(unsigned int out[2], int clear) {
+    if (cudaMemcpyFromSymbol(out, sdpa::fwd2::g_status, 2 * sizeof(unsigned int)) != cudaSuccess)
+        return SDPA_ERR_CUDA;
+    if (clear) {
+        const unsigned int z[2] = {0u, 0u};
+        if (cudaMemcpyToSymbol(sdpa::fwd2::g_status, z, sizeof z) != cudaSuccess) return SDPA_ERR_CUDA;
+    }
+    return SDPA_OK;
+}
+
+}  // namespace sdpa_host

@@ -7,12 +7,13 @@ rows (first, last, tile-boundary and seeded random rows of every (batch,
 head)), which the oracle computes one by one.
 
 Tolerances.  LSE (fp32 output): max abs error <= 1e-3 (bf16 / fp16 inputs)
-and <= 2e-3 (FP8).  O: max abs error <= 1e-2 (bf16 / fp16) and <= 6e-2 (FP8)
-for the kernel's own error, on top of the half-ulp rounding every value
-stored in a 16-bit output carries: |O - O_ref| <= tol + ulp(O_ref)/2 in the
-output format.  A stored bf16 value cannot be closer than that to the exact
-result (half an ulp is 0.0156 for 4 <= |O| < 8, above 1e-2 by itself); the
-codelab's own bf16 comparison (section 6) is looser, rtol = atol = 1e-2.
+and <= 2e-3 (FP8).  O: max abs error <= 1e-2 (bf16 / fp16) and <= 6e-2 (FP8),
+as stated, on every element whose exact value has |O_ref| < 4.  Where
+|O_ref| >= 4 a stored bf16 value cannot meet 1e-2 at all (half an ulp is
+0.0156 for 4 <= |O| < 8), so there the bound applies to the kernel's own error
+on top of that rounding: |O - O_ref| <= tol + ulp(O_ref)/2 in the output
+format.  The codelab's own bf16 comparison (section 6) is looser, rtol = atol
+= 1e-2.
 """
 import math
 
@@ -42,11 +43,21 @@ def half_ulp(ref, dtype):
     return np.where(a > 0, 2.0 ** (e - MANT_BITS[dtype]) / 2.0, 0.0)
 
 
+# below this magnitude the stated bound is met as stated; at and above it a
+# 16-bit output's own rounding (half an ulp) is allowed on top of it
+PLAIN_BOUND_BELOW = 4.0
+
+
+def o_allowance(ref, tol, dtype):
+    """Per-element O bound: tol where |ref| < 4, tol + ulp(ref)/2 elsewhere."""
+    return tol + np.where(np.abs(ref) < PLAIN_BOUND_BELOW, 0.0, half_ulp(ref, dtype))
+
+
 def check_o(got, ref, tol, dtype, what):
     err = np.abs(got - ref)
-    excess = err - half_ulp(ref, dtype)
+    excess = err - o_allowance(ref, tol, dtype)
     i = int(np.argmax(excess))
-    assert excess.flat[i] <= tol, "%s: |dO| %.4g at flat index %d (ref %.5g, got %.5g), max|dO| %.4g" % (
+    assert excess.flat[i] <= 0.0, "%s: |dO| %.4g at flat index %d (ref %.5g, got %.5g), max|dO| %.4g" % (
         what, err.flat[i], i, ref.flat[i], got.flat[i], err.max())
     return float(err.max())
 
