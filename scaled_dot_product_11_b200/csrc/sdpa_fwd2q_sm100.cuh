@@ -47,22 +47,26 @@
 #include "sm100_ptx.cuh"
 
 // Pairs e (0..15) of a 32-column chunk whose exponentials are evaluated on
-// the FMA pipe (exp2_poly_x2) instead of the MUFU: bit (e & 7) of the mask.
+// the FMA pipe (exp2_poly_x2) instead of the MUFU: bit (e & 7) of the mask,
+// for 16-bit inputs and for e4m3 (whose products take half the tensor time,
+// so that the MUFU bounds it sooner).
 #ifndef SDPA2_POLY_MASK
 #define SDPA2_POLY_MASK 0x00
 #endif
+#ifndef SDPA2_POLY_MASK_FP8
+#define SDPA2_POLY_MASK_FP8 0x11
+#endif
 // Register budgets (setmaxnreg) of the softmax, epilogue and producer/MMA
 // warp groups: 8 * S + 4 * E + 4 * W <= 16 * 128 (the launch allocation; per
-// SM sub-partition 2 * S + E + W <= 512).  The MMA issue loops stay rolled so
-// that their descriptor arithmetic is not hoisted into registers.
+// SM sub-partition 2 * S + E + W <= 512).
 #ifndef SDPA2_REGS_SOFTMAX
-#define SDPA2_REGS_SOFTMAX 192
+#define SDPA2_REGS_SOFTMAX 184
 #endif
 #ifndef SDPA2_REGS_EPILOGUE
-#define SDPA2_REGS_EPILOGUE 64
+#define SDPA2_REGS_EPILOGUE 56
 #endif
 #ifndef SDPA2_REGS_OTHER
-#define SDPA2_REGS_OTHER 64
+#define SDPA2_REGS_OTHER 88
 #endif
 static_assert(8 * SDPA2_REGS_SOFTMAX + 4 * SDPA2_REGS_EPILOGUE + 4 * SDPA2_REGS_OTHER <= 16 * 128,
               "register split exceeds the launch allocation");
@@ -198,8 +202,9 @@ __device__ __forceinline__ bool wait_sleep(uint32_t bar, uint32_t parity, uint32
     return wait_slow(bar, parity, abort_addr, status, where, SDPA2_EPI_SLEEP_NS);
 }
 
+template <int KIND>
 __device__ __forceinline__ constexpr bool poly_pair(int e) {
-    return ((SDPA2_POLY_MASK >> (e & 7)) & 1) != 0;
+    return (((KIND == K2_E4M3 ? SDPA2_POLY_MASK_FP8 : SDPA2_POLY_MASK) >> (e & 7)) & 1) != 0;
 }
 
 // Maximum of 128 registers (3-input max, four chains).
@@ -288,15 +293,12 @@ __device__ __forceinline__ int stage_tiles(const Unit& u, int s) { return s ? u.
 struct Cursor {
     Unit u;
     int j;   // tile within the unit
-    int g;   // tile within the stream
 };
 __device__ __forceinline__ void cur_first(const Params& p, Cursor& c) {
     unit_first(p, c.u);
     c.j = 0;
-    c.g = 0;
 }
 __device__ __forceinline__ void cur_next(const Params& p, Cursor& c) {
-    ++c.g;
     if (++c.j == c.u.n) {
         unit_next(p, c.u);
         c.j = 0;
@@ -477,9 +479,17 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             constexpr uint32_t fmt = (KIND == K2_BF16) ? 1u : 0u;
             constexpr uint32_t idesc_qk = make_idesc(fmt, false, kRows, kKeys);
             constexpr uint32_t idesc_pv = make_idesc(fmt, true, kRows, D);
-            const uint64_t desc_q = make_smem_desc(sQ, 16, C::kSbo, C::kSwLayout);
-            const uint64_t desc_k = make_smem_desc(sKV, 16, C::kSbo, C::kSwLayout);
-            const uint64_t desc_v = make_smem_desc(sKV, C::kSwBlockBytes, C::kSbo, C::kSwLayout);
+            // Shared-memory descriptors: the high word (stride offset, fixed
+            // bits, swizzle) is the same for every operand; the low word is
+            // start address >> 4 plus the leading offset, and stepping
+            // through a tile only adds to the start address (no carry: the
+            // addresses stay below 2^18).
+            const uint64_t dq0 = make_smem_desc(sQ, 16, C::kSbo, C::kSwLayout);
+            const uint64_t dk0 = make_smem_desc(sKV, 16, C::kSbo, C::kSwLayout);
+            const uint64_t dv0 = make_smem_desc(sKV, C::kSwBlockBytes, C::kSbo, C::kSwLayout);
+            const uint32_t desc_hi = (uint32_t)(dq0 >> 32);
+            const uint32_t dq_lo = (uint32_t)dq0, dk_lo = (uint32_t)dk0, dv_lo = (uint32_t)dv0;
+            auto desc = [&](uint32_t lo) -> uint64_t { return ((uint64_t)desc_hi << 32) | lo; };
             bool ok = true;
             int cq[2] = {0, 0};    // S_s tiles issued (S_full phase)
             int cp[2] = {0, 0};    // P_s tiles consumed (P_full phase)
@@ -494,19 +504,22 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 if (leader) mma_commit(b_);
                 __syncwarp();
             };
+            // The issue loops are unrolled: every MMA's descriptors are one
+            // add of an immediate to a 32-bit base, so the single issuing
+            // thread keeps up with the tensor pipe.
             auto issue_qk = [&](int s, int qb, int slot) {
                 const uint32_t d_tmem = tmem + (s ? C::kColS1 : C::kColS0);
-                const uint64_t dq = desc_q + (uint64_t)(((s * QB + qb) * C::kTileBytes) >> 4);
-                const uint64_t dk = desc_k + (uint64_t)((slot * C::kTileBytes) >> 4);
+                const uint32_t aq = dq_lo + (uint32_t)(((s * QB + qb) * C::kTileBytes) >> 4);
+                const uint32_t bk = dk_lo + (uint32_t)((slot * C::kTileBytes) >> 4);
                 if (leader) {
-#pragma unroll 1
+#pragma unroll
                     for (int kk = 0; kk < C::kQkSteps; ++kk) {
-                        const uint64_t off = (uint64_t)(((kk / C::kStepsPerBlock) * C::kSwBlockBytes +
-                                                         (kk % C::kStepsPerBlock) * 32) >> 4);
+                        constexpr int kBlk = C::kSwBlockBytes, kSpb = C::kStepsPerBlock;
+                        const uint32_t off = (uint32_t)(((kk / kSpb) * kBlk + (kk % kSpb) * 32) >> 4);
                         if constexpr (KIND == K2_E4M3)
-                            mma_f8_ss(d_tmem, dq + off, dk + off, idesc_qk, kk > 0);
+                            mma_f8_ss(d_tmem, desc(aq + off), desc(bk + off), idesc_qk, kk > 0);
                         else
-                            mma_f16_ss(d_tmem, dq + off, dk + off, idesc_qk, kk > 0);
+                            mma_f16_ss(d_tmem, desc(aq + off), desc(bk + off), idesc_qk, kk > 0);
                     }
                 }
                 __syncwarp();
@@ -514,16 +527,16 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             auto issue_pv = [&](int s, int slot, bool acc) {
                 const uint32_t d_tmem = tmem + (s ? C::kColO1 : C::kColO0);
                 const uint32_t a_tmem = tmem + (s ? C::kColS1 : C::kColS0);
-                const uint64_t dv = desc_v + (uint64_t)((slot * C::kTileBytes) >> 4);
+                const uint32_t bv = dv_lo + (uint32_t)((slot * C::kTileBytes) >> 4);
                 if (leader) {
-#pragma unroll 1
+#pragma unroll
                     for (int kk = 0; kk < C::kPvSteps; ++kk) {
-                        const uint64_t off = (uint64_t)((kk * C::kPvKeysPerStep * C::kSwBytes) >> 4);
+                        const uint32_t off = (uint32_t)((kk * C::kPvKeysPerStep * C::kSwBytes) >> 4);
                         const uint32_t accum = (acc || kk > 0) ? 1u : 0u;
                         if constexpr (KIND == K2_E4M3)
-                            mma_f8_ts(d_tmem, a_tmem + kk * 8, dv + off, idesc_pv, accum);
+                            mma_f8_ts(d_tmem, a_tmem + kk * 8, desc(bv + off), idesc_pv, accum);
                         else
-                            mma_f16_ts(d_tmem, a_tmem + kk * 8, dv + off, idesc_pv, accum);
+                            mma_f16_ts(d_tmem, a_tmem + kk * 8, desc(bv + off), idesc_pv, accum);
                     }
                 }
                 __syncwarp();
@@ -581,7 +594,7 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             while (ok && vc.u.valid) {
                 const int slotV = t % NS;
                 ok = wait_all(bar(C::kBarKVFull + slotV), (uint32_t)(t / NS) & 1u,
-                              0x22000u | (uint32_t)(vc.g & 0xfff));
+                              0x22000u | (uint32_t)(t & 0xfff));
                 if (!ok) break;
                 const int slotK = (t + 1) % NS;
                 bool k_ready = false;
@@ -590,7 +603,7 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                     if (ok && kc.u.valid && kc.j < stage_tiles(kc.u, s)) {
                         if (!k_ready) {
                             ok = wait_all(bar(C::kBarKVFull + slotK), (uint32_t)((t + 1) / NS) & 1u,
-                                          0x21000u | (uint32_t)(kc.g & 0xfff));
+                                          0x21000u | (uint32_t)((t + 1) & 0xfff));
                             k_ready = true;
                         }
                         if (ok) ok = qk_stage(kc, s, slotK);
@@ -646,7 +659,7 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 float x0, x1;
                 f2_unpack(x2, x0, x1);
                 uint64_t p2;
-                if (poly_pair(e))
+                if (poly_pair<KIND>(e))
                     p2 = exp2_poly_x2(f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f)));
                 else
                     p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
