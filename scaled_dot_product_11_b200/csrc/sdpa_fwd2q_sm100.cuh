@@ -24,7 +24,10 @@
 //                stage, off the softmax groups' path
 //   warp 12      TMA producer: Q tiles per unit, K/V tiles in stream order
 //                K_0 V_0 K_1 V_1 ... (the ring spans unit boundaries)
-//   warp 13      MMA issuer (one elected lane) and TMEM owner
+//   warp 13      MMA issuer (one elected lane) and TMEM owner; a single
+//                in-order issuer keeps each stage's PV + QK block contiguous
+//                in the tensor pipe (two issuers, one per stage, interleave
+//                the blocks and lengthen both stages' chains)
 //   warps 14-15  idle (they complete the fourth warp group's register split)
 // Tensor memory (128 lanes x 512 columns, fp32):
 //   [0,128) S_0   [128,256) S_1   [256,256+d) O_0   [256+d,256+2d) O_1
@@ -127,10 +130,16 @@ struct Cfg {
     static constexpr int kPvSteps = kKeys / kPvKeysPerStep;
     static constexpr int kPWordsPer32 = 32 * kElem / 4;    // TMEM columns of P per 32 keys
     // lazy rescale: the running max only moves when a tile's max exceeds it
-    // by more than this (log2 units); FP8 moves it on every rise so that the
-    // e4m3 weights never exceed 448
-    static constexpr float kRescaleThreshold = (KIND == K2_E4M3) ? 0.0f : 8.0f;
-    static constexpr float kPLog2 = (KIND == K2_E4M3) ? 8.807354922057604f : 0.0f;   // log2(448)
+    // by more than this (log2 units), so a weight 2^(s - m_run) can reach
+    // 2^threshold
+    static constexpr float kRescaleThreshold = (KIND == K2_E4M3) ? 4.0f : 8.0f;
+    // log2 of the factor applied to the weights before they are rounded for
+    // the PV product: for e4m3, 448 * 2^-threshold, so that the largest
+    // weight (2^threshold) maps to the format's largest value, 448
+    static constexpr float kPLog2 = (KIND == K2_E4M3) ? 8.807354922057604f - 4.0f : 0.0f;
+    // weights before the tile max (16-bit P); e4m3 takes the max first, whose
+    // register footprint leaves room for its packing and polynomial
+    static constexpr bool kWeightsFirst = KIND != K2_E4M3;
     // shared memory (offsets from a 1024-byte aligned base)
     static constexpr int kSmemQ = 0;                                 // [2 stages][QB] tiles
     static constexpr int kSmemKV = 2 * QB * kTileBytes;              // [NS] tiles
@@ -491,7 +500,6 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             const uint32_t dq_lo = (uint32_t)dq0, dk_lo = (uint32_t)dk0, dv_lo = (uint32_t)dv0;
             auto desc = [&](uint32_t lo) -> uint64_t { return ((uint64_t)desc_hi << 32) | lo; };
             bool ok = true;
-            int cq[2] = {0, 0};    // S_s tiles issued (S_full phase)
             int cp[2] = {0, 0};    // P_s tiles consumed (P_full phase)
             int kqk[2] = {0, 0};   // units started, QK side (Q_full phase)
             int kpv[2] = {0, 0};   // units started, PV side (O_empty phase)
@@ -554,7 +562,6 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                     commit(bar(C::kBarQEmpty + 2 * s + qb));   // Q_s buffer free
                     ++kqk[s];
                 }
-                ++cq[s];
                 return true;
             };
             // O_s (+)= P_s V for stream tile vc (V landed in slotV)
@@ -650,11 +657,17 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
 
         // weights of 32 scores against nm2 = (-m + log2 of the P scale) x 2,
         // rounded for the PV product into chunk c of P; returns the fp32 sum
-        auto exp_chunk = [&](const float* sc, uint64_t nm2, int c) -> uint64_t {
+        // and, in cmax, the largest of the 32 raw scores
+        auto exp_chunk = [&](const float* sc, uint64_t nm2, int c, float& cmax) -> uint64_t {
             uint64_t sum2[2] = {0ull, 0ull};
             uint32_t pk[16];
+            float mx0 = sc[0], mx1 = sc[1];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
+                if (e > 0) {
+                    if (e & 1) mx1 = fmax3(mx1, sc[2 * e], sc[2 * e + 1]);
+                    else mx0 = fmax3(mx0, sc[2 * e], sc[2 * e + 1]);
+                }
                 const uint64_t x2 = f2_fma(f2_pack(sc[2 * e], sc[2 * e + 1]), sl2, nm2);
                 float x0, x1;
                 f2_unpack(x2, x0, x1);
@@ -673,6 +686,7 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                     pk[e] = (KIND == K2_BF16) ? pack_bf16x2(q0, q1) : pack_f16x2(q0, q1);
                 }
             }
+            cmax = fmaxf(mx0, mx1);
             if constexpr (KIND == K2_E4M3)
                 tmem_st8(tS + C::kPWordsPer32 * c, pk);
             else
@@ -718,39 +732,77 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                     for (int c = 0; c < kKeys; ++c)
                         if (c >= lim) sc[c] = -INFINITY;
                 }
-                const float tmax = max128(sc) * sl;
-                // lazy rescale: the reference max moves only when this tile's
-                // max exceeds it by more than the threshold; O_s and l share
-                // the reference max at all times
-                const bool need = tmax > m_run + C::kRescaleThreshold;
-                if (__any_sync(0xffffffffu, need)) {
-                    float alpha = 1.0f;
-                    if (need) {
-                        alpha = ex2_approx(m_run - tmax);   // 0 on the first live tile
-                        m_run = tmax;
-                    }
-                    l_run *= alpha;
-                    // O_s += P_s V of the previous tile has completed (it was
-                    // issued before the Q K^T that produced this S)
-                    if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+                // Lazy rescale: the reference max m_run moves only when a
+                // tile's max exceeds it by more than the threshold; O_s and l
+                // share the reference max at all times.  With kWeightsFirst,
+                // past the unit's first tile the weights are computed against
+                // m_run at once and the tile's max is found alongside them,
+                // off the MUFU; in the rare case that it exceeds m_run by more
+                // than the threshold, m_run moves, l and O_s are rescaled and
+                // the weights are computed again (the PV product has not been
+                // released yet).  Otherwise the max comes first.
+                // all weights against m_run; tmax receives the tile's max
+                // raw score
+                auto all_weights = [&](float& tmax) -> uint64_t {
+                    const float nm = C::kPLog2 - m_run;
+                    const uint64_t nm2 = f2_pack(nm, nm);
+                    float c0, c1, c2, c3;
+                    uint64_t a = exp_chunk(&sc[0], nm2, 0, c0);
+                    a = f2_add(a, exp_chunk(&sc[32], nm2, 1, c1));
+                    a = f2_add(a, exp_chunk(&sc[64], nm2, 2, c2));
+                    a = f2_add(a, exp_chunk(&sc[96], nm2, 3, c3));
+                    tmax = fmaxf(fmaxf(c0, c1), fmaxf(c2, c3));
+                    return a;
+                };
+                uint64_t acc;
+                float traw;
+                // O_s *= alpha row by row; O_s += P_s V of the previous tile
+                // has completed (it was issued before the Q K^T that produced
+                // this S)
+                auto rescale_o = [&](float alpha) {
 #pragma unroll 1
-                        for (int c = 0; c < D / 32; ++c) {
-                            float o[32];
-                            tmem_ld32(tO + 32 * c, o);
-                            tmem_wait_ld();
-                            reg_fence32(o);
+                    for (int c = 0; c < D / 32; ++c) {
+                        float o[32];
+                        tmem_ld32(tO + 32 * c, o);
+                        tmem_wait_ld();
+                        reg_fence32(o);
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) o[e] *= alpha;
-                            tmem_st32(tO + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(o));
+                        for (int e = 0; e < 32; ++e) o[e] *= alpha;
+                        tmem_st32(tO + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(o));
+                    }
+                };
+                if (j == 0) {
+                    // every row of the unit's first tile has a visible key
+                    m_run = max128(sc) * sl;
+                    acc = all_weights(traw);
+                } else if constexpr (!C::kWeightsFirst) {
+                    const float tmax = max128(sc) * sl;
+                    const bool need = tmax > m_run + C::kRescaleThreshold;
+                    if (__any_sync(0xffffffffu, need)) {
+                        float alpha = 1.0f;
+                        if (need) {
+                            alpha = ex2_approx(m_run - tmax);
+                            m_run = tmax;
                         }
+                        l_run *= alpha;
+                        rescale_o(alpha);
+                    }
+                    acc = all_weights(traw);
+                } else {
+                    acc = all_weights(traw);
+                    const float tmax = traw * sl;
+                    const bool need = tmax > m_run + C::kRescaleThreshold;
+                    if (__any_sync(0xffffffffu, need)) {
+                        float alpha = 1.0f;
+                        if (need) {
+                            alpha = ex2_approx(m_run - tmax);
+                            m_run = tmax;
+                        }
+                        l_run *= alpha;
+                        rescale_o(alpha);
+                        acc = all_weights(traw);   // P_s overwritten in place
                     }
                 }
-                const float nm = (m_run == -INFINITY) ? 0.0f : C::kPLog2 - m_run;
-                const uint64_t nm2 = f2_pack(nm, nm);
-                uint64_t acc = exp_chunk(&sc[0], nm2, 0);
-                acc = f2_add(acc, exp_chunk(&sc[32], nm2, 1));
-                acc = f2_add(acc, exp_chunk(&sc[64], nm2, 2));
-                acc = f2_add(acc, exp_chunk(&sc[96], nm2, 3));
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(bar(C::kBarPFull + s));
@@ -807,27 +859,26 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 const uint32_t tO = tmem + lane_base + (s ? C::kColO1 : C::kColO0);
                 uint16_t* obase = reinterpret_cast<uint16_t*>(p.o) + o_offset<D, STRIDED>(p, u.bh, live ? row : 0);
 #pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    float x[32];
-                    tmem_ld32(tO + 32 * c, x);
+                for (int c = 0; c < D / 16; ++c) {
+                    float x[16];
+                    tmem_ld16(tO + 16 * c, x);
                     tmem_wait_ld();
-                    reg_fence32(x);
-                    if (c == D / 32 - 1) {
+                    reg_fence16(x);
+                    if (c == D / 16 - 1) {
                         // O_s is read: the next unit's first product may overwrite it
                         tc_fence_before();
                         mbar_arrive(bar(C::kBarOEmpty + s));
                     }
-                    uint32_t w[16];
+                    uint32_t w[8];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
+                    for (int e = 0; e < 8; ++e) {
                         const float v0 = x[2 * e] * cmul, v1 = x[2 * e + 1] * cmul;
                         w[e] = (KIND == K2_FP16) ? pack_f16x2(v0, v1) : pack_bf16x2(v0, v1);
                     }
                     if (live) {
-                        uint4* dst = reinterpret_cast<uint4*>(obase + 32 * c);
-#pragma unroll
-                        for (int v4 = 0; v4 < 4; ++v4)
-                            dst[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+                        uint4* dst = reinterpret_cast<uint4*>(obase + 16 * c);
+                        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
                     }
                 }
                 ++ks[s];
