@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd"],
                     help="bwd: time sdpa_bwd (dQ, dK, dV) on the workload, one GPU")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-config measurements added to the JSON line (1 GPU only)")
     ap.add_argument("--ref-budget-s", type=float, default=90.0,
                     help="host seconds the reference (oracle) arm spends over all its steps")
     return ap.parse_args()
@@ -278,6 +280,98 @@ def run_backward(args, w):
         "clocks": clk, "gpu_launches": 2 * args.steps}))
 
 
+def roofline_of(w, ms, peaks, src, fwd=True):
+    """Roofline of one launch of workload w taking `ms`: the tensor peak of
+    the inputs' dtype (e4m3: the measured bf16 figure x 2, the nominal ratio)
+    when the algorithmic arithmetic intensity is above the ridge, HBM
+    otherwise; the backward's five contractions are 2.5x the forward's."""
+    fp8 = w.dtype == "e4m3"
+    flops = w.flops * (1.0 if fwd else 2.5)
+    peak = float(peaks["bf16_tflops"]) * (2.0 if fp8 else 1.0)
+    ridge = peak * 1e12 / (float(peaks["hbm_gbs"]) * 1e9)
+    ai = flops / w.min_hbm_bytes
+    if ai < ridge:
+        achieved = w.min_hbm_bytes / (ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": achieved, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                "frac": achieved / float(peaks["hbm_gbs"]), "arithmetic_intensity": ai,
+                "peak_source": "%s hbm_gbs (copy)" % src}
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "arithmetic_intensity": ai,
+            "peak_source": "%s bf16_tflops (burst)%s" % (src, " x 2 (nominal fp8/bf16)" if fp8 else "")}
+
+
+def config_sweep(dev, launches=20, warmup=3):
+    """Every BASELINE-shaped workload besides the headline, one GPU: device
+    time over `launches` launches after `warmup`, TFLOP/s, roofline fraction,
+    and the largest |O - O_ref| over sampled rows against the oracle; then the
+    backward on the causal LM shape (timing only)."""
+    import numpy as np
+    import torch
+    import oracle
+    import scaled_dot_product_11_b200 as sdpa
+    from sdpa_workloads import WORKLOADS, make_qkv, make_qkv_fp8, sample_rows, sweep
+    peaks, src = load_peaks()
+    names = ["tiny", "vit", "gqa", "mqa", "fp8"]
+    todo = [WORKLOADS[n] for n in names] + [sweep(False)[5], sweep(True)[0]]
+    stream = torch.cuda.current_stream(dev)
+    out = []
+    for w in todo:
+        fp8 = w.dtype == "e4m3"
+        if fp8:
+            q, k, v, ds, _ = make_qkv_fp8(w, dev)
+            run = lambda: sdpa.attention_fp8(q, k, v, ds, causal=w.causal, scale=w.scale, out=o, lse=lse)
+            o = torch.empty((w.B, w.Hq, w.Sq, w.d), dtype=torch.bfloat16, device=dev)
+        else:
+            q, k, v = make_qkv(w, dev)
+            ds = (1.0, 1.0, 1.0)
+            run = lambda: sdpa.attention(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse)
+            o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device=dev)
+        for _ in range(warmup):
+            run()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(launches):
+            run()
+        e1.record(stream)
+        e1.synchronize()
+        ms = e0.elapsed_time(e1) / launches
+        st, detail = sdpa.sdpa_device_status(clear=True)
+        rows = sample_rows(w, n_random=32)
+        rows = rows[:: max(1, len(rows) // 64)]
+        ro, _ = oracle.sdpa_rows(*(t.contiguous().cpu() for t in (q, k, v)), rows, w.scale, w.causal,
+                                 descales=ds)
+        go = o.reshape(-1, w.d).index_select(0, torch.tensor(rows, device=dev)).double().cpu().numpy()
+        out.append({"workload": w.name, "ms": ms, "tflops": w.flops / (ms * 1e-3) / 1e12,
+                    "launches": launches, "roofline": roofline_of(w, ms, peaks, src),
+                    "parity": {"rows": len(rows), "max_abs_o": float(np.abs(go - ro).max())},
+                    "device_status": st})
+        del q, k, v, o, lse
+    # backward on the causal LM shape
+    w = WORKLOADS["lm_causal"]
+    q, k, v = make_qkv(w, dev)
+    g = torch.Generator(device="cpu").manual_seed(w.seed + 1)
+    dout = torch.randn(q.shape, generator=g).to(q.dtype).to(dev)
+    o, lse = sdpa.attention(q, k, v, causal=w.causal, scale=w.scale)
+    run = lambda: sdpa.attention_backward(q, k, v, o, lse, dout, causal=w.causal, scale=w.scale)
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(launches):
+        run()
+    e1.record(stream)
+    e1.synchronize()
+    ms = e0.elapsed_time(e1) / launches
+    st, _ = sdpa.sdpa_device_status(clear=True)
+    out.append({"workload": w.name, "pass": "bwd", "ms": ms, "tflops": 2.5 * w.flops / (ms * 1e-3) / 1e12,
+                "launches": launches, "roofline": roofline_of(w, ms, peaks, src, fwd=False),
+                "device_status": st})
+    return out
+
+
 def main():
     args = parse()
     from sdpa_workloads import WORKLOADS, make_inputs, make_qkv_fp8, sample_rows, with_shape
@@ -446,6 +540,8 @@ def main():
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+        if world == 1 and not args.no_configs:
+            line["configs"] = config_sweep(dev)
         print(json.dumps(line), flush=True)
 
     if world > 1:

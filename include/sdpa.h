@@ -152,9 +152,13 @@ SDPA_API int sdpa_fwd_strided(const void* q, const void* k, const void* v, void*
  *   o                bf16 [B,Hq,Sq,d]
  *   lse              float32 [B,Hq,Sq] or NULL
  *
- * The softmax weights p in [0, 1] are themselves quantised to e4m3 as
- * e4m3(448 * p) (the amax rule with amax(p) = 1) for the P*V product, whose
- * result is multiplied back by descale_v / 448; row sums use fp32 p.
+ * The softmax weights are themselves quantised to e4m3 for the P*V product,
+ * by the amax rule: against a reference max m_ref that is moved only when a
+ * tile's scores exceed it by more than 4 (log2 units), a weight is
+ * 2^(s - m_ref) <= 2^4 and is stored as e4m3(448 * 2^-4 * 2^(s - m_ref)), so
+ * that the largest possible weight maps to 448; the product is multiplied
+ * back by descale_v and divided by the fp32 row sum of the same scaled
+ * weights.
  * Errors as sdpa_fwd; d must be 128 (SDPA_ERR_UNSUPPORTED otherwise).
  */
 SDPA_API int sdpa_fwd_fp8(const void* q8, const void* k8, const void* v8,
@@ -207,8 +211,14 @@ SDPA_API int sdpa_bwd(const void* q, const void* k, const void* v, const void* o
  * when B*Hq*Sq is above SDPA_BWD_NOALLOC_MAX_ROWS.  The call allocates
  * nothing.
  *
- * The first call on a device looks the array's device address up with that
- * device current; make that first call before any stream capture begins.
+ * The array belongs to the library's device code, which the CUDA runtime
+ * loads into a device's context on the first call of any library entry point
+ * on that device (lazy module loading, the default since CUDA 12): that load
+ * places the array in device memory and may synchronise the device.  Make one
+ * call on each device before entering a region that must not allocate or
+ * synchronise (a stream capture included).  Every call looks the array's
+ * address up in the current context, so a context recreated in between
+ * (cudaDeviceReset) is followed correctly.
  * All calls on a device share the one array, which keeps the D values of the
  * last call: nothing in it has to start at zero, since every call writes each
  * row's D before reading it.  Calls whose kernels overlap on the GPU (on
@@ -239,6 +249,38 @@ SDPA_API int sdpa_device_status(int* status, int* detail, int clear);
 /* Number of kernel launches sdpa_fwd / sdpa_fwd_strided / sdpa_fwd_fp8 issue
  * per call (1); sdpa_bwd and sdpa_bwd_noalloc issue 2. */
 SDPA_API int sdpa_launches_per_call(void);
+
+/*
+ * Self-tests of the kernels' device-side machinery.  They are not part of the
+ * attention path; the library's test suite calls them to check, on the GPU,
+ * behaviour that the attention kernels only show when something goes wrong
+ * or that sits deep inside them.
+ *
+ * sdpa_selftest_wait -- runs the attention kernels' bounded-wait path (the
+ * forward kernel's) on an mbarrier that nothing ever completes: one CTA, two
+ * warps.  Warp 0 waits with a limit of limit_us microseconds, gives up,
+ * raises the CTA's abort flag and records SDPA_ERR_DEVICE_TIMEOUT with
+ * location code 0x7e000 in the device status word (read it with
+ * sdpa_device_status); warp 1 waits on the same barrier with the kernels'
+ * full one-second limit and must give up as soon as it sees the abort flag.
+ * No trap, no fault: the kernel returns and the context stays usable.
+ *   limit_us  1 .. 1000000
+ *   out       device memory, 4 x uint32, 4-byte aligned: warp 0's wait result
+ *             (0 = gave up), the abort flag after it (1), warp 1's wait result
+ *             (0), the abort flag warp 1 saw (1)
+ * Returns SDPA_OK after the launch, SDPA_ERR_INVALID_ARG for a null or
+ * misaligned out or a limit outside the range, SDPA_ERR_UNSUPPORTED off
+ * sm_100, SDPA_ERR_CUDA for a launch error.
+ *
+ * sdpa_selftest_exp2 -- evaluates 2^x for n floats x (device memory, x in
+ * [-126, 64]) both with the FMA-pipe polynomial the softmax can use for part
+ * of its exponentials (range reduction to [-1/2, 1/2] by rounding, a cubic
+ * fitted to the relative error of 2^f, the exponent added to the result's
+ * bits) and with the MUFU instruction ex2.approx; results to poly and mufu
+ * (device memory, n floats each).  Errors as sdpa_selftest_wait.
+ */
+SDPA_API int sdpa_selftest_wait(unsigned int limit_us, unsigned int* out, void* stream);
+SDPA_API int sdpa_selftest_exp2(const float* x, float* poly, float* mufu, int n, void* stream);
 
 #ifdef __cplusplus
 }

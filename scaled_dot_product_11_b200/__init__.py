@@ -20,7 +20,8 @@ __all__ = [
     "SDPA_BWD_NOALLOC_MAX_ROWS", "sdpa_bwd_noalloc", "SdpaError", "LIB_PATH",
     "SDPA_NO_MASK", "SDPA_CAUSAL", "SDPA_CAUSAL_BOTTOM_RIGHT",
     "sdpa_fwd", "sdpa_fwd_strided", "sdpa_fwd_fp8", "sdpa_bwd", "attention_backward", "sdpa_strerror", "sdpa_device_status",
-    "sdpa_launches_per_call", "attention", "attention_fp8",
+    "sdpa_launches_per_call", "attention", "attention_fp8", "sdpa_selftest_wait",
+    "sdpa_selftest_exp2",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -69,6 +70,10 @@ _lib.sdpa_device_status.argtypes = [ctypes.POINTER(_i), ctypes.POINTER(_i), _i]
 _lib.sdpa_device_status.restype = _i
 _lib.sdpa_launches_per_call.argtypes = []
 _lib.sdpa_launches_per_call.restype = _i
+_lib.sdpa_selftest_wait.argtypes = [ctypes.c_uint, _vp, _vp]
+_lib.sdpa_selftest_wait.restype = _i
+_lib.sdpa_selftest_exp2.argtypes = [_vp, _vp, _vp, _i, _vp]
+_lib.sdpa_selftest_exp2.restype = _i
 
 
 # ---- the C entry points, same names, raw arguments ------------------------
@@ -129,6 +134,18 @@ def sdpa_device_status(clear: bool = True):
 
 def sdpa_launches_per_call() -> int:
     return int(_lib.sdpa_launches_per_call())
+
+
+def sdpa_selftest_wait(limit_us, out, stream) -> int:
+    """Raw call: the kernels' bounded wait on a barrier nothing completes;
+    out is the device address of 4 uint32 (see include/sdpa.h)."""
+    return int(_lib.sdpa_selftest_wait(int(limit_us), out, stream or None))
+
+
+def sdpa_selftest_exp2(x, poly, mufu, n, stream) -> int:
+    """Raw call: 2^x for n device floats by the FMA-pipe polynomial and by
+    ex2.approx (device addresses as ints)."""
+    return int(_lib.sdpa_selftest_exp2(x, poly, mufu, int(n), stream or None))
 
 
 # ---- torch conveniences -------------------------------------------------------

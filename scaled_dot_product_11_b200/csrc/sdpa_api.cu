@@ -439,6 +439,21 @@ extern "C" int sdpa_device_status(int* status, int* detail, int clear) {
 
 extern "C" int sdpa_launches_per_call(void) { return 1; }
 
+extern "C" int sdpa_selftest_wait(unsigned int limit_us, unsigned int* out, void* stream) {
+    if (!out || limit_us == 0 || limit_us > 1000000u || (reinterpret_cast<uintptr_t>(out) & 3u))
+        return SDPA_ERR_INVALID_ARG;
+    const int rc = check_device();
+    if (rc != SDPA_OK) return rc;
+    return sdpa_host::selftest_wait(limit_us, out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int sdpa_selftest_exp2(const float* x, float* poly, float* mufu, int n, void* stream) {
+    if (!x || !poly || !mufu || n <= 0) return SDPA_ERR_INVALID_ARG;
+    const int rc = check_device();
+    if (rc != SDPA_OK) return rc;
+    return sdpa_host::selftest_exp2(x, poly, mufu, n, reinterpret_cast<cudaStream_t>(stream));
+}
+
 // ---------------------------------------------------------------------------
 // sdpa_bwd_noalloc: the backward for callers that cannot allocate device
 // memory (a host framework that owns every allocation, or a path on which

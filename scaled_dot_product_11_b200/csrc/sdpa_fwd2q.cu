@@ -75,8 +75,13 @@ int launch_fwd2q(const Fwd2Request& r, cudaStream_t stream) {
     const long long n_items = (long long)r.B * r.Hq * prm.items_per_head;
     if (n_items > INT32_MAX) return SDPA_ERR_INVALID_ARG;
     prm.n_items = (int)n_items;
-    // about two waves of items per group of (batch, head) pairs
-    int gh = (2 * sm_count() + prm.items_per_head - 1) / prm.items_per_head;
+    // about one wave of items per group of (batch, head) pairs, so that the
+    // K/V of the heads in flight (2 MB per head at S = 4096, d = 128) stay
+    // well inside the L2
+#ifndef SDPA2_GROUP_WAVES
+#define SDPA2_GROUP_WAVES 1
+#endif
+    int gh = (SDPA2_GROUP_WAVES * sm_count() + prm.items_per_head - 1) / prm.items_per_head;
     if (gh < 1) gh = 1;
     if (gh > r.B * r.Hq) gh = r.B * r.Hq;
     prm.group_heads = gh;
@@ -101,6 +106,17 @@ int launch_fwd2q(const Fwd2Request& r, cudaStream_t stream) {
     default:
         return SDPA_ERR_UNSUPPORTED;
     }
+}
+
+int selftest_wait(unsigned int limit_us, unsigned int* out, cudaStream_t stream) {
+    sdpa::fwd2::selftest_wait_kernel<<<1, 64, 0, stream>>>((uint64_t)limit_us * 1000ull, out);
+    return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
+int selftest_exp2(const float* x, float* poly, float* mufu, int n, cudaStream_t stream) {
+    const int pairs = (n + 1) / 2;
+    sdpa::fwd2::selftest_exp2_kernel<<<(pairs + 255) / 256, 256, 0, stream>>>(x, poly, mufu, n);
+    return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
 }
 
 int fwd2q_status(unsigned int out[2], int clear) {

@@ -185,14 +185,15 @@ __device__ __forceinline__ void sts_u32(uint32_t addr, uint32_t v) {
 }
 
 __device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, uint32_t abort_addr,
-                                       unsigned int* status, uint32_t where, uint32_t sleep_ns) {
+                                          unsigned int* status, uint32_t where, uint32_t sleep_ns,
+                                          uint64_t limit_ns = kWaitLimitNs) {
     const uint64_t t0 = global_timer_ns();
     for (uint32_t k = 1;; ++k) {
         if (sleep_ns) __nanosleep(sleep_ns);
         if (mbar_try_wait(bar, parity)) return true;
         if ((k & 15u) == 0) {
             if (lds_u32(abort_addr) != 0u) return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs) {
+            if (global_timer_ns() - t0 > limit_ns) {
                 sts_u32(abort_addr, 1u);
                 if (atomicCAS(&status[0], 0u, 4u) == 0u) atomicExch(&status[1], where);
                 return false;
@@ -857,7 +858,18 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t tO = tmem + lane_base + (s ? C::kColO1 : C::kColO0);
-                uint16_t* obase = reinterpret_cast<uint16_t*>(p.o) + o_offset<D, STRIDED>(p, u.bh, live ? row : 0);
+                // Stores in whole 32-byte sectors: lanes 2i and 2i+1 swap
+                // halves of each 16-column chunk, so that one store
+                // instruction writes 16 bytes of each of the pair's rows
+                // next to each other (16 full sectors per instruction).
+                const bool odd = (lane & 1) != 0;
+                const int prow = (2 * u.m + s) * kRows + (r ^ 1);   // the partner's row
+                const bool plive = prow < p.Sq;
+                uint16_t* const rowA = reinterpret_cast<uint16_t*>(p.o) +
+                                       o_offset<D, STRIDED>(p, u.bh, odd ? (plive ? prow : 0) : (live ? row : 0));
+                uint16_t* const rowB = reinterpret_cast<uint16_t*>(p.o) +
+                                       o_offset<D, STRIDED>(p, u.bh, odd ? (live ? row : 0) : (plive ? prow : 0));
+                const bool liveA = odd ? plive : live, liveB = odd ? live : plive;
 #pragma unroll 1
                 for (int c = 0; c < D / 16; ++c) {
                     float x[16];
@@ -875,11 +887,18 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const float v0 = x[2 * e] * cmul, v1 = x[2 * e + 1] * cmul;
                         w[e] = (KIND == K2_FP16) ? pack_f16x2(v0, v1) : pack_bf16x2(v0, v1);
                     }
-                    if (live) {
-                        uint4* dst = reinterpret_cast<uint4*>(obase + 16 * c);
-                        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-                    }
+                    // even lanes keep columns 0-7 of the chunk and receive the
+                    // partner's; odd lanes keep columns 8-15 and receive the
+                    // partner's
+                    uint32_t y[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) y[e] = __shfl_xor_sync(0xffffffffu, odd ? w[e] : w[4 + e], 1);
+                    // first store: the even row of the pair; second: the odd row
+                    const uint4 first = odd ? make_uint4(y[0], y[1], y[2], y[3]) : make_uint4(w[0], w[1], w[2], w[3]);
+                    const uint4 second = odd ? make_uint4(w[4], w[5], w[6], w[7]) : make_uint4(y[0], y[1], y[2], y[3]);
+                    const int colA = 16 * c + (odd ? 8 : 0);
+                    if (liveA) *reinterpret_cast<uint4*>(rowA + colA) = first;
+                    if (liveB) *reinterpret_cast<uint4*>(rowB + colA) = second;
                 }
                 ++ks[s];
             }
@@ -887,6 +906,56 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
         tc_fence_before();
         named_bar_sync(1, C::kTmemUsers);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// self-test kernels (not part of the attention path)
+// ---------------------------------------------------------------------------
+// The kernels' bounded-wait path on a barrier that nothing completes: warp 0
+// waits with a limit of limit_ns, gives up, raises the CTA's abort flag and
+// records SDPA_ERR_DEVICE_TIMEOUT with location kSelftestWhere in the status
+// word; warp 1 waits on the same barrier with the full limit and must give up
+// as soon as it sees the abort flag.  out[0..3]: warp 0's wait result, the
+// abort flag after it, warp 1's wait result, the abort flag warp 1 saw.
+constexpr uint32_t kSelftestWhere = 0x7e000u;
+__global__ void __launch_bounds__(64, 1) selftest_wait_kernel(uint64_t limit_ns, unsigned int* out) {
+    __shared__ __align__(8) uint64_t bar_word;
+    __shared__ uint32_t abort_word;
+    const uint32_t bar = smem_u32(&bar_word), abort_addr = smem_u32(&abort_word);
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        sts_u32(abort_addr, 0u);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5;
+    bool ok;
+    if (warp == 0)
+        ok = wait_slow(bar, 0u, abort_addr, g_status, kSelftestWhere, 0u, limit_ns);
+    else
+        ok = wait_slow(bar, 0u, abort_addr, g_status, kSelftestWhere + 1u, 0u, kWaitLimitNs);
+    ok = __all_sync(0xffffffffu, ok);
+    if ((threadIdx.x & 31) == 0) {
+        out[2 * warp] = ok ? 1u : 0u;
+        out[2 * warp + 1] = lds_u32(abort_addr);
+    }
+}
+
+// 2^x by the FMA-pipe polynomial (exp2_poly_x2) and by ex2.approx, for n
+// inputs (pairs of consecutive elements through the packed form; an odd last
+// element is paired with itself).
+__global__ void selftest_exp2_kernel(const float* x, float* poly, float* mufu, int n) {
+    const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    const float a = x[i], b = (i + 1 < n) ? x[i + 1] : a;
+    float p0, p1;
+    f2_unpack(exp2_poly_x2(f2_pack(a, b)), p0, p1);
+    poly[i] = p0;
+    mufu[i] = ex2_approx(a);
+    if (i + 1 < n) {
+        poly[i + 1] = p1;
+        mufu[i + 1] = ex2_approx(b);
     }
 }
 

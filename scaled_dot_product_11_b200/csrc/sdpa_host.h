@@ -93,5 +93,8 @@ struct Fwd2Request {
 int launch_fwd2q(const Fwd2Request& r, cudaStream_t stream);
 // Read (and with clear, reset) that kernel's device status word; synchronous.
 int fwd2q_status(unsigned int out[2], int clear);
+// Self-tests of that translation unit's device helpers (sdpa_selftest_*).
+int selftest_wait(unsigned int limit_us, unsigned int* out, cudaStream_t stream);
+int selftest_exp2(const float* x, float* poly, float* mufu, int n, cudaStream_t stream);
 
 }  // namespace sdpa_host
