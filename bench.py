@@ -344,8 +344,10 @@ def config_sweep(dev, launches=20, warmup=3):
         ro, _ = oracle.sdpa_rows(*(t.contiguous().cpu() for t in (q, k, v)), rows, w.scale, w.causal,
                                  descales=ds)
         go = o.reshape(-1, w.d).index_select(0, torch.tensor(rows, device=dev)).double().cpu().numpy()
+        roof = roofline_of(w, ms, peaks, src)
+        roof["traffic"] = load_traffic(w.name)
         out.append({"workload": w.name, "ms": ms, "tflops": w.flops / (ms * 1e-3) / 1e12,
-                    "launches": launches, "roofline": roofline_of(w, ms, peaks, src),
+                    "launches": launches, "roofline": roof,
                     "parity": {"rows": len(rows), "max_abs_o": float(np.abs(go - ro).max())},
                     "device_status": st})
         del q, k, v, o, lse

@@ -681,8 +681,9 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 float q0, q1;
                 f2_unpack(p2, q0, q1);
                 if constexpr (KIND == K2_E4M3) {
-                    if (e & 1) pk[e >> 1] |= pack_e4m3x4(0.f, 0.f, q0, q1) & 0xFFFF0000u;
-                    else pk[e >> 1] = pack_e4m3x4(q0, q1, 0.f, 0.f) & 0x0000FFFFu;
+                    // one conversion per pair; pairs 2i and 2i+1 share a word
+                    if (e & 1) pk[e >> 1] |= pack_e4m3x2(q0, q1) << 16;
+                    else pk[e >> 1] = pack_e4m3x2(q0, q1);
                 } else {
                     pk[e] = (KIND == K2_BF16) ? pack_bf16x2(q0, q1) : pack_f16x2(q0, q1);
                 }
