@@ -73,6 +73,10 @@
 #endif
 static_assert(8 * SDPA2_REGS_SOFTMAX + 4 * SDPA2_REGS_EPILOGUE + 4 * SDPA2_REGS_OTHER <= 16 * 128,
               "register split exceeds the launch allocation");
+// 1: 16-bit inputs compute the weights before the tile max (see the softmax)
+#ifndef SDPA2_WEIGHTS_FIRST
+#define SDPA2_WEIGHTS_FIRST 1
+#endif
 #ifndef SDPA2_EPI_SLEEP_NS
 #define SDPA2_EPI_SLEEP_NS 128
 #endif
@@ -139,7 +143,7 @@ struct Cfg {
     static constexpr float kPLog2 = (KIND == K2_E4M3) ? 8.807354922057604f - 4.0f : 0.0f;
     // weights before the tile max (16-bit P); e4m3 takes the max first, whose
     // register footprint leaves room for its packing and polynomial
-    static constexpr bool kWeightsFirst = KIND != K2_E4M3;
+    static constexpr bool kWeightsFirst = SDPA2_WEIGHTS_FIRST && KIND != K2_E4M3;
     // shared memory (offsets from a 1024-byte aligned base)
     static constexpr int kSmemQ = 0;                                 // [2 stages][QB] tiles
     static constexpr int kSmemKV = 2 * QB * kTileBytes;              // [NS] tiles
