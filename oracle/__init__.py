@@ -25,8 +25,12 @@ Parity status of each function (what pins it, in ``tests/test_oracle.py``):
   sdpa_rows        pinned: equals sdpa_fwd on the same rows (same per-row code
                    reached through a different index path) and the pins above.
   sdpa_bruteforce  pinned: mpmath evaluation, weights-sum, V = identity.
-  decode_*         pinned: all 256 e4m3 codes and all 65536 fp16 / bf16 codes
-                   against torch's own casts.
+  sdpa_bwd_fp8     pinned: equals sdpa_bwd on the decoded values (the same
+                   code path reached with E4M3 / E5M2 loads and descales),
+                   a power-of-two descale scaling each gradient exactly, and
+                   central differences of sdpa_fwd on the decoded inputs.
+  decode_*         pinned: all 256 e4m3 and e5m2 codes and all 65536 fp16 /
+                   bf16 codes against torch's own casts.
 """
 from __future__ import annotations
 
@@ -40,7 +44,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "sdpa_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
-F64, BF16, F16, E4M3 = 0, 1, 2, 3
+F64, BF16, F16, E4M3, E5M2 = 0, 1, 2, 3, 4
 
 _lib = None
 
@@ -71,12 +75,17 @@ def _load():
         lib.oracle_sdpa_bwd.argtypes = [vp, vp, vp, vp, i32, vp, vp, vp,
                                         i32, i32, i32, i32, i32, i32, f64, i32, i32]
         lib.oracle_sdpa_bwd.restype = i32
+        lib.oracle_sdpa_bwd_fp8.argtypes = [vp, vp, vp, vp, f64, f64, f64, f64, vp, vp, vp,
+                                            i32, i32, i32, i32, i32, i32, f64, i32, i32]
+        lib.oracle_sdpa_bwd_fp8.restype = i32
         lib.oracle_decode_bf16.argtypes = [ctypes.c_uint16]
         lib.oracle_decode_bf16.restype = f64
         lib.oracle_decode_f16.argtypes = [ctypes.c_uint16]
         lib.oracle_decode_f16.restype = f64
         lib.oracle_decode_e4m3.argtypes = [ctypes.c_uint8]
         lib.oracle_decode_e4m3.restype = f64
+        lib.oracle_decode_e5m2.argtypes = [ctypes.c_uint8]
+        lib.oracle_decode_e5m2.restype = f64
         for fn in (lib.oracle_sdpa_fwd, lib.oracle_sdpa_rows, lib.oracle_sdpa_bruteforce):
             fn.restype = i32
         lib.oracle_max_threads.restype = i32
@@ -102,6 +111,8 @@ def _raw(x):
             return x.view(torch.int16).numpy().view(np.uint16), F16
         if x.dtype == torch.float8_e4m3fn:
             return x.view(torch.uint8).numpy(), E4M3
+        if x.dtype == torch.float8_e5m2:
+            return x.view(torch.uint8).numpy(), E5M2
         return x.to(torch.float64).numpy(), F64
     a = np.ascontiguousarray(x)
     if a.dtype != np.float64:
@@ -201,6 +212,30 @@ def sdpa_bwd(q, k, v, dout, scale: float, causal=False, nthreads: int | None = N
     return dq, dk, dv
 
 
+def sdpa_bwd_fp8(q8, k8, v8, dout8, descales, scale: float, causal=False,
+                 nthreads: int | None = None):
+    """Gradients (dQ, dK, dV) float64 for the FP8 hybrid recipe: q8, k8, v8
+    float8_e4m3fn codes, dout8 float8_e5m2 codes, descales = (dq, dk, dv, ddo)
+    so that value = code * descale."""
+    lib = _load()
+    qa, ka, va, t = _prep(q8, k8, v8)
+    da, td = _raw(dout8)
+    if t != E4M3 or td != E5M2:
+        raise ValueError("q8, k8, v8 must be float8_e4m3fn and dout8 float8_e5m2")
+    B, Hq, Hkv, Sq, Sk, d = _shape(q8, k8)
+    if tuple(da.shape) != (B, Hq, Sq, d):
+        raise ValueError("dout8 must have q8's shape")
+    dq = np.empty((B, Hq, Sq, d), np.float64)
+    dk = np.empty((B, Hkv, Sk, d), np.float64)
+    dv = np.empty((B, Hkv, Sk, d), np.float64)
+    nt = nthreads or max_threads()
+    _check(lib.oracle_sdpa_bwd_fp8(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, da.ctypes.data,
+                                   *(float(x) for x in descales), dq.ctypes.data, dk.ctypes.data,
+                                   dv.ctypes.data, B, Hq, Hkv, Sq, Sk, d, float(scale),
+                                   _mask(causal), nt))
+    return dq, dk, dv
+
+
 def sdpa_bruteforce(q, k, v, scale: float, causal: bool = False, descales=(1.0, 1.0, 1.0),
                     return_weights: bool = False):
     """Explicit-matrix forward for tiny inputs.  Returns (O, LSE) or
@@ -229,3 +264,7 @@ def decode_f16(bits: int) -> float:
 
 def decode_e4m3(code: int) -> float:
     return float(_load().oracle_decode_e4m3(int(code)))
+
+
+def decode_e5m2(code: int) -> float:
+    return float(_load().oracle_decode_e5m2(int(code)))

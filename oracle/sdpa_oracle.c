@@ -47,7 +47,7 @@
 #include <omp.h>
 #endif
 
-enum { ORC_F64 = 0, ORC_BF16 = 1, ORC_F16 = 2, ORC_E4M3 = 3 };
+enum { ORC_F64 = 0, ORC_BF16 = 1, ORC_F16 = 2, ORC_E4M3 = 3, ORC_E5M2 = 4 };
 
 /* ---- exact widening of the storage formats to double ------------------- */
 
@@ -92,11 +92,29 @@ double oracle_decode_e4m3(uint8_t c) {
     return sign ? -mag : mag;
 }
 
+/* OCP FP8 E5M2: 1 sign, 5 exponent (bias 15), 2 fraction bits; IEEE-like,
+ * exponent 31 holds the infinities and NaNs; the largest finite is 57344. */
+double oracle_decode_e5m2(uint8_t c) {
+    int sign = (c >> 7) & 1;
+    int e = (c >> 2) & 0x1f;
+    int f = c & 0x3;
+    double mag;
+    if (e == 31) {
+        mag = f ? NAN : INFINITY;
+    } else if (e == 0) {
+        mag = ldexp((double)f, -16);            /* subnormal: f/4 * 2^-14 */
+    } else {
+        mag = ldexp((double)(4 + f), e - 17);   /* (1 + f/4) * 2^(e-15) */
+    }
+    return sign ? -mag : mag;
+}
+
 static double load_elem(const void* base, int dtype, size_t idx, double descale) {
     switch (dtype) {
     case ORC_BF16: return oracle_decode_bf16(((const uint16_t*)base)[idx]);
     case ORC_F16:  return oracle_decode_f16(((const uint16_t*)base)[idx]);
     case ORC_E4M3: return oracle_decode_e4m3(((const uint8_t*)base)[idx]) * descale;
+    case ORC_E5M2: return oracle_decode_e5m2(((const uint8_t*)base)[idx]) * descale;
     default:       return ((const double*)base)[idx];
     }
 }
@@ -319,14 +337,15 @@ int oracle_max_threads(void) {
  * dout has Q's shape and storage type.  dq: [B,Hq,Sq,d], dk, dv: [B,Hkv,Sk,d]
  * doubles.  Work is split by (b, hk), so every dK/dV row has one writer.
  */
-int oracle_sdpa_bwd(const void* q, const void* k, const void* v, const void* dout, int dtype,
+static int bwd_impl(const void* q, const void* k, const void* v, const void* dout, int dtype,
+                    int dout_dtype, double dsq, double dsk, double dsv, double dsdo,
                     double* dq_out, double* dk_out, double* dv_out,
                     int B, int Hq, int Hkv, int Sq, int Sk, int d,
                     double scale, int causal, int nthreads) {
-    problem_t p = {q, k, v, dtype, 1.0, 1.0, 1.0, B, Hq, Hkv, Sq, Sk, d, scale, causal};
+    problem_t p = {q, k, v, dtype, dsq, dsk, dsv, B, Hq, Hkv, Sq, Sk, d, scale, causal};
     int rc = check_problem(&p);
     if (rc) return rc;
-    if (!dout || !dq_out || !dk_out || !dv_out || dtype == ORC_E4M3) return 1;
+    if (!dout || !dq_out || !dk_out || !dv_out) return 1;
     memset(dk_out, 0, sizeof(double) * (size_t)B * Hkv * Sk * d);
     memset(dv_out, 0, sizeof(double) * (size_t)B * Hkv * Sk * d);
     const int group = Hq / Hkv;
@@ -352,10 +371,10 @@ int oracle_sdpa_bwd(const void* q, const void* k, const void* v, const void* dou
                         for (int j = 0; j < nkeys; ++j) {
                             double acc = 0.0, accd = 0.0;
                             for (int c = 0; c < d; ++c) {
-                                acc += load_elem(q, dtype, qoff + c, 1.0) *
-                                       load_elem(k, dtype, (kvhead + j) * d + c, 1.0);
-                                accd += load_elem(dout, dtype, qoff + c, 1.0) *
-                                        load_elem(v, dtype, (kvhead + j) * d + c, 1.0);
+                                acc += load_elem(q, dtype, qoff + c, dsq) *
+                                       load_elem(k, dtype, (kvhead + j) * d + c, dsk);
+                                accd += load_elem(dout, dout_dtype, qoff + c, dsdo) *
+                                        load_elem(v, dtype, (kvhead + j) * d + c, dsv);
                             }
                             s[j] = scale * acc;
                             dp[j] = accd;
@@ -378,9 +397,9 @@ int oracle_sdpa_bwd(const void* q, const void* k, const void* v, const void* dou
                             double* dkj = dk_out + (kvhead + j) * d;
                             double* dvj = dv_out + (kvhead + j) * d;
                             for (int c = 0; c < d; ++c) {
-                                dqi[c] += scale * ds * load_elem(k, dtype, (kvhead + j) * d + c, 1.0);
-                                dkj[c] += scale * ds * load_elem(q, dtype, qoff + c, 1.0);
-                                dvj[c] += s[j] * load_elem(dout, dtype, qoff + c, 1.0);
+                                dqi[c] += scale * ds * load_elem(k, dtype, (kvhead + j) * d + c, dsk);
+                                dkj[c] += scale * ds * load_elem(q, dtype, qoff + c, dsq);
+                                dvj[c] += s[j] * load_elem(dout, dout_dtype, qoff + c, dsdo);
                             }
                         }
                     }
@@ -390,4 +409,27 @@ int oracle_sdpa_bwd(const void* q, const void* k, const void* v, const void* dou
         }
     }
     return failed ? 3 : 0;
+}
+
+/* 16-bit inputs: dout has Q's storage type. */
+int oracle_sdpa_bwd(const void* q, const void* k, const void* v, const void* dout, int dtype,
+                    double* dq_out, double* dk_out, double* dv_out,
+                    int B, int Hq, int Hkv, int Sq, int Sk, int d,
+                    double scale, int causal, int nthreads) {
+    if (dtype == ORC_E4M3 || dtype == ORC_E5M2) return 1;
+    return bwd_impl(q, k, v, dout, dtype, dtype, 1.0, 1.0, 1.0, 1.0, dq_out, dk_out, dv_out,
+                    B, Hq, Hkv, Sq, Sk, d, scale, causal, nthreads);
+}
+
+/* The FP8 hybrid recipe (codelab section 10: E4M3 for the forward tensors,
+ * E5M2 for gradients): Q, K, V as E4M3 codes times their per-tensor
+ * descales, dO as E5M2 codes times its descale; the same exact gradients. */
+int oracle_sdpa_bwd_fp8(const void* q8, const void* k8, const void* v8, const void* dout8,
+                        double descale_q, double descale_k, double descale_v, double descale_do,
+                        double* dq_out, double* dk_out, double* dv_out,
+                        int B, int Hq, int Hkv, int Sq, int Sk, int d,
+                        double scale, int causal, int nthreads) {
+    return bwd_impl(q8, k8, v8, dout8, ORC_E4M3, ORC_E5M2, descale_q, descale_k, descale_v,
+                    descale_do, dq_out, dk_out, dv_out, B, Hq, Hkv, Sq, Sk, d, scale, causal,
+                    nthreads);
 }

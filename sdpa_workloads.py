@@ -10,7 +10,9 @@ ViT-B/16 example, 196 tokens and 12 heads, section 1).  No dataset is used.
 Recipe: ``torch.Generator('cpu').manual_seed(seed)``, then Q, K, V drawn in
 that order as fp32 N(0,1) and rounded to the storage dtype by torch's cast
 (round to nearest even).  FP8 inputs: fp32 N(0,1) per tensor, per-tensor
-descale = amax(|x|) / 448, codes = e4m3fn(x / descale) by torch's cast.
+descale = amax(|x|) / 448, codes = e4m3fn(x / descale) by torch's cast;
+output gradients for the FP8 backward: per-tensor descale = amax(|x|) / 57344,
+codes = e5m2(x / descale).
 """
 from __future__ import annotations
 
@@ -156,6 +158,7 @@ def make_qkv_btnh(w: Workload, device="cpu"):
 
 
 E4M3_MAX = 448.0
+E5M2_MAX = 57344.0
 
 
 def quantize_e4m3(x: torch.Tensor):
@@ -164,6 +167,24 @@ def quantize_e4m3(x: torch.Tensor):
     descale = amax / E4M3_MAX if amax > 0 else 1.0
     codes = (x / descale).to(torch.float8_e4m3fn)
     return codes, descale
+
+
+def quantize_e5m2(x: torch.Tensor):
+    """Per-tensor current scaling for gradients (the FP8 hybrid recipe's E5M2
+    format): descale = amax/57344, codes = e5m2(x/descale) by torch's cast."""
+    amax = float(x.abs().max())
+    descale = amax / E5M2_MAX if amax > 0 else 1.0
+    codes = (x / descale).to(torch.float8_e5m2)
+    return codes, descale
+
+
+def make_dout_e5m2(w: Workload, device="cpu"):
+    """(do8, descale_do, do32): an output gradient of q's shape drawn as fp32
+    N(0,1) from w.seed + 1 and quantised to e5m2."""
+    g = torch.Generator(device="cpu").manual_seed(w.seed + 1)
+    do = torch.randn(w.B, w.Hq, w.Sq, w.d, generator=g, dtype=torch.float32)
+    do8, dd = quantize_e5m2(do)
+    return do8.to(device), dd, do
 
 
 def make_qkv_fp8(w: Workload, device="cpu"):

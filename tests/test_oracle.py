@@ -15,7 +15,7 @@ import pytest
 import torch
 
 import oracle
-from sdpa_workloads import quantize_e4m3
+from sdpa_workloads import quantize_e4m3, quantize_e5m2
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 rng = np.random.default_rng(20261202)
@@ -38,6 +38,17 @@ def test_decode_e4m3_all_codes():
     assert nan.sum() == 2                      # 0x7f and 0xff only
     assert np.array_equal(ref[~nan], got[~nan])
     assert got[0x7e] == 448.0 and got[0x01] == 2.0 ** -9
+
+
+def test_decode_e5m2_all_codes():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e5m2).to(torch.float64).numpy()
+    got = np.array([oracle.decode_e5m2(c) for c in range(256)])
+    nan = np.isnan(ref)
+    assert np.array_equal(nan, np.isnan(got))
+    assert nan.sum() == 6                      # 0x7d-0x7f and 0xfd-0xff
+    assert np.array_equal(ref[~nan], got[~nan])
+    assert got[0x7b] == 57344.0 and got[0x7c] == np.inf and got[0x01] == 2.0 ** -16
 
 
 def test_decode_bf16_and_f16_all_codes():
@@ -496,3 +507,68 @@ def test_backward_zero_queries_closed_form(causal):
         for j in seen:
             expect[:, :, j, :] += dout[:, :, i, :] / len(seen)
     np.testing.assert_allclose(dv, expect, rtol=0, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# FP8 backward (E4M3 forward tensors, E5M2 output gradient; codelab section 10)
+# --------------------------------------------------------------------------
+
+def _fp8_problem(B=1, Hq=2, Hkv=1, Sq=9, Sk=13, d=8, seed=5):
+    g = torch.Generator().manual_seed(seed)
+    q, ds_q = quantize_e4m3(torch.randn(B, Hq, Sq, d, generator=g))
+    k, ds_k = quantize_e4m3(torch.randn(B, Hkv, Sk, d, generator=g))
+    v, ds_v = quantize_e4m3(torch.randn(B, Hkv, Sk, d, generator=g))
+    do, ds_do = quantize_e5m2(torch.randn(B, Hq, Sq, d, generator=g))
+    return (q, k, v, do), (ds_q, ds_k, ds_v, ds_do)
+
+
+def _decoded(t, ds):
+    return t.to(torch.float64).numpy() * ds
+
+
+@pytest.mark.parametrize("causal", [0, 2])
+def test_fp8_backward_matches_finite_differences_of_the_forward(causal):
+    """dQ, dK, dV of the FP8 recipe against central differences of the
+    pinned forward on the decoded values (the loss is <O, dO>)."""
+    (q8, k8, v8, do8), ds = _fp8_problem()
+    scale = 0.35
+    gq, gk, gv = oracle.sdpa_bwd_fp8(q8, k8, v8, do8, ds, scale, causal)
+    q, k, v = _decoded(q8, ds[0]), _decoded(k8, ds[1]), _decoded(v8, ds[2])
+    do = _decoded(do8, ds[3])
+
+    def loss(qq, kk, vv):
+        o, _ = oracle.sdpa_fwd(qq, kk, vv, scale, causal)
+        return float((o * do).sum())
+
+    h = 1e-6
+    picks = [(q, gq, (0, 1, 3, 2)), (k, gk, (0, 0, 7, 5)), (v, gv, (0, 0, 12, 1)), (k, gk, (0, 0, 0, 0))]
+    for arr, grad, idx in picks:
+        plus, minus = arr.copy(), arr.copy()
+        plus[idx] += h
+        minus[idx] -= h
+        args_p = [plus if a is arr else a for a in (q, k, v)]
+        args_m = [minus if a is arr else a for a in (q, k, v)]
+        fd = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        assert abs(fd - grad[idx]) <= 1e-6 * max(1.0, abs(fd)), (idx, fd, grad[idx])
+
+
+def test_fp8_backward_equals_backward_on_decoded_values():
+    (q8, k8, v8, do8), ds = _fp8_problem(B=2, Hq=4, Hkv=2, Sq=20, Sk=31, d=16, seed=9)
+    got = oracle.sdpa_bwd_fp8(q8, k8, v8, do8, ds, 0.25, 0)
+    ref = oracle.sdpa_bwd(_decoded(q8, ds[0]), _decoded(k8, ds[1]), _decoded(v8, ds[2]),
+                          _decoded(do8, ds[3]), 0.25, 0)
+    for a, b in zip(got, ref):
+        assert np.array_equal(a, b)
+
+
+def test_fp8_backward_descales_scale_the_gradients_exactly():
+    """Doubling dO's descale doubles every gradient; doubling V's doubles dQ
+    and dK (through dP) and leaves dV = P^T dO unchanged."""
+    (q8, k8, v8, do8), ds = _fp8_problem(seed=11)
+    base = oracle.sdpa_bwd_fp8(q8, k8, v8, do8, ds, 0.3, 0)
+    two_do = oracle.sdpa_bwd_fp8(q8, k8, v8, do8, (ds[0], ds[1], ds[2], 2 * ds[3]), 0.3, 0)
+    two_v = oracle.sdpa_bwd_fp8(q8, k8, v8, do8, (ds[0], ds[1], 2 * ds[2], ds[3]), 0.3, 0)
+    for a, b in zip(two_do, base):
+        assert np.array_equal(a, 2 * b)
+    assert np.array_equal(two_v[0], 2 * base[0]) and np.array_equal(two_v[1], 2 * base[1])
+    assert np.array_equal(two_v[2], base[2])
