@@ -40,6 +40,8 @@
 #ifndef SDPA_B200_H
 #define SDPA_B200_H
 
+#include <stddef.h>
+
 #if defined(__GNUC__)
 #define SDPA_API __attribute__((visibility("default")))
 #else
@@ -196,6 +198,43 @@ SDPA_API int sdpa_bwd(const void* q, const void* k, const void* v, const void* o
                       float scale, int causal, int dtype, void* stream);
 
 /*
+ * sdpa_bwd_fp8 -- gradients of sdpa_fwd_fp8 under the codelab's FP8 hybrid
+ * recipe ("JAX on GPU, Lab 5: attention on GPU", section 10: E4M3 for the
+ * forward tensors, E5M2 for the gradients): E4M3 Q/K/V codes with their
+ * per-tensor descales (as passed to sdpa_fwd_fp8), the forward's bf16 O and
+ * fp32 LSE, and the output gradient as E5M2 codes with its own per-tensor
+ * descale (current scaling: descale_do = amax(|dO|) / 57344).  The weights are
+ * recomputed from LSE (article "Self-attention, CUDA kernels and
+ * FlashAttention", section 3).
+ *
+ *   q8               E4M3 [B,Hq,Sq,d];  k8, v8  E4M3 [B,Hkv,Sk,d]
+ *   o                bf16 [B,Hq,Sq,d], lse float32 [B,Hq,Sq] (sdpa_fwd_fp8's)
+ *   dout8            E5M2 [B,Hq,Sq,d]
+ *   descale_q/k/v/do host floats, > 0 and finite
+ *   dq               bf16 [B,Hq,Sq,d];  dk, dv  bf16 [B,Hkv,Sk,d] (out; for GQA
+ *                    summed over the query heads sharing each K/V head)
+ *   workspace        device memory owned by the caller, 256-byte aligned, at
+ *                    least sdpa_bwd_fp8_workspace_bytes(B, Hq, Hkv, Sq, Sk, d)
+ *                    bytes; overwritten
+ *   d                128
+ *
+ * Three launches: the codes are widened exactly to bf16 into the workspace
+ * (both formats' values are bf16 values), then the two tensor-core backward
+ * kernels of sdpa_bwd run on them with the descales folded into the score
+ * scale and into their output multipliers, so no value is rounded twice; P
+ * and dS are rounded to bf16 for their products, accumulation is fp32.
+ * Deterministic.  Errors as sdpa_bwd, plus SDPA_ERR_INVALID_ARG for a
+ * non-positive or non-finite descale, a null or misaligned workspace or one
+ * smaller than required, and SDPA_ERR_UNSUPPORTED for d != 128.
+ */
+SDPA_API size_t sdpa_bwd_fp8_workspace_bytes(int B, int Hq, int Hkv, int Sq, int Sk, int d);
+SDPA_API int sdpa_bwd_fp8(const void* q8, const void* k8, const void* v8, const void* o,
+                          const void* dout8, const float* lse, float descale_q, float descale_k,
+                          float descale_v, float descale_do, void* dq, void* dk, void* dv,
+                          void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv,
+                          int Sq, int Sk, int d, float scale, int causal, void* stream);
+
+/*
  * sdpa_bwd_noalloc -- sdpa_bwd without the delta argument, for callers that
  * cannot allocate device memory: code running inside a host framework that
  * owns every device allocation and lends none to its extensions, or code on
@@ -247,7 +286,7 @@ SDPA_API const char* sdpa_strerror(int status);
 SDPA_API int sdpa_device_status(int* status, int* detail, int clear);
 
 /* Number of kernel launches sdpa_fwd / sdpa_fwd_strided / sdpa_fwd_fp8 issue
- * per call (1); sdpa_bwd and sdpa_bwd_noalloc issue 2. */
+ * per call (1); sdpa_bwd and sdpa_bwd_noalloc issue 2, sdpa_bwd_fp8 3. */
 SDPA_API int sdpa_launches_per_call(void);
 
 /*

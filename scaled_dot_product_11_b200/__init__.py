@@ -21,7 +21,7 @@ __all__ = [
     "SDPA_NO_MASK", "SDPA_CAUSAL", "SDPA_CAUSAL_BOTTOM_RIGHT",
     "sdpa_fwd", "sdpa_fwd_strided", "sdpa_fwd_fp8", "sdpa_bwd", "attention_backward", "sdpa_strerror", "sdpa_device_status",
     "sdpa_launches_per_call", "attention", "attention_fp8", "sdpa_selftest_wait",
-    "sdpa_selftest_exp2",
+    "sdpa_selftest_exp2", "sdpa_bwd_fp8", "sdpa_bwd_fp8_workspace_bytes", "attention_backward_fp8",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -70,6 +70,10 @@ _lib.sdpa_device_status.argtypes = [ctypes.POINTER(_i), ctypes.POINTER(_i), _i]
 _lib.sdpa_device_status.restype = _i
 _lib.sdpa_launches_per_call.argtypes = []
 _lib.sdpa_launches_per_call.restype = _i
+_lib.sdpa_bwd_fp8_workspace_bytes.argtypes = [_i] * 6
+_lib.sdpa_bwd_fp8_workspace_bytes.restype = ctypes.c_size_t
+_lib.sdpa_bwd_fp8.argtypes = [_vp] * 6 + [_f] * 4 + [_vp] * 4 + [ctypes.c_size_t] + [_i] * 6 + [_f, _i, _vp]
+_lib.sdpa_bwd_fp8.restype = _i
 _lib.sdpa_selftest_wait.argtypes = [ctypes.c_uint, _vp, _vp]
 _lib.sdpa_selftest_wait.restype = _i
 _lib.sdpa_selftest_exp2.argtypes = [_vp, _vp, _vp, _i, _vp]
@@ -117,6 +121,22 @@ def sdpa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Sq, Sk, d, s
     int; calls on one device must not overlap on the GPU."""
     return int(_lib.sdpa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Sq, Sk, d,
                                      float(scale), int(causal), int(dtype), stream or None))
+
+
+def sdpa_bwd_fp8_workspace_bytes(B, Hq, Hkv, Sq, Sk, d) -> int:
+    """Bytes of device workspace sdpa_bwd_fp8 needs (0 for invalid sizes)."""
+    return int(_lib.sdpa_bwd_fp8_workspace_bytes(B, Hq, Hkv, Sq, Sk, d))
+
+
+def sdpa_bwd_fp8(q8, k8, v8, o, dout8, lse, descale_q, descale_k, descale_v, descale_do,
+                 dq, dk, dv, workspace, workspace_bytes, B, Hq, Hkv, Sq, Sk, d, scale, causal,
+                 stream) -> int:
+    """Raw FP8 backward call: device addresses as ints (E4M3 q8/k8/v8, bf16 o,
+    E5M2 dout8, fp32 lse; bf16 dq/dk/dv; a 256-byte aligned workspace)."""
+    return int(_lib.sdpa_bwd_fp8(q8, k8, v8, o, dout8, lse, float(descale_q), float(descale_k),
+                                 float(descale_v), float(descale_do), dq, dk, dv, workspace,
+                                 int(workspace_bytes), B, Hq, Hkv, Sq, Sk, d, float(scale),
+                                 int(causal), stream or None))
 
 
 def sdpa_strerror(status: int) -> str:
@@ -290,4 +310,36 @@ def attention_backward(q, k, v, o, lse, dout, causal=False, scale: float | None 
                       SDPA_BF16 if q.dtype == torch.bfloat16 else SDPA_FP16, _stream_handle(stream))
     if rc != SDPA_OK:
         raise SdpaError(rc, "sdpa_bwd")
+    return dq, dk, dv
+
+
+def attention_backward_fp8(q8, k8, v8, o, lse, dout8, descales, causal=False,
+                           scale: float | None = None, stream=None):
+    """(dQ, dK, dV) bf16 for the FP8 forward: q8/k8/v8 float8_e4m3fn codes,
+    o (bf16) and lse from attention_fp8 with the same causal and scale,
+    dout8 float8_e5m2 codes, descales = (dq, dk, dv, ddo) with value =
+    code * descale.  The workspace is allocated with torch."""
+    import torch
+    B, Hq, Hkv, Sq, Sk, d = _dims(q8, k8, v8)
+    causal = _causal_code(causal)
+    for t in (q8, k8, v8):
+        if t.dtype != torch.float8_e4m3fn:
+            raise ValueError("q8, k8, v8 must be float8_e4m3fn")
+    _check_buffer(o, "o", (B, Hq, Sq, d), torch.bfloat16, q8.device)
+    _check_buffer(dout8, "dout8", (B, Hq, Sq, d), torch.float8_e5m2, q8.device)
+    _check_buffer(lse, "lse", (B, Hq, Sq), torch.float32, q8.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    with torch.cuda.device(q8.device):
+        dq = torch.empty((B, Hq, Sq, d), dtype=torch.bfloat16, device=q8.device)
+        dk = torch.empty((B, Hkv, Sk, d), dtype=torch.bfloat16, device=q8.device)
+        dv = torch.empty((B, Hkv, Sk, d), dtype=torch.bfloat16, device=q8.device)
+        nbytes = sdpa_bwd_fp8_workspace_bytes(B, Hq, Hkv, Sq, Sk, d)
+        ws = torch.empty(nbytes + 256, dtype=torch.uint8, device=q8.device)
+        base = (ws.data_ptr() + 255) // 256 * 256
+        rc = sdpa_bwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), o.data_ptr(), dout8.data_ptr(),
+                          lse.data_ptr(), descales[0], descales[1], descales[2], descales[3],
+                          dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), base, nbytes,
+                          B, Hq, Hkv, Sq, Sk, d, scale, causal, _stream_handle(stream))
+    if rc != SDPA_OK:
+        raise SdpaError(rc, "sdpa_bwd_fp8")
     return dq, dk, dv

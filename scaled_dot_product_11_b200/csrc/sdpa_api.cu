@@ -6,6 +6,7 @@
 #include <cstring>
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <cuda_fp16.h>
 
 #include "sdpa.h"
 #include "sdpa_host.h"
@@ -350,6 +351,7 @@ int launch_bwd_tc(const void* q, const void* k, const void* v, const sdpa::BwdPa
     tp.dq = bp.dq; tp.dk = bp.dk; tp.dv = bp.dv;
     tp.B = bp.B; tp.Hq = bp.Hq; tp.Hkv = bp.Hkv; tp.Sq = bp.Sq; tp.Sk = bp.Sk; tp.group = bp.group;
     tp.causal = bp.causal; tp.causal_off = bp.causal_off; tp.scale = bp.scale;
+    tp.dq_mul = bp.dq_mul; tp.dk_mul = bp.dk_mul; tp.dv_mul = bp.dv_mul; tp.d_mul = bp.d_mul;
     auto kdkdv = sdpa::sdpa_bwd_dkdv_tc_kernel<D, BF16>;
     auto kdq = sdpa::sdpa_bwd_dq_tc_kernel<D, BF16>;
     static bool attr_set[64];
@@ -395,6 +397,10 @@ extern "C" int sdpa_bwd(const void* q, const void* k, const void* v, const void*
     bp.causal = causal != 0 ? 1 : 0;
     bp.causal_off = causal == SDPA_CAUSAL_BOTTOM_RIGHT ? Sk - Sq : 0;
     bp.scale = scale;
+    bp.dq_mul = scale;
+    bp.dk_mul = scale;
+    bp.dv_mul = 1.0f;
+    bp.d_mul = 1.0f;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool bf = dtype == SDPA_BF16;
     if (d == 32) return bf ? launch_bwd<32, true>(bp, s) : launch_bwd<32, false>(bp, s);
@@ -404,6 +410,145 @@ extern "C" int sdpa_bwd(const void* q, const void* k, const void* v, const void*
     }
     if (d == 64) return bf ? launch_bwd<64, true>(bp, s) : launch_bwd<64, false>(bp, s);
     return bf ? launch_bwd<128, true>(bp, s) : launch_bwd<128, false>(bp, s);
+}
+
+// ---------------------------------------------------------------------------
+// sdpa_bwd_fp8: the backward of the FP8 forward under the codelab's hybrid
+// recipe (section 10: E4M3 for the forward tensors, E5M2 for gradients).
+// One launch widens the E4M3 Q/K/V codes and the E5M2 dO codes to bf16 --
+// exactly, since both formats' values are bf16 values (3 and 2 fraction bits,
+// exponents inside bf16's range) -- into the caller's workspace; the
+// tensor-core backward then runs on the codes, with the per-tensor descales
+// folded into the score scale and into its output and D multipliers, so that
+// no value is rounded twice.  With codes q', k', v', g' (dO) and descales
+// a_q, a_k, a_v, a_g:
+//   scores        scale * a_q a_k (q' . k')            = scale * (q . k)
+//   dP' = g' v'^T = dP / (a_g a_v);  D' = (g' . O) / a_v = D / (a_g a_v)
+//   dS' = P (dP' - D') = dS / (a_g a_v)
+//   dQ = (scale a_g a_v a_k) dS' k',  dK = (scale a_g a_v a_q) dS'^T q',
+//   dV = a_g P^T g'.
+// ---------------------------------------------------------------------------
+namespace {
+
+struct WidenSeg {
+    const uint8_t* src;
+    uint16_t* dst;
+    long long n;      // elements
+    int e5m2;         // 0: E4M3 codes, 1: E5M2 codes
+};
+struct WidenParams {
+    WidenSeg seg[4];
+    long long start[5];   // first 16-code chunk of each segment; start[4] = all chunks
+};
+
+// Two codes (low byte first) to bf16x2, exactly.
+__device__ __forceinline__ uint32_t widen2(uint16_t two, int e5m2) {
+    uint32_t h2;
+    if (e5m2) {
+        // an E5M2 code is the high byte of the binary16 with the same value
+        h2 = ((uint32_t)(two & 0xffu) << 8) | ((uint32_t)(two & 0xff00u) << 16);
+    } else {
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(two));
+    }
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+    return sdpa::pack_bf16x2(f.x, f.y);
+}
+
+__global__ void widen_fp8_kernel(const WidenParams wp) {
+    const long long total = wp.start[4];
+    for (long long c = (long long)blockIdx.x * blockDim.x + threadIdx.x; c < total;
+         c += (long long)gridDim.x * blockDim.x) {
+        const int s = (c >= wp.start[1]) + (c >= wp.start[2]) + (c >= wp.start[3]);
+        const WidenSeg sg = wp.seg[s];
+        const long long i = (c - wp.start[s]) * 16;
+        if (i + 16 <= sg.n) {
+            const uint4 in = *reinterpret_cast<const uint4*>(sg.src + i);
+            const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+            uint32_t o[8];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                o[2 * e] = widen2((uint16_t)(w[e] & 0xffffu), sg.e5m2);
+                o[2 * e + 1] = widen2((uint16_t)(w[e] >> 16), sg.e5m2);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(sg.dst + i);
+            dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+            dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+        } else {
+            for (long long e = i; e < sg.n; ++e) {
+                const uint32_t two = widen2((uint16_t)sg.src[e], sg.e5m2);
+                sg.dst[e] = (uint16_t)(two & 0xffffu);
+            }
+        }
+    }
+}
+
+// Byte offsets of the workspace's parts, each 256-byte aligned: widened Q,
+// K, V, dO (bf16), then D (fp32); returns the total.
+size_t fp8_bwd_layout(int B, int Hq, int Hkv, int Sq, int Sk, int d, size_t off[5]) {
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t nq = (size_t)B * Hq * Sq * d, nk = (size_t)B * Hkv * Sk * d;
+    off[0] = 0;
+    off[1] = off[0] + up(nq * 2);
+    off[2] = off[1] + up(nk * 2);
+    off[3] = off[2] + up(nk * 2);
+    off[4] = off[3] + up(nq * 2);
+    return off[4] + up((size_t)B * Hq * Sq * 4);
+}
+
+}  // namespace
+
+extern "C" size_t sdpa_bwd_fp8_workspace_bytes(int B, int Hq, int Hkv, int Sq, int Sk, int d) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Sq <= 0 || Sk <= 0 || d <= 0) return 0;
+    size_t off[5];
+    return fp8_bwd_layout(B, Hq, Hkv, Sq, Sk, d, off);
+}
+
+extern "C" int sdpa_bwd_fp8(const void* q8, const void* k8, const void* v8, const void* o,
+                            const void* dout8, const float* lse, float descale_q, float descale_k,
+                            float descale_v, float descale_do, void* dq, void* dk, void* dv,
+                            void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv,
+                            int Sq, int Sk, int d, float scale, int causal, void* stream) {
+    int rc = check_args(q8, k8, v8, o, lse, B, Hq, Hkv, Sq, Sk, d, scale, causal);
+    if (rc != SDPA_OK) return rc;
+    if (!dout8 || !lse || !dq || !dk || !dv || !workspace) return SDPA_ERR_INVALID_ARG;
+    if (!aligned16(dout8) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return SDPA_ERR_INVALID_ARG;
+    for (float ds : {descale_q, descale_k, descale_v, descale_do})
+        if (!std::isfinite(ds) || !(ds > 0.0f)) return SDPA_ERR_INVALID_ARG;
+    if ((long long)B * Hq > 65535) return SDPA_ERR_INVALID_ARG;   // grid rows
+    if (d != 128) return SDPA_ERR_UNSUPPORTED;
+    size_t off[5];
+    if (workspace_bytes < fp8_bwd_layout(B, Hq, Hkv, Sq, Sk, d, off)) return SDPA_ERR_INVALID_ARG;
+    rc = check_device();
+    if (rc != SDPA_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint16_t *q16 = reinterpret_cast<uint16_t*>(ws + off[0]), *k16 = reinterpret_cast<uint16_t*>(ws + off[1]);
+    uint16_t *v16 = reinterpret_cast<uint16_t*>(ws + off[2]), *g16 = reinterpret_cast<uint16_t*>(ws + off[3]);
+    const long long nq = (long long)B * Hq * Sq * d, nk = (long long)B * Hkv * Sk * d;
+    WidenParams wp;
+    wp.seg[0] = WidenSeg{static_cast<const uint8_t*>(q8), q16, nq, 0};
+    wp.seg[1] = WidenSeg{static_cast<const uint8_t*>(k8), k16, nk, 0};
+    wp.seg[2] = WidenSeg{static_cast<const uint8_t*>(v8), v16, nk, 0};
+    wp.seg[3] = WidenSeg{static_cast<const uint8_t*>(dout8), g16, nq, 1};
+    wp.start[0] = 0;
+    for (int i = 0; i < 4; ++i) wp.start[i + 1] = wp.start[i] + (wp.seg[i].n + 15) / 16;
+    const long long blocks = (wp.start[4] + 255) / 256;
+    widen_fp8_kernel<<<(unsigned)(blocks < 4 * sm_count() ? blocks : 4 * sm_count()), 256, 0, s>>>(wp);
+    if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
+    sdpa::BwdParams bp;
+    bp.q = q16; bp.k = k16; bp.v = v16; bp.o = o; bp.dout = g16; bp.lse = lse;
+    bp.dq = dq; bp.dk = dk; bp.dv = dv; bp.delta = reinterpret_cast<float*>(ws + off[4]);
+    bp.B = B; bp.Hq = Hq; bp.Hkv = Hkv; bp.Sq = Sq; bp.Sk = Sk; bp.group = Hq / Hkv;
+    bp.causal = causal != 0 ? 1 : 0;
+    bp.causal_off = causal == SDPA_CAUSAL_BOTTOM_RIGHT ? Sk - Sq : 0;
+    bp.scale = scale * descale_q * descale_k;
+    bp.dq_mul = scale * descale_do * descale_v * descale_k;
+    bp.dk_mul = scale * descale_do * descale_v * descale_q;
+    bp.dv_mul = descale_do;
+    bp.d_mul = 1.0f / descale_v;
+    return launch_bwd_tc<128, true>(q16, k16, v16, bp, s);
 }
 
 extern "C" const char* sdpa_strerror(int status) {

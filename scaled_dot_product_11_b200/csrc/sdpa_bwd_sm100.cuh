@@ -36,6 +36,10 @@ struct BwdParams {
     int B, Hq, Hkv, Sq, Sk, group;
     int causal, causal_off;          // key j visible to query i iff j <= i + causal_off
     float scale;
+    // multipliers of the tensor-core kernels' outputs and of D (the 16-bit
+    // path: scale, scale, 1, 1; the FP8 path folds the per-tensor descales
+    // into them)
+    float dq_mul, dk_mul, dv_mul, d_mul;
 };
 
 template <int D>

@@ -45,7 +45,11 @@ struct BwdTcParams {
     void *dq, *dk, *dv;
     int B, Hq, Hkv, Sq, Sk, group;
     int causal, causal_off;
-    float scale;
+    float scale;                     // score scale (P = exp(scale * s - LSE))
+    // output multipliers: dQ = dq_mul * (dS K), dK = dk_mul * (dS^T Q),
+    // dV = dv_mul * (P^T dO), and D = d_mul * (dO . O); 16-bit inputs use
+    // scale, scale, 1, 1
+    float dq_mul, dk_mul, dv_mul, d_mul;
 };
 
 template <int D>
@@ -280,7 +284,7 @@ sdpa_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     const float lse_r = row < p.Sq ? p.lse[(size_t)bh * p.Sq + row] * kL2e : 0.0f;
     dpart[threadIdx.x] = bt_row_dot<D, BF16>(p, (size_t)bh * p.Sq * D, row, half);
     bool ok = __syncthreads_and(bt_wait(sm.bar_in[0], 0, 0x50000u));
-    const float d_r = dpart[r] + dpart[r + 128];
+    const float d_r = (dpart[r] + dpart[r + 128]) * p.d_mul;
     if (half == 0 && row < p.Sq) p.delta[(size_t)bh * p.Sq + row] = d_r;   // for the dK/dV kernel
 
     // this thread's own wait results since the last block-wide check
@@ -368,10 +372,10 @@ sdpa_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
                                                       ((size_t)bh * p.Sq + row) * D + 32 * c);
 #pragma unroll
                 for (int v4 = 0; v4 < 4; ++v4)
-                    dst[v4] = make_uint4(bt_pack<BF16>(x[8 * v4] * p.scale, x[8 * v4 + 1] * p.scale),
-                                         bt_pack<BF16>(x[8 * v4 + 2] * p.scale, x[8 * v4 + 3] * p.scale),
-                                         bt_pack<BF16>(x[8 * v4 + 4] * p.scale, x[8 * v4 + 5] * p.scale),
-                                         bt_pack<BF16>(x[8 * v4 + 6] * p.scale, x[8 * v4 + 7] * p.scale));
+                    dst[v4] = make_uint4(bt_pack<BF16>(x[8 * v4] * p.dq_mul, x[8 * v4 + 1] * p.dq_mul),
+                                         bt_pack<BF16>(x[8 * v4 + 2] * p.dq_mul, x[8 * v4 + 3] * p.dq_mul),
+                                         bt_pack<BF16>(x[8 * v4 + 4] * p.dq_mul, x[8 * v4 + 5] * p.dq_mul),
+                                         bt_pack<BF16>(x[8 * v4 + 6] * p.dq_mul, x[8 * v4 + 7] * p.dq_mul));
             }
         }
     }
@@ -553,7 +557,7 @@ sdpa_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         // are warp-collective, the stores per key.  Warps 0-3 write dV, 4-7 dK.
         const size_t orow = ((size_t)bk * p.Sk + (size_t)key) * D;
         void* out = half ? p.dk : p.dv;
-        const float mul = half ? p.scale : 1.0f;
+        const float mul = half ? p.dk_mul : p.dv_mul;
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
             float x[32];

@@ -21,7 +21,8 @@ def test_header_declares_the_entry_points():
     assert set(declared_symbols()) == {"sdpa_fwd", "sdpa_fwd_strided", "sdpa_fwd_fp8",
                                        "sdpa_bwd", "sdpa_bwd_noalloc", "sdpa_strerror",
                                        "sdpa_device_status", "sdpa_launches_per_call",
-                                       "sdpa_selftest_wait", "sdpa_selftest_exp2"}
+                                       "sdpa_selftest_wait", "sdpa_selftest_exp2",
+                                       "sdpa_bwd_fp8", "sdpa_bwd_fp8_workspace_bytes"}
 
 
 def test_library_exports_every_declared_symbol():
@@ -219,3 +220,27 @@ def test_wrapper_buffer_check_refuses_mismatches(bad):
     t = _FakeCudaTensor(shape, dtype, device, strides, cuda)
     with pytest.raises(ValueError):
         _check_buffer(t, "out", (2, 4, 100, 64), torch.bfloat16, dev, contiguous=False)
+
+
+def test_fp8_backward_workspace_size_and_argument_checks():
+    """sdpa_bwd_fp8: the workspace holds widened Q, K, V, dO (bf16) and D
+    (fp32), each part 256-byte aligned; bad arguments are refused before any
+    device call."""
+    import scaled_dot_product_11_b200 as sdpa
+    up = lambda x: (x + 255) // 256 * 256
+    B, Hq, Hkv, Sq, Sk, d = 2, 8, 2, 300, 500, 128
+    want = 2 * up(B * Hq * Sq * d * 2) + 2 * up(B * Hkv * Sk * d * 2) + up(B * Hq * Sq * 4)
+    assert sdpa.sdpa_bwd_fp8_workspace_bytes(B, Hq, Hkv, Sq, Sk, d) == want
+    assert sdpa.sdpa_bwd_fp8_workspace_bytes(0, Hq, Hkv, Sq, Sk, d) == 0
+    p = 1 << 20          # an aligned stand-in address; never dereferenced
+    ws = 1 << 24
+    args = dict(q8=p, k8=p, v8=p, o=p, dout8=p, lse=p, descale_q=0.01, descale_k=0.01,
+                descale_v=0.01, descale_do=1e-4, dq=p, dk=p, dv=p, workspace=ws,
+                workspace_bytes=want, B=B, Hq=Hq, Hkv=Hkv, Sq=Sq, Sk=Sk, d=d, scale=0.088,
+                causal=0, stream=0)
+    bad = [dict(dout8=0), dict(workspace=0), dict(workspace=ws + 16), dict(workspace_bytes=want - 1),
+           dict(descale_do=0.0), dict(descale_q=float("inf")), dict(descale_v=-1.0), dict(lse=0)]
+    for b in bad:
+        assert sdpa.sdpa_bwd_fp8(**{**args, **b}) == sdpa.SDPA_ERR_INVALID_ARG, b
+    w64 = sdpa.sdpa_bwd_fp8_workspace_bytes(B, Hq, Hkv, Sq, Sk, 64)
+    assert sdpa.sdpa_bwd_fp8(**{**args, "d": 64, "workspace_bytes": w64}) == sdpa.SDPA_ERR_UNSUPPORTED
