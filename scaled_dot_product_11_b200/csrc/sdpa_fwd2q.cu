@@ -8,15 +8,26 @@
 #include "sdpa_host.h"
 #include "sdpa_fwd2q_sm100.cuh"
 
-// K/V ring depth and Q buffers per stage: 16-bit head dim 128 (32 KB tiles:
-// 2 Q tiles + 5 ring slots fill the 227 KB), 16-bit head dim 64 and e4m3
-// head dim 128 (16 KB tiles: 2 x 2 Q tiles + 8 ring slots).
+// Forms and K/V ring depths.  16-bit head dim 128 takes the one-warp-per-row
+// softmax (two 32 KB Q tiles + 5 ring slots fill the 227 KB); head dim 64 and
+// e4m3 head dim 128 (16 KB tiles: 2 x 2 Q tiles + 8 ring slots) take the split
+// softmax (two warps per row, each over 64 of the 128 scores), which measured
+// faster there and slower at 16-bit head dim 128.
 #ifndef SDPA2_STAGES_D128
 #define SDPA2_STAGES_D128 5
 #endif
 #ifndef SDPA2_STAGES_16K
 #define SDPA2_STAGES_16K 8
 #endif
+#ifndef SDPA2_SPLIT_D128
+#define SDPA2_SPLIT_D128 0
+#endif
+#ifndef SDPA2_SPLIT_16K
+#define SDPA2_SPLIT_16K 1
+#endif
+// the split form needs room for its halves' statistics and exchange: its
+// 16-bit head dim 128 ring has 4 slots
+static constexpr int kStagesD128 = SDPA2_SPLIT_D128 ? 4 : SDPA2_STAGES_D128;
 
 namespace sdpa_host {
 namespace {
@@ -24,9 +35,9 @@ namespace {
 using sdpa::fwd2::Cfg;
 using sdpa::fwd2::Params;
 
-template <int D, int KIND, int NS, int QB, bool STRIDED>
+template <int D, int KIND, int NS, int QB, bool SPLIT, bool STRIDED>
 int launch_cfg(const Fwd2Request& r, const Params& prm, cudaStream_t stream) {
-    using C = Cfg<D, KIND, NS, QB>;
+    using C = Cfg<D, KIND, NS, QB, SPLIT>;
     const CUtensorMapDataType dt = KIND == sdpa::fwd2::K2_BF16   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                    : KIND == sdpa::fwd2::K2_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                                  : CU_TENSOR_MAP_DATA_TYPE_UINT8;
@@ -35,7 +46,7 @@ int launch_cfg(const Fwd2Request& r, const Params& prm, cudaStream_t stream) {
         !encode_view(&tk, dt, C::kElem, r.k, D, r.Sk, r.Hkv, r.B, r.vk, C::kElemsPerSw, !STRIDED) ||
         !encode_view(&tv, dt, C::kElem, r.v, D, r.Sk, r.Hkv, r.B, r.vv, C::kElemsPerSw, !STRIDED))
         return SDPA_ERR_CUDA;
-    auto kern = sdpa::fwd2::sdpa_fwd2q_sm100_kernel<D, KIND, NS, QB, STRIDED>;
+    auto kern = sdpa::fwd2::sdpa_fwd2q_sm100_kernel<D, KIND, NS, QB, SPLIT, STRIDED>;
     static bool attr_set[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return SDPA_ERR_CUDA;
@@ -50,10 +61,10 @@ int launch_cfg(const Fwd2Request& r, const Params& prm, cudaStream_t stream) {
     return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
 }
 
-template <int D, int KIND, int NS, int QB>
+template <int D, int KIND, int NS, int QB, bool SPLIT>
 int launch_form(const Fwd2Request& r, const Params& prm, cudaStream_t stream) {
-    return r.contiguous ? launch_cfg<D, KIND, NS, QB, false>(r, prm, stream)
-                        : launch_cfg<D, KIND, NS, QB, true>(r, prm, stream);
+    return r.contiguous ? launch_cfg<D, KIND, NS, QB, SPLIT, false>(r, prm, stream)
+                        : launch_cfg<D, KIND, NS, QB, SPLIT, true>(r, prm, stream);
 }
 
 }  // namespace
@@ -93,16 +104,17 @@ int launch_fwd2q(const Fwd2Request& r, cudaStream_t stream) {
     prm.o_sh = r.vo.sh;
     prm.o_ss = r.vo.ss;
     using namespace sdpa::fwd2;
+    constexpr bool kSplitD128 = SDPA2_SPLIT_D128 != 0, kSplit16K = SDPA2_SPLIT_16K != 0;
     switch (r.kind) {
     case K2_BF16:
-        return r.d == 64 ? launch_form<64, K2_BF16, SDPA2_STAGES_16K, 2>(r, prm, stream)
-                         : launch_form<128, K2_BF16, SDPA2_STAGES_D128, 1>(r, prm, stream);
+        return r.d == 64 ? launch_form<64, K2_BF16, SDPA2_STAGES_16K, 2, kSplit16K>(r, prm, stream)
+                         : launch_form<128, K2_BF16, kStagesD128, 1, kSplitD128>(r, prm, stream);
     case K2_FP16:
-        return r.d == 64 ? launch_form<64, K2_FP16, SDPA2_STAGES_16K, 2>(r, prm, stream)
-                         : launch_form<128, K2_FP16, SDPA2_STAGES_D128, 1>(r, prm, stream);
+        return r.d == 64 ? launch_form<64, K2_FP16, SDPA2_STAGES_16K, 2, kSplit16K>(r, prm, stream)
+                         : launch_form<128, K2_FP16, kStagesD128, 1, kSplitD128>(r, prm, stream);
     case K2_E4M3:
         if (!r.contiguous || r.d != 128) return SDPA_ERR_UNSUPPORTED;
-        return launch_cfg<128, K2_E4M3, SDPA2_STAGES_16K, 2, false>(r, prm, stream);
+        return launch_cfg<128, K2_E4M3, SDPA2_STAGES_16K, 2, kSplit16K, false>(r, prm, stream);
     default:
         return SDPA_ERR_UNSUPPORTED;
     }

@@ -29,6 +29,13 @@
 //                in the tensor pipe (two issuers, one per stage, interleave
 //                the blocks and lengthen both stages' chains)
 //   warps 14-15  idle (they complete the fourth warp group's register split)
+// The split form (768 threads) doubles the softmax warps: warps 0-7 stage 0,
+// 8-15 stage 1, two warps per TMEM lane quarter, each over 64 of a row's 128
+// scores (the halves exchange tile maxima through shared memory and keep
+// their own row sums); the epilogue, producer and MMA warps follow (16-19,
+// 20, 21).  It halves each softmax warp's serial work, at the price of a
+// 32-score register budget (80 registers a thread at launch), so its scores
+// are read from TMEM twice (max, then weights).
 // Tensor memory (128 lanes x 512 columns, fp32):
 //   [0,128) S_0   [128,256) S_1   [256,256+d) O_0   [256+d,256+2d) O_1
 // The weights P_s (16-bit pairs, or e4m3 quads, per column) overwrite the
@@ -73,6 +80,25 @@
 #endif
 static_assert(8 * SDPA2_REGS_SOFTMAX + 4 * SDPA2_REGS_EPILOGUE + 4 * SDPA2_REGS_OTHER <= 16 * 128,
               "register split exceeds the launch allocation");
+// The split form (two softmax warps per lane quarter and stage, 768 threads)
+// is launched with 80 registers a thread (65536 / 768, rounded down to a
+// multiple of 8); setmaxnreg moves registers only within that allocation, so
+// per SM sub-partition (4 softmax, 1 epilogue, 1 other warp) 4 S + E + W <= 6 * 80.
+#ifndef SDPA2S_REGS_SOFTMAX
+#define SDPA2S_REGS_SOFTMAX 88
+#endif
+#ifndef SDPA2S_REGS_EPILOGUE
+#define SDPA2S_REGS_EPILOGUE 48
+#endif
+#ifndef SDPA2S_REGS_OTHER
+#define SDPA2S_REGS_OTHER 80
+#endif
+static_assert(4 * SDPA2S_REGS_SOFTMAX + SDPA2S_REGS_EPILOGUE + SDPA2S_REGS_OTHER <= 6 * 80,
+              "split register budget exceeds the launch allocation");
+// 1: the MMA warp commits a step's K/V slot releases at the next step's top
+#ifndef SDPA2_DEFER_RELEASE
+#define SDPA2_DEFER_RELEASE 1
+#endif
 // 1: 16-bit inputs compute the weights before the tile max (see the softmax)
 #ifndef SDPA2_WEIGHTS_FIRST
 #define SDPA2_WEIGHTS_FIRST 1
@@ -112,13 +138,19 @@ struct Params {
     long long o_sb, o_sh, o_ss;   // O's batch, head, row strides in elements
 };
 
-template <int D, int KIND, int NS, int QB>
+template <int D, int KIND, int NS, int QB, bool SPLIT = false>
 struct Cfg {
-    static constexpr int kThreads = 512;
-    static constexpr int kEpiWarp0 = 8;
-    static constexpr int kLoadWarp = 12;
-    static constexpr int kMmaWarp = 13;
-    static constexpr int kTmemUsers = 256 + 128 + 32;   // softmax, epilogue, MMA threads
+    // SPLIT: two softmax warps per TMEM lane quarter and stage, each over 64
+    // of a row's 128 scores (16 softmax warps); else one (8 softmax warps)
+    static constexpr int kSmWarpsPerStage = SPLIT ? 8 : 4;
+    static constexpr int kSoftmaxWarps = 2 * kSmWarpsPerStage;
+    static constexpr int kSmThreadsPerStage = 32 * kSmWarpsPerStage;
+    static constexpr int kThreads = SPLIT ? 768 : 512;
+    static constexpr int kEpiWarp0 = kSoftmaxWarps;
+    static constexpr int kLoadWarp = kSoftmaxWarps + 4;
+    static constexpr int kMmaWarp = kLoadWarp + 1;
+    static constexpr int kTmemUsers = 2 * kSmThreadsPerStage + 128 + 32;   // softmax, epilogue, MMA
+    static constexpr int kThreadKeys = SPLIT ? 64 : 128;   // scores per softmax thread and tile
     static constexpr int kElem = (KIND == K2_E4M3) ? 1 : 2;
     static constexpr int kRowBytes = D * kElem;
     static constexpr int kSwBytes = 128;                   // 128-byte swizzle rows
@@ -133,6 +165,10 @@ struct Cfg {
     static constexpr int kPvKeysPerStep = 32 / kElem;
     static constexpr int kPvSteps = kKeys / kPvKeysPerStep;
     static constexpr int kPWordsPer32 = 32 * kElem / 4;    // TMEM columns of P per 32 keys
+    // PV products per 64-key half: a half's weights sit in its own score
+    // columns (S_s + 64 h) in the split form, so the A operand address jumps
+    // by 64 columns between the halves
+    static constexpr int kPvStepsPerHalf = kThreadKeys / kPvKeysPerStep;
     // lazy rescale: the running max only moves when a tile's max exceeds it
     // by more than this (log2 units), so a weight 2^(s - m_run) can reach
     // 2^threshold
@@ -147,8 +183,12 @@ struct Cfg {
     // shared memory (offsets from a 1024-byte aligned base)
     static constexpr int kSmemQ = 0;                                 // [2 stages][QB] tiles
     static constexpr int kSmemKV = 2 * QB * kTileBytes;              // [NS] tiles
-    static constexpr int kSmemStats = kSmemKV + NS * kTileBytes;     // [2 stages][128 rows][m, l]
-    static constexpr int kSmemBar = kSmemStats + 2 * 128 * 2 * 4;
+    // [2 stages][halves][128 rows][m, l], then (split) the halves' tile-max
+    // exchange [2 stages][2 tile parities][2 halves][128 rows]
+    static constexpr int kSmemStats = kSmemKV + NS * kTileBytes;
+    static constexpr int kStatsBytes = (SPLIT ? 2 : 1) * 2 * 128 * 2 * 4;
+    static constexpr int kSmemXchg = kSmemStats + kStatsBytes;
+    static constexpr int kSmemBar = kSmemXchg + (SPLIT ? 2 * 2 * 2 * 128 * 4 : 0);
     // barriers
     static constexpr int kBarQFull = 0;            // [2 stages][2 buffers]
     static constexpr int kBarQEmpty = 4;           // [2][2]
@@ -161,7 +201,8 @@ struct Cfg {
     static constexpr int kBarStFull = 16 + 2 * NS; // [2], softmax -> epilogue
     static constexpr int kBarStEmpty = 18 + 2 * NS;// [2], epilogue -> softmax
     static constexpr int kBarDrain = 20 + 2 * NS;
-    static constexpr int kNumBars = 21 + 2 * NS;
+    static constexpr int kBarXchg = 21 + 2 * NS;   // split: [2 stages][4 lane quarters], both halves arrive
+    static constexpr int kNumBars = 29 + 2 * NS;
     static constexpr int kSmemTmemSlot = kSmemBar + 8 * kNumBars;
     static constexpr int kSmemAbort = kSmemTmemSlot + 4;
     static constexpr int kSmemUsed = kSmemAbort + 4;
@@ -234,6 +275,17 @@ __device__ __forceinline__ float max128(const float* s) {
     a = fmax3(a, s[124], s[125]);
     b = fmax3(b, s[126], s[127]);
     return fmax3(fmaxf(a, b), c, d);
+}
+
+// Maximum of 32 registers.
+__device__ __forceinline__ float max32(const float* s) {
+    float a = s[0], b = s[1];
+#pragma unroll
+    for (int i = 2; i + 4 <= 32; i += 4) {
+        a = fmax3(a, s[i], s[i + 1]);
+        b = fmax3(b, s[i + 2], s[i + 3]);
+    }
+    return fmax3(fmaxf(a, b), s[30], s[31]);
 }
 
 // K/V tiles the query rows [row0, row0 + 128) need (0 when the tile starts
@@ -329,13 +381,13 @@ __device__ __forceinline__ long long o_offset(const Params& p, int bh, int row) 
     }
 }
 
-template <int D, int KIND, int NS, int QB, bool STRIDED>
-__global__ void __launch_bounds__(512, 1)
+template <int D, int KIND, int NS, int QB, bool SPLIT, bool STRIDED>
+__global__ void __launch_bounds__(SPLIT ? 768 : 512, 1)
 sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV,
                         const Params p) {
-    using C = Cfg<D, KIND, NS, QB>;
+    using C = Cfg<D, KIND, NS, QB, SPLIT>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -363,13 +415,14 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar(C::kBarSFull + s), 1);
-            mbar_init(bar(C::kBarPFull + s), kRows);
+            mbar_init(bar(C::kBarPFull + s), C::kSmThreadsPerStage);
             mbar_init(bar(C::kBarOFull + s), 1);
             mbar_init(bar(C::kBarOEmpty + s), kRows);
-            mbar_init(bar(C::kBarStFull + s), kRows);
+            mbar_init(bar(C::kBarStFull + s), C::kSmThreadsPerStage);
             mbar_init(bar(C::kBarStEmpty + s), kRows);
         }
         mbar_init(bar(C::kBarDrain), 1);
+        for (int i = 0; i < 8; ++i) mbar_init(bar(C::kBarXchg + i), 64);
         sts_u32(abort_addr, 0u);
         fence_barrier_init();
     }
@@ -389,8 +442,9 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     const uint32_t sQ = sbase + C::kSmemQ;
     const uint32_t sKV = sbase + C::kSmemKV;
 
-    if (warp >= 12) {
-        regs_dec<SDPA2_REGS_OTHER>();
+    if (warp >= C::kLoadWarp) {
+        if constexpr (SPLIT) regs_dec<SDPA2S_REGS_OTHER>();
+        else regs_dec<SDPA2_REGS_OTHER>();
         if (warp == C::kLoadWarp && lane == 0) {
             // ================= TMA producer ==============================
             bool ok = true;
@@ -546,10 +600,12 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                     for (int kk = 0; kk < C::kPvSteps; ++kk) {
                         const uint32_t off = (uint32_t)((kk * C::kPvKeysPerStep * C::kSwBytes) >> 4);
                         const uint32_t accum = (acc || kk > 0) ? 1u : 0u;
+                        constexpr int kPh = C::kPvStepsPerHalf;
+                        const uint32_t a_col = (uint32_t)((kk / kPh) * 64 + (kk % kPh) * 8);
                         if constexpr (KIND == K2_E4M3)
-                            mma_f8_ts(d_tmem, a_tmem + kk * 8, desc(bv + off), idesc_pv, accum);
+                            mma_f8_ts(d_tmem, a_tmem + a_col, desc(bv + off), idesc_pv, accum);
                         else
-                            mma_f16_ts(d_tmem, a_tmem + kk * 8, desc(bv + off), idesc_pv, accum);
+                            mma_f16_ts(d_tmem, a_tmem + a_col, desc(bv + off), idesc_pv, accum);
                     }
                 }
                 __syncwarp();
@@ -603,11 +659,22 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 ++t;
                 cur_next(p, kc);
             }
+            // Release commits of the previous step's K/V slots, deferred to
+            // the top of the next step: a tcgen05.commit holds the issuing
+            // thread until its queued MMAs have been taken by the pipe, and
+            // here the thread is about to wait for weights anyway.
+            int pend_v = -1, pend_k = -1;
+            auto release = [&]() {
+                if (pend_v >= 0) commit(bar(C::kBarKVEmpty + pend_v));
+                if (pend_k >= 0) commit(bar(C::kBarKVEmpty + pend_k));
+                pend_v = pend_k = -1;
+            };
             while (ok && vc.u.valid) {
                 const int slotV = t % NS;
                 ok = wait_all(bar(C::kBarKVFull + slotV), (uint32_t)(t / NS) & 1u,
                               0x22000u | (uint32_t)(t & 0xfff));
                 if (!ok) break;
+                if (SDPA2_DEFER_RELEASE) release();
                 const int slotK = (t + 1) % NS;
                 bool k_ready = false;
                 for (int s = 0; s < 2 && ok; ++s) {
@@ -622,17 +689,19 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                     }
                 }
                 if (!ok) break;
-                commit(bar(C::kBarKVEmpty + slotV));
+                pend_v = slotV;
                 ++t;
                 if (kc.u.valid) {
                     // a unit whose stage tiles are all inactive on this K
                     // tile does not exist (stage 1's count is the unit's)
-                    commit(bar(C::kBarKVEmpty + slotK));
+                    pend_k = slotK;
                     ++t;
                     cur_next(p, kc);
                 }
+                if (!SDPA2_DEFER_RELEASE) release();
                 cur_next(p, vc);
             }
+            if (ok) release();
             if (!ok) {
                 // make sure no MMA is still writing tensor memory at exit
                 commit(bar(C::kBarDrain));
@@ -645,7 +714,7 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             tc_fence_after();
             tmem_dealloc(tmem, kTmemCols);
         }
-    } else if (warp < 8) {
+    } else if (warp < C::kSoftmaxWarps && !SPLIT) {
         // ================= softmax, one stage per warp group ==============
         regs_inc<SDPA2_REGS_SOFTMAX>();
         const int s = warp >> 2;                 // stage
@@ -832,9 +901,180 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
         tc_fence_before();
         named_bar_sync(1, C::kTmemUsers);
+    } else if (warp < C::kSoftmaxWarps) {
+        // ================= softmax, split form: two warps per lane quarter
+        // and stage, each over 64 of a row's 128 scores ====================
+        // The two halves of a row share its reference max m_run (moved on
+        // both sides by the same decision) and keep their own row sums; once
+        // per tile they exchange their tile maxima (shared memory and a
+        // two-warp mbarrier), which is all a rescale decision needs.  A
+        // half's weights go into its own score columns, S_s + 64 h.
+        if constexpr (SPLIT) regs_inc<SDPA2S_REGS_SOFTMAX>();
+        const int s = warp / C::kSmWarpsPerStage;               // stage
+        const int quarter = warp & 3;                            // TMEM lane quarter
+        const int h = (warp % C::kSmWarpsPerStage) >> 2;         // key half
+        const int r = quarter * 32 + lane;                       // row within the stage tile
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        const uint32_t tS = tmem + lane_base + (s ? C::kColS1 : C::kColS0) + 64 * h;
+        const uint32_t tO = tmem + lane_base + (s ? C::kColO1 : C::kColO0) + h * (D / 2);
+        float* const xchg = reinterpret_cast<float*>(smem_raw + (sbase - raw) + C::kSmemXchg);
+        const uint32_t xbar = bar(C::kBarXchg + 4 * s + quarter);
+        const float sl = p.score_log2;
+        const uint64_t sl2 = f2_pack(sl, sl);
+        bool ok = true;
+        int cs = 0;   // tiles of this stage so far (S_full / P_full / exchange phase)
+        int ks = 0;   // units of this stage so far (stats phase)
+
+        // weights of 32 scores against nm2 = (-m + log2 of the P scale) x 2,
+        // rounded into chunk c of this half's P; returns the fp32 sum
+        auto exp_chunk = [&](const float* sc, uint64_t nm2, int c) -> uint64_t {
+            uint64_t sum2[2] = {0ull, 0ull};
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const uint64_t x2 = f2_fma(f2_pack(sc[2 * e], sc[2 * e + 1]), sl2, nm2);
+                float x0, x1;
+                f2_unpack(x2, x0, x1);
+                uint64_t p2;
+                if (poly_pair<KIND>(e))
+                    p2 = exp2_poly_x2(f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f)));
+                else
+                    p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+                sum2[e & 1] = f2_add(sum2[e & 1], p2);
+                float q0, q1;
+                f2_unpack(p2, q0, q1);
+                if constexpr (KIND == K2_E4M3) {
+                    if (e & 1) pk[e >> 1] |= pack_e4m3x2(q0, q1) << 16;
+                    else pk[e >> 1] = pack_e4m3x2(q0, q1);
+                } else {
+                    pk[e] = (KIND == K2_BF16) ? pack_bf16x2(q0, q1) : pack_f16x2(q0, q1);
+                }
+            }
+            if constexpr (KIND == K2_E4M3)
+                tmem_st8(tS + C::kPWordsPer32 * c, pk);
+            else
+                tmem_st16(tS + C::kPWordsPer32 * c, pk);
+            return f2_add(sum2[0], sum2[1]);
+        };
+
+        Unit u;
+        unit_first(p, u);
+        while (ok && u.valid) {
+            const int ns = stage_tiles(u, s);
+            if (ns == 0) {
+                unit_next(p, u);
+                continue;
+            }
+            const int row0 = (2 * u.m + s) * kRows;
+            const int row = row0 + r;
+            float m_run = -INFINITY;   // the row's reference max (log2 units), shared by the halves
+            float l_run = 0.0f;        // this half's sum of 2^(s*sl - m_run + kPLog2)
+            for (int j = 0; j < ns && ok; ++j, ++cs) {
+                ok = wait(bar(C::kBarSFull + s), (uint32_t)cs & 1u, abort_addr, status,
+                          0x30000u | (s << 12) | (uint32_t)(cs & 0xfff));
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                tc_fence_after();
+                const int key0 = j * kKeys + 64 * h;
+                const bool edge = (key0 + 64 > p.Sk) || (p.causal && key0 + 63 > row0 + p.causal_off);
+                int lim = 64;
+                if (edge) {
+                    lim = p.Sk - key0;
+                    if (p.causal) lim = min(lim, row + p.causal_off - key0 + 1);
+                }
+                // 32 scores of the half (chunk c), masked past Sk and after
+                // row + causal_off
+                auto load32 = [&](int c, float (&sc)[32]) {
+                    tmem_ld32(tS + 32 * c, sc);
+                    tmem_wait_ld();
+                    reg_fence32(sc);
+                    if (edge) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (32 * c + e >= lim) sc[e] = -INFINITY;
+                    }
+                };
+                // The max comes first, one chunk at a time; the scores are
+                // read again for the weights (the chunk-0 weights overwrite
+                // only chunk-0 columns), so 32 of them are live at a time.
+                float hm;
+                {
+                    float sc[32];
+                    load32(0, sc);
+                    hm = max32(sc);
+                    load32(1, sc);
+                    hm = fmaxf(hm, max32(sc));
+                }
+                // the row's tile max: this half's and the partner's, through
+                // shared memory (slots alternate with the tile parity)
+                const int par = cs & 1;
+                xchg[((s * 2 + par) * 2 + h) * kRows + r] = hm * sl;
+                mbar_arrive(xbar);
+                ok = wait(xbar, (uint32_t)par, abort_addr, status, 0x33000u | (s << 11) | (uint32_t)(cs & 0x7ff));
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                const float tmax = fmaxf(hm * sl, xchg[((s * 2 + par) * 2 + (1 - h)) * kRows + r]);
+                // lazy rescale, as in the one-warp form; both halves take the
+                // same decision on the same m_run
+                const bool need = tmax > m_run + C::kRescaleThreshold;
+                if (__any_sync(0xffffffffu, need)) {
+                    float alpha = 1.0f;
+                    if (need) {
+                        alpha = ex2_approx(m_run - tmax);   // 0 on the first live tile
+                        m_run = tmax;
+                    }
+                    l_run *= alpha;
+                    if (j > 0) {
+                        // this half's columns of O_s; O_s += P_s V of the
+                        // previous tile has completed
+#pragma unroll 1
+                        for (int c = 0; c < D / 64; ++c) {
+                            float o[32];
+                            tmem_ld32(tO + 32 * c, o);
+                            tmem_wait_ld();
+                            reg_fence32(o);
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+                            tmem_st32(tO + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(o));
+                        }
+                    }
+                }
+                const float nm = C::kPLog2 - m_run;
+                const uint64_t nm2 = f2_pack(nm, nm);
+                uint64_t acc;
+                {
+                    float sc[32];
+                    load32(0, sc);
+                    acc = exp_chunk(sc, nm2, 0);
+                    load32(1, sc);
+                    acc = f2_add(acc, exp_chunk(sc, nm2, 1));
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(C::kBarPFull + s));
+                float a0, a1;
+                f2_unpack(acc, a0, a1);
+                l_run += a0 + a1;
+            }
+            if (!ok) break;
+            if (ks > 0) {
+                ok = wait(bar(C::kBarStEmpty + s), (uint32_t)(ks - 1) & 1u, abort_addr, status,
+                          0x40000u | (s << 12) | (uint32_t)(ks & 0xfff));
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+            }
+            stats[((s * 2 + h) * kRows + r) * 2] = m_run;
+            stats[((s * 2 + h) * kRows + r) * 2 + 1] = l_run;
+            mbar_arrive(bar(C::kBarStFull + s));
+            ++ks;
+            unit_next(p, u);
+        }
+        tc_fence_before();
+        named_bar_sync(1, C::kTmemUsers);
     } else {
-        // ================= epilogue (warps 8-11) ==========================
-        regs_dec<SDPA2_REGS_EPILOGUE>();
+        // ================= epilogue (4 warps after the softmax warps) =====
+        if constexpr (SPLIT) regs_dec<SDPA2S_REGS_EPILOGUE>();
+        else regs_dec<SDPA2_REGS_EPILOGUE>();
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;       // row within the stage tile = TMEM lane
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
@@ -850,7 +1090,15 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                                 0x41000u | (s << 11) | (uint32_t)(ks[s] & 0x7ff));
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
-                const float m = stats[(s * kRows + r) * 2], l = stats[(s * kRows + r) * 2 + 1];
+                float m, l;
+                if constexpr (SPLIT) {
+                    // the halves share m; their sums add
+                    m = stats[((s * 2) * kRows + r) * 2];
+                    l = stats[((s * 2) * kRows + r) * 2 + 1] + stats[((s * 2 + 1) * kRows + r) * 2 + 1];
+                } else {
+                    m = stats[(s * kRows + r) * 2];
+                    l = stats[(s * kRows + r) * 2 + 1];
+                }
                 mbar_arrive(bar(C::kBarStEmpty + s));
                 const float cmul = p.out_mul / l;
                 const int row = (2 * u.m + s) * kRows + r;
