@@ -13,6 +13,7 @@
 #include "sdpa_fwd_sm100.cuh"
 #include "sdpa_bwd_sm100.cuh"
 #include "sdpa_bwd_tc_sm100.cuh"
+#include "sdpa_bwd_pipe_sm100.cuh"
 
 namespace {
 
@@ -334,6 +335,60 @@ int launch_bwd(const sdpa::BwdParams& bp, cudaStream_t stream) {
 #ifndef SDPA_BWD_TC
 #define SDPA_BWD_TC 1
 #endif
+// The pipelined tensor-core backward (sdpa_bwd_pipe_sm100.cuh): 1, or the
+// one-tile form (sdpa_bwd_tc_sm100.cuh): 0.
+#ifndef SDPA_BWD_PIPE
+#define SDPA_BWD_PIPE 1
+#endif
+
+template <int D, bool BF16>
+int launch_bwd_pipe(const void* q, const void* k, const void* v, const sdpa::BwdParams& bp,
+                    cudaStream_t stream) {
+    using C = sdpa::bwdp::Cfg<D>;
+    const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    // each kernel keeps one pair resident (128-row boxes) and streams the
+    // other in 64-row boxes
+    CUtensorMap tq128, tdo128, tk128, tv128, tq64, tdo64, tk64, tv64;
+    const View vq = bhsd(bp.Hq, bp.Sq, D), vk = bhsd(bp.Hkv, bp.Sk, D);
+    for (int rows : {128, 64}) {
+        CUtensorMap* mq = rows == 128 ? &tq128 : &tq64;
+        CUtensorMap* mdo = rows == 128 ? &tdo128 : &tdo64;
+        CUtensorMap* mk = rows == 128 ? &tk128 : &tk64;
+        CUtensorMap* mv = rows == 128 ? &tv128 : &tv64;
+        if (!encode_view(mq, dt, 2, q, D, bp.Sq, bp.Hq, bp.B, vq, C::kElemsPerSw, true, rows) ||
+            !encode_view(mdo, dt, 2, bp.dout, D, bp.Sq, bp.Hq, bp.B, vq, C::kElemsPerSw, true, rows) ||
+            !encode_view(mk, dt, 2, k, D, bp.Sk, bp.Hkv, bp.B, vk, C::kElemsPerSw, true, rows) ||
+            !encode_view(mv, dt, 2, v, D, bp.Sk, bp.Hkv, bp.B, vk, C::kElemsPerSw, true, rows))
+            return SDPA_ERR_CUDA;
+    }
+    sdpa::BwdTcParams tp;
+    tp.o = bp.o; tp.dout = bp.dout; tp.lse = bp.lse; tp.delta = bp.delta;
+    tp.dq = bp.dq; tp.dk = bp.dk; tp.dv = bp.dv;
+    tp.B = bp.B; tp.Hq = bp.Hq; tp.Hkv = bp.Hkv; tp.Sq = bp.Sq; tp.Sk = bp.Sk; tp.group = bp.group;
+    tp.causal = bp.causal; tp.causal_off = bp.causal_off; tp.scale = bp.scale;
+    tp.dq_mul = bp.dq_mul; tp.dk_mul = bp.dk_mul; tp.dv_mul = bp.dv_mul; tp.d_mul = bp.d_mul;
+    auto kdkdv = sdpa::bwdp::sdpa_bwd_dkdv_pipe_kernel<D, BF16>;
+    auto kdq = sdpa::bwdp::sdpa_bwd_dq_pipe_kernel<D, BF16>;
+    static bool attr_set[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        if (cudaFuncSetAttribute(kdkdv, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+                cudaSuccess)
+            return SDPA_ERR_CUDA;
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+    const dim3 gkv((bp.Sk + 127) / 128, bp.B * bp.Hkv);
+    const dim3 gq((bp.Sq + 127) / 128, bp.B * bp.Hq);
+    // dQ first: it writes D of every row, which the dK/dV kernel reads
+    kdq<<<gq, sdpa::bwdp::kThreads, C::kSmemBytes, stream>>>(tq128, tk64, tv64, tdo128, tp);
+    if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
+    kdkdv<<<gkv, sdpa::bwdp::kThreads, C::kSmemBytes, stream>>>(tq64, tk128, tv128, tdo64, tp);
+    return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
 template <int D, bool BF16>
 int launch_bwd_tc(const void* q, const void* k, const void* v, const sdpa::BwdParams& bp,
                   cudaStream_t stream) {
@@ -405,6 +460,11 @@ extern "C" int sdpa_bwd(const void* q, const void* k, const void* v, const void*
     const bool bf = dtype == SDPA_BF16;
     if (d == 32) return bf ? launch_bwd<32, true>(bp, s) : launch_bwd<32, false>(bp, s);
     if (SDPA_BWD_TC) {
+        if (SDPA_BWD_PIPE) {
+            if (d == 64)
+                return bf ? launch_bwd_pipe<64, true>(q, k, v, bp, s) : launch_bwd_pipe<64, false>(q, k, v, bp, s);
+            return bf ? launch_bwd_pipe<128, true>(q, k, v, bp, s) : launch_bwd_pipe<128, false>(q, k, v, bp, s);
+        }
         if (d == 64) return bf ? launch_bwd_tc<64, true>(q, k, v, bp, s) : launch_bwd_tc<64, false>(q, k, v, bp, s);
         return bf ? launch_bwd_tc<128, true>(q, k, v, bp, s) : launch_bwd_tc<128, false>(q, k, v, bp, s);
     }
@@ -548,7 +608,8 @@ extern "C" int sdpa_bwd_fp8(const void* q8, const void* k8, const void* v8, cons
     bp.dk_mul = scale * descale_do * descale_v * descale_q;
     bp.dv_mul = descale_do;
     bp.d_mul = 1.0f / descale_v;
-    return launch_bwd_tc<128, true>(q16, k16, v16, bp, s);
+    return SDPA_BWD_PIPE ? launch_bwd_pipe<128, true>(q16, k16, v16, bp, s)
+                         : launch_bwd_tc<128, true>(q16, k16, v16, bp, s);
 }
 
 extern "C" const char* sdpa_strerror(int status) {
