@@ -275,7 +275,7 @@ def run_backward(args, w):
         "data": "synthetic", "config": dict(w.describe(), pass_="bwd"),
         "roofline": {"bound": bound, "achieved": value, "peak": peak, "unit": "TFLOP/s",
                      "frac": value / peak, "traffic": load_traffic("bwd:" + w.name),
-                     "traffic_kernel": "sdpa_bwd_dkdv_tc_kernel (the larger of the two launches)",
+                     "traffic_kernel": "sdpa_bwd_dkdv_pipe_kernel (the larger of the two launches)",
                      "peak_source": peak_source},
         "clocks": clk, "gpu_launches": 2 * args.steps}))
 

@@ -12,7 +12,6 @@
 #include "sdpa_host.h"
 #include "sdpa_fwd_sm100.cuh"
 #include "sdpa_bwd_sm100.cuh"
-#include "sdpa_bwd_tc_sm100.cuh"
 #include "sdpa_bwd_pipe_sm100.cuh"
 
 namespace {
@@ -330,17 +329,8 @@ int launch_bwd(const sdpa::BwdParams& bp, cudaStream_t stream) {
     return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
 }
 
-// Tensor-core backward (head dims 64, 128): 3-D maps over (d, S, B*H) of
-// Q, K, V, dO, then the dK/dV and dQ kernels.
-#ifndef SDPA_BWD_TC
-#define SDPA_BWD_TC 1
-#endif
-// The pipelined tensor-core backward (sdpa_bwd_pipe_sm100.cuh): 1, or the
-// one-tile form (sdpa_bwd_tc_sm100.cuh): 0.
-#ifndef SDPA_BWD_PIPE
-#define SDPA_BWD_PIPE 1
-#endif
-
+// Tensor-core backward (head dims 64, 128; sdpa_bwd_pipe_sm100.cuh): 3-D
+// maps over (d, S, B*H) of Q, K, V, dO, then the dQ and dK/dV kernels.
 template <int D, bool BF16>
 int launch_bwd_pipe(const void* q, const void* k, const void* v, const sdpa::BwdParams& bp,
                     cudaStream_t stream) {
@@ -389,46 +379,6 @@ int launch_bwd_pipe(const void* q, const void* k, const void* v, const sdpa::Bwd
     return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
 }
 
-template <int D, bool BF16>
-int launch_bwd_tc(const void* q, const void* k, const void* v, const sdpa::BwdParams& bp,
-                  cudaStream_t stream) {
-    using C = sdpa::BtCfg<D>;
-    const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-    CUtensorMap tq, tk, tv, tdo;
-    const View vq = bhsd(bp.Hq, bp.Sq, D), vk = bhsd(bp.Hkv, bp.Sk, D);
-    if (!encode_view(&tq, dt, 2, q, D, bp.Sq, bp.Hq, bp.B, vq, C::kElemsPerSw, true) ||
-        !encode_view(&tk, dt, 2, k, D, bp.Sk, bp.Hkv, bp.B, vk, C::kElemsPerSw, true) ||
-        !encode_view(&tv, dt, 2, v, D, bp.Sk, bp.Hkv, bp.B, vk, C::kElemsPerSw, true) ||
-        !encode_view(&tdo, dt, 2, bp.dout, D, bp.Sq, bp.Hq, bp.B, vq, C::kElemsPerSw, true))
-        return SDPA_ERR_CUDA;
-    sdpa::BwdTcParams tp;
-    tp.o = bp.o; tp.dout = bp.dout; tp.lse = bp.lse; tp.delta = bp.delta;
-    tp.dq = bp.dq; tp.dk = bp.dk; tp.dv = bp.dv;
-    tp.B = bp.B; tp.Hq = bp.Hq; tp.Hkv = bp.Hkv; tp.Sq = bp.Sq; tp.Sk = bp.Sk; tp.group = bp.group;
-    tp.causal = bp.causal; tp.causal_off = bp.causal_off; tp.scale = bp.scale;
-    tp.dq_mul = bp.dq_mul; tp.dk_mul = bp.dk_mul; tp.dv_mul = bp.dv_mul; tp.d_mul = bp.d_mul;
-    auto kdkdv = sdpa::sdpa_bwd_dkdv_tc_kernel<D, BF16>;
-    auto kdq = sdpa::sdpa_bwd_dq_tc_kernel<D, BF16>;
-    static bool attr_set[64];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-        if (cudaFuncSetAttribute(kdkdv, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
-                cudaSuccess ||
-            cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
-                cudaSuccess)
-            return SDPA_ERR_CUDA;
-        if (dev >= 0 && dev < 64) attr_set[dev] = true;
-    }
-    const dim3 gkv((bp.Sk + 127) / 128, bp.B * bp.Hkv);
-    const dim3 gq((bp.Sq + 127) / 128, bp.B * bp.Hq);
-    // dQ first: it writes D of every row, which the dK/dV kernel reads
-    kdq<<<gq, sdpa::kBtThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, tp);
-    if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
-    kdkdv<<<gkv, sdpa::kBtThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, tp);
-    return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
-}
-
 }  // namespace
 
 extern "C" int sdpa_bwd(const void* q, const void* k, const void* v, const void* o,
@@ -459,17 +409,8 @@ extern "C" int sdpa_bwd(const void* q, const void* k, const void* v, const void*
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool bf = dtype == SDPA_BF16;
     if (d == 32) return bf ? launch_bwd<32, true>(bp, s) : launch_bwd<32, false>(bp, s);
-    if (SDPA_BWD_TC) {
-        if (SDPA_BWD_PIPE) {
-            if (d == 64)
-                return bf ? launch_bwd_pipe<64, true>(q, k, v, bp, s) : launch_bwd_pipe<64, false>(q, k, v, bp, s);
-            return bf ? launch_bwd_pipe<128, true>(q, k, v, bp, s) : launch_bwd_pipe<128, false>(q, k, v, bp, s);
-        }
-        if (d == 64) return bf ? launch_bwd_tc<64, true>(q, k, v, bp, s) : launch_bwd_tc<64, false>(q, k, v, bp, s);
-        return bf ? launch_bwd_tc<128, true>(q, k, v, bp, s) : launch_bwd_tc<128, false>(q, k, v, bp, s);
-    }
-    if (d == 64) return bf ? launch_bwd<64, true>(bp, s) : launch_bwd<64, false>(bp, s);
-    return bf ? launch_bwd<128, true>(bp, s) : launch_bwd<128, false>(bp, s);
+    if (d == 64) return bf ? launch_bwd_pipe<64, true>(q, k, v, bp, s) : launch_bwd_pipe<64, false>(q, k, v, bp, s);
+    return bf ? launch_bwd_pipe<128, true>(q, k, v, bp, s) : launch_bwd_pipe<128, false>(q, k, v, bp, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -608,8 +549,7 @@ extern "C" int sdpa_bwd_fp8(const void* q8, const void* k8, const void* v8, cons
     bp.dk_mul = scale * descale_do * descale_v * descale_q;
     bp.dv_mul = descale_do;
     bp.d_mul = 1.0f / descale_v;
-    return SDPA_BWD_PIPE ? launch_bwd_pipe<128, true>(q16, k16, v16, bp, s)
-                         : launch_bwd_tc<128, true>(q16, k16, v16, bp, s);
+    return launch_bwd_pipe<128, true>(q16, k16, v16, bp, s);
 }
 
 extern "C" const char* sdpa_strerror(int status) {

@@ -5,8 +5,7 @@
 // 3): the weights are recomputed from the kept row statistics,
 //   P = exp(scale * S - LSE),  dP = dO V^T,  D_i = dO_i . O_i,
 //   dS = P * (dP - D),  dQ = scale * dS K,  dK = scale * dS^T Q,  dV = P^T dO,
-// the same arithmetic as sdpa_bwd_tc_sm100.cuh, arranged so that the tensor
-// pipe and the elementwise warps overlap.
+// arranged so that the tensor pipe and the elementwise warps overlap.
 //
 // Both kernels walk their streamed operand in steps of 64 rows, so that the
 // two products the elementwise step reads (S and dP, 64 fp32 columns each)
@@ -45,9 +44,65 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include "sm100_ptx.cuh"
-#include "sdpa_bwd_tc_sm100.cuh"
 
 namespace sdpa {
+
+struct BwdTcParams {
+    const void* o;                   // [B,Hq,Sq,D] (for D_i = dO_i . O_i)
+    const void* dout;                // [B,Hq,Sq,D]
+    const float* lse;                // [B,Hq,Sq]
+    float* delta;                    // [B,Hq,Sq] D_i, written by the dQ kernel
+    void *dq, *dk, *dv;
+    int B, Hq, Hkv, Sq, Sk, group;
+    int causal, causal_off;
+    float scale;                     // score scale (P = exp(scale * s - LSE))
+    // output multipliers: dQ = dq_mul * (dS K), dK = dk_mul * (dS^T Q),
+    // dV = dv_mul * (P^T dO), and D = d_mul * (dO . O); 16-bit inputs use
+    // scale, scale, 1, 1
+    float dq_mul, dk_mul, dv_mul, d_mul;
+};
+
+template <bool BF16>
+__device__ __forceinline__ uint32_t bt_pack(float a, float b) {
+    return BF16 ? pack_bf16x2(a, b) : pack_f16x2(a, b);
+}
+
+template <bool BF16>
+__device__ __forceinline__ float2 bt_unpack(uint32_t w) {
+    if constexpr (BF16)
+        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    else
+        return __half22float2(*reinterpret_cast<const __half2*>(&w));
+}
+
+// Half `half` (columns [half*D/2, (half+1)*D/2)) of D_i = dO_i . O_i of row
+// `row` (0 past the end); 16-byte loads
+template <int D, bool BF16>
+__device__ __forceinline__ float bt_row_dot(const BwdTcParams& p, size_t head, int row, int half) {
+    if (row >= p.Sq) return 0.0f;
+    const size_t off = head + (size_t)row * D + (size_t)half * (D / 2);
+    const uint4* g = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.dout) + off);
+    const uint4* o = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.o) + off);
+    uint4 gv[D / 16], ov[D / 16];
+#pragma unroll
+    for (int v = 0; v < D / 16; ++v) {
+        gv[v] = g[v];
+        ov[v] = o[v];
+    }
+    float acc = 0.0f;
+#pragma unroll
+    for (int v = 0; v < D / 16; ++v) {
+        const uint32_t gw[4] = {gv[v].x, gv[v].y, gv[v].z, gv[v].w};
+        const uint32_t ow[4] = {ov[v].x, ov[v].y, ov[v].z, ov[v].w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const float2 a = bt_unpack<BF16>(gw[u]), b = bt_unpack<BF16>(ow[u]);
+            acc = fmaf(a.x, b.x, fmaf(a.y, b.y, acc));
+        }
+    }
+    return acc;
+}
+
 namespace bwdp {
 
 constexpr int kEwWarps = 16;      // elementwise warps 0-15

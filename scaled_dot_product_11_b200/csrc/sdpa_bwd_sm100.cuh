@@ -17,7 +17,8 @@
 //                         head), looping over the key tiles they see.
 // Arithmetic is fp32 on the CUDA cores (register-blocked 4x4 tiles from
 // shared memory); inputs and outputs are bf16 or fp16, contiguous
-// [B, H, S, d].
+// [B, H, S, d].  This form serves head dim 32; head dims 64 and 128 take the
+// tensor-core kernels of sdpa_bwd_pipe_sm100.cuh.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
