@@ -1,24 +1,29 @@
 """Model check of the backward kernels' synchronisation protocol (no GPU).
 
 compute-sanitizer is not available for these kernels, so the protocol they
-follow -- mbarrier phases, the double-buffered streamed tiles, the queued MMA
-commits and the CTA barriers -- is restated here as a small discrete-event
-model and run under many random interleavings of the warps, the TMA engine
-and the in-order tensor pipe.  The model checks, at every step:
+follow -- mbarrier phases, the ring of streamed 64-row tiles, the two TMEM
+buffers of S and dP, the separate commits of S and dP, and the in-order
+tensor pipe -- is restated here as a small discrete-event model and run under
+many random interleavings of the warps, the TMA engine and the tensor pipe.
+The model checks, at every step:
 
 - a parity wait only succeeds on the phase it means (never one phase early,
   never aliased two phases late);
-- a TMA copy never lands in a buffer an issued, unfinished MMA still reads,
-  and every MMA reads the tile of its own step;
-- the elementwise warps read S/dP only after the MMAs that produce them
-  completed, and the accumulating MMAs read P/dS only after every warp wrote
-  them;
-- the per-step statistics are not overwritten while a warp still reads them;
-- every role finishes (no deadlock).
+- a TMA copy never lands in a ring slot an issued, unfinished product still
+  reads, and every product reads the tiles of its own step;
+- the elementwise warps read S (and dP) of a buffer only after the products
+  that write them completed, and only while they hold their own step;
+- a product that overwrites S or dP of a buffer never runs before the
+  accumulating product that reads P or dS from it, and the accumulating
+  products read P/dS only after every elementwise warp wrote them;
+- the per-step statistics in a ring slot are not rewritten while a warp still
+  reads them;
+- every role finishes (no deadlock) and nothing is in flight at exit.
 
-Planted mistakes (a copy issued before its buffer is free, a wrong parity)
-must be caught, so the model is known to be able to fail.  Each role mirrors
-the kernel it is named after in csrc/sdpa_bwd_tc_sm100.cuh.
+Planted mistakes (a copy issued before its slot is free, a wrong parity, the
+next S issued before the product that reads the buffer) must be caught, so the
+model is known to be able to fail.  Each role mirrors the warp of the same name
+in csrc/sdpa_bwd_pipe_sm100.cuh.
 """
 import random
 
@@ -135,159 +140,176 @@ def run(machine, roles, limit=400000):
     raise ModelError("no progress: deadlock")
 
 
-# ---------------------------------------------------------------------------
-# dK/dV kernel: K, V once; Q/dO tiles of step s in buffer s & 1; one commit
-# per step queues dV/dK of step s and S^T/dP^T of step s+1; LSE/D of the
-# step's rows in one shared buffer, rewritten by warps 1-7 after the barrier
-# that ends the step's reads.
-# ---------------------------------------------------------------------------
-def dkdv_model(nsteps, seed, plant=None):
-    m = Machine(seed)
-    bar_kv, bar_mma = Bar("kv"), Bar("mma")
-    bar_in = [Bar("in0"), Bar("in1")]
-    tm = {"S": None, "P": None, "P_writers": set()}     # TMEM S^T/dP^T and P^T/dS^T
-    stats = {"step": None, "readers": set()}
+RING = 4          # ring slots of 64-row tile pairs (head dim 128)
+N_EW = 4          # elementwise warps modelled (the kernel has 16, one arrival each)
 
-    def mma1_done(s):
+
+def pipe_model(nsteps, seed, kind, plant=None):
+    """kind "dkdv": K, V resident; Q, dO and the step's statistics streamed;
+    per step dV(st) [reads S_b], S(st+2) [writes S_b], dK(st) [reads dP_b],
+    ring slot released, dP(st+2) [writes dP_b].  kind "dq": Q, dO resident;
+    K, V streamed; per step dQ(jt) [reads S_b], ring slot released, S(jt+2),
+    dP(jt+2)."""
+    m = Machine(seed)
+    res_full, done = Bar("res_full"), Bar("done")
+    ring_full = [Bar("ring_full%d" % i) for i in range(RING)]
+    ring_empty = [Bar("ring_empty%d" % i) for i in range(RING)]
+    s_full = [Bar("s_full%d" % b) for b in range(2)]
+    dp_full = [Bar("dp_full%d" % b) for b in range(2)]
+    p_full = [Bar("p_full%d" % b, count=N_EW) for b in range(2)]
+    # TMEM buffers, per column chunk (warp w owns chunk w of each buffer):
+    # what the chunk holds ("S"/"P" or "dP"/"dS", step); and per buffer the
+    # unfinished products reading it
+    tm = {(x, b, w): None for x in ("S", "D") for b in range(2) for w in range(N_EW)}
+    tm_readers = {(x, b): 0 for x in ("S", "D") for b in range(2)}
+    stats = [{"step": None, "readers": set()} for _ in range(RING)]
+    stream = "q" if kind == "dkdv" else "kv"
+
+    def par(intended):
+        """Parity of completion number `intended` (a planted mistake flips it)."""
+        p = intended & 1
+        return 1 - p if plant == "wrong_parity" else p
+
+    def write_tm(key, step):      # a product overwriting S_b or dP_b completes
         def f():
-            tm["S"] = s
+            check(tm_readers[key] == 0, "S/dP overwritten before the product reading P/dS ran", key, step)
+            for w in range(N_EW):
+                tm[key + (w,)] = ("S" if key[0] == "S" else "dP", step)
         return f
 
-    def issue_qk(s):           # warp 0: wait for step s's tiles, queue S^T, dP^T
-        b = s & 1
-        par = (s >> 1) & 1 if plant != "wrong_parity" else 1 - ((s >> 1) & 1)
-        while not bar_in[b].ready(par, s >> 1):
-            yield
-        m.mma([("q", b)], s, mma1_done(s))
+    def read_tm(keys, step):      # an accumulating product reads P/dS of `step`
+        for k in keys:
+            want = ("P" if k[0] == "S" else "dS", step)
+            for w in range(N_EW):
+                check(tm[k + (w,)] == want, "accumulating product before every warp wrote P/dS", k, w, step,
+                      tm[k + (w,)])
+            tm_readers[k] += 1
 
-    def warp(w):
-        if w == 0:
-            bar_kv.arrive(tx=1)
-            m.tma.append((bar_kv, "kv", 0))
-            if nsteps > 0:
-                m.copy(bar_in[0], ("q", 0), 0)
-        while not bar_kv.ready(0, 0):
-            yield
-        yield from m.syncthreads()
-        if nsteps > 0:
-            if w != 0:
-                stats["step"] = 0
-            if w == 0:
-                yield from issue_qk(0)
-                m.commit(bar_mma)
-        for it in range(nsteps):
-            if plant == "early_copy" and w == 0 and it + 1 < nsteps:
-                m.copy(bar_in[(it + 1) & 1], ("q", (it + 1) & 1), it + 1)
-            while not bar_mma.ready(it & 1, it):
-                yield
-            yield from m.syncthreads()
-            if w == 0 and it + 1 < nsteps and plant != "early_copy":
-                m.copy(bar_in[(it + 1) & 1], ("q", (it + 1) & 1), it + 1)
-            # elementwise: S^T/dP^T of step it, statistics of step it
-            check(tm["S"] == it, "elementwise reads S before its MMAs", w, it, tm["S"])
-            check(stats["step"] == it, "statistics of another step", w, it, stats["step"])
-            stats["readers"].add(w)
-            yield
-            stats["readers"].discard(w)
-            if tm["P"] != it:
-                tm["P"], tm["P_writers"] = it, set()
-            tm["P_writers"].add(w)
-            yield from m.syncthreads()
-            if w == 0:
-                check(tm["P_writers"] == set(range(8)), "dV/dK MMAs before every warp wrote P", it)
-                m.mma([("q", it & 1)], it)
-                if it + 1 < nsteps:
-                    yield from issue_qk(it + 1)
-                m.commit(bar_mma)
-            if it + 1 < nsteps and w != 0:
-                check(not stats["readers"], "statistics rewritten while read", w, it)
-                stats["step"] = it + 1
-        if nsteps > 0:
-            while not bar_mma.ready(nsteps & 1, nsteps):
-                yield
-        yield from m.syncthreads()
+        def f():
+            for k in keys:
+                tm_readers[k] -= 1
+        return f
 
-    run(m, [warp(w) for w in range(8)])
+    def producer():
+        m.buf["res"] = None
+        res_full.arrive(tx=1)
+        m.tma.append((res_full, "res", 0))
+        for st in range(nsteps):
+            slot = st % RING
+            if plant == "early_copy" and st >= RING:
+                pass
+            elif st >= RING:
+                n = st // RING - 1
+                while not ring_empty[slot].ready(par(n), n):
+                    yield
+            if kind == "dkdv":
+                check(not stats[slot]["readers"], "statistics rewritten while read", slot, st)
+                stats[slot]["step"] = st
+            m.copy(ring_full[slot], (stream, slot), st)
+            yield
+
+    def mma():
+        while not res_full.ready(0, 0):
+            yield
+
+        def wait_in(st):
+            n = st // RING
+            while not ring_full[st % RING].ready(par(n), n):
+                yield
+
+        def issue_s(st):
+            b = st & 1
+            m.mma([(stream, st % RING)], st, write_tm(("S", b), st))
+            m.commit(s_full[b])
+
+        def issue_dp(st):
+            b = st & 1
+            m.mma([(stream, st % RING)], st, write_tm(("D", b), st))
+            m.commit(dp_full[b])
+
+        for st in range(min(2, nsteps)):
+            yield from wait_in(st)
+            issue_s(st)
+            issue_dp(st)
+        for st in range(nsteps):
+            b, slot, nxt = st & 1, st % RING, st + 2 < nsteps
+            n = st >> 1
+            while not p_full[b].ready(par(n), n):
+                yield
+            if nxt:
+                yield from wait_in(st + 2)
+            if kind == "dkdv":
+                if plant == "early_overwrite" and nxt:
+                    issue_s(st + 2)
+                m.mma([(stream, slot)], st, read_tm([("S", b)], st))        # dV += P^T dO
+                if nxt and plant != "early_overwrite":
+                    issue_s(st + 2)
+                m.mma([(stream, slot)], st, read_tm([("D", b)], st))        # dK += dS^T Q
+                m.commit(ring_empty[slot])
+                if nxt:
+                    issue_dp(st + 2)
+            else:
+                if plant == "early_overwrite" and nxt:
+                    issue_s(st + 2)
+                m.mma([(stream, slot)], st, read_tm([("S", b)], st))        # dQ += dS K
+                m.commit(ring_empty[slot])
+                if nxt:
+                    if plant != "early_overwrite":
+                        issue_s(st + 2)
+                    issue_dp(st + 2)
+            yield
+        m.commit(done)
+
+    def elementwise(w):
+        for st in range(nsteps):
+            b, slot, n = st & 1, st % RING, st >> 1
+            if kind == "dkdv":
+                nr = st // RING
+                while not ring_full[slot].ready(par(nr), nr):
+                    yield
+                check(stats[slot]["step"] == st, "statistics of another step", w, st, stats[slot]["step"])
+                stats[slot]["readers"].add(w)
+            while not s_full[b].ready(par(n), n):
+                yield
+            check(tm[("S", b, w)] == ("S", st), "elementwise reads S before its product", w, st, tm[("S", b, w)])
+            yield
+            # P^T (dK/dV) written over this warp's chunk of S_b now; dS (dQ)
+            # after dP
+            if kind == "dkdv":
+                tm[("S", b, w)] = ("P", st)
+            while not dp_full[b].ready(par(n), n):
+                yield
+            check(tm[("D", b, w)] == ("dP", st), "elementwise reads dP before its product", w, st, tm[("D", b, w)])
+            yield
+            if kind == "dkdv":
+                tm[("D", b, w)] = ("dS", st)
+                stats[slot]["readers"].discard(w)
+            else:
+                tm[("S", b, w)] = ("P", st)
+            p_full[b].arrive()
+            yield
+        if nsteps > 0:
+            while not done.ready(0, 0):
+                yield
+
+    run(m, [producer(), mma()] + [elementwise(w) for w in range(N_EW)])
     check(not m.pipe and not m.tma, "work left in flight at exit")
 
 
-# ---------------------------------------------------------------------------
-# dQ kernel: Q, dO once; K/V tiles of tile j in buffer j & 1; one commit per
-# tile queues dQ of tile j and S/dP of tile j+1.
-# ---------------------------------------------------------------------------
-def dq_model(ntiles, seed, plant=None):
-    m = Machine(seed)
-    bar_in, bar_mma = Bar("in"), Bar("mma")
-    bar_kv = [Bar("kv0"), Bar("kv1")]
-    tm = {"S": None, "P_writers": set(), "P": None}
-
-    def mma1_done(j):
-        def f():
-            tm["S"] = j
-        return f
-
-    def issue_qk(j):
-        b = j & 1
-        par = (j >> 1) & 1 if plant != "wrong_parity" else 1 - ((j >> 1) & 1)
-        while not bar_kv[b].ready(par, j >> 1):
-            yield
-        m.mma([("kv", b)], j, mma1_done(j))
-
-    def warp(w):
-        if w == 0:
-            bar_in.arrive(tx=1)
-            m.tma.append((bar_in, "q", 0))
-            if ntiles > 0:
-                m.copy(bar_kv[0], ("kv", 0), 0)
-        while not bar_in.ready(0, 0):
-            yield
-        yield from m.syncthreads()
-        if ntiles > 0 and w == 0:
-            yield from issue_qk(0)
-            m.commit(bar_mma)
-        for jt in range(ntiles):
-            if plant == "early_copy" and w == 0 and jt + 1 < ntiles:
-                m.copy(bar_kv[(jt + 1) & 1], ("kv", (jt + 1) & 1), jt + 1)
-            while not bar_mma.ready(jt & 1, jt):
-                yield
-            yield from m.syncthreads()
-            if w == 0 and jt + 1 < ntiles and plant != "early_copy":
-                m.copy(bar_kv[(jt + 1) & 1], ("kv", (jt + 1) & 1), jt + 1)
-            check(tm["S"] == jt, "elementwise reads S before its MMAs", w, jt, tm["S"])
-            yield
-            if tm["P"] != jt:
-                tm["P"], tm["P_writers"] = jt, set()
-            tm["P_writers"].add(w)
-            yield from m.syncthreads()
-            if w == 0:
-                check(tm["P_writers"] == set(range(8)), "dQ MMAs before every warp wrote dS", jt)
-                m.mma([("kv", jt & 1)], jt)
-                if jt + 1 < ntiles:
-                    yield from issue_qk(jt + 1)
-                m.commit(bar_mma)
-        if ntiles > 0:
-            while not bar_mma.ready(ntiles & 1, ntiles):
-                yield
-        yield from m.syncthreads()
-
-    run(m, [warp(w) for w in range(8)])
-    check(not m.pipe and not m.tma, "work left in flight at exit")
-
-
-@pytest.mark.parametrize("model", [dkdv_model, dq_model], ids=["dkdv", "dq"])
-@pytest.mark.parametrize("n", [0, 1, 2, 3, 4, 7])
-def test_protocol_holds_under_random_interleavings(model, n):
+@pytest.mark.parametrize("kind", ["dkdv", "dq"])
+@pytest.mark.parametrize("n", [0, 1, 2, 3, 4, 5, 9])
+def test_protocol_holds_under_random_interleavings(kind, n):
     for seed in range(30):
-        model(n, seed)
+        pipe_model(n, seed, kind)
 
 
-@pytest.mark.parametrize("model", [dkdv_model, dq_model], ids=["dkdv", "dq"])
-@pytest.mark.parametrize("plant", ["early_copy", "wrong_parity"])
-def test_planted_mistakes_are_caught(model, plant):
+@pytest.mark.parametrize("kind", ["dkdv", "dq"])
+@pytest.mark.parametrize("plant", ["early_copy", "wrong_parity", "early_overwrite"])
+def test_planted_mistakes_are_caught(kind, plant):
     caught = 0
     for seed in range(20):
         try:
-            model(5, seed, plant=plant)
+            pipe_model(7, seed, kind, plant=plant)
         except ModelError:
             caught += 1
     assert caught > 0, plant
