@@ -54,6 +54,15 @@ CASES = [
     (1, 2, 2, 77, 77, 32, 1, "fp16"),        # head dim 32
     (1, 3, 3, 65, 190, 128, 0, "fp16"),
     (1, 4, 4, 1024, 1024, 128, 1, "bf16"),   # many tiles
+    # the tensor-core kernels walk 64-row steps through a ring of 4 (d=128)
+    # or 8 (d=64) slots, with S and dP double-buffered
+    (1, 2, 2, 40, 40, 128, 0, "bf16"),       # one partial step
+    (1, 2, 2, 33, 33, 64, 1, "fp16"),        # one partial causal step
+    (1, 2, 2, 320, 320, 128, 1, "bf16"),     # causal starts on 64-row steps inside 128-key tiles
+    (1, 8, 2, 257, 257, 128, 1, "bf16"),     # GQA: steps of four query heads wrap the ring
+    (1, 2, 2, 190, 450, 128, 2, "bf16"),     # end-aligned causal, Sk > Sq
+    (2, 2, 2, 130, 131, 64, 2, "fp16"),      # ragged rows and keys, d=64, end-aligned causal
+    (1, 2, 1, 1536, 1536, 64, 0, "bf16"),    # long: the 8-slot ring wraps many times
 ]
 
 
