@@ -12,10 +12,11 @@
 // fit twice in tensor memory next to the accumulators: while the sixteen
 // elementwise warps turn step t's S, dP into P, dS (written back over them,
 // 16-bit), the tensor pipe runs step t-1's accumulating products and step
-// t+1's S and dP.  A TMA producer warp streams the 64-row tiles through a
-// ring; an MMA warp issues every product from one elected lane (in issue
-// order, so a product that overwrites a buffer cannot overtake the one that
-// reads it).
+// t+1's S and dP (committed separately, so that step t+1's exponentials can
+// start before its dP lands).  A TMA producer warp streams the 64-row tiles
+// through a ring; an MMA warp issues every product from one elected lane (in
+// issue order, so a product that overwrites a buffer cannot overtake the one
+// that reads it, which is issued just before it).
 //
 // dK/dV kernel, one CTA per 128 keys of one (batch, K/V head); TMEM lane =
 // key; steps = 64 query rows of one query head of the group:
