@@ -336,21 +336,18 @@ int launch_bwd_pipe(const void* q, const void* k, const void* v, const sdpa::Bwd
                     cudaStream_t stream) {
     using C = sdpa::bwdp::Cfg<D>;
     const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-    // each kernel keeps one pair resident (128-row boxes) and streams the
-    // other in 64-row boxes
-    CUtensorMap tq128, tdo128, tk128, tv128, tq64, tdo64, tk64, tv64;
+    // the dK/dV kernel streams Q, dO in 64-row boxes; everything else moves
+    // in 128-row boxes
+    CUtensorMap tq128, tdo128, tk128, tv128, tq64, tdo64;
     const View vq = bhsd(bp.Hq, bp.Sq, D), vk = bhsd(bp.Hkv, bp.Sk, D);
-    for (int rows : {128, 64}) {
-        CUtensorMap* mq = rows == 128 ? &tq128 : &tq64;
-        CUtensorMap* mdo = rows == 128 ? &tdo128 : &tdo64;
-        CUtensorMap* mk = rows == 128 ? &tk128 : &tk64;
-        CUtensorMap* mv = rows == 128 ? &tv128 : &tv64;
-        if (!encode_view(mq, dt, 2, q, D, bp.Sq, bp.Hq, bp.B, vq, C::kElemsPerSw, true, rows) ||
-            !encode_view(mdo, dt, 2, bp.dout, D, bp.Sq, bp.Hq, bp.B, vq, C::kElemsPerSw, true, rows) ||
-            !encode_view(mk, dt, 2, k, D, bp.Sk, bp.Hkv, bp.B, vk, C::kElemsPerSw, true, rows) ||
-            !encode_view(mv, dt, 2, v, D, bp.Sk, bp.Hkv, bp.B, vk, C::kElemsPerSw, true, rows))
-            return SDPA_ERR_CUDA;
-    }
+    const int sw = C::kElemsPerSw;
+    if (!encode_view(&tq128, dt, 2, q, D, bp.Sq, bp.Hq, bp.B, vq, sw, true, 128) ||
+        !encode_view(&tdo128, dt, 2, bp.dout, D, bp.Sq, bp.Hq, bp.B, vq, sw, true, 128) ||
+        !encode_view(&tk128, dt, 2, k, D, bp.Sk, bp.Hkv, bp.B, vk, sw, true, 128) ||
+        !encode_view(&tv128, dt, 2, v, D, bp.Sk, bp.Hkv, bp.B, vk, sw, true, 128) ||
+        !encode_view(&tq64, dt, 2, q, D, bp.Sq, bp.Hq, bp.B, vq, sw, true, 64) ||
+        !encode_view(&tdo64, dt, 2, bp.dout, D, bp.Sq, bp.Hq, bp.B, vq, sw, true, 64))
+        return SDPA_ERR_CUDA;
     sdpa::BwdTcParams tp;
     tp.o = bp.o; tp.dout = bp.dout; tp.lse = bp.lse; tp.delta = bp.delta;
     tp.dq = bp.dq; tp.dk = bp.dk; tp.dv = bp.dv;
@@ -359,21 +356,21 @@ int launch_bwd_pipe(const void* q, const void* k, const void* v, const sdpa::Bwd
     tp.dq_mul = bp.dq_mul; tp.dk_mul = bp.dk_mul; tp.dv_mul = bp.dv_mul; tp.d_mul = bp.d_mul;
     auto kdkdv = sdpa::bwdp::sdpa_bwd_dkdv_pipe_kernel<D, BF16>;
     auto kdq = sdpa::bwdp::sdpa_bwd_dq_pipe_kernel<D, BF16>;
+    const int dq_smem = sdpa::bwdp::CfgQ<D>::kSmemBytes;
     static bool attr_set[64];
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_set[dev]) {
         if (cudaFuncSetAttribute(kdkdv, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
                 cudaSuccess ||
-            cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
-                cudaSuccess)
+            cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, dq_smem) != cudaSuccess)
             return SDPA_ERR_CUDA;
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
     const dim3 gkv((bp.Sk + 127) / 128, bp.B * bp.Hkv);
     const dim3 gq((bp.Sq + 127) / 128, bp.B * bp.Hq);
     // dQ first: it writes D of every row, which the dK/dV kernel reads
-    kdq<<<gq, sdpa::bwdp::kThreads, C::kSmemBytes, stream>>>(tq128, tk64, tv64, tdo128, tp);
+    kdq<<<gq, sdpa::bwdp::kThreads, dq_smem, stream>>>(tq128, tk128, tv128, tdo128, tp);
     if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
     kdkdv<<<gkv, sdpa::bwdp::kThreads, C::kSmemBytes, stream>>>(tq64, tk128, tv128, tdo64, tp);
     return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;

@@ -7,9 +7,9 @@
 //   dS = P * (dP - D),  dQ = scale * dS K,  dK = scale * dS^T Q,  dV = P^T dO,
 // arranged so that the tensor pipe and the elementwise warps overlap.
 //
-// Both kernels walk their streamed operand in steps of 64 rows, so that the
+// The dK/dV kernel walks its streamed operand in steps of 64 rows, so that the
 // two products the elementwise step reads (S and dP, 64 fp32 columns each)
-// fit twice in tensor memory next to the accumulators: while the sixteen
+// fit twice in tensor memory next to the two accumulators: while the sixteen
 // elementwise warps turn step t's S, dP into P, dS (written back over them,
 // 16-bit), the tensor pipe runs step t-1's accumulating products and step
 // t+1's S and dP (committed separately, so that step t+1's exponentials can
@@ -23,16 +23,17 @@
 //   S^T = K Q^T, dP^T = V dO^T            (M 128 keys, N 64 rows, K d)
 //   dV += P^T dO, dK += dS^T Q            (A = P^T / dS^T from TMEM, K 64)
 // dQ kernel, one CTA per 128 query rows of one (batch, query head); TMEM lane
-// = row; steps = 64 keys:
-//   S = Q K^T, dP = dO V^T                (M 128 rows, N 64 keys, K d)
-//   dQ += dS K                            (A = dS from TMEM, K 64)
+// = row; steps = 128 keys (its one accumulator leaves room for two 128-column
+// S buffers and one dP, see CfgQ):
+//   S = Q K^T, dP = dO V^T                (M 128 rows, N 128 keys, K d)
+//   dQ += dS K                            (A = dS from TMEM, K 128)
 // The dQ kernel runs first and writes D_i of every row to the caller's
 // workspace, which the dK/dV kernel's producer reads per step with the LSE.
-// Tensor memory (512 columns): S_b at [64 b, 64 b + 64), dP_b at
-// [128 + 64 b, ...) for buffers b = 0, 1; accumulators from column 256 (dQ;
-// or dV then dK).  The 16-bit P / dS of a buffer's 16-column chunk c (owned
-// by warps 4c..4c+3) are packed over the chunk's first 8 columns, which is
-// where the accumulating product's k-th 16-row slice reads them (k = c).
+// dK/dV tensor memory (512 columns): S_b at [64 b, 64 b + 64), dP_b at
+// [128 + 64 b, ...) for buffers b = 0, 1; dV, dK from column 256.  The 16-bit
+// P / dS of a buffer's 16-column chunk c (owned by warps 4c..4c+3) are packed
+// over the chunk's first 8 columns, which is where the accumulating product's
+// k-th 16-row slice reads them (k = c).
 // Warps: 0-15 elementwise (four per TMEM lane quarter, warp w on quarter
 // w & 3 and chunk w >> 2: four warps per SM sub-partition to hide the
 // latencies of one step's short chain), 16 TMA producer, 17 MMA issuer and
@@ -111,9 +112,10 @@ constexpr int kEwThreads = 32 * kEwWarps;
 constexpr int kLoadWarp = kEwWarps;
 constexpr int kMmaWarp = kEwWarps + 1;
 constexpr int kThreads = kEwThreads + 64;
-constexpr int kStep = 64;         // rows (dK/dV) or keys (dQ) per step
-constexpr int kChunk = 16;        // columns of a step per elementwise warp
+constexpr int kStep = 64;         // query rows per dK/dV step
+constexpr int kChunk = 16;        // columns of a dK/dV step per elementwise warp
 
+// dK/dV kernel layout (the dQ kernel's is CfgQ below)
 template <int D>
 struct Cfg {
     static constexpr int kRowBytes = D * 2;
@@ -124,12 +126,11 @@ struct Cfg {
     static constexpr int kTile128 = 128 * kRowBytes;
     static constexpr int kTile64 = 64 * kRowBytes;
     static constexpr int kQkSteps = kRowBytes / 32;         // K steps of 16 elements
-    // ring of streamed 64-row tile pairs (Q, dO or K, V): 4 slots at d = 128,
-    // 8 at d = 64 (32 KB / 16 KB a slot)
+    // ring of streamed 64-row (Q, dO) tile pairs: 4 slots at d = 128, 8 at
+    // d = 64 (32 KB / 16 KB a slot)
     static constexpr int kRing = D == 128 ? 4 : 8;
     // shared memory: resident pair (2 x 128-row tiles), ring, per-slot
-    // statistics (64 -LSE + 64 D floats; the dQ kernel keeps its D partial
-    // sums there), barriers, TMEM slot, abort flag
+    // statistics (64 -LSE + 64 D floats), barriers, TMEM slot, abort flag
     static constexpr int kSmemRes = 0;
     static constexpr int kSmemRing = 2 * kTile128;
     static constexpr int kSmemStats = kSmemRing + kRing * 2 * kTile64;
@@ -155,7 +156,6 @@ struct Cfg {
     static_assert(D == 64 || D == 128, "pipelined backward: head dims 64 and 128");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
     static_assert(kSmemBytes > 116 * 1024, "one CTA per SM (each allocates all of TMEM)");
-    static_assert(kRing * 2 * kStep >= 4 * 128, "room for the dQ kernel's D partial sums");
 };
 
 __device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
@@ -541,22 +541,92 @@ sdpa_bwd_dkdv_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
     teardown<D>(base, tmem, mma_ok);
 }
 
-// dQ: one CTA per 128 query rows of one (batch, query head); also writes
-// D_i = dO_i . O_i of its rows for the dK/dV kernel.
+// ---------------------------------------------------------------------------
+// The dQ kernel takes 128-key steps.  It needs only S double-buffered:
+// its dS goes over S, and dP is free as soon as the elementwise step has read
+// it, so S_b [128 b, 128 b + 128) (b = 0, 1), one dP [256, 384) and dQ
+// [384, 384 + d) fit 512 TMEM columns at N = 128: per 128 keys 24 products at
+// the full rate (an N = 128 Q K^T-form product takes 64 cycles, two N = 64
+// ones 96) and one step's turnaround instead of two.  K and V stream through
+// separate rings (V is free after dP, K only after dQ), sized to the 227 KB:
+// 3 K and 2 V slots at d = 128, 4 and 4 at d = 64.
+// ---------------------------------------------------------------------------
+template <int D>
+struct CfgQ {
+    static constexpr int kRowBytes = D * 2;
+    static constexpr int kElemsPerSw = 64;
+    static constexpr int kSwBlocks = kRowBytes / 128;
+    static constexpr int kBlock = 128 * 128;                 // swizzle block of a 128-row tile
+    static constexpr int kTile = 128 * kRowBytes;
+    static constexpr int kQkSteps = kRowBytes / 32;
+    static constexpr int kRingK = D == 128 ? 3 : 4;
+    static constexpr int kRingV = D == 128 ? 2 : 4;
+    static constexpr int kSmemQ = 0, kSmemDO = kTile, kSmemK = 2 * kTile;
+    static constexpr int kSmemV = kSmemK + kRingK * kTile;
+    static constexpr int kSmemPart = kSmemV + kRingV * kTile;   // D_i partial sums [2][128]
+    static constexpr int kSmemBar = kSmemPart + 2 * 128 * 4;
+    static constexpr int kBarResFull = 0;
+    static constexpr int kBarKFull = 1;
+    static constexpr int kBarKEmpty = 1 + kRingK;
+    static constexpr int kBarVFull = 1 + 2 * kRingK;
+    static constexpr int kBarVEmpty = 1 + 2 * kRingK + kRingV;
+    static constexpr int kBarSFull = 1 + 2 * kRingK + 2 * kRingV;   // [2]
+    static constexpr int kBarDPFull = kBarSFull + 2;
+    static constexpr int kBarPFull = kBarDPFull + 1;               // [2]
+    static constexpr int kBarDone = kBarPFull + 2;
+    static constexpr int kBarDrain = kBarDone + 1;
+    static constexpr int kNumBars = kBarDrain + 1;
+    static constexpr int kSmemSlot = kSmemBar + 8 * kNumBars;
+    static constexpr int kSmemAbort = kSmemSlot + 4;
+    static constexpr int kSmemUsed = kSmemAbort + 4;
+    static constexpr int kSmemBytes = kSmemUsed + 1024;
+    static constexpr uint32_t kColS = 0, kColDP = 256, kColAcc = 384;
+    static_assert(D == 64 || D == 128, "pipelined backward: head dims 64 and 128");
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+// d[128][128] = A[128 rows][D] . B[128 rows][D]^T, both K-major 128-row tiles
+template <int D, bool BF16>
+__device__ __forceinline__ void mma_qk128(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
+    using C = CfgQ<D>;
+    constexpr uint32_t idesc = make_idesc(BF16 ? 1u : 0u, false, 128, 128);
+    const uint64_t da = make_smem_desc(a_smem, 16, 1024), db = make_smem_desc(b_smem, 16, 1024);
+#pragma unroll
+    for (int kk = 0; kk < C::kQkSteps; ++kk) {
+        const uint64_t off = (uint64_t)(((kk >> 2) * C::kBlock + (kk & 3) * 32) >> 4);
+        mma_f16_ss(d_tmem, da + off, db + off, idesc, kk > 0);
+    }
+}
+
+// d[128][D] (+)= A (TMEM, 128 x 128, 16-bit; 32-column chunk c packed over
+// its first 16 columns) . B[128 rows][D] (MN-major 128-row tile)
+template <int D, bool BF16>
+__device__ __forceinline__ void mma_pv128(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, bool acc) {
+    using C = CfgQ<D>;
+    constexpr uint32_t idesc = make_idesc(BF16 ? 1u : 0u, true, 128, D);
+    const uint64_t db = make_smem_desc(b_smem, C::kBlock, 1024);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {    // 16 keys per product
+        const uint64_t off = (uint64_t)((kk * 16 * 128) >> 4);
+        mma_f16_ts(d_tmem, a_tmem + 32 * (kk >> 1) + 8 * (kk & 1), db + off, idesc, (acc || kk > 0) ? 1u : 0u);
+    }
+}
+
+// dQ: one CTA per 128 query rows of one (batch, query head), 128-key steps;
+// also writes D_i = dO_i . O_i of its rows for the dK/dV kernel.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
 sdpa_bwd_dq_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                         const BwdTcParams p) {
-    using C = Cfg<D>;
+    using C = CfgQ<D>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
-    const uint32_t sQ = base + C::kSmemRes, sdO = sQ + C::kTile128;
-    auto sK = [&](int slot) -> uint32_t { return base + C::kSmemRing + (uint32_t)slot * 2u * C::kTile64; };
-    auto sV = [&](int slot) -> uint32_t { return sK(slot) + C::kTile64; };
-    // the two halves' partial dot products of D_i
-    float* const dpart = reinterpret_cast<float*>(smem_raw + (base - raw) + C::kSmemStats);
+    const uint32_t sQ = base + C::kSmemQ, sdO = base + C::kSmemDO;
+    auto sK = [&](int slot) -> uint32_t { return base + C::kSmemK + (uint32_t)slot * C::kTile; };
+    auto sV = [&](int slot) -> uint32_t { return base + C::kSmemV + (uint32_t)slot * C::kTile; };
+    float* const dpart = reinterpret_cast<float*>(smem_raw + (base - raw) + C::kSmemPart);
     auto bar = [&](int i) -> uint32_t { return base + C::kSmemBar + 8u * (uint32_t)i; };
     const uint32_t abort_addr = base + C::kSmemAbort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -566,11 +636,37 @@ sdpa_bwd_dq_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
     const int bh = blockIdx.y;
     const int b = bh / p.Hq, hq = bh - b * p.Hq;
     const int kvrow = b * p.Hkv + hq / p.group;        // 3-D map index of the K/V head
-    // steps: 64 keys, up to the last key a row of the tile sees
     const int kend = p.causal ? min(p.Sk, i0 + 128 + p.causal_off) : p.Sk;
-    const int nsteps = kend > 0 ? (kend + kStep - 1) / kStep : 0;
+    const int nsteps = kend > 0 ? (kend + 127) / 128 : 0;
 
-    const uint32_t tmem = setup<D>(base);
+    if (threadIdx.x == 0) {
+        mbar_init(bar(C::kBarResFull), 1);
+        for (int i = 0; i < C::kRingK; ++i) {
+            mbar_init(bar(C::kBarKFull + i), 1);
+            mbar_init(bar(C::kBarKEmpty + i), 1);
+        }
+        for (int i = 0; i < C::kRingV; ++i) {
+            mbar_init(bar(C::kBarVFull + i), 1);
+            mbar_init(bar(C::kBarVEmpty + i), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(C::kBarSFull + i), 1);
+            mbar_init(bar(C::kBarPFull + i), kEwWarps);   // one arrival per warp
+        }
+        mbar_init(bar(C::kBarDPFull), 1);
+        mbar_init(bar(C::kBarDone), 1);
+        mbar_init(bar(C::kBarDrain), 1);
+        sts_u32(abort_addr, 0u);
+        fence_barrier_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(base + C::kSmemSlot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = lds_u32(base + C::kSmemSlot);
     bool mma_ok = true;
 
     if (warp == kLoadWarp) {
@@ -580,28 +676,46 @@ sdpa_bwd_dq_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
             prefetch_tmap(&tmdO);
-            mbar_arrive_expect_tx(bar(C::kBarResFull), 2 * C::kTile128);
+            mbar_arrive_expect_tx(bar(C::kBarResFull), 2 * C::kTile);
             for (int kb = 0; kb < C::kSwBlocks; ++kb) {
-                tma_load_3d(sQ + kb * C::kBlock128, &tmQ, bar(C::kBarResFull), kb * C::kElemsPerSw, i0, bh);
-                tma_load_3d(sdO + kb * C::kBlock128, &tmdO, bar(C::kBarResFull), kb * C::kElemsPerSw, i0, bh);
+                tma_load_3d(sQ + kb * C::kBlock, &tmQ, bar(C::kBarResFull), kb * C::kElemsPerSw, i0, bh);
+                tma_load_3d(sdO + kb * C::kBlock, &tmdO, bar(C::kBarResFull), kb * C::kElemsPerSw, i0, bh);
             }
             bool ok = true;
-            int issued = 0;
+            int kiss = 0, viss = 0;   // K / V tiles issued
             for (int jt = 0; jt < nsteps && ok; ++jt) {
-                const int slot = jt % C::kRing;
-                if (jt >= C::kRing)
-                    ok = wait(bar(C::kBarRingEmpty + slot), (uint32_t)(jt / C::kRing - 1) & 1u, abort_addr,
-                              0x69000u | (uint32_t)(jt & 0xfff));
+                const int ks = jt % C::kRingK, vs = jt % C::kRingV;
+                if (jt >= C::kRingK)
+                    ok = wait(bar(C::kBarKEmpty + ks), (uint32_t)(jt / C::kRingK - 1) & 1u, abort_addr,
+                              0x71000u | (uint32_t)(jt & 0xfff));
                 if (!ok) break;
-                const uint32_t fb = bar(C::kBarRingFull + slot);
-                mbar_arrive_expect_tx(fb, 2 * C::kTile64);
-                for (int kb = 0; kb < C::kSwBlocks; ++kb) {
-                    tma_load_3d(sK(slot) + kb * C::kBlock64, &tmK, fb, kb * C::kElemsPerSw, jt * kStep, kvrow);
-                    tma_load_3d(sV(slot) + kb * C::kBlock64, &tmV, fb, kb * C::kElemsPerSw, jt * kStep, kvrow);
-                }
-                issued = jt + 1;
+                mbar_arrive_expect_tx(bar(C::kBarKFull + ks), C::kTile);
+                for (int kb = 0; kb < C::kSwBlocks; ++kb)
+                    tma_load_3d(sK(ks) + kb * C::kBlock, &tmK, bar(C::kBarKFull + ks), kb * C::kElemsPerSw,
+                                jt * 128, kvrow);
+                kiss = jt + 1;
+                if (jt >= C::kRingV)
+                    ok = wait(bar(C::kBarVEmpty + vs), (uint32_t)(jt / C::kRingV - 1) & 1u, abort_addr,
+                              0x72000u | (uint32_t)(jt & 0xfff));
+                if (!ok) break;
+                mbar_arrive_expect_tx(bar(C::kBarVFull + vs), C::kTile);
+                for (int kb = 0; kb < C::kSwBlocks; ++kb)
+                    tma_load_3d(sV(vs) + kb * C::kBlock, &tmV, bar(C::kBarVFull + vs), kb * C::kElemsPerSw,
+                                jt * 128, kvrow);
+                viss = jt + 1;
             }
-            drain_loads<D>(base, issued);
+            // let the copies already issued land before the CTA ends
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(bar(C::kBarResFull), 0) && global_timer_ns() - t0 < 100000000ull) {
+            }
+            for (int jt = kiss > C::kRingK ? kiss - C::kRingK : 0; jt < kiss; ++jt)
+                while (!mbar_try_wait(bar(C::kBarKFull + jt % C::kRingK), (uint32_t)(jt / C::kRingK) & 1u) &&
+                       global_timer_ns() - t0 < 100000000ull) {
+                }
+            for (int jt = viss > C::kRingV ? viss - C::kRingV : 0; jt < viss; ++jt)
+                while (!mbar_try_wait(bar(C::kBarVFull + jt % C::kRingV), (uint32_t)(jt / C::kRingV) & 1u) &&
+                       global_timer_ns() - t0 < 100000000ull) {
+                }
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
@@ -614,52 +728,55 @@ sdpa_bwd_dq_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             if (leader) mma_commit(b_);
             __syncwarp();
         };
-        // Step jt's K / V landed (its ring slot)
-        auto wait_in = [&](int jt) -> bool {
-            return wait_all(bar(C::kBarRingFull + jt % C::kRing), (uint32_t)(jt / C::kRing) & 1u,
-                            0x6a000u | (uint32_t)(jt & 0xfff));
-        };
-        // S (or dP) of step jt into buffer jt & 1, with its own commit
-        auto issue_s = [&](int jt) {
-            if (leader) mma_qk<D, BF16>(tmem + C::kColS + 64 * (jt & 1), sQ, sK(jt % C::kRing));
+        // S of step jt into buffer jt & 1 (its K landed)
+        auto issue_s = [&](int jt) -> bool {
+            const int ks = jt % C::kRingK;
+            if (!wait_all(bar(C::kBarKFull + ks), (uint32_t)(jt / C::kRingK) & 1u, 0x73000u | (uint32_t)(jt & 0xfff)))
+                return false;
+            tc_fence_after();
+            if (leader) mma_qk128<D, BF16>(tmem + C::kColS + 128 * (jt & 1), sQ, sK(ks));
             __syncwarp();
             commit(bar(C::kBarSFull + (jt & 1)));
+            return true;
         };
-        auto issue_dp = [&](int jt) {
-            if (leader) mma_qk<D, BF16>(tmem + C::kColDP + 64 * (jt & 1), sdO, sV(jt % C::kRing));
-            __syncwarp();
-            commit(bar(C::kBarDPFull + (jt & 1)));
-        };
-        bool ok = wait_all(bar(C::kBarResFull), 0, 0x68000u);
-        for (int jt = 0; jt < 2 && jt < nsteps && ok; ++jt) {
-            ok = wait_in(jt);
-            if (!ok) break;
+        // dP of step jt (its V landed); V's slot is free once it has run
+        auto issue_dp = [&](int jt) -> bool {
+            const int vs = jt % C::kRingV;
+            if (!wait_all(bar(C::kBarVFull + vs), (uint32_t)(jt / C::kRingV) & 1u, 0x74000u | (uint32_t)(jt & 0xfff)))
+                return false;
             tc_fence_after();
-            issue_s(jt);
-            issue_dp(jt);
-        }
-        // Per step, in issue order: dQ(jt) (reads dS over S_b), S(jt+2)
-        // (overwrites it), dP(jt+2) (dP_b was read before dS was written)
+            if (leader) mma_qk128<D, BF16>(tmem + C::kColDP, sdO, sV(vs));
+            __syncwarp();
+            commit(bar(C::kBarDPFull));
+            commit(bar(C::kBarVEmpty + vs));
+            return true;
+        };
+        bool ok = wait_all(bar(C::kBarResFull), 0, 0x70000u);
+        if (ok && nsteps > 0) ok = issue_s(0);
+        if (ok && nsteps > 0) ok = issue_dp(0);
+        if (ok && nsteps > 1) ok = issue_s(1);
+        // Per step, in issue order: dP(jt+1) (the single dP buffer was read
+        // by the elementwise step jt), dQ(jt) (reads dS over S_b; K's slot is
+        // then free), S(jt+2) (overwrites S_b)
         for (int jt = 0; jt < nsteps && ok; ++jt) {
-            const int slot = jt % C::kRing, bf = jt & 1;
-            const bool next = jt + 2 < nsteps;
-            ok = wait_all(bar(C::kBarPFull + bf), (uint32_t)(jt >> 1) & 1u, 0x6b000u | (uint32_t)(jt & 0xfff));
-            if (ok && next) ok = wait_in(jt + 2);
+            const int bf = jt & 1, ks = jt % C::kRingK;
+            ok = wait_all(bar(C::kBarPFull + bf), (uint32_t)(jt >> 1) & 1u, 0x75000u | (uint32_t)(jt & 0xfff));
             if (!ok) break;
             tc_fence_after();
-            if (leader) mma_pv<D, BF16>(tmem + C::kColAcc, tmem + C::kColS + 64 * bf, sK(slot), jt > 0);  // dQ += dS K
-            __syncwarp();
-            commit(bar(C::kBarRingEmpty + slot));
-            if (next) {
-                issue_s(jt + 2);
-                issue_dp(jt + 2);
+            if (jt + 1 < nsteps) {
+                ok = issue_dp(jt + 1);
+                if (!ok) break;
             }
+            if (leader) mma_pv128<D, BF16>(tmem + C::kColAcc, tmem + C::kColS + 128 * bf, sK(ks), jt > 0);  // dQ += dS K
+            __syncwarp();
+            commit(bar(C::kBarKEmpty + ks));
+            if (jt + 2 < nsteps) ok = issue_s(jt + 2);
         }
         if (ok) commit(bar(C::kBarDone));
         mma_ok = ok;
     } else {
         // ================= elementwise (warps 0-15) =======================
-        const int quarter = warp & 3, c = warp >> 2;   // lane quarter, column chunk
+        const int quarter = warp & 3, c = warp >> 2;   // lane quarter, 32-column chunk
         const int r = quarter * 32 + lane, row = i0 + r;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         const float sl = p.scale * kL2e;
@@ -675,28 +792,28 @@ sdpa_bwd_dq_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         if (c == 0 && row < p.Sq) p.delta[(size_t)bh * p.Sq + row] = d_r;
         bool ok = true;
         for (int jt = 0; jt < nsteps && ok; ++jt) {
-            const int bf = jt & 1, j0 = jt * kStep;
+            const int bf = jt & 1, j0 = jt * 128;
             ok = __all_sync(0xffffffffu, wait(bar(C::kBarSFull + bf), (uint32_t)(jt >> 1) & 1u, abort_addr,
-                                              0x6c000u | (uint32_t)(jt & 0xfff)));
+                                              0x76000u | (uint32_t)(jt & 0xfff)));
             if (!ok) break;
             tc_fence_after();
-            const uint32_t tS = tmem + lane_base + C::kColS + 64 * bf + kChunk * c;
-            const uint32_t tP = tmem + lane_base + C::kColDP + 64 * bf + kChunk * c;
-            float s[16];
-            tmem_ld16(tS, s);
+            const uint32_t tS = tmem + lane_base + C::kColS + 128 * bf + 32 * c;
+            const uint32_t tP = tmem + lane_base + C::kColDP + 32 * c;
+            float s[32];
+            tmem_ld32(tS, s);
             tmem_wait_ld();
-            reg_fence16(s);
+            reg_fence32(s);
             // P = 2^(s sl - LSE) (0 where masked), while dP is computed
-            float pv[16];
+            float pv[32];
             auto weights = [&](auto masked) {
                 constexpr bool kMask = decltype(masked)::value;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
+                for (int e = 0; e < 16; ++e) {
                     float x0, x1;
                     f2_unpack(f2_fma(f2_pack(s[2 * e], s[2 * e + 1]), sl2, nl2), x0, x1);
                     float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
                     if constexpr (kMask) {
-                        const int key = j0 + kChunk * c + 2 * e;
+                        const int key = j0 + 32 * c + 2 * e;
                         const bool rin = row < p.Sq;
                         p0 = (rin && key < p.Sk && (!p.causal || key <= row + p.causal_off)) ? p0 : 0.0f;
                         p1 = (rin && key + 1 < p.Sk && (!p.causal || key + 1 <= row + p.causal_off)) ? p1 : 0.0f;
@@ -705,27 +822,27 @@ sdpa_bwd_dq_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                     pv[2 * e + 1] = p1;
                 }
             };
-            if (i0 + 128 <= p.Sq && j0 + kStep <= p.Sk && (!p.causal || j0 + kStep - 1 <= i0 + p.causal_off))
+            if (i0 + 128 <= p.Sq && j0 + 128 <= p.Sk && (!p.causal || j0 + 127 <= i0 + p.causal_off))
                 weights(std::false_type{});
             else
                 weights(std::true_type{});
             // dS = P (dP - D)
-            ok = __all_sync(0xffffffffu, wait(bar(C::kBarDPFull + bf), (uint32_t)(jt >> 1) & 1u, abort_addr,
-                                              0x6e000u | (uint32_t)(jt & 0xfff)));
+            ok = __all_sync(0xffffffffu, wait(bar(C::kBarDPFull), (uint32_t)jt & 1u, abort_addr,
+                                              0x77000u | (uint32_t)(jt & 0xfff)));
             if (!ok) break;
             tc_fence_after();
-            float dp[16];
-            tmem_ld16(tP, dp);
+            float dp[32];
+            tmem_ld32(tP, dp);
             tmem_wait_ld();
-            reg_fence16(dp);
-            uint32_t w[8];
+            reg_fence32(dp);
+            uint32_t w[16];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
+            for (int e = 0; e < 16; ++e) {
                 float d0, d1;
                 f2_unpack(f2_mul(f2_pack(pv[2 * e], pv[2 * e + 1]), f2_sub(f2_pack(dp[2 * e], dp[2 * e + 1]), d2)), d0, d1);
                 w[e] = bt_pack<BF16>(d0, d1);
             }
-            tmem_st8(tS, w);    // dS
+            tmem_st16(tS, w);    // dS
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -733,7 +850,7 @@ sdpa_bwd_dq_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         }
         // dQ row, this warp's quarter of the columns; zero when the row sees
         // no key
-        if (ok && nsteps > 0) ok = __all_sync(0xffffffffu, wait(bar(C::kBarDone), 0, abort_addr, 0x6d000u));
+        if (ok && nsteps > 0) ok = __all_sync(0xffffffffu, wait(bar(C::kBarDone), 0, abort_addr, 0x78000u));
         if (ok) {
             tc_fence_after();
             const int col0 = c * (D / 4);
@@ -744,7 +861,18 @@ sdpa_bwd_dq_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                                     row < p.Sq);
         }
     }
-    teardown<D>(base, tmem, mma_ok);
+    // end: after a failed wait no MMA may still write TMEM when it is freed
+    if (warp == kMmaWarp && !mma_ok) {
+        if (elect_one()) mma_commit(bar(C::kBarDrain));
+        __syncwarp();
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(bar(C::kBarDrain), 0) && global_timer_ns() - t0 < 100000000ull) {
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace bwdp

@@ -140,16 +140,15 @@ def run(machine, roles, limit=400000):
     raise ModelError("no progress: deadlock")
 
 
-RING = 4          # ring slots of 64-row tile pairs (head dim 128)
+RING = 4          # dK/dV kernel at head dim 128: ring slots of 64-row (Q, dO) tile pairs
 N_EW = 4          # elementwise warps modelled (the kernel has 16, one arrival each)
 
 
-def pipe_model(nsteps, seed, kind, plant=None):
-    """kind "dkdv": K, V resident; Q, dO and the step's statistics streamed;
-    per step dV(st) [reads S_b], S(st+2) [writes S_b], dK(st) [reads dP_b],
-    ring slot released, dP(st+2) [writes dP_b].  kind "dq": Q, dO resident;
-    K, V streamed; per step dQ(jt) [reads S_b], ring slot released, S(jt+2),
-    dP(jt+2)."""
+def dkdv_model(nsteps, seed, plant=None):
+    """The dK/dV kernel (64-row steps): K, V resident; Q, dO and the step's
+    statistics streamed through one ring; S and dP double-buffered.  Per step
+    dV(st) [reads S_b], S(st+2) [writes S_b], dK(st) [reads dP_b], ring slot
+    released, dP(st+2) [writes dP_b]."""
     m = Machine(seed)
     res_full, done = Bar("res_full"), Bar("done")
     ring_full = [Bar("ring_full%d" % i) for i in range(RING)]
@@ -163,7 +162,6 @@ def pipe_model(nsteps, seed, kind, plant=None):
     tm = {(x, b, w): None for x in ("S", "D") for b in range(2) for w in range(N_EW)}
     tm_readers = {(x, b): 0 for x in ("S", "D") for b in range(2)}
     stats = [{"step": None, "readers": set()} for _ in range(RING)]
-    stream = "q" if kind == "dkdv" else "kv"
 
     def par(intended):
         """Parity of completion number `intended` (a planted mistake flips it)."""
@@ -177,17 +175,15 @@ def pipe_model(nsteps, seed, kind, plant=None):
                 tm[key + (w,)] = ("S" if key[0] == "S" else "dP", step)
         return f
 
-    def read_tm(keys, step):      # an accumulating product reads P/dS of `step`
-        for k in keys:
-            want = ("P" if k[0] == "S" else "dS", step)
-            for w in range(N_EW):
-                check(tm[k + (w,)] == want, "accumulating product before every warp wrote P/dS", k, w, step,
-                      tm[k + (w,)])
-            tm_readers[k] += 1
+    def read_tm(key, step):       # an accumulating product reads P/dS of `step`
+        want = ("P" if key[0] == "S" else "dS", step)
+        for w in range(N_EW):
+            check(tm[key + (w,)] == want, "accumulating product before every warp wrote P/dS", key, w, step,
+                  tm[key + (w,)])
+        tm_readers[key] += 1
 
         def f():
-            for k in keys:
-                tm_readers[k] -= 1
+            tm_readers[key] -= 1
         return f
 
     def producer():
@@ -196,16 +192,13 @@ def pipe_model(nsteps, seed, kind, plant=None):
         m.tma.append((res_full, "res", 0))
         for st in range(nsteps):
             slot = st % RING
-            if plant == "early_copy" and st >= RING:
-                pass
-            elif st >= RING:
+            if st >= RING and plant != "early_copy":
                 n = st // RING - 1
                 while not ring_empty[slot].ready(par(n), n):
                     yield
-            if kind == "dkdv":
-                check(not stats[slot]["readers"], "statistics rewritten while read", slot, st)
-                stats[slot]["step"] = st
-            m.copy(ring_full[slot], (stream, slot), st)
+            check(not stats[slot]["readers"], "statistics rewritten while read", slot, st)
+            stats[slot]["step"] = st
+            m.copy(ring_full[slot], ("q", slot), st)
             yield
 
     def mma():
@@ -218,74 +211,53 @@ def pipe_model(nsteps, seed, kind, plant=None):
                 yield
 
         def issue_s(st):
-            b = st & 1
-            m.mma([(stream, st % RING)], st, write_tm(("S", b), st))
-            m.commit(s_full[b])
+            m.mma([("q", st % RING)], st, write_tm(("S", st & 1), st))
+            m.commit(s_full[st & 1])
 
         def issue_dp(st):
-            b = st & 1
-            m.mma([(stream, st % RING)], st, write_tm(("D", b), st))
-            m.commit(dp_full[b])
+            m.mma([("q", st % RING)], st, write_tm(("D", st & 1), st))
+            m.commit(dp_full[st & 1])
 
         for st in range(min(2, nsteps)):
             yield from wait_in(st)
             issue_s(st)
             issue_dp(st)
         for st in range(nsteps):
-            b, slot, nxt = st & 1, st % RING, st + 2 < nsteps
-            n = st >> 1
+            b, slot, nxt, n = st & 1, st % RING, st + 2 < nsteps, st >> 1
             while not p_full[b].ready(par(n), n):
                 yield
             if nxt:
                 yield from wait_in(st + 2)
-            if kind == "dkdv":
-                if plant == "early_overwrite" and nxt:
-                    issue_s(st + 2)
-                m.mma([(stream, slot)], st, read_tm([("S", b)], st))        # dV += P^T dO
-                if nxt and plant != "early_overwrite":
-                    issue_s(st + 2)
-                m.mma([(stream, slot)], st, read_tm([("D", b)], st))        # dK += dS^T Q
-                m.commit(ring_empty[slot])
-                if nxt:
-                    issue_dp(st + 2)
-            else:
-                if plant == "early_overwrite" and nxt:
-                    issue_s(st + 2)
-                m.mma([(stream, slot)], st, read_tm([("S", b)], st))        # dQ += dS K
-                m.commit(ring_empty[slot])
-                if nxt:
-                    if plant != "early_overwrite":
-                        issue_s(st + 2)
-                    issue_dp(st + 2)
+            if plant == "early_overwrite" and nxt:
+                issue_s(st + 2)
+            m.mma([("q", slot)], st, read_tm(("S", b), st))             # dV += P^T dO
+            if nxt and plant != "early_overwrite":
+                issue_s(st + 2)
+            m.mma([("q", slot)], st, read_tm(("D", b), st))             # dK += dS^T Q
+            m.commit(ring_empty[slot])
+            if nxt:
+                issue_dp(st + 2)
             yield
         m.commit(done)
 
     def elementwise(w):
         for st in range(nsteps):
-            b, slot, n = st & 1, st % RING, st >> 1
-            if kind == "dkdv":
-                nr = st // RING
-                while not ring_full[slot].ready(par(nr), nr):
-                    yield
-                check(stats[slot]["step"] == st, "statistics of another step", w, st, stats[slot]["step"])
-                stats[slot]["readers"].add(w)
+            b, slot, n, nr = st & 1, st % RING, st >> 1, st // RING
+            while not ring_full[slot].ready(par(nr), nr):
+                yield
+            check(stats[slot]["step"] == st, "statistics of another step", w, st, stats[slot]["step"])
+            stats[slot]["readers"].add(w)
             while not s_full[b].ready(par(n), n):
                 yield
             check(tm[("S", b, w)] == ("S", st), "elementwise reads S before its product", w, st, tm[("S", b, w)])
             yield
-            # P^T (dK/dV) written over this warp's chunk of S_b now; dS (dQ)
-            # after dP
-            if kind == "dkdv":
-                tm[("S", b, w)] = ("P", st)
+            tm[("S", b, w)] = ("P", st)           # P^T over this warp's chunk of S_b
             while not dp_full[b].ready(par(n), n):
                 yield
             check(tm[("D", b, w)] == ("dP", st), "elementwise reads dP before its product", w, st, tm[("D", b, w)])
             yield
-            if kind == "dkdv":
-                tm[("D", b, w)] = ("dS", st)
-                stats[slot]["readers"].discard(w)
-            else:
-                tm[("S", b, w)] = ("P", st)
+            tm[("D", b, w)] = ("dS", st)          # dS^T over its chunk of dP_b
+            stats[slot]["readers"].discard(w)
             p_full[b].arrive()
             yield
         if nsteps > 0:
@@ -296,20 +268,168 @@ def pipe_model(nsteps, seed, kind, plant=None):
     check(not m.pipe and not m.tma, "work left in flight at exit")
 
 
-@pytest.mark.parametrize("kind", ["dkdv", "dq"])
+RING_K, RING_V = 3, 2   # dQ kernel at head dim 128: K and V rings of 128-row tiles
+
+
+def dq_model(nsteps, seed, plant=None):
+    """The dQ kernel (128-key steps): Q, dO resident; K and V in separate
+    rings; S double-buffered, dP single (free once every warp has read it).
+    Per step: dP(jt+1) [after the weights of jt], dQ(jt) [reads dS over S_b],
+    K's slot released, S(jt+2) [overwrites S_b]."""
+    m = Machine(seed)
+    res_full, done = Bar("res_full"), Bar("done")
+    k_full = [Bar("k_full%d" % i) for i in range(RING_K)]
+    k_empty = [Bar("k_empty%d" % i) for i in range(RING_K)]
+    v_full = [Bar("v_full%d" % i) for i in range(RING_V)]
+    v_empty = [Bar("v_empty%d" % i) for i in range(RING_V)]
+    s_full = [Bar("s_full%d" % b) for b in range(2)]
+    dp_full = Bar("dp_full")
+    p_full = [Bar("p_full%d" % b, count=N_EW) for b in range(2)]
+    tm = {("S", b, w): None for b in range(2) for w in range(N_EW)}
+    tm.update({("D", w): None for w in range(N_EW)})
+    readers = {("S", b): 0 for b in range(2)}
+
+    def par(intended):
+        p = intended & 1
+        return 1 - p if plant == "wrong_parity" else p
+
+    def write_s(b, jt):
+        def f():
+            check(readers[("S", b)] == 0, "S overwritten before the dQ product reading dS ran", b, jt)
+            for w in range(N_EW):
+                tm[("S", b, w)] = ("S", jt)
+        return f
+
+    def write_dp(jt):
+        def f():
+            for w in range(N_EW):
+                check(jt == 0 or tm[("D", w)] == ("read", jt - 1), "dP overwritten before a warp read it", w, jt,
+                      tm[("D", w)])
+                tm[("D", w)] = ("dP", jt)
+        return f
+
+    def read_ds(b, jt):
+        for w in range(N_EW):
+            check(tm[("S", b, w)] == ("dS", jt), "dQ product before every warp wrote dS", b, w, jt,
+                  tm[("S", b, w)])
+        readers[("S", b)] += 1
+
+        def f():
+            readers[("S", b)] -= 1
+        return f
+
+    def producer():
+        m.buf["res"] = None
+        res_full.arrive(tx=1)
+        m.tma.append((res_full, "res", 0))
+        for jt in range(nsteps):
+            ks, vs = jt % RING_K, jt % RING_V
+            if jt >= RING_K and plant != "early_copy":
+                n = jt // RING_K - 1
+                while not k_empty[ks].ready(par(n), n):
+                    yield
+            m.copy(k_full[ks], ("k", ks), jt)
+            yield
+            if jt >= RING_V:
+                n = jt // RING_V - 1
+                while not v_empty[vs].ready(par(n), n):
+                    yield
+            m.copy(v_full[vs], ("v", vs), jt)
+            yield
+
+    def mma():
+        while not res_full.ready(0, 0):
+            yield
+
+        def issue_s(jt):
+            ks, n = jt % RING_K, jt // RING_K
+            while not k_full[ks].ready(par(n), n):
+                yield
+            m.mma([("k", ks)], jt, write_s(jt & 1, jt))
+            m.commit(s_full[jt & 1])
+
+        def issue_dp(jt):
+            vs, n = jt % RING_V, jt // RING_V
+            while not v_full[vs].ready(par(n), n):
+                yield
+            m.mma([("v", vs)], jt, write_dp(jt))
+            m.commit(dp_full)
+            m.commit(v_empty[vs])
+
+        if nsteps > 0:
+            yield from issue_s(0)
+            yield from issue_dp(0)
+        if nsteps > 1:
+            yield from issue_s(1)
+        for jt in range(nsteps):
+            b, n = jt & 1, jt >> 1
+            if plant == "early_dp" and jt + 1 < nsteps:
+                yield from issue_dp(jt + 1)
+            while not p_full[b].ready(par(n), n):
+                yield
+            if jt + 1 < nsteps and plant != "early_dp":
+                yield from issue_dp(jt + 1)
+            if plant == "early_overwrite" and jt + 2 < nsteps:
+                yield from issue_s(jt + 2)
+            m.mma([("k", jt % RING_K)], jt, read_ds(b, jt))       # dQ += dS K
+            m.commit(k_empty[jt % RING_K])
+            if jt + 2 < nsteps and plant != "early_overwrite":
+                yield from issue_s(jt + 2)
+            yield
+        m.commit(done)
+
+    def elementwise(w):
+        for jt in range(nsteps):
+            b, n = jt & 1, jt >> 1
+            while not s_full[b].ready(par(n), n):
+                yield
+            check(tm[("S", b, w)] == ("S", jt), "elementwise reads S before its product", w, jt, tm[("S", b, w)])
+            yield
+            while not dp_full.ready(par(jt), jt):
+                yield
+            check(tm[("D", w)] == ("dP", jt), "elementwise reads dP before its product", w, jt, tm[("D", w)])
+            tm[("D", w)] = ("read", jt)
+            yield
+            tm[("S", b, w)] = ("dS", jt)
+            p_full[b].arrive()
+            yield
+        if nsteps > 0:
+            while not done.ready(0, 0):
+                yield
+
+    run(m, [producer(), mma()] + [elementwise(w) for w in range(N_EW)])
+    check(not m.pipe and not m.tma, "work left in flight at exit")
+
+
 @pytest.mark.parametrize("n", [0, 1, 2, 3, 4, 5, 9])
-def test_protocol_holds_under_random_interleavings(kind, n):
+def test_dkdv_protocol_holds_under_random_interleavings(n):
     for seed in range(30):
-        pipe_model(n, seed, kind)
+        dkdv_model(n, seed)
 
 
-@pytest.mark.parametrize("kind", ["dkdv", "dq"])
+@pytest.mark.parametrize("n", [0, 1, 2, 3, 4, 5, 9])
+def test_dq_protocol_holds_under_random_interleavings(n):
+    for seed in range(30):
+        dq_model(n, seed)
+
+
 @pytest.mark.parametrize("plant", ["early_copy", "wrong_parity", "early_overwrite"])
-def test_planted_mistakes_are_caught(kind, plant):
+def test_dkdv_planted_mistakes_are_caught(plant):
     caught = 0
     for seed in range(20):
         try:
-            pipe_model(7, seed, kind, plant=plant)
+            dkdv_model(7, seed, plant=plant)
+        except ModelError:
+            caught += 1
+    assert caught > 0, plant
+
+
+@pytest.mark.parametrize("plant", ["early_copy", "wrong_parity", "early_overwrite", "early_dp"])
+def test_dq_planted_mistakes_are_caught(plant):
+    caught = 0
+    for seed in range(20):
+        try:
+            dq_model(7, seed, plant=plant)
         except ModelError:
             caught += 1
     assert caught > 0, plant
