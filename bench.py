@@ -301,6 +301,20 @@ def roofline_of(w, ms, peaks, src, fwd=True):
             "peak_source": "%s bf16_tflops (burst)%s" % (src, " x 2 (nominal fp8/bf16)" if fp8 else "")}
 
 
+def median_launch_ms(run, stream, n):
+    """Median device time of one launch over n launches, each bracketed by its
+    own pair of CUDA events on the launching stream (run outside the timed
+    region, after the warm-ups)."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for a, b in evs:
+        a.record(stream)
+        run()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in evs)
+
+
 def config_sweep(dev, launches=20, warmup=3):
     """Every BASELINE-shaped workload besides the headline, one GPU: device
     time over `launches` launches after `warmup`, TFLOP/s, roofline fraction,
@@ -338,6 +352,7 @@ def config_sweep(dev, launches=20, warmup=3):
         e1.record(stream)
         e1.synchronize()
         ms = e0.elapsed_time(e1) / launches
+        med = median_launch_ms(run, stream, launches)
         st, detail = sdpa.sdpa_device_status(clear=True)
         rows = sample_rows(w, n_random=32)
         rows = rows[:: max(1, len(rows) // 64)]
@@ -347,7 +362,8 @@ def config_sweep(dev, launches=20, warmup=3):
         roof = roofline_of(w, ms, peaks, src)
         roof["traffic"] = load_traffic(w.name)
         out.append({"workload": w.name, "ms": ms, "tflops": w.flops / (ms * 1e-3) / 1e12,
-                    "launches": launches, "roofline": roof,
+                    "launches": launches, "median_ms": med, "median_tflops": w.flops / (med * 1e-3) / 1e12,
+                    "roofline": roof,
                     "parity": {"rows": len(rows), "max_abs_o": float(np.abs(go - ro).max())},
                     "device_status": st})
         del q, k, v, o, lse
@@ -367,9 +383,11 @@ def config_sweep(dev, launches=20, warmup=3):
     e1.record(stream)
     e1.synchronize()
     ms = e0.elapsed_time(e1) / launches
+    med = median_launch_ms(run, stream, launches)
     st, _ = sdpa.sdpa_device_status(clear=True)
     out.append({"workload": w.name, "pass": "bwd", "ms": ms, "tflops": 2.5 * w.flops / (ms * 1e-3) / 1e12,
-                "launches": launches, "roofline": roofline_of(w, ms, peaks, src, fwd=False),
+                "launches": launches, "median_ms": med, "median_tflops": 2.5 * w.flops / (med * 1e-3) / 1e12,
+                "roofline": roofline_of(w, ms, peaks, src, fwd=False),
                 "device_status": st})
     return out
 
@@ -462,6 +480,11 @@ def main():
         raise SystemExit("device status %d (%#x) after timing" % (st, detail))
     ms_per_step = ms_total / args.steps
     value = job_throughput(world, w.flops, args.steps, ms_total)
+    # per-launch device times, after the timed region: the median of up to 50
+    # launches, each with its own event pair (max over ranks)
+    n_med = min(50, args.steps)
+    med_ms = max_over_ranks(median_launch_ms(run, stream, n_med))
+    median = {"ms": med_ms, "value": job_throughput(world, w.flops, 1, med_ms), "launches": n_med}
 
     # end to end through the public API: pinned host inputs -> device -> fused
     # forward -> O and LSE back to pinned host memory, all inside the region
@@ -538,6 +561,7 @@ def main():
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
             "gpu_launches": args.steps * sdpa.sdpa_launches_per_call(),
+            "median": median,
             "parity": parity,
         }
         if world == 1 and not args.no_cpu_baseline:
