@@ -170,12 +170,10 @@ __device__ __forceinline__ void sts_u32(uint32_t addr, uint32_t v) {
 // Bounded wait on `bar`'s phase `parity`: gives up after 1 s (records a
 // device timeout at `where` and raises the CTA's abort flag) or when another
 // warp has raised the flag.
-__device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, uint32_t abort_addr, uint32_t where,
-                                     uint32_t sleep_ns = 0) {
+__device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, uint32_t abort_addr, uint32_t where) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t k = 1;; ++k) {
-        if (sleep_ns) __nanosleep(sleep_ns);
         if (mbar_try_wait(bar, parity)) return true;
         if ((k & 15u) == 0) {
             if (lds_u32(abort_addr) != 0u) return false;
