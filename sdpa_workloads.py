@@ -114,6 +114,9 @@ def batch_sweep():
 
 
 WORKLOADS.update({"bsweep_b%d" % w.B: w for w in batch_sweep()})
+# the sequence sweep's points by name (e.g. sweep_s16384_full), so that
+# bench.py --workload can select one
+WORKLOADS.update({w.name: w for causal in (False, True) for w in sweep(causal)})
 
 
 def with_shape(w: Workload, **kw) -> Workload:
