@@ -27,16 +27,16 @@ using sdpa_host::sm_count;
 
 // 0 ok, else an sdpa_status.  Caches the answer per device.
 int check_device() {
-    static int verdict[64];   // 0 unknown, 1 ok, 2 unsupported
+    static int support[64];   // 0 unknown, 1 ok, 2 unsupported
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return SDPA_ERR_CUDA;
-    if (dev >= 0 && dev < 64 && verdict[dev] != 0) return verdict[dev] == 1 ? SDPA_OK : SDPA_ERR_UNSUPPORTED;
+    if (dev >= 0 && dev < 64 && support[dev] != 0) return support[dev] == 1 ? SDPA_OK : SDPA_ERR_UNSUPPORTED;
     int major = 0, minor = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
         return SDPA_ERR_CUDA;
     const bool ok = (major == 10 && minor == 0);
-    if (dev >= 0 && dev < 64) verdict[dev] = ok ? 1 : 2;
+    if (dev >= 0 && dev < 64) support[dev] = ok ? 1 : 2;
     return ok ? SDPA_OK : SDPA_ERR_UNSUPPORTED;
 }
 
