@@ -58,13 +58,13 @@
 
 // Pairs e (0..15) of a 32-column chunk whose exponentials are evaluated on
 // the FMA pipe (exp2_poly_x2) instead of the MUFU: bit (e & 7) of the mask,
-// for 16-bit inputs and for e4m3 (whose products take half the tensor time,
-// so that the MUFU bounds it sooner).
+// for 16-bit inputs and for e4m3.  None measured fastest in the forms that
+// are launched (the split e4m3 form was fastest with 0x11 or 0x01).
 #ifndef SDPA2_POLY_MASK
 #define SDPA2_POLY_MASK 0x00
 #endif
 #ifndef SDPA2_POLY_MASK_FP8
-#define SDPA2_POLY_MASK_FP8 0x11
+#define SDPA2_POLY_MASK_FP8 0x00
 #endif
 // Register budgets (setmaxnreg) of the softmax, epilogue and producer/MMA
 // warp groups: 8 * S + 4 * E + 4 * W <= 16 * 128 (the launch allocation; per
@@ -99,7 +99,7 @@ static_assert(4 * SDPA2S_REGS_SOFTMAX + SDPA2S_REGS_EPILOGUE + SDPA2S_REGS_OTHER
 #ifndef SDPA2_DEFER_RELEASE
 #define SDPA2_DEFER_RELEASE 1
 #endif
-// 1: 16-bit inputs compute the weights before the tile max (see the softmax)
+// 1: the one-warp form computes the weights before the tile max (see the softmax)
 #ifndef SDPA2_WEIGHTS_FIRST
 #define SDPA2_WEIGHTS_FIRST 1
 #endif
@@ -177,9 +177,9 @@ struct Cfg {
     // the PV product: for e4m3, 448 * 2^-threshold, so that the largest
     // weight (2^threshold) maps to the format's largest value, 448
     static constexpr float kPLog2 = (KIND == K2_E4M3) ? 8.807354922057604f - 4.0f : 0.0f;
-    // weights before the tile max (16-bit P); e4m3 takes the max first, whose
-    // register footprint leaves room for its packing and polynomial
-    static constexpr bool kWeightsFirst = SDPA2_WEIGHTS_FIRST && KIND != K2_E4M3;
+    // one-warp form: weights against the running max before the tile max
+    // (recomputed in the rare tile whose max moves it)
+    static constexpr bool kWeightsFirst = SDPA2_WEIGHTS_FIRST != 0;
     // shared memory (offsets from a 1024-byte aligned base)
     static constexpr int kSmemQ = 0;                                 // [2 stages][QB] tiles
     static constexpr int kSmemKV = 2 * QB * kTileBytes;              // [NS] tiles
