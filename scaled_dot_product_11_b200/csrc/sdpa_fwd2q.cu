@@ -101,6 +101,13 @@ int launch_fwd2q(const Fwd2Request& r, cudaStream_t stream) {
     if (gh < 1) gh = 1;
     if (gh > r.B * r.Hq) gh = r.B * r.Hq;
     prm.group_heads = gh;
+    using sdpa::fwd2::make_fastdiv;
+    prm.div_items = make_fastdiv(gh * prm.items_per_head);
+    prm.div_gh = make_fastdiv(gh);
+    const int n_bh = r.B * r.Hq;
+    prm.div_gh_last = make_fastdiv(n_bh - ((n_bh - 1) / gh) * gh);
+    prm.div_hq = make_fastdiv(r.Hq);
+    prm.div_group = make_fastdiv(prm.group);
     prm.causal = r.causal ? 1 : 0;
     prm.causal_off = r.causal_off;
     prm.score_log2 = r.score_log2;

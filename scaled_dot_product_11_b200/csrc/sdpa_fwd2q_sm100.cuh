@@ -122,6 +122,28 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;   // bounded waits: 1 s
 // timed out, 5 = the shared-memory layout does not fit), [1] location code.
 __device__ unsigned int g_status[2];
 
+// n / d for 0 <= n < 2^31 by one multiply and a shift: m = ceil(2^(31+l) / d)
+// with l = ceil(log2 d) satisfies 2^(31+l) <= m d <= 2^(31+l) + 2^l, which
+// makes floor(m n / 2^(31+l)) = floor(n / d) for every 31-bit n (Granlund and
+// Montgomery, "Division by invariant integers using multiplication", 1994,
+// Theorem 4.2).  The schedule decodes every unit with a few of these in the
+// MMA issuer's thread, where a 64-bit division cost over a thousand cycles.
+struct FastDiv {
+    unsigned int m;
+    int s;   // 31 + l
+};
+inline FastDiv make_fastdiv(int d) {
+    int l = 0;
+    while ((1ull << l) < (unsigned long long)d) ++l;
+    FastDiv f;
+    f.m = (unsigned int)(((1ull << (31 + l)) + (unsigned long long)d - 1) / (unsigned long long)d);
+    f.s = 31 + l;
+    return f;
+}
+__device__ __forceinline__ int fdiv(int n, FastDiv f) {
+    return (int)(((unsigned long long)(unsigned int)n * f.m) >> f.s);
+}
+
 struct Params {
     void* o;                // [B,Hq,Sq,D] view, 16-bit, D contiguous (strides below)
     float* lse;             // [B,Hq,Sq] contiguous, or null
@@ -131,6 +153,11 @@ struct Params {
     int items_per_head;     // schedule items per (batch, head): causal ceil(n_pairs/2), else n_pairs
     int n_items;            // B * Hq * items_per_head
     int group_heads;        // (batch, head) pairs per schedule group
+    FastDiv div_items;      // by group_heads * items_per_head (items per group)
+    FastDiv div_gh;         // by group_heads
+    FastDiv div_gh_last;    // by the size of the last group (B * Hq - its first pair)
+    FastDiv div_hq;         // by Hq
+    FastDiv div_group;      // by Hq / Hkv
     int causal;             // 0 / 1
     int causal_off;         // query row i sees keys 0 .. i + causal_off
     float score_log2;       // raw MMA score -> log2 units
@@ -310,15 +337,17 @@ struct Unit {
 };
 
 __device__ __forceinline__ bool sched(const Params& p, int k, int sub, int& bh, int& m) {
-    const long long item = (long long)blockIdx.x + (long long)k * gridDim.x;
-    if (item >= p.n_items) return false;
-    const int n_bh = p.B * p.Hq;
+    // item < n_items < 2^31 once the bound holds; the sum cannot wrap 32 bits
+    const unsigned int item = blockIdx.x + (unsigned int)k * gridDim.x;
+    if (item >= (unsigned int)p.n_items) return false;
     const int per_group = p.group_heads * p.items_per_head;
-    const int grp = (int)(item / per_group);
-    const int within = (int)(item - (long long)grp * per_group);
-    const int gsize = min(p.group_heads, n_bh - grp * p.group_heads);
-    const int j = within / gsize;
-    bh = grp * p.group_heads + within % gsize;
+    const int grp = fdiv((int)item, p.div_items);
+    const int within = (int)item - grp * per_group;
+    const int rest = p.B * p.Hq - grp * p.group_heads;   // pairs from this group's first on
+    const bool last = rest < p.group_heads;
+    const int gsize = last ? rest : p.group_heads;
+    const int j = fdiv(within, last ? p.div_gh_last : p.div_gh);
+    bh = grp * p.group_heads + (within - j * gsize);
     const int hi = p.n_pairs - 1 - j;
     if (sub == 0) {
         m = hi;
@@ -344,7 +373,7 @@ __device__ __forceinline__ void unit_first(const Params& p, Unit& u) {
     unit_load(p, u);
 }
 __device__ __forceinline__ void unit_next(const Params& p, Unit& u) {
-    if (u.sub == 0) {
+    if (u.sub == 0 && p.causal) {   // only causal items hold a second unit
         u.sub = 1;
         unit_load(p, u);
         if (u.valid) return;
@@ -374,7 +403,7 @@ __device__ __forceinline__ void cur_next(const Params& p, Cursor& c) {
 template <int D, bool STRIDED>
 __device__ __forceinline__ long long o_offset(const Params& p, int bh, int row) {
     if constexpr (STRIDED) {
-        const int b = bh / p.Hq;
+        const int b = fdiv(bh, p.div_hq);
         return (long long)b * p.o_sb + (long long)(bh - b * p.Hq) * p.o_sh + (long long)row * p.o_ss;
     } else {
         return ((long long)bh * p.Sq + row) * D;
@@ -454,7 +483,7 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 const int row0 = (2 * u.m + s) * kRows;
                 for (int kb = 0; kb < C::kSwBlocks; ++kb) {
                     if constexpr (STRIDED) {
-                        const int b = u.bh / p.Hq;
+                        const int b = fdiv(u.bh, p.div_hq);
                         tma_load_4d(dst + kb * C::kSwBlockBytes, &tmQ, fb, kb * C::kElemsPerSw, row0,
                                     u.bh - b * p.Hq, b);
                     } else {
@@ -468,7 +497,7 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const int row0 = (2 * u.m + s) * kRows;
                     for (int kb = 0; kb < C::kSwBlocks; ++kb) {
                         if constexpr (STRIDED) {
-                            const int b = u.bh / p.Hq;
+                            const int b = fdiv(u.bh, p.div_hq);
                             tma_prefetch_l2_4d(&tmQ, kb * C::kElemsPerSw, row0, u.bh - b * p.Hq, b);
                         } else {
                             tma_prefetch_l2_3d(&tmQ, kb * C::kElemsPerSw, row0, u.bh);
@@ -481,8 +510,8 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 if (!wait(bar(C::kBarKVEmpty + slot), ((uint32_t)(t / NS) & 1u) ^ 1u, abort_addr, status,
                           0x10000u | (uint32_t)(t & 0xffff)))
                     return false;
-                const int b = u.bh / p.Hq;
-                const int kvh = (u.bh - b * p.Hq) / p.group;
+                const int b = fdiv(u.bh, p.div_hq);
+                const int kvh = fdiv(u.bh - b * p.Hq, p.div_group);
                 const uint32_t fb = bar(C::kBarKVFull + slot);
                 mbar_arrive_expect_tx(fb, C::kTileBytes);
                 for (int kb = 0; kb < C::kSwBlocks; ++kb) {
