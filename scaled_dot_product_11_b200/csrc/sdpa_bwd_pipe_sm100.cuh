@@ -77,23 +77,26 @@ __device__ __forceinline__ float2 bt_unpack(uint32_t w) {
         return __half22float2(*reinterpret_cast<const __half2*>(&w));
 }
 
-// Half `half` (columns [half*D/2, (half+1)*D/2)) of D_i = dO_i . O_i of row
-// `row` (0 past the end); 16-byte loads
+// Half of D_i = dO_i . O_i for row r of a 128-row tile, from the dO and O
+// tiles in shared memory (128-byte swizzle: 16-byte unit u of a row's
+// 128-byte segment sits at unit u ^ (row & 7)); half h covers columns
+// [h D/2, (h + 1) D/2), summed in column order.
 template <int D, bool BF16>
-__device__ __forceinline__ float bt_row_dot(const BwdTcParams& p, size_t head, int row, int half) {
-    if (row >= p.Sq) return 0.0f;
-    const size_t off = head + (size_t)row * D + (size_t)half * (D / 2);
-    const uint4* g = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.dout) + off);
-    const uint4* o = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.o) + off);
-    uint4 gv[D / 16], ov[D / 16];
+__device__ __forceinline__ float bt_row_dot_smem(uint32_t sdo, uint32_t so, int r, int half) {
+    constexpr int kUnits = D / 16;   // 16-byte units per half row
+    uint4 gv[kUnits], ov[kUnits];
 #pragma unroll
-    for (int v = 0; v < D / 16; ++v) {
-        gv[v] = g[v];
-        ov[v] = o[v];
+    for (int v = 0; v < kUnits; ++v) {
+        const int gu = half * kUnits + v;
+        const uint32_t off = (uint32_t)((gu >> 3) * 128 * 128 + r * 128 + (((gu & 7) ^ (r & 7)) << 4));
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(gv[v].x), "=r"(gv[v].y), "=r"(gv[v].z), "=r"(gv[v].w) : "r"(sdo + off));
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(ov[v].x), "=r"(ov[v].y), "=r"(ov[v].z), "=r"(ov[v].w) : "r"(so + off));
     }
     float acc = 0.0f;
 #pragma unroll
-    for (int v = 0; v < D / 16; ++v) {
+    for (int v = 0; v < kUnits; ++v) {
         const uint32_t gw[4] = {gv[v].x, gv[v].y, gv[v].z, gv[v].w};
         const uint32_t ow[4] = {ov[v].x, ov[v].y, ov[v].z, ov[v].w};
 #pragma unroll
@@ -573,12 +576,17 @@ struct CfgQ {
     static constexpr int kBarPFull = kBarDPFull + 1;               // [2]
     static constexpr int kBarDone = kBarPFull + 2;
     static constexpr int kBarDrain = kBarDone + 1;
-    static constexpr int kNumBars = kBarDrain + 1;
+    static constexpr int kBarOFull = kBarDrain + 1;   // the O tile landed (in V slot kOSlot)
+    static constexpr int kBarOFree = kBarOFull + 1;   // D_i computed: V slot kOSlot is free
+    static constexpr int kNumBars = kBarOFree + 1;
     static constexpr int kSmemSlot = kSmemBar + 8 * kNumBars;
     static constexpr int kSmemAbort = kSmemSlot + 4;
     static constexpr int kSmemUsed = kSmemAbort + 4;
     static constexpr int kSmemBytes = kSmemUsed + 1024;
     static constexpr uint32_t kColS = 0, kColDP = 256, kColAcc = 384;
+    // the rows' O tile borrows the last V slot until D_i is computed (its
+    // first V tile, kOSlot, is loaded after that)
+    static constexpr int kOSlot = kRingV - 1;
     static_assert(D == 64 || D == 128, "pipelined backward: head dims 64 and 128");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
@@ -611,12 +619,13 @@ __device__ __forceinline__ void mma_pv128(uint32_t d_tmem, uint32_t a_tmem, uint
 }
 
 // dQ: one CTA per 128 query rows of one (batch, query head), 128-key steps;
-// also writes D_i = dO_i . O_i of its rows for the dK/dV kernel.
+// also writes D_i = dO_i . O_i of its rows for the dK/dV kernel (from a TMA-loaded
+// O tile that borrows the last V slot, and the resident dO).
 template <int D, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
 sdpa_bwd_dq_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                        const BwdTcParams p) {
+                        const __grid_constant__ CUtensorMap tmO, const BwdTcParams p) {
     using C = CfgQ<D>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -654,6 +663,8 @@ sdpa_bwd_dq_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         mbar_init(bar(C::kBarDPFull), 1);
         mbar_init(bar(C::kBarDone), 1);
         mbar_init(bar(C::kBarDrain), 1);
+        mbar_init(bar(C::kBarOFull), 1);
+        mbar_init(bar(C::kBarOFree), 1);
         sts_u32(abort_addr, 0u);
         fence_barrier_init();
     }
@@ -674,11 +685,15 @@ sdpa_bwd_dq_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
             prefetch_tmap(&tmdO);
+            prefetch_tmap(&tmO);
             mbar_arrive_expect_tx(bar(C::kBarResFull), 2 * C::kTile);
             for (int kb = 0; kb < C::kSwBlocks; ++kb) {
                 tma_load_3d(sQ + kb * C::kBlock, &tmQ, bar(C::kBarResFull), kb * C::kElemsPerSw, i0, bh);
                 tma_load_3d(sdO + kb * C::kBlock, &tmdO, bar(C::kBarResFull), kb * C::kElemsPerSw, i0, bh);
             }
+            mbar_arrive_expect_tx(bar(C::kBarOFull), C::kTile);
+            for (int kb = 0; kb < C::kSwBlocks; ++kb)
+                tma_load_3d(sV(C::kOSlot) + kb * C::kBlock, &tmO, bar(C::kBarOFull), kb * C::kElemsPerSw, i0, bh);
             bool ok = true;
             int kiss = 0, viss = 0;   // K / V tiles issued
             for (int jt = 0; jt < nsteps && ok; ++jt) {
@@ -695,6 +710,8 @@ sdpa_bwd_dq_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                 if (jt >= C::kRingV)
                     ok = wait(bar(C::kBarVEmpty + vs), (uint32_t)(jt / C::kRingV - 1) & 1u, abort_addr,
                               0x72000u | (uint32_t)(jt & 0xfff));
+                else if (jt == C::kOSlot)   // the O tile there has been read
+                    ok = wait(bar(C::kBarOFree), 0, abort_addr, 0x7a000u);
                 if (!ok) break;
                 mbar_arrive_expect_tx(bar(C::kBarVFull + vs), C::kTile);
                 for (int kb = 0; kb < C::kSwBlocks; ++kb)
@@ -705,6 +722,8 @@ sdpa_bwd_dq_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             // let the copies already issued land before the CTA ends
             const uint64_t t0 = global_timer_ns();
             while (!mbar_try_wait(bar(C::kBarResFull), 0) && global_timer_ns() - t0 < 100000000ull) {
+            }
+            while (!mbar_try_wait(bar(C::kBarOFull), 0) && global_timer_ns() - t0 < 100000000ull) {
             }
             for (int jt = kiss > C::kRingK ? kiss - C::kRingK : 0; jt < kiss; ++jt)
                 while (!mbar_try_wait(bar(C::kBarKFull + jt % C::kRingK), (uint32_t)(jt / C::kRingK) & 1u) &&
@@ -782,13 +801,19 @@ sdpa_bwd_dq_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         const float nlse_r = row < p.Sq ? -(p.lse[(size_t)bh * p.Sq + row] * kL2e) : 0.0f;
         const uint64_t nl2 = f2_pack(nlse_r, nlse_r);
         // D_i: chunks 0 and 1 compute the two halves of the row's dot
-        // product, summed through shared memory
-        if (c < 2) dpart[c * 128 + r] = bt_row_dot<D, BF16>(p, (size_t)bh * p.Sq * D, row, c);
+        // product from the dO and O tiles (rows past Sq were filled with
+        // zeros), summed through shared memory; then O's slot is released
+        bool ok = true;
+        if (c < 2) {
+            ok = wait(bar(C::kBarResFull), 0, abort_addr, 0x79000u) &&
+                 wait(bar(C::kBarOFull), 0, abort_addr, 0x7b000u);
+            dpart[c * 128 + r] = ok ? bt_row_dot_smem<D, BF16>(sdO, sV(C::kOSlot), r, c) : 0.0f;
+        }
         named_bar_sync(1, kEwThreads);
+        if (threadIdx.x == 0) mbar_arrive(bar(C::kBarOFree));
         const float d_r = (dpart[r] + dpart[128 + r]) * p.d_mul;
         const uint64_t d2 = f2_pack(d_r, d_r);
         if (c == 0 && row < p.Sq) p.delta[(size_t)bh * p.Sq + row] = d_r;
-        bool ok = true;
         for (int jt = 0; jt < nsteps && ok; ++jt) {
             const int bf = jt & 1, j0 = jt * 128;
             ok = __all_sync(0xffffffffu, wait(bar(C::kBarSFull + bf), (uint32_t)(jt >> 1) & 1u, abort_addr,

@@ -275,9 +275,15 @@ def dq_model(nsteps, seed, plant=None):
     """The dQ kernel (128-key steps): Q, dO resident; K and V in separate
     rings; S double-buffered, dP single (free once every warp has read it).
     Per step: dP(jt+1) [after the weights of jt], dQ(jt) [reads dS over S_b],
-    K's slot released, S(jt+2) [overwrites S_b]."""
+    K's slot released, S(jt+2) [overwrites S_b].  The rows' O tile lands in
+    the last V slot first; half of the elementwise warps read it (with the
+    resident dO) for D_i, all of them meet at a named barrier, and one arrival
+    on o_free lets the producer load that slot's first V tile."""
     m = Machine(seed)
     res_full, done = Bar("res_full"), Bar("done")
+    o_full, o_free = Bar("o_full"), Bar("o_free")
+    o_slot = ("v", RING_V - 1)
+    ew_bar = {"arrived": 0, "gen": 0}
     k_full = [Bar("k_full%d" % i) for i in range(RING_K)]
     k_empty = [Bar("k_empty%d" % i) for i in range(RING_K)]
     v_full = [Bar("v_full%d" % i) for i in range(RING_V)]
@@ -322,6 +328,7 @@ def dq_model(nsteps, seed, plant=None):
         m.buf["res"] = None
         res_full.arrive(tx=1)
         m.tma.append((res_full, "res", 0))
+        m.copy(o_full, o_slot, "O")
         for jt in range(nsteps):
             ks, vs = jt % RING_K, jt % RING_V
             if jt >= RING_K and plant != "early_copy":
@@ -333,6 +340,9 @@ def dq_model(nsteps, seed, plant=None):
             if jt >= RING_V:
                 n = jt // RING_V - 1
                 while not v_empty[vs].ready(par(n), n):
+                    yield
+            elif ("v", vs) == o_slot and plant != "early_v":
+                while not o_free.ready(0, 0):
                     yield
             m.copy(v_full[vs], ("v", vs), jt)
             yield
@@ -379,6 +389,22 @@ def dq_model(nsteps, seed, plant=None):
         m.commit(done)
 
     def elementwise(w):
+        if w < N_EW // 2:   # D_i from dO (resident) and the O tile
+            while not (res_full.ready(0, 0) and o_full.ready(0, 0)):
+                yield
+            check(m.buf.get(o_slot) == "O", "D_i reads O before it landed", w, m.buf.get(o_slot))
+            m.readers[o_slot] = m.readers.get(o_slot, 0) + 1
+            yield
+            check(m.buf.get(o_slot) == "O", "O overwritten while D_i reads it", w, m.buf.get(o_slot))
+            m.readers[o_slot] -= 1
+        gen = ew_bar["gen"]   # named barrier of the elementwise warps
+        ew_bar["arrived"] += 1
+        if ew_bar["arrived"] == N_EW:
+            ew_bar["arrived"], ew_bar["gen"] = 0, gen + 1
+        while ew_bar["gen"] == gen:
+            yield
+        if w == 0:
+            o_free.arrive()
         for jt in range(nsteps):
             b, n = jt & 1, jt >> 1
             while not s_full[b].ready(par(n), n):
@@ -424,7 +450,7 @@ def test_dkdv_planted_mistakes_are_caught(plant):
     assert caught > 0, plant
 
 
-@pytest.mark.parametrize("plant", ["early_copy", "wrong_parity", "early_overwrite", "early_dp"])
+@pytest.mark.parametrize("plant", ["early_copy", "wrong_parity", "early_overwrite", "early_dp", "early_v"])
 def test_dq_planted_mistakes_are_caught(plant):
     caught = 0
     for seed in range(20):
