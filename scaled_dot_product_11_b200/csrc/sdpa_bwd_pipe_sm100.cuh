@@ -365,6 +365,17 @@ sdpa_bwd_dkdv_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
                           0x61000u | (uint32_t)(st & 0xfff));
             if (!ok) break;
             const int bh = step_bh(st), i0 = step_i0(st);
+            // the tiles first (their bytes are expected before the copies
+            // start), then the statistics, whose load latency overlaps the
+            // copies; lane 0's arrival after them completes the slot
+            const uint32_t fb = bar(C::kBarRingFull + slot);
+            if (lane == 0) {
+                mbar_expect_tx(fb, 2 * C::kTile64);
+                for (int kb = 0; kb < C::kSwBlocks; ++kb) {
+                    tma_load_3d(sQ(slot) + kb * C::kBlock64, &tmQ, fb, kb * C::kElemsPerSw, i0, bh);
+                    tma_load_3d(sdO(slot) + kb * C::kBlock64, &tmdO, fb, kb * C::kElemsPerSw, i0, bh);
+                }
+            }
             float* const st_lse = stats + slot * 2 * kStep;
             const size_t rows = (size_t)bh * p.Sq;
             for (int i = lane; i < kStep; i += 32) {
@@ -373,14 +384,7 @@ sdpa_bwd_dkdv_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
                 st_lse[kStep + i] = qr < p.Sq ? p.delta[rows + qr] : 0.0f;
             }
             __syncwarp();
-            if (lane == 0) {
-                const uint32_t fb = bar(C::kBarRingFull + slot);
-                mbar_arrive_expect_tx(fb, 2 * C::kTile64);
-                for (int kb = 0; kb < C::kSwBlocks; ++kb) {
-                    tma_load_3d(sQ(slot) + kb * C::kBlock64, &tmQ, fb, kb * C::kElemsPerSw, i0, bh);
-                    tma_load_3d(sdO(slot) + kb * C::kBlock64, &tmdO, fb, kb * C::kElemsPerSw, i0, bh);
-                }
-            }
+            if (lane == 0) mbar_arrive(fb);
             __syncwarp();
             issued = st + 1;
         }
