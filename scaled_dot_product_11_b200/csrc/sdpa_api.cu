@@ -338,7 +338,7 @@ int launch_bwd_pipe(const void* q, const void* k, const void* v, const sdpa::Bwd
     const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     // the dK/dV kernel streams Q, dO in 64-row boxes; everything else moves
     // in 128-row boxes
-    CUtensorMap tq128, tdo128, tk128, tv128, tq64, tdo64, to128;
+    CUtensorMap tq128, tdo128, tk128, tv128, tq64, tdo64, to128, tdq128, tdk128, tdv128;
     const View vq = bhsd(bp.Hq, bp.Sq, D), vk = bhsd(bp.Hkv, bp.Sk, D);
     const int sw = C::kElemsPerSw;
     if (!encode_view(&tq128, dt, 2, q, D, bp.Sq, bp.Hq, bp.B, vq, sw, true, 128) ||
@@ -347,7 +347,10 @@ int launch_bwd_pipe(const void* q, const void* k, const void* v, const sdpa::Bwd
         !encode_view(&tv128, dt, 2, v, D, bp.Sk, bp.Hkv, bp.B, vk, sw, true, 128) ||
         !encode_view(&tq64, dt, 2, q, D, bp.Sq, bp.Hq, bp.B, vq, sw, true, 64) ||
         !encode_view(&tdo64, dt, 2, bp.dout, D, bp.Sq, bp.Hq, bp.B, vq, sw, true, 64) ||
-        !encode_view(&to128, dt, 2, bp.o, D, bp.Sq, bp.Hq, bp.B, vq, sw, true, 128))
+        !encode_view(&to128, dt, 2, bp.o, D, bp.Sq, bp.Hq, bp.B, vq, sw, true, 128) ||
+        !encode_view(&tdq128, dt, 2, bp.dq, D, bp.Sq, bp.Hq, bp.B, vq, sw, true, 128) ||
+        !encode_view(&tdk128, dt, 2, bp.dk, D, bp.Sk, bp.Hkv, bp.B, vk, sw, true, 128) ||
+        !encode_view(&tdv128, dt, 2, bp.dv, D, bp.Sk, bp.Hkv, bp.B, vk, sw, true, 128))
         return SDPA_ERR_CUDA;
     sdpa::BwdTcParams tp;
     tp.o = bp.o; tp.dout = bp.dout; tp.lse = bp.lse; tp.delta = bp.delta;
@@ -371,9 +374,9 @@ int launch_bwd_pipe(const void* q, const void* k, const void* v, const sdpa::Bwd
     const dim3 gkv((bp.Sk + 127) / 128, bp.B * bp.Hkv);
     const dim3 gq((bp.Sq + 127) / 128, bp.B * bp.Hq);
     // dQ first: it writes D of every row, which the dK/dV kernel reads
-    kdq<<<gq, sdpa::bwdp::kThreads, dq_smem, stream>>>(tq128, tk128, tv128, tdo128, to128, tp);
+    kdq<<<gq, sdpa::bwdp::kThreads, dq_smem, stream>>>(tq128, tk128, tv128, tdo128, to128, tdq128, tp);
     if (cudaGetLastError() != cudaSuccess) return SDPA_ERR_CUDA;
-    kdkdv<<<gkv, sdpa::bwdp::kThreads, C::kSmemBytes, stream>>>(tq64, tk128, tv128, tdo64, tp);
+    kdkdv<<<gkv, sdpa::bwdp::kThreads, C::kSmemBytes, stream>>>(tq64, tk128, tv128, tdo64, tdk128, tdv128, tp);
     return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
 }
 

@@ -288,9 +288,12 @@ __device__ __forceinline__ void drain_loads(uint32_t base, int issued) {
 }
 
 // One row's 16-column accumulator chunk (TMEM address t): times `mul` (or
-// zeros), rounded, 32 bytes to dst_row
+// zeros), rounded, into the row's 32 bytes at 16-bit column `col` of a
+// 128-row tile in shared memory, in the 128-byte swizzled layout its TMA
+// store reads (64-column blocks of 128 rows x 128 bytes; 16-byte unit u of a
+// row segment at u ^ (row & 7)).
 template <bool BF16>
-__device__ __forceinline__ void store_chunk16(uint32_t t, void* dst_row, float mul, bool zero, bool live) {
+__device__ __forceinline__ void stage_chunk16(uint32_t t, uint32_t tile, int r, int col, float mul, bool zero) {
     float x[16];
     tmem_ld16(t, x);
     tmem_wait_ld();
@@ -299,14 +302,17 @@ __device__ __forceinline__ void store_chunk16(uint32_t t, void* dst_row, float m
 #pragma unroll
         for (int e = 0; e < 16; ++e) x[e] = 0.0f;
     }
-    if (!live) return;
-    uint4* dst = reinterpret_cast<uint4*>(dst_row);
 #pragma unroll
-    for (int v4 = 0; v4 < 2; ++v4)
-        dst[v4] = make_uint4(bt_pack<BF16>(x[8 * v4] * mul, x[8 * v4 + 1] * mul),
-                             bt_pack<BF16>(x[8 * v4 + 2] * mul, x[8 * v4 + 3] * mul),
-                             bt_pack<BF16>(x[8 * v4 + 4] * mul, x[8 * v4 + 5] * mul),
-                             bt_pack<BF16>(x[8 * v4 + 6] * mul, x[8 * v4 + 7] * mul));
+    for (int v4 = 0; v4 < 2; ++v4) {
+        const int gu = col / 8 + v4;
+        const uint32_t addr = tile + (uint32_t)((gu >> 3) * 128 * 128 + r * 128 + (((gu & 7) ^ (r & 7)) << 4));
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                     "r"(bt_pack<BF16>(x[8 * v4] * mul, x[8 * v4 + 1] * mul)),
+                     "r"(bt_pack<BF16>(x[8 * v4 + 2] * mul, x[8 * v4 + 3] * mul)),
+                     "r"(bt_pack<BF16>(x[8 * v4 + 4] * mul, x[8 * v4 + 5] * mul)),
+                     "r"(bt_pack<BF16>(x[8 * v4 + 6] * mul, x[8 * v4 + 7] * mul))
+                     : "memory");
+    }
 }
 
 // dK, dV: one CTA per 128 keys of one (batch, K/V head).
@@ -314,6 +320,7 @@ template <int D, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
 sdpa_bwd_dkdv_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                          const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
                           const BwdTcParams p) {
     using C = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -528,19 +535,30 @@ sdpa_bwd_dkdv_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
             if (lane == 0) mbar_arrive(bar(C::kBarPFull + bf));
         }
         // dV (chunks 0, 1: columns [0, D/2), [D/2, D)) and dK (chunks 2, 3)
-        // rows; zero when no query row sees these keys
+        // rows, zero when no query row sees these keys, staged in the ring's
+        // first 64 KB (every product that read the ring has completed) and
+        // written by two TMA stores (rows past Sk are not written)
         if (ok && nsteps > 0) ok = __all_sync(0xffffffffu, wait(bar(C::kBarDone), 0, abort_addr, 0x66000u));
+        const uint32_t tile_v = base + C::kSmemRing, tile_k = tile_v + C::kTile128;
         if (ok) {
             tc_fence_after();
             const bool is_k = c >= 2;
-            void* const out = is_k ? p.dk : p.dv;
             const float mul = is_k ? p.dk_mul : p.dv_mul;
             const int col0 = (c & 1) * (D / 2);
-            uint16_t* const orow = reinterpret_cast<uint16_t*>(out) + ((size_t)bk * p.Sk + (size_t)key) * D + col0;
             const uint32_t tacc = tmem + lane_base + C::kColAcc + (is_k ? D : 0) + col0;
 #pragma unroll 1
             for (int cc = 0; cc < D / 2; cc += 16)
-                store_chunk16<BF16>(tacc + cc, orow + cc, mul, nsteps == 0, key < p.Sk);
+                stage_chunk16<BF16>(tacc + cc, is_k ? tile_k : tile_v, r, col0 + cc, mul, nsteps == 0);
+            fence_proxy_async_smem();
+        }
+        named_bar_sync(1, kEwThreads);
+        if (ok && threadIdx.x == 0) {
+            for (int kb = 0; kb < C::kSwBlocks; ++kb) {
+                tma_store_3d(&tmdV, tile_v + kb * C::kBlock128, kb * C::kElemsPerSw, j0, bk);
+                tma_store_3d(&tmdK, tile_k + kb * C::kBlock128, kb * C::kElemsPerSw, j0, bk);
+            }
+            bulk_commit_group();
+            bulk_wait_group_read0();   // the stores have read the tiles before the CTA ends
         }
     }
     teardown<D>(base, tmem, mma_ok);
@@ -629,7 +647,8 @@ template <int D, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
 sdpa_bwd_dq_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                        const __grid_constant__ CUtensorMap tmO, const BwdTcParams p) {
+                        const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmdQ,
+                        const BwdTcParams p) {
     using C = CfgQ<D>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -875,17 +894,27 @@ sdpa_bwd_dq_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(C::kBarPFull + bf));
         }
-        // dQ row, this warp's quarter of the columns; zero when the row sees
-        // no key
+        // dQ row, this warp's quarter of the columns, zero when the row sees
+        // no key, staged in K slot 0 (every product that read K has
+        // completed) and written by one TMA store (rows past Sq are not
+        // written)
         if (ok && nsteps > 0) ok = __all_sync(0xffffffffu, wait(bar(C::kBarDone), 0, abort_addr, 0x78000u));
+        const uint32_t tile = sK(0);
         if (ok) {
             tc_fence_after();
             const int col0 = c * (D / 4);
-            uint16_t* const orow = reinterpret_cast<uint16_t*>(p.dq) + ((size_t)bh * p.Sq + (size_t)row) * D + col0;
 #pragma unroll 1
             for (int cc = 0; cc < D / 4; cc += 16)
-                store_chunk16<BF16>(tmem + lane_base + C::kColAcc + col0 + cc, orow + cc, p.dq_mul, nsteps == 0,
-                                    row < p.Sq);
+                stage_chunk16<BF16>(tmem + lane_base + C::kColAcc + col0 + cc, tile, r, col0 + cc, p.dq_mul,
+                                    nsteps == 0);
+            fence_proxy_async_smem();
+        }
+        named_bar_sync(1, kEwThreads);
+        if (ok && threadIdx.x == 0) {
+            for (int kb = 0; kb < C::kSwBlocks; ++kb)
+                tma_store_3d(&tmdQ, tile + kb * C::kBlock, kb * C::kElemsPerSw, i0, bh);
+            bulk_commit_group();
+            bulk_wait_group_read0();   // the store has read the tile before the CTA ends
         }
     }
     // end: after a failed wait no MMA may still write TMEM when it is freed
