@@ -662,7 +662,9 @@ sdpa_bwd_dq_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const float kL2e = 1.44269504088896340736f;
 
-    const int i0 = blockIdx.x * 128;
+    // causal: a head's last query tiles (the most keys) first, so that the
+    // light ones end the launch
+    const int i0 = (p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x) * 128;
     const int bh = blockIdx.y;
     const int b = bh / p.Hq, hq = bh - b * p.Hq;
     const int kvrow = b * p.Hkv + hq / p.group;        // 3-D map index of the K/V head
