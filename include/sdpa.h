@@ -318,8 +318,18 @@ SDPA_API int sdpa_launches_per_call(void);
  * bits) and with the MUFU instruction ex2.approx; results to poly and mufu
  * (device memory, n floats each).  Errors as sdpa_selftest_wait.
  */
+/*
+ * sdpa_selftest_fastdiv -- host only, needs no GPU: q[i] = floor(n[i] / d[i])
+ * for count pairs (host memory, n[i] >= 0, d[i] >= 1) by the multiply-and-
+ * shift division the forward's schedule decodes its units with (a magic
+ * number m = ceil(2^(31+l) / d), l = ceil(log2 d), computed on the host;
+ * q = (n m) >> (31 + l); Granlund and Montgomery 1994, Theorem 4.2).
+ * SDPA_ERR_INVALID_ARG for a null pointer, count < 0 or a pair out of range
+ * (q is then filled up to that pair).
+ */
 SDPA_API int sdpa_selftest_wait(unsigned int limit_us, unsigned int* out, void* stream);
 SDPA_API int sdpa_selftest_exp2(const float* x, float* poly, float* mufu, int n, void* stream);
+SDPA_API int sdpa_selftest_fastdiv(const int* n, const int* d, int count, int* q);
 
 #ifdef __cplusplus
 }

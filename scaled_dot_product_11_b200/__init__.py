@@ -21,7 +21,8 @@ __all__ = [
     "SDPA_NO_MASK", "SDPA_CAUSAL", "SDPA_CAUSAL_BOTTOM_RIGHT",
     "sdpa_fwd", "sdpa_fwd_strided", "sdpa_fwd_fp8", "sdpa_bwd", "attention_backward", "sdpa_strerror", "sdpa_device_status",
     "sdpa_launches_per_call", "attention", "attention_fp8", "sdpa_selftest_wait",
-    "sdpa_selftest_exp2", "sdpa_bwd_fp8", "sdpa_bwd_fp8_workspace_bytes", "attention_backward_fp8",
+    "sdpa_selftest_exp2", "sdpa_selftest_fastdiv", "sdpa_bwd_fp8", "sdpa_bwd_fp8_workspace_bytes",
+    "attention_backward_fp8",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -77,6 +78,8 @@ _lib.sdpa_bwd_fp8.restype = _i
 _lib.sdpa_selftest_wait.argtypes = [ctypes.c_uint, _vp, _vp]
 _lib.sdpa_selftest_wait.restype = _i
 _lib.sdpa_selftest_exp2.argtypes = [_vp, _vp, _vp, _i, _vp]
+_lib.sdpa_selftest_fastdiv.argtypes = [_vp, _vp, _i, _vp]
+_lib.sdpa_selftest_fastdiv.restype = _i
 _lib.sdpa_selftest_exp2.restype = _i
 
 
@@ -160,6 +163,12 @@ def sdpa_selftest_wait(limit_us, out, stream) -> int:
     """Raw call: the kernels' bounded wait on a barrier nothing completes;
     out is the device address of 4 uint32 (see include/sdpa.h)."""
     return int(_lib.sdpa_selftest_wait(int(limit_us), out, stream or None))
+
+
+def sdpa_selftest_fastdiv(n, d, count, q) -> int:
+    """Raw call (host memory, no GPU): q[i] = n[i] // d[i] by the schedule's
+    multiply-and-shift division (host addresses as ints)."""
+    return int(_lib.sdpa_selftest_fastdiv(n, d, int(count), q))
 
 
 def sdpa_selftest_exp2(x, poly, mufu, n, stream) -> int:

@@ -594,6 +594,11 @@ extern "C" int sdpa_selftest_wait(unsigned int limit_us, unsigned int* out, void
     return sdpa_host::selftest_wait(limit_us, out, reinterpret_cast<cudaStream_t>(stream));
 }
 
+extern "C" int sdpa_selftest_fastdiv(const int* n, const int* d, int count, int* q) {
+    if (!n || !d || !q || count < 0) return SDPA_ERR_INVALID_ARG;
+    return sdpa_host::selftest_fastdiv(n, d, count, q);
+}
+
 extern "C" int sdpa_selftest_exp2(const float* x, float* poly, float* mufu, int n, void* stream) {
     if (!x || !poly || !mufu || n <= 0) return SDPA_ERR_INVALID_ARG;
     const int rc = check_device();

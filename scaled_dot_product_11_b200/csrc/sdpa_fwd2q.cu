@@ -144,6 +144,14 @@ int selftest_exp2(const float* x, float* poly, float* mufu, int n, cudaStream_t 
     return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
 }
 
+int selftest_fastdiv(const int* n, const int* d, int count, int* q) {
+    for (int i = 0; i < count; ++i) {
+        if (n[i] < 0 || d[i] < 1) return SDPA_ERR_INVALID_ARG;
+        q[i] = sdpa::fwd2::fdiv(n[i], sdpa::fwd2::make_fastdiv(d[i]));
+    }
+    return SDPA_OK;
+}
+
 int fwd2q_status(unsigned int out[2], int clear) {
     if (cudaMemcpyFromSymbol(out, sdpa::fwd2::g_status, 2 * sizeof(unsigned int)) != cudaSuccess)
         return SDPA_ERR_CUDA;

@@ -140,7 +140,7 @@ inline FastDiv make_fastdiv(int d) {
     f.s = 31 + l;
     return f;
 }
-__device__ __forceinline__ int fdiv(int n, FastDiv f) {
+__host__ __device__ __forceinline__ int fdiv(int n, FastDiv f) {
     return (int)(((unsigned long long)(unsigned int)n * f.m) >> f.s);
 }
 

@@ -96,5 +96,7 @@ int fwd2q_status(unsigned int out[2], int clear);
 // Self-tests of that translation unit's device helpers (sdpa_selftest_*).
 int selftest_wait(unsigned int limit_us, unsigned int* out, cudaStream_t stream);
 int selftest_exp2(const float* x, float* poly, float* mufu, int n, cudaStream_t stream);
+// the schedule's multiply-and-shift division, on the host
+int selftest_fastdiv(const int* n, const int* d, int count, int* q);
 
 }  // namespace sdpa_host

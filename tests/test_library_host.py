@@ -21,7 +21,7 @@ def test_header_declares_the_entry_points():
     assert set(declared_symbols()) == {"sdpa_fwd", "sdpa_fwd_strided", "sdpa_fwd_fp8",
                                        "sdpa_bwd", "sdpa_bwd_noalloc", "sdpa_strerror",
                                        "sdpa_device_status", "sdpa_launches_per_call",
-                                       "sdpa_selftest_wait", "sdpa_selftest_exp2",
+                                       "sdpa_selftest_wait", "sdpa_selftest_exp2", "sdpa_selftest_fastdiv",
                                        "sdpa_bwd_fp8", "sdpa_bwd_fp8_workspace_bytes"}
 
 
