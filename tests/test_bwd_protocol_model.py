@@ -144,11 +144,12 @@ RING = 4          # dK/dV kernel at head dim 128: ring slots of 64-row (Q, dO) t
 N_EW = 4          # elementwise warps modelled (the kernel has 16, one arrival each)
 
 
-def dkdv_model(nsteps, seed, plant=None):
+def dkdv_model(nsteps, seed, plant=None, ring=RING):
     """The dK/dV kernel (64-row steps): K, V resident; Q, dO and the step's
     statistics streamed through one ring; S and dP double-buffered.  Per step
     dV(st) [reads S_b], S(st+2) [writes S_b], dK(st) [reads dP_b], ring slot
     released, dP(st+2) [writes dP_b]."""
+    RING = ring
     m = Machine(seed)
     res_full, done = Bar("res_full"), Bar("done")
     ring_full = [Bar("ring_full%d" % i) for i in range(RING)]
@@ -427,10 +428,11 @@ def dq_model(nsteps, seed, plant=None):
     check(not m.pipe and not m.tma, "work left in flight at exit")
 
 
-@pytest.mark.parametrize("n", [0, 1, 2, 3, 4, 5, 9])
-def test_dkdv_protocol_holds_under_random_interleavings(n):
+@pytest.mark.parametrize("ring", [4, 8])
+@pytest.mark.parametrize("n", [0, 1, 2, 3, 4, 5, 9, 17])
+def test_dkdv_protocol_holds_under_random_interleavings(n, ring):
     for seed in range(30):
-        dkdv_model(n, seed)
+        dkdv_model(n, seed, ring=ring)
 
 
 @pytest.mark.parametrize("n", [0, 1, 2, 3, 4, 5, 9])
