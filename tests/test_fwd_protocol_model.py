@@ -25,8 +25,10 @@ P_s ran; P_s is read only after the softmax wrote it; O_s is rescaled only
 after the previous product into it ran, restarted only after the epilogue read
 it, and read by the epilogue only when complete; the statistics are not
 rewritten before they are read; nothing deadlocks and nothing is in flight at
-exit.  Planted mistakes must be caught, so the model is known to be able to
-fail.
+exit.  A second, smaller model covers the split form's exchange of tile
+maxima between the two half warps of a row (a two-parity slot and a two-warp
+barrier).  Planted mistakes must be caught, so the models are known to be able
+to fail.
 """
 import random
 
@@ -289,6 +291,54 @@ def test_fwd_planted_mistakes_are_caught(plant):
     for seed in range(30):
         try:
             fwd_model(CASES["mixed"], seed, plant=plant)
+        except ModelError:
+            caught += 1
+    assert caught > 0, plant
+
+
+def xchg_model(ntiles, seed, plant=None):
+    """The split form's tile-max exchange within one stage and lane quarter:
+    two half warps (keys 0-63 and 64-127 of the same rows) each write their
+    tile max into slot (tile parity, half), arrive on a shared barrier
+    (count 2) and, once both have, read the other half's value.  The slot of
+    a tile parity is rewritten two tiles later, which the barrier of the tile
+    in between orders after the other half's read."""
+    m = Machine(seed)
+    xbar = Bar("xchg", count=2)
+    slots = {}
+
+    def par(intended):
+        p = intended & 1
+        return 1 - p if plant == "wrong_parity" else p
+
+    def half(h):
+        for cs in range(ntiles):
+            slot = (0 if plant == "single_buffer" else cs & 1, h)
+            slots[slot] = (h, cs)
+            yield
+            xbar.arrive()
+            while not xbar.ready(par(cs), cs):
+                yield
+            other = (slot[0], 1 - h)
+            yield
+            check(slots.get(other) == (1 - h, cs), "exchange slot holds another tile's max", h, cs, slots.get(other))
+            yield
+
+    run(m, [half(0), half(1)])
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 8, 17])
+def test_xchg_protocol_holds(n):
+    for seed in range(40):
+        xchg_model(n, seed)
+
+
+@pytest.mark.parametrize("plant", ["single_buffer", "wrong_parity"])
+def test_xchg_planted_mistakes_are_caught(plant):
+    caught = 0
+    for seed in range(40):
+        try:
+            xchg_model(8, seed, plant=plant)
         except ModelError:
             caught += 1
     assert caught > 0, plant
