@@ -316,7 +316,8 @@ def median_launch_ms(run, stream, n):
 
 
 def config_sweep(dev, launches=20, warmup=3):
-    """Every BASELINE-shaped workload besides the headline, one GPU: device
+    """Every other workload the pages measure (tiny, ViT, GQA, MQA, FP8, two
+    sequence-sweep points), one GPU: device
     time over `launches` launches after `warmup`, TFLOP/s, roofline fraction,
     and the largest |O - O_ref| over sampled rows against the oracle; then the
     backward on the causal LM shape (timing only)."""
