@@ -187,6 +187,16 @@ def cpu_baseline(w, seconds):
                       % (nrows, w.name, t)}
 
 
+def arm_config(w, world):
+    """The `config` object of the JSON line; both arms print the same one."""
+    elt = 1 if w.dtype == "e4m3" else 2
+    in_mb = (w.B * w.Hq * w.Sq + 2 * w.B * w.Hkv * w.Sk) * w.d * elt / 1e6
+    l2_note = ("inputs %.0f MB per GPU > 126 MB L2; no flush" % in_mb if in_mb > 126
+               else "inputs %.0f MB per GPU fit in L2: L2-warm timing" % in_mb)
+    return dict(w.describe(), global_batch=w.B * world,
+                parallelism="dp%d (independent batches per GPU)" % world, l2=l2_note)
+
+
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -211,7 +221,7 @@ def run_reference(args, w):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": dict(w.describe(), parallelism="none (host cores)"),
+        "config": arm_config(w, args.gpus),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": nt, "kind": "oracle",
                          "sample": "%d random rows per step of %s, fp64 C oracle, OpenMP"
                                    % (rows_per_step, w.name)},
@@ -555,9 +565,6 @@ def main():
         torch.cuda.synchronize()
 
     if rank == 0:
-        in_mb = sum(t.numel() * t.element_size() for t in (q, k, v)) / 1e6
-        l2_note = ("inputs %.0f MB per GPU > 126 MB L2; no flush" % in_mb if in_mb > 126
-                   else "inputs %.0f MB per GPU fit in L2: L2-warm timing" % in_mb)
         peaks, src = load_peaks()
         # a contraction takes the peak of its own dtype: e4m3 is the measured
         # bf16 figure times the nominal dense fp8 / bf16 ratio (2)
@@ -586,9 +593,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3" if fp8 else w.dtype, "data": "synthetic",
-            "config": dict(w.describe(), global_batch=w.B * world,
-                           parallelism="dp%d (independent batches per GPU)" % world,
-                           l2=l2_note),
+            "config": arm_config(w, world),
             "roofline": roofline,
             "clocks": clk,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
