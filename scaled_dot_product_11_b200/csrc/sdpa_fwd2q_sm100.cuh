@@ -99,6 +99,11 @@ static_assert(4 * SDPA2S_REGS_SOFTMAX + SDPA2S_REGS_EPILOGUE + SDPA2S_REGS_OTHER
 #ifndef SDPA2_DEFER_RELEASE
 #define SDPA2_DEFER_RELEASE 1
 #endif
+// 1: split form, edge tiles: a 32-key chunk that every row of a warp has
+// masked gets zero weights without exponentials
+#ifndef SDPA2_SKIP_MASKED
+#define SDPA2_SKIP_MASKED 1
+#endif
 // 1: the one-warp form computes the weights before the tile max (see the softmax)
 #ifndef SDPA2_WEIGHTS_FIRST
 #define SDPA2_WEIGHTS_FIRST 1
@@ -284,6 +289,17 @@ __device__ __forceinline__ bool wait_sleep(uint32_t bar, uint32_t parity, uint32
     return wait_slow(bar, parity, abort_addr, status, where, SDPA2_EPI_SLEEP_NS);
 }
 
+// Zero weights into chunk c (32 keys) of a P tile starting at TMEM address tP.
+template <int KIND, int WORDS_PER_32>
+__device__ __forceinline__ void zero_p_chunk(uint32_t tP, int c) {
+    uint32_t z[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) z[i] = 0u;
+    if constexpr (KIND == K2_E4M3)
+        tmem_st8(tP + WORDS_PER_32 * c, z);
+    else
+        tmem_st16(tP + WORDS_PER_32 * c, z);
+}
 template <int KIND>
 __device__ __forceinline__ constexpr bool poly_pair(int e) {
     return (((KIND == K2_E4M3 ? SDPA2_POLY_MASK_FP8 : SDPA2_POLY_MASK) >> (e & 7)) & 1) != 0;
@@ -1007,9 +1023,12 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 const int key0 = j * kKeys + 64 * h;
                 const bool edge = (key0 + 64 > p.Sk) || (p.causal && key0 + 63 > row0 + p.causal_off);
                 int lim = 64;
+                int nch = 2;   // leading 32-key chunks of the half not masked for the whole warp
                 if (edge) {
                     lim = p.Sk - key0;
                     if (p.causal) lim = min(lim, row + p.causal_off - key0 + 1);
+                    if (SDPA2_SKIP_MASKED)
+                        nch = min(2, max(0, (__reduce_max_sync(0xffffffffu, lim) + 31) >> 5));
                 }
                 // 32 scores of the half (chunk c), masked past Sk and after
                 // row + causal_off
@@ -1026,13 +1045,15 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 // The max comes first, one chunk at a time; the scores are
                 // read again for the weights (the chunk-0 weights overwrite
                 // only chunk-0 columns), so 32 of them are live at a time.
-                float hm;
-                {
+                float hm = -INFINITY;
+                if (nch > 0) {
                     float sc[32];
                     load32(0, sc);
                     hm = max32(sc);
-                    load32(1, sc);
-                    hm = fmaxf(hm, max32(sc));
+                    if (nch > 1) {
+                        load32(1, sc);
+                        hm = fmaxf(hm, max32(sc));
+                    }
                 }
                 // the row's tile max: this half's and the partner's, through
                 // shared memory (slots alternate with the tile parity)
@@ -1070,13 +1091,16 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 }
                 const float nm = C::kPLog2 - m_run;
                 const uint64_t nm2 = f2_pack(nm, nm);
-                uint64_t acc;
-                {
-                    float sc[32];
-                    load32(0, sc);
-                    acc = exp_chunk(sc, nm2, 0);
-                    load32(1, sc);
-                    acc = f2_add(acc, exp_chunk(sc, nm2, 1));
+                uint64_t acc = 0ull;
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    if (c < nch) {
+                        float sc[32];
+                        load32(c, sc);
+                        acc = f2_add(acc, exp_chunk(sc, nm2, c));
+                    } else {
+                        zero_p_chunk<KIND, C::kPWordsPer32>(tS, c);
+                    }
                 }
                 tmem_wait_st();
                 tc_fence_before();

@@ -134,6 +134,11 @@ SMALL = [
     (1, 2, 2, 200, 3200, 128, False),
     (1, 4, 2, 130, 3329, 128, False),
     (1, 2, 2, 100, 3100, 64, False),
+    # head dim 64, edge tiles whose last 32 or 64 keys every row of a warp
+    # has masked (zero weights written without exponentials)
+    (1, 2, 2, 150, 130, 64, False),
+    (1, 2, 2, 160, 160, 64, True),
+    (2, 3, 1, 200, 196, 64, False),
     # head dim 32 (64-byte rows, 64-byte swizzle)
     (1, 2, 2, 256, 256, 32, False),
     (1, 3, 3, 300, 300, 32, True),
