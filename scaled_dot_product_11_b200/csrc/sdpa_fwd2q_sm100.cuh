@@ -80,6 +80,19 @@
 #endif
 static_assert(8 * SDPA2_REGS_SOFTMAX + 4 * SDPA2_REGS_EPILOGUE + 4 * SDPA2_REGS_OTHER <= 16 * 128,
               "register split exceeds the launch allocation");
+// e4m3 inputs (one-warp form): the softmax holds packed e4m3 words besides
+// the fp32 scores and takes more, the other groups less
+#ifndef SDPA2_REGS_SOFTMAX_FP8
+#define SDPA2_REGS_SOFTMAX_FP8 200
+#endif
+#ifndef SDPA2_REGS_EPILOGUE_FP8
+#define SDPA2_REGS_EPILOGUE_FP8 40
+#endif
+#ifndef SDPA2_REGS_OTHER_FP8
+#define SDPA2_REGS_OTHER_FP8 72
+#endif
+static_assert(8 * SDPA2_REGS_SOFTMAX_FP8 + 4 * SDPA2_REGS_EPILOGUE_FP8 + 4 * SDPA2_REGS_OTHER_FP8 <= 16 * 128,
+              "register split exceeds the launch allocation");
 // The split form (two softmax warps per lane quarter and stage, 768 threads)
 // is launched with 80 registers a thread (65536 / 768, rounded down to a
 // multiple of 8); setmaxnreg moves registers only within that allocation, so
@@ -489,7 +502,7 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
 
     if (warp >= C::kLoadWarp) {
         if constexpr (SPLIT) regs_dec<SDPA2S_REGS_OTHER>();
-        else regs_dec<SDPA2_REGS_OTHER>();
+        else regs_dec<KIND == K2_E4M3 ? SDPA2_REGS_OTHER_FP8 : SDPA2_REGS_OTHER>();
         if (warp == C::kLoadWarp && lane == 0) {
             // ================= TMA producer ==============================
             bool ok = true;
@@ -761,7 +774,7 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
     } else if (warp < C::kSoftmaxWarps && !SPLIT) {
         // ================= softmax, one stage per warp group ==============
-        regs_inc<SDPA2_REGS_SOFTMAX>();
+        regs_inc<KIND == K2_E4M3 ? SDPA2_REGS_SOFTMAX_FP8 : SDPA2_REGS_SOFTMAX>();
         const int s = warp >> 2;                 // stage
         const int quarter = warp & 3;            // TMEM lane quarter
         const int r = (int)(threadIdx.x & 127);  // row within the stage tile
@@ -1127,7 +1140,7 @@ sdpa_fwd2q_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     } else {
         // ================= epilogue (4 warps after the softmax warps) =====
         if constexpr (SPLIT) regs_dec<SDPA2S_REGS_EPILOGUE>();
-        else regs_dec<SDPA2_REGS_EPILOGUE>();
+        else regs_dec<KIND == K2_E4M3 ? SDPA2_REGS_EPILOGUE_FP8 : SDPA2_REGS_EPILOGUE>();
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;       // row within the stage tile = TMEM lane
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
