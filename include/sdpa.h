@@ -31,6 +31,15 @@
  * legacy default stream) and errors raised while it runs surface at the
  * caller's next synchronisation.
  *
+ * CUDA graphs: the compute entry points may be called while `stream` is being
+ * captured.  The host work (argument checks, tensor-map encoding) runs at
+ * capture time and the captured graph holds only the kernel launches, whose
+ * arguments -- including every device pointer -- are fixed then; a replay
+ * reads the inputs found at those addresses at replay time.  Make one call of
+ * each entry point on the device before the capture: the first call sets the
+ * kernels' shared-memory attribute and (with lazy module loading) loads the
+ * module.
+ *
  * Errors: every entry point returns an sdpa_status.  There is no fallback
  * path: a request the kernels cannot serve is refused with a status (the
  * codelab's cuDNN back-end likewise raises instead of silently falling back,
